@@ -1,0 +1,417 @@
+"""Pins of the CPU oracle to what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a
+hand-worked example (tests/golden/worked_examples.json), an identity the
+zaya page prints, a textbook routine the block reduces to in a special
+case, or a brute-force structural property (causality, window reach).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import zaya_oracle as Z
+from synthetic import gen_block_weights, gen_prefill_inputs, get_config
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = get_config("tiny")
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    out = Z.block_prefill(cfg, W, inp["x"], inp["attn_mask"], inp["router_state_in"])
+    return cfg, W, inp, out
+
+
+# ---------------------------------------------------------------- worked examples
+
+def test_conv_worked_examples():
+    g = _load("worked_examples.json")
+    for key in ("conv_fresh", "conv_with_state"):
+        ex = g[key]
+        w = np.array([ex["taps_t-2_t-1_t"]])
+        y = Z.causal_conv(np.array(ex["u"])[:, None], w, np.array([ex["bias"]]), np.array(ex["hist"])[:, None])
+        np.testing.assert_allclose(y[:, 0], ex["y"], rtol=0, atol=1e-12)
+
+
+def test_cca_residual_worked_example():
+    ex = _load("worked_examples.json")["cca_mean_residual"]
+    q = np.array(ex["q_pre"])[None, :, None]
+    k = np.array(ex["k_pre"])[None, :, None]
+    qr, kr = Z.cca_mean_residual(q, k, ex["n_q"], ex["n_kv"])
+    np.testing.assert_allclose(qr.ravel(), ex["q_res"], atol=1e-12)
+    np.testing.assert_allclose(kr.ravel(), ex["k_res"], atol=1e-12)
+
+
+def test_norms_rope_merge_worked_examples():
+    g = _load("worked_examples.json")
+    ex = g["l2_to_sqrt_d"]
+    np.testing.assert_allclose(Z.l2_to_sqrt_d(np.array(ex["x"]), 1e-6), ex["y"], atol=1e-12)
+    ex = g["rms_norm"]
+    np.testing.assert_allclose(Z.rms_norm(np.array(ex["x"]), np.array(ex["w"]), ex["eps"]), ex["y"], atol=1e-12)
+    ex = g["rope_half"]
+    for a, b in (("x_a", "y_a"), ("x_b", "y_b")):
+        y = Z.rope(np.array(ex[a])[None, None, :], [ex["pos"]], ex["rot"], ex["theta"])
+        np.testing.assert_allclose(y.ravel(), ex[b], atol=1e-12)
+    ex = g["merge"]
+    p = np.array([[ex["hb"]], [ex["hs"]], [ex["rb"]], [ex["rs"]]])
+    c, s = Z.merge(np.array([ex["o"]]), np.array([ex["r"]]), p)
+    assert c[0] == ex["contribution"] and s[0] == ex["stream"]
+
+
+def test_activations_closed_form():
+    ex = _load("worked_examples.json")["activations"]
+    for x, y in ex["gelu"]:
+        assert Z.gelu(np.array(x)) == pytest.approx(y, abs=1e-15)
+    for x, y in ex["silu"]:
+        assert Z.silu(np.array(x)) == pytest.approx(y, abs=1e-15)
+
+
+def test_selection_worked_examples():
+    ex = _load("worked_examples.json")["selection"]
+    for c in ex["cases"]:
+        cls, idx, w, p, gap = Z.select(np.array([c["logits"]]), np.array(c["bias"]), ex["n_experts"])
+        assert int(cls[0]) == c["cls"], c["note"]
+        assert int(idx[0]) == c["idx"], c["note"]
+        assert w[0] == pytest.approx(c["w"], abs=1e-7), c["note"]
+
+
+# ---------------------------------------------------------------- page identities
+
+def test_contribution_identity(tiny):
+    """layer_output == (layer_mid + m.rb) * m.rs + mlp_output and
+    layer_mid == (layer_input + a.rb) * a.rs + attention_output, in float32
+    (zaya page, 'The contributions are the merges' scaled terms')."""
+    cfg, W, inp, o = tiny
+    f = lambda a: torch.tensor(a, dtype=torch.float32)
+    a, m = W["merge_a"], W["merge_m"]
+    h = (f(o["layer_input"]) + a[2]) * a[3] + f(o["attention_output"])
+    torch.testing.assert_close(h, f(o["layer_mid"]))
+    out = (f(o["layer_mid"]) + m[2]) * m[3] + f(o["mlp_output"])
+    torch.testing.assert_close(out, f(o["layer_output"]))
+
+
+def test_router_identity_and_skip(tiny):
+    """softmax(router_logits.float()).gather(idx) == expert_weights where an
+    expert was chosen; skip slots read (0, 0) and leave mlp_output =
+    hidden_states_bias * hidden_states_scale (zaya page, 'One expert per
+    token' and 'Ablating an expert leaves the merge's bias')."""
+    cfg, W, inp, o = tiny
+    E = cfg.n_experts
+    logits = torch.tensor(o["router_logits"], dtype=torch.float32)
+    probs = logits.softmax(-1)
+    idx = torch.tensor(o["expert_indices"]).long()
+    w = torch.tensor(o["expert_weights"], dtype=torch.float32)
+    cls = o["expert_cls"]
+    chose = torch.tensor(cls != E)
+    assert chose.any() and (~chose).any(), "the tiny workload must route some tokens to skip"
+    g = probs.gather(-1, idx[..., None])[..., 0]
+    torch.testing.assert_close(g[chose], w[chose])
+    assert (idx[~chose] == 0).all() and (w[~chose] == 0).all()
+    skip = cls == E
+    assert np.all(o["routed_output"][skip] == 0)
+    hb, hs = Z.as64(W["merge_m"][0]), Z.as64(W["merge_m"][1])
+    np.testing.assert_array_equal(o["mlp_output"][skip], np.broadcast_to(Z.round_bf16(hb * hs), o["mlp_output"][skip].shape))
+
+
+def test_expert_ablation(tiny):
+    """Zeroing expert e's weight changes mlp_output exactly at the tokens
+    with (idx == e) & (w > 0) (zaya page, 'Ablating an expert ...')."""
+    cfg, W, inp, o = tiny
+    m_in = o["mlp_norm_output"][0]
+    cls, w = o["expert_cls"][0], o["expert_weights"][0]
+    h = o["layer_mid"][0]
+    for e in range(cfg.n_experts):
+        w_abl = np.where(o["expert_indices"][0] == e, 0.0, w)
+        routed = Z.moe(cfg, W, m_in, cls, w_abl)
+        ablated, _ = Z.merge(routed, h, Z.as64(W["merge_m"]))
+        changed = (ablated != o["mlp_output"][0]).any(-1)
+        chose = (o["expert_indices"][0] == e) & (w > 0)
+        np.testing.assert_array_equal(changed, chose)
+
+
+def test_zero_attention_contribution(tiny):
+    """hidden_states_scale = 0 on the first merge leaves (x + rb) * rs
+    (zaya page, 'Zeroing attention_output removes the term ...')."""
+    cfg, W, inp, _ = tiny
+    W2 = dict(W)
+    ma = W["merge_a"].clone()
+    ma[1] = 0.0
+    W2["merge_a"] = ma
+    o = Z.block_prefill(cfg, W2, inp["x"], None, inp["router_state_in"])
+    assert np.all(o["attention_output"] == 0)
+    x = Z.as64(inp["x"])
+    np.testing.assert_array_equal(o["layer_mid"], Z.round_f32((x + Z.as64(ma[2])) * Z.as64(ma[3])))
+
+
+# ---------------------------------------------------------------- special cases
+
+def test_temp_zero_uniform_attention():
+    """temp = 0 zeroes every key, so each query mixes the values of its
+    visible window uniformly (zaya page, family docstring: 'at its initial
+    value of zero every key is zero and the pattern uniform').  Uses 2 kv
+    heads with 2 query heads each, so the head -> kv-head map is pinned."""
+    cfg = get_config("tiny").with_(n_q=4, n_kv=2, temp_mode="zero", window=8, seq=20)
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    o = Z.block_prefill(cfg, W, inp["x"], None, inp["router_state_in"])
+    assert np.all(o["attention_keys"] == 0)
+    v = o["attention_values"][0]            # [nkv, S, d]
+    S, d = cfg.seq, cfg.head_dim
+    prem = o["attention_premix"][0].reshape(S, cfg.n_q, d)
+    for i in range(S):
+        lo = max(0, i - cfg.window + 1)
+        for h in range(cfg.n_q):
+            np.testing.assert_allclose(prem[i, h], v[h // 2, lo:i + 1].mean(axis=0), rtol=1e-12, atol=1e-12)
+
+
+def test_plain_gqa_special_case():
+    """With conv taps (0,0,1), zero conv bias, no CCA residual, no delayed
+    values, no rotation and a window >= S, the attention half is plain
+    L2-normed causal GQA: compared with torch's scaled_dot_product_attention
+    in float64."""
+    cfg = get_config("tiny").with_(n_q=4, n_kv=2, cca_mean_residual=0, v_delayed=0, rot_dim=0,
+                                   window=1000, seq=24)
+    W = dict(gen_block_weights(cfg))
+    cw = torch.zeros_like(W["conv_w"])
+    cw[:, 2] = 1.0
+    W["conv_w"], W["conv_b"] = cw, torch.zeros_like(W["conv_b"])
+    inp = gen_prefill_inputs(cfg)
+    o = Z.block_prefill(cfg, W, inp["x"], None, inp["router_state_in"])
+    S, d, H = cfg.seq, cfg.head_dim, cfg.hidden
+    a_in = torch.tensor(o["attention_norm_output"][0])
+    proj = a_in @ W["w_qkv"].double().T
+    proj = torch.tensor(Z.round_bf16(proj.numpy()))
+    q = proj[:, :cfg.q_dim].reshape(S, cfg.n_q, d).transpose(0, 1)
+    k = proj[:, cfg.q_dim:cfg.q_dim + cfg.kv_dim].reshape(S, cfg.n_kv, d).transpose(0, 1)
+    vc = proj[:, cfg.q_dim + cfg.kv_dim:cfg.q_dim + cfg.kv_dim + cfg.v_half]
+    vd = proj[:, cfg.q_dim + cfg.kv_dim + cfg.v_half:]
+    hd = d // 2
+    v = torch.stack([torch.cat([vc[:, g * hd:(g + 1) * hd], vd[:, g * hd:(g + 1) * hd]], -1)
+                     for g in range(cfg.n_kv)])
+    q = torch.nn.functional.normalize(q, dim=-1) * math.sqrt(d)
+    k = torch.nn.functional.normalize(k, dim=-1) * math.sqrt(d)
+    k = torch.tensor(Z.round_bf16(k.numpy()))
+    v = torch.tensor(Z.round_bf16(v.numpy()))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q[None], k[None], v[None], is_causal=True, enable_gqa=True)[0]
+    np.testing.assert_allclose(o["attention_premix"][0], ref.transpose(0, 1).reshape(S, -1).numpy(),
+                               rtol=1e-10, atol=1e-10)
+
+
+def test_rope_is_complex_rotation_and_relative():
+    """Rotate-half RoPE on dims (i, i+rot/2) is multiplication of
+    x_i + j x_{i+rot/2} by exp(j * pos * inv_freq_i); scores depend only on
+    the position difference."""
+    rng = np.random.default_rng(0)
+    rot, theta = 32, 1e4
+    x = rng.standard_normal((5, 1, 64))
+    pos = np.array([0, 1, 7, 30, 63])
+    y = Z.rope(x, pos, rot, theta)
+    inv = Z.rope_inv_freq(rot, theta)
+    ang = Z.round_f32(pos[:, None] * inv[None, :])
+    z = (x[:, 0, :16] + 1j * x[:, 0, 16:32]) * np.exp(1j * ang)
+    np.testing.assert_allclose(y[:, 0, :16], z.real, atol=1e-12)
+    np.testing.assert_allclose(y[:, 0, 16:32], z.imag, atol=1e-12)
+    np.testing.assert_array_equal(y[:, 0, 32:], x[:, 0, 32:])
+    q, k = rng.standard_normal((1, 1, 64)), rng.standard_normal((1, 1, 64))
+    s0 = (Z.rope(q, [10], rot, theta) * Z.rope(k, [3], rot, theta)).sum()
+    s1 = (Z.rope(q, [50], rot, theta) * Z.rope(k, [43], rot, theta)).sum()
+    assert s0 == pytest.approx(s1, rel=1e-5)
+
+
+def test_expert_permutation_closed_form():
+    """An expert whose gate is a permutation sigma, up the identity and down
+    a permutation tau gives y_i = silu(x[sigma(tau(i))]) * x[tau(i)];
+    sigma and tau are not involutions, so a transposed operand fails."""
+    n = 6
+    sigma = np.array([1, 2, 3, 4, 5, 0])
+    tau = np.array([2, 0, 4, 1, 5, 3])
+    P = lambda perm: np.eye(n)[perm]                 # (P @ x)[j] = x[perm[j]]
+    wgu = np.concatenate([P(sigma), np.eye(n)], axis=0)
+    x = np.array([[0.3, -1.2, 2.0, 0.7, -0.4, 1.5]])
+    y = Z.expert_ffn(x, wgu, P(tau), n)
+    expect = [Z.silu(x[0, sigma[tau[i]]]) * x[0, tau[i]] for i in range(n)]
+    np.testing.assert_allclose(y[0], expect, atol=1e-14)
+
+
+# ---------------------------------------------------------------- brute force
+
+def _perturbed(cfg, W, inp, t):
+    x2 = inp["x"].clone()
+    x2[0, t] += 0.5
+    return Z.block_prefill(cfg, W, x2, None, inp["router_state_in"])
+
+
+def test_causality_brute_force(tiny):
+    """Perturbing token t leaves every output before t bit-identical."""
+    cfg, W, inp, o = tiny
+    for t in (0, 5, 31, 63):
+        o2 = _perturbed(cfg, W, inp, t)
+        for key in ("layer_output", "router_state", "router_logits", "attention_premix"):
+            np.testing.assert_array_equal(o2[key][0, :t], o[key][0, :t])
+        assert not np.array_equal(o2["layer_output"][0, t], o["layer_output"][0, t])
+
+
+def test_window_and_conv_reach(tiny):
+    """Keys j in {t, t+1, t+2} depend on token t (width-3 conv and the
+    delayed value half), and a query i sees keys with 0 <= i-j < W.  So
+    outputs at i >= t+W+2 are bit-identical and the output at t+W+1
+    changes; reading the window as i-j <= W would move that edge by one."""
+    cfg, W, inp, o = tiny
+    Wn = cfg.window
+    for t in (0, 10, 20):
+        o2 = _perturbed(cfg, W, inp, t)
+        edge = t + Wn + 1
+        assert edge < cfg.seq - 1
+        np.testing.assert_array_equal(o2["attention_premix"][0, edge + 1:], o["attention_premix"][0, edge + 1:])
+        np.testing.assert_array_equal(o2["layer_output"][0, edge + 1:], o["layer_output"][0, edge + 1:])
+        assert not np.array_equal(o2["attention_premix"][0, edge], o["attention_premix"][0, edge])
+
+
+def test_decode_continues_prefill(tiny):
+    """prefill(S) then one decode step equals prefill(S+1) at position S,
+    for the outputs and the state it leaves (KV, conv_state, prev_hs)."""
+    cfg, W, inp, _ = tiny
+    S = cfg.seq
+    x = inp["x"]
+    r = inp["router_state_in"]
+    full = Z.block_prefill(cfg, W, x, None, r)
+    part = Z.block_prefill(cfg.with_(seq=S - 1), W, x[:, :S - 1], None, r[:, :S - 1])
+    st = part["state"]
+    cap = S + 3
+    B = 1
+    kc = np.zeros((B, cfg.n_kv, cap, cfg.head_dim))
+    vc = np.zeros_like(kc)
+    kc[:, :, :S - 1] = st["k_cache"]
+    vc[:, :, :S - 1] = st["v_cache"]
+    state = dict(k_cache=kc, v_cache=vc, conv_state=st["conv_state"], prev_hs=st["prev_hs"],
+                 cache_len=st["cache_len"])
+    dec = Z.block_decode(cfg, W, x[:, S - 1], state, r[:, S - 1])
+    for key in ("layer_output", "router_state", "attention_output", "mlp_output"):
+        np.testing.assert_allclose(dec[key], full[key][:, S - 1], rtol=1e-9, atol=1e-9)
+    np.testing.assert_array_equal(dec["expert_cls"], full["expert_cls"][:, S - 1])
+    np.testing.assert_allclose(dec["state"]["k_cache"][:, :, :S], full["state"]["k_cache"], rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(dec["state"]["v_cache"][:, :, :S], full["state"]["v_cache"], rtol=1e-9, atol=1e-9)
+    np.testing.assert_array_equal(dec["state"]["conv_state"], full["state"]["conv_state"])
+    np.testing.assert_array_equal(dec["state"]["prev_hs"], full["state"]["prev_hs"])
+    assert int(dec["state"]["cache_len"][0]) == S
+
+
+@pytest.mark.parametrize("rot", [0, 32])
+def test_left_padding_equals_unpadded(tiny, rot):
+    """A left-padded sequence's real rows equal the unpadded sequence's
+    (padding is absent; RoPE sees only position differences).  Without
+    rotation the match is exact up to summation order; with it, the fp32
+    angles differ by rounding, which can move a bf16-rounded contribution
+    by one unit in the last place."""
+    cfg, W, inp, _ = tiny
+    cfg = cfg.with_(rot_dim=rot)
+    S, P = cfg.seq, 9
+    x = inp["x"][:, :S - P]
+    r = inp["router_state_in"][:, :S - P]
+    ref = Z.block_prefill(cfg.with_(seq=S - P), W, x, None, r)
+    g = torch.Generator().manual_seed(5)
+    xp = torch.cat([torch.randn(1, P, cfg.hidden, generator=g), x], dim=1)
+    rp = torch.cat([torch.randn(1, P, cfg.router_hidden, generator=g), r], dim=1)
+    mask = torch.ones(1, S, dtype=torch.int32)
+    mask[0, :P] = 0
+    o = Z.block_prefill(cfg, W, xp, mask, rp)
+    tol = 1e-9 if rot == 0 else 8e-3
+    np.testing.assert_allclose(o["layer_output"][0, P:], ref["layer_output"][0], rtol=tol, atol=tol)
+    np.testing.assert_array_equal(o["expert_cls"][0, P:], ref["expert_cls"][0])
+    np.testing.assert_array_equal(o["expert_cls"][0, :P], cfg.n_experts)
+
+
+# ---------------------------------------------------------------- printed sizes
+
+def test_page_sizes():
+    facts = _load("page_facts.json")
+    cfg = get_config("prefill_4k")
+    kv = facts["kv_cache_bytes_per_token"]
+    assert kv["layers"] * 2 * cfg.n_kv * cfg.head_dim * 2 == kv["value"]
+    e = facts["embed_bytes"]
+    assert e["shape"][0] * e["shape"][1] * e["dtype_bytes"] == e["value"]
+    assert e["shape"][1] == cfg.hidden
+    pr = facts["projections"]
+    assert pr["q"][1] == cfg.q_dim and pr["k"][1] == cfg.kv_dim
+    assert pr["v_current"][1] == cfg.v_half and pr["v_delayed"][1] == cfg.v_half
+    assert pr["o"] == [cfg.q_dim, cfg.hidden]
+    assert pr["router_down"][1] == cfg.router_hidden and pr["router_out"][1] == cfg.n_experts + 1
+    assert facts["conv_channels"]["value"] == cfg.qk_channels
+    assert facts["conv_state_shape"]["value"][1] == cfg.qk_channels
+    assert facts["prev_hs_shape"]["value"][1] == cfg.hidden
+
+
+# ---------------------------------------------------------------- router MLP order, stack
+
+def test_router_mlp_order_special_case():
+    """With fc1 = 2*I, fc2 = I, zero biases, unit norm weight, out_proj
+    = the first E+1 unit rows and a constant router state, the router MLP
+    reduces to gelu(gelu(2 * 1)) in every logit (norm -> fc1 -> GELU ->
+    fc2 -> GELU -> out_proj); computed here with math.erf."""
+    R, E = 8, 3
+    W = {"router_norm_w": np.ones(R), "fc1_w": 2 * np.eye(R), "fc1_b": np.zeros(R),
+         "fc2_w": np.eye(R), "fc2_b": np.zeros(R), "out_w": np.eye(R)[:E + 1]}
+    r = np.full((2, R), 3.7)
+    g = lambda x: 0.5 * x * (1 + math.erf(x / math.sqrt(2)))
+    expect = np.float32(g(g(2.0)))
+    logits = Z.router_mlp(r, W, 0.0)
+    np.testing.assert_allclose(logits, np.full((2, E + 1), expect), rtol=1e-6)
+
+
+def test_embed_and_head_closed_form():
+    """stream0 = fp32((E[id] + shift) * mult); logits = norm(x) @ E^T with
+    the tied table: for x = c * e_k, norm(x) = sqrt(H) * w_k * e_k."""
+    cfg = get_config("tiny").with_(emb_shift=0.25)
+    V, H = 7, cfg.hidden
+    table = np.arange(V, dtype=np.float64)[:, None] * np.ones((1, H)) / 8.0
+    ids = np.array([[3, 0, 6]])
+    te, x = Z.embed(cfg, table, ids)
+    np.testing.assert_array_equal(x[0, :, 0], Z.round_f32((np.array([3, 0, 6]) / 8.0 + 0.25) * cfg.emb_mult))
+    k = 5
+    xs = np.zeros((1, H))
+    xs[0, k] = 3.0
+    wn = np.ones(H)
+    wn[k] = 0.5
+    tab = np.zeros((V, H))
+    tab[:, k] = np.arange(V) / 4.0
+    fn, logits = Z.lm_head(cfg, tab, wn, xs)
+    expect = Z.round_bf16(Z.round_bf16(math.sqrt(H) * 0.5 / math.sqrt(1 + cfg.rms_eps * H / 9.0)) * np.arange(V) / 4.0)
+    np.testing.assert_allclose(logits[0], expect, rtol=1e-12)
+
+
+def test_stack_with_silent_sublayers():
+    """With hidden_states_scale = 0 on both merges of every block, each
+    block maps the stream to ((x + a.rb) * a.rs + m.rb) * m.rs (each merge
+    rounded to fp32), block after block in order."""
+    cfg = get_config("tiny").with_(seq=6)
+    blocks = []
+    for i in range(3):
+        W = dict(gen_block_weights(cfg, block=i))
+        for m in ("merge_a", "merge_m"):
+            t = W[m].clone()
+            t[1] = 0.0
+            W[m] = t
+        blocks.append(W)
+    V = cfg.vocab
+    extra = {"embed": torch.randn(V, cfg.hidden, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16),
+             "final_norm_w": torch.ones(cfg.hidden, dtype=torch.bfloat16)}
+    ids = np.array([[1, 2, 3, 4, 5, 6]])
+    out = Z.stack_prefill(cfg, blocks, extra, ids)
+    _, x = Z.embed(cfg, extra["embed"], ids)
+    for W in blocks:
+        a, m = Z.as64(W["merge_a"]), Z.as64(W["merge_m"])
+        x = Z.round_f32((x + a[2]) * a[3])
+        x = Z.round_f32((x + m[2]) * m[3])
+    np.testing.assert_array_equal(out["final_stream"], x)
