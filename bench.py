@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Throughput of the ZAYA1 block forward on B200, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole block (every stage of the hot path) over one
+batch of the workload's synthetic input; the default workload is the
+full-width single-block prefill, B1 x S4096.  Under torchrun (N > 1) every
+rank runs its own replica on its own GPU (independent sequences, no data
+exchange: weak scaling); NCCL carries only the barrier and the max-over-ranks
+of the device time.  Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; between steps (outside the events) the input stream
+is restored and a 256 MiB buffer is written to flush L2.  The whole timed
+region is bracketed by a barrier and a device synchronisation.  A second pass
+of K steps with per-stage CUDA events gives the dominant kernel's duration for
+the roofline; a third pass measures end to end from pinned host buffers.
+`--impl reference` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ZAYA block tokens/s on 1×B200 (prefill, decode) + % of TC/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_4k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stages", action="store_true", help="print the per-stage table to stderr")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(cfg):
+    return (f"{cfg.name}: one ZAYA1 block prefill, B{cfg.batch} x S{cfg.seq}, hidden {cfg.hidden}, "
+            f"{cfg.n_q}q/{cfg.n_kv}kv heads x {cfg.head_dim}, conv_qk width 3 over {cfg.qk_channels} ch, "
+            f"partial RoPE {cfg.rot_dim} dims, window {cfg.window}, {cfg.n_experts} SwiGLU experts x {cfg.inter} "
+            f"+ skip, router hidden {cfg.router_hidden}")
+
+
+# ---------------------------------------------------------------- algorithmic work per stage
+def stage_work(cfg, routed_tokens, pairs):
+    """Algorithmic work of one launch of each stage: (bound, amount, unit).
+    tensor: FLOPs (2 per multiply-add); hbm: bytes that must move once."""
+    M = cfg.batch * cfg.seq
+    H, R, E1, I = cfg.hidden, cfg.router_hidden, cfg.n_experts + 1, cfg.inter
+    qd, kvd = cfg.q_dim, cfg.kv_dim
+    nqkv = cfg.n_qkv
+    d = cfg.head_dim
+    return {
+        "rmsnorm_attn": ("hbm", M * H * (4 + 2) + H * 2, "B"),
+        "qkv_gemm": ("tensor", 2.0 * M * H * nqkv, "FLOP"),
+        "cca": ("hbm", M * nqkv * 2 + M * (qd + 2 * kvd) * 2, "B"),
+        "attention": ("tensor", 4.0 * d * pairs * cfg.n_q, "FLOP"),
+        "o_proj_merge": ("tensor", 2.0 * M * qd * H, "FLOP"),
+        "rmsnorm_mlp": ("hbm", M * H * (4 + 2) + H * 2, "B"),
+        "router_down": ("tensor", 2.0 * M * H * R, "FLOP"),
+        "router_mlp": ("alu", 2.0 * M * (2 * R * R + R * E1), "FLOP"),
+        "permute": ("hbm", M * 4 * 3, "B"),
+        "dispatch": ("hbm", routed_tokens * H * 2 * 2 + (M - routed_tokens) * H * 8, "B"),
+        "experts_gate_up": ("tensor", 2.0 * routed_tokens * H * 2 * I, "FLOP"),
+        "experts_down_merge": ("tensor", 2.0 * routed_tokens * I * H, "FLOP"),
+    }
+
+
+def attention_pairs(cfg, mask):
+    """Visible (query, key) pairs over real queries: the window's pairs only."""
+    import numpy as np
+    S, W = cfg.seq, cfg.window
+    total = 0
+    for b in range(cfg.batch):
+        valid = np.ones(S, dtype=bool) if mask is None else mask[b].cpu().numpy() != 0
+        cum = np.concatenate([[0], np.cumsum(valid)])
+        i = np.arange(S)
+        lo = np.maximum(0, i - W + 1)
+        vis = cum[i + 1] - cum[lo]
+        total += int(vis[valid].sum())
+    return total
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index):
+        self.dev = dev_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"zaya_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower().startswith("active")})
+        load = [r[0] for r in rows if r[0] > 0.3 * r[1]] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return world, rank, local          # CPU only: rank 0 times the oracle, the others exit
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_tokens(total_tokens, world):
+    """Tokens each rank processes: every rank runs a full replica."""
+    return [total_tokens] * world
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import torch
+    import top_moe_block_b200 as ZB
+    from synthetic import gen_block_weights, gen_prefill_inputs, get_config
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    from top_moe_block_b200 import build
+    build.build()
+    cfg = get_config(args.workload)
+    if cfg.mode != "prefill" or cfg.n_blocks != 1:
+        raise SystemExit(f"workload {cfg.name}: only single-block prefill workloads are timed by bench.py")
+    dev = torch.device("cuda", local)
+    W = gen_block_weights(cfg)
+    Wd = {k: v.to(dev).contiguous() for k, v in W.items()}
+    inp = gen_prefill_inputs(cfg)
+    B, S, H, R = cfg.batch, cfg.seq, cfg.hidden, cfg.router_hidden
+    M = B * S
+    x0 = inp["x"].to(dev)
+    mask = None if inp["attn_mask"] is None else inp["attn_mask"].to(dev)
+    rin = None if inp["router_state_in"] is None else inp["router_state_in"].to(dev)
+    hidden = x0.clone()
+    rout = torch.empty(B, S, R, dtype=torch.float32, device=dev)
+    state = dict(
+        k_cache=torch.zeros(B, cfg.n_kv, S, cfg.head_dim, dtype=torch.bfloat16, device=dev),
+        v_cache=torch.zeros(B, cfg.n_kv, S, cfg.head_dim, dtype=torch.bfloat16, device=dev),
+        cache_len=torch.zeros(B, dtype=torch.int32, device=dev),
+        conv_state=torch.zeros(B, cfg.qk_channels, 2, dtype=torch.bfloat16, device=dev),
+        prev_hs=torch.zeros(B, H, dtype=torch.bfloat16, device=dev))
+    c = ZB.make_config(cfg)
+    ws = torch.zeros(ZB.zaya_workspace_size(c, ZB.ZAYA_PREFILL, B, S), dtype=torch.uint8, device=dev)
+    w_s, st_s = ZB.make_weights(Wd), ZB.make_state(state)
+    taps_w = torch.empty(M, dtype=torch.float32, device=dev)
+    taps = ZB.make_taps({"expert_weights": taps_w})
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(with_taps=False):
+        ZB.zaya_block_prefill(c, w_s, cfg.block_idx, B, S, hidden, mask, rin, rout, st_s,
+                              taps if with_taps else None, ws, stream=stream)
+
+    for i in range(args.warmup):
+        hidden.copy_(x0)
+        step(with_taps=(i == 0))
+    torch.cuda.synchronize()
+    assert ZB.zaya_device_status(ws, stream) == 0
+    routed = int((taps_w > 0).sum().item())
+
+    # ---- pass 1: the timed steps
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = ZB.zaya_launch_count()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            hidden.copy_(x0)
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    launches = ZB.zaya_launch_count() - n0
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    local_total = sum(step_ms)
+    total_ms = max_over_ranks(local_total, world)
+    clocks = clk.summary()
+
+    # ---- pass 2: per-stage durations (CUDA events around each launch)
+    ZB.zaya_profile_reset()
+    ZB.zaya_profile_enable(True)
+    for i in range(K):
+        hidden.copy_(x0)
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    stages = ZB.zaya_profile_read()
+    ZB.zaya_profile_enable(False)
+
+    # ---- pass 3: end to end from pinned host buffers (H2D in, D2H out, per step)
+    x_h = x0.cpu().pin_memory()
+    rin_h = None if rin is None else rin.cpu().pin_memory()
+    out_h = torch.empty_like(x_h).pin_memory()
+    rout_h = torch.empty(B, S, R, dtype=torch.float32).pin_memory()
+    e2e = []
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        hidden.copy_(x_h, non_blocking=True)
+        if rin is not None:
+            rin.copy_(rin_h, non_blocking=True)
+        step()
+        out_h.copy_(hidden, non_blocking=True)
+        rout_h.copy_(rout, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e.append(a.elapsed_time(b))
+    e2e_ms = max_over_ranks(sum(e2e), world) / K
+    h2d = x_h.numel() * 4 + (0 if rin_h is None else rin_h.numel() * 4)
+    d2h = out_h.numel() * 4 + rout_h.numel() * 4
+
+    ms_per_step = total_ms / K
+    tokens = sum(shard_tokens(M, world))
+    value = tokens / (ms_per_step / 1e3)
+    pairs = attention_pairs(cfg, mask)
+    work = stage_work(cfg, routed, pairs)
+    peaks, peak_src = load_peaks()
+    roof = roofline(stages, work, peaks, peak_src, cfg)
+    if rank == 0 and args.stages:
+        tot = sum(v[0] for v in stages.values())
+        for name, (ms, n) in sorted(stages.items(), key=lambda kv: -kv[1][0]):
+            bound, amt, unit = work.get(name, ("?", 0, ""))
+            per = ms / max(n, 1)
+            rate = amt / (per / 1e3) / (1e12 if unit == "FLOP" else 1e9) if amt else 0
+            print(f"{name:22s} {per * 1e3:9.1f} us  {100 * ms / tot:5.1f}%  {bound:6s} "
+                  f"{rate:9.1f} {'TFLOP/s' if unit == 'FLOP' else 'GB/s'}", file=sys.stderr)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) stream, random-init weights of the ZAYA1-8B block shapes)",
+        "config": {"workload": workload_desc(cfg), "batch": B, "seq_len": S, "tokens_per_step": M,
+                   "routed_tokens": routed, "attention_pairs": pairs,
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)"},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items()},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def kernel_source_sha(name):
+    files = {"attention": "attn_prefill.cu", "experts_gate_up": "gemm_tc.cu", "experts_down_merge": "gemm_tc.cu",
+             "qkv_gemm": "gemm_tc.cu", "o_proj_merge": "gemm_tc.cu", "router_down": "gemm_tc.cu",
+             "router_mlp": "router.cu", "permute": "router.cu", "dispatch": "router.cu", "cca": "cca.cu",
+             "rmsnorm_attn": "norm.cu", "rmsnorm_mlp": "norm.cu"}
+    f = files.get(name)
+    if not f:
+        return None
+    with open(os.path.join(ROOT, "top_moe_block_b200", "csrc", f), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def roofline(stages, work, peaks, peak_src, cfg):
+    if not stages:
+        return None
+    name = max(stages, key=lambda k: stages[k][0])
+    ms, n = stages[name]
+    bound, amount, unit = work.get(name, ("hbm", 0, "B"))
+    per_ms = ms / max(n, 1)
+    if bound == "tensor":
+        achieved = amount / (per_ms / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+        u = "TFLOP/s"
+        peak_note = f"bf16 dense, {peak_src} sustained (kernel timed inside the block step)"
+    elif bound == "alu":
+        achieved = amount / (per_ms / 1e3) / 1e12
+        peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
+        u = "TFLOP/s"
+        peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"
+    else:
+        achieved = amount / (per_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        u = "GB/s"
+        peak_note = f"HBM copy, {peak_src}"
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tr = json.load(f)
+        ent = tr.get(cfg.name, {}).get(name)
+        if ent and ent.get("source_sha") == kernel_source_sha(name):
+            traffic = ent.get("dram_bytes_per_launch")
+    return {"kernel": name, "bound": "hbm" if bound == "hbm" else ("alu" if bound == "alu" else "tensor"),
+            "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": u, "frac": round(achieved / peak, 4),
+            "traffic": traffic, "algorithmic_per_launch": amount, "launch_us": round(per_ms * 1e3, 2),
+            "peak_note": peak_note}
+
+
+def cpu_baseline(cfg):
+    """The oracle as it stands, on the host cores, over the whole workload."""
+    from oracle import zaya_oracle as Z
+    from synthetic import gen_block_weights, gen_prefill_inputs
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    t0 = time.perf_counter()
+    Z.block_prefill(cfg, W, inp["x"], inp["attn_mask"], inp["router_state_in"])
+    dt = time.perf_counter() - t0
+    return {"value": round(cfg.batch * cfg.seq / dt, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"one full block prefill of the workload (B{cfg.batch} x S{cfg.seq}), float64 numpy oracle, "
+                      f"{dt:.1f} s", "host_cpus": os.cpu_count()}
+
+
+# ---------------------------------------------------------------- reference arm: the oracle
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    from oracle import zaya_oracle as Z
+    from synthetic import gen_block_weights, gen_prefill_inputs, get_config
+    cfg = get_config(args.workload)
+    sample = cfg.with_(seq=min(cfg.seq, 1024), batch=1)
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    x = inp["x"][:1, :sample.seq]
+    m = None if inp["attn_mask"] is None else inp["attn_mask"][:1, :sample.seq]
+    r = None if inp["router_state_in"] is None else inp["router_state_in"][:1, :sample.seq]
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    for _ in range(args.warmup):
+        Z.block_prefill(sample, W, x, m, r)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        Z.block_prefill(sample, W, x, m, r)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = sample.seq / (ms / 1e3)
+    desc = f"first {sample.seq} tokens of {cfg.name} (B1), one block prefill, float64 numpy oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "sample": desc},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1 and args.impl != "reference":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

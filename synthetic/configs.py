@@ -105,9 +105,11 @@ CONFIGS = {
         # N(0, 0.02) router-MLP weights make the 5 logits equal to ~1e-3 and send
         # every token to one class; 1/sqrt(R) keeps the choice token-dependent.
         router_w_std=1.0 / math.sqrt(32.0), calibrated=1, skip_frac=0.25),
-    # Full-width single block prefill, B1 x S4096, skip never wins (bias -1).
+    # Full-width single block prefill, B1 x S4096; balancing biases fitted to
+    # roughly uniform expert loads with no skip (the random-init router alone
+    # sends half the tokens to one expert).
     "prefill_4k": BlockConfig(
-        name="prefill_4k", batch=1, seq=4096, seed=1, skip_bias=-1.0,
+        name="prefill_4k", batch=1, seq=4096, seed=1, calibrated=1, skip_frac=0.0,
         input_dtype="bf16", **_FULL),
     # Batched prefill, B8 x S2048, left pads U{0..256}, Zipf(1.1) loads, ~20% skip.
     "prefill_skewed_8x2k": BlockConfig(

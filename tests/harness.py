@@ -1,0 +1,200 @@
+"""Test harness: runs the CUDA path through the C ABI and compares it with
+the CPU oracle on the same seeded inputs.
+
+Comparison protocol (the block's tolerances):
+  * router choices, teacher-forced: the oracle's router (down_proj, router
+    MLP, fp32 scoring) is run on the GPU's own mlp_norm_output and incoming
+    router state; its class must equal the GPU's for every token except
+    near-ties (top-two selection scores within 1e-5 relative), which are
+    counted and reported;
+  * floating point, per block: the oracle block is run on the GPU's block
+    input (and state), with the GPU's expert choices forced where the
+    oracle's own choice flips from upstream rounding (flips counted);
+    layer_output must satisfy max|err| / rms(oracle) <= 2e-2 and
+    cosine >= 0.9995.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import top_moe_block_b200 as ZB
+from oracle import zaya_oracle as Z
+
+TOL_REL_MAX = 2e-2
+TOL_COS = 0.9995
+NEAR_TIE = 1e-5
+
+
+def dev_weights(W: dict, dev="cuda") -> dict:
+    return {k: v.to(dev).contiguous() for k, v in W.items()}
+
+
+def new_state(cfg, B, cap, dev="cuda") -> dict:
+    return dict(
+        k_cache=torch.zeros(B, cfg.n_kv, cap, cfg.head_dim, dtype=torch.bfloat16, device=dev),
+        v_cache=torch.zeros(B, cfg.n_kv, cap, cfg.head_dim, dtype=torch.bfloat16, device=dev),
+        cache_len=torch.zeros(B, dtype=torch.int32, device=dev),
+        conv_state=torch.zeros(B, cfg.qk_channels, 2, dtype=torch.bfloat16, device=dev),
+        prev_hs=torch.zeros(B, cfg.hidden, dtype=torch.bfloat16, device=dev))
+
+
+def new_taps(cfg, B, S, dev="cuda") -> dict:
+    M, H, E1 = B * S, cfg.hidden, cfg.n_experts + 1
+    bf, f32 = torch.bfloat16, torch.float32
+    return dict(
+        router_logits=torch.full((M, E1), float("nan"), dtype=f32, device=dev),
+        expert_indices=torch.full((M,), -1, dtype=torch.int32, device=dev),
+        expert_weights=torch.full((M,), float("nan"), dtype=f32, device=dev),
+        attention_norm_output=torch.empty(M, H, dtype=bf, device=dev),
+        attention_output=torch.empty(M, H, dtype=bf, device=dev),
+        layer_mid=torch.empty(M, H, dtype=f32, device=dev),
+        mlp_norm_output=torch.empty(M, H, dtype=bf, device=dev),
+        mlp_output=torch.empty(M, H, dtype=bf, device=dev),
+        attention_queries=torch.empty(B, cfg.n_q, S, cfg.head_dim, dtype=bf, device=dev))
+
+
+def workspace(nbytes, dev="cuda", poison=True) -> torch.Tensor:
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if poison:
+        ws.fill_(0xFF)           # NaN bit patterns: a read before write shows up as a mismatch
+    ws[:256].zero_()             # status word
+    return ws
+
+
+def gpu_prefill(cfg, Wd, x, mask=None, rin=None, block_idx=None, cap=None, taps=True, state=None):
+    """One block prefill on the GPU; returns outputs and taps as CPU tensors."""
+    bidx = cfg.block_idx if block_idx is None else block_idx
+    B, S, H, R = x.shape[0], x.shape[1], cfg.hidden, cfg.router_hidden
+    cap = cap or S
+    hidden = x.to("cuda", torch.float32).contiguous().clone()
+    m = None if mask is None else mask.to("cuda", torch.int32).contiguous()
+    r_in = None if (rin is None or bidx == 0) else rin.to("cuda", torch.float32).contiguous()
+    r_out = torch.full((B, S, R), float("nan"), dtype=torch.float32, device="cuda")
+    st = state if state is not None else new_state(cfg, B, cap)
+    tp = new_taps(cfg, B, S) if taps else None
+    c = ZB.make_config(cfg)
+    ws = workspace(ZB.zaya_workspace_size(c, ZB.ZAYA_PREFILL, B, S))
+    ZB.zaya_block_prefill(c, ZB.make_weights(Wd), bidx, B, S, hidden, m, r_in, r_out, ZB.make_state(st),
+                          ZB.make_taps(tp), ws)
+    status = ZB.zaya_device_status(ws)
+    assert status == 0, f"device status {status}: {ZB.zaya_status_string(status)}"
+    out = dict(layer_output=hidden.cpu(), router_state=r_out.cpu(), state={k: v.cpu() for k, v in st.items()})
+    if tp:
+        out.update({k: v.cpu() for k, v in tp.items()})
+    return out
+
+
+def gpu_decode(cfg, Wd, x, state, rin=None, block_idx=None, taps=True):
+    """One decode step of one block on the GPU; `state` (device tensors) is updated in place."""
+    bidx = cfg.block_idx if block_idx is None else block_idx
+    B, H, R = x.shape[0], cfg.hidden, cfg.router_hidden
+    hidden = x.to("cuda", torch.float32).contiguous().clone()
+    r_in = None if (rin is None or bidx == 0) else rin.to("cuda", torch.float32).contiguous()
+    r_out = torch.full((B, R), float("nan"), dtype=torch.float32, device="cuda")
+    tp = new_taps(cfg, B, 1) if taps else None
+    c = ZB.make_config(cfg)
+    ws = workspace(ZB.zaya_workspace_size(c, ZB.ZAYA_DECODE, B, 1))
+    ZB.zaya_block_decode(c, ZB.make_weights(Wd), bidx, B, hidden, r_in, r_out, ZB.make_state(state),
+                         ZB.make_taps(tp), ws)
+    status = ZB.zaya_device_status(ws)
+    assert status == 0, f"device status {status}: {ZB.zaya_status_string(status)}"
+    out = dict(layer_output=hidden.cpu(), router_state=r_out.cpu())
+    if tp:
+        out.update({k: v.cpu() for k, v in tp.items()})
+    return out
+
+
+def gpu_classes(cfg, gpu) -> np.ndarray:
+    """Class per token from the GPU taps: expert index, or E (skip) where the weight is 0."""
+    idx = gpu["expert_indices"].numpy().astype(np.int64)
+    w = gpu["expert_weights"].numpy()
+    return np.where(w > 0, idx, cfg.n_experts)
+
+
+def router_teacher_forced(cfg, W, m_in, rin, block_idx, real=None):
+    """The oracle's router on the GPU's mlp_norm_output: returns (cls, gap, r, logits)."""
+    m = Z.as64(m_in)
+    r = m @ Z.as64(W["router_down_w"]).T + Z.as64(W["router_down_b"])
+    if block_idx > 0 and rin is not None:
+        r = r + Z.as64(rin) * Z.as64(W["router_state_scale"])
+    r = Z.round_f32(r)
+    logits = Z.router_mlp(r, W, cfg.rms_eps)
+    cls, idx, w, p, gap = Z.select(logits, Z.as64(W["balancing"]), cfg.n_experts)
+    if real is not None:
+        cls = np.where(real, cls, cfg.n_experts)
+    return cls, gap, r, logits
+
+
+def rel_max(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    rms = np.sqrt(np.mean(b * b))
+    return float(np.max(np.abs(a - b)) / max(rms, 1e-30))
+
+
+def cosine(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64).ravel()
+    b = np.asarray(b, dtype=np.float64).ravel()
+    return float(a @ b / max(np.linalg.norm(a) * np.linalg.norm(b), 1e-300))
+
+
+def report(name, gpu, ref) -> dict:
+    return {"name": name, "rel_max": rel_max(gpu, ref), "cos": cosine(gpu, ref)}
+
+
+def check_prefill_block(cfg, W, inp, gpu, block_idx=None, verbose=True):
+    """Full comparison of one GPU prefill block against the oracle."""
+    bidx = cfg.block_idx if block_idx is None else block_idx
+    B, S = inp["x"].shape[:2]
+    M = B * S
+    E = cfg.n_experts
+    real = np.ones(M, dtype=bool) if inp.get("attn_mask") is None else inp["attn_mask"].numpy().reshape(-1) != 0
+    rin = inp.get("router_state_in")
+    rin2 = None if rin is None else rin.reshape(M, -1)
+    g_cls = gpu_classes(cfg, gpu)
+    t_cls, gap, t_r, t_logits = router_teacher_forced(cfg, W, gpu["mlp_norm_output"], rin2, bidx, real)
+    near = gap < NEAR_TIE
+    mism = (t_cls != g_cls) & ~near
+    res = {"tokens": M, "near_ties": int((near & real).sum()), "router_mismatch": int(mism.sum())}
+    res["router_state"] = report("router_state", gpu["router_state"].reshape(M, -1).numpy(), t_r)
+    res["router_logits"] = report("router_logits", gpu["router_logits"].numpy(), t_logits)
+    o = Z.block_prefill(cfg, W, inp["x"], inp.get("attn_mask"), rin, bidx, force_cls=g_cls.reshape(B, S))
+    res["flips"] = int((o["router_own_cls"].reshape(-1) != g_cls)[real].sum())
+    for key in ("layer_output", "attention_output", "mlp_output", "layer_mid", "attention_norm_output",
+                "mlp_norm_output"):
+        gv = gpu[key].float().numpy().reshape(M, -1)
+        ov = o[key].reshape(M, -1)
+        res[key] = report(key, gv, ov)
+        res[key]["bf16_ok"] = close_bf16(gv, ov)
+    res["attention_queries"] = report("q", gpu["attention_queries"].float().numpy(), o["attention_queries"])
+    st = gpu["state"]
+    res["attention_queries"]["bf16_ok"] = close_bf16(gpu["attention_queries"].float().numpy(), o["attention_queries"])
+    res["k_cache"] = report("k", st["k_cache"][:, :, :S].float().numpy(), o["state"]["k_cache"])
+    res["k_cache"]["bf16_ok"] = close_bf16(st["k_cache"][:, :, :S].float().numpy(), o["state"]["k_cache"])
+    res["v_cache"] = report("v", st["v_cache"][:, :, :S].float().numpy(), o["state"]["v_cache"])
+    res["v_cache"]["bf16_ok"] = close_bf16(st["v_cache"][:, :, :S].float().numpy(), o["state"]["v_cache"])
+    res["conv_state"] = report("conv", st["conv_state"].float().numpy(), o["state"]["conv_state"])
+    res["prev_hs"] = report("prev_hs", st["prev_hs"].float().numpy(), o["state"]["prev_hs"])
+    res["cache_len_ok"] = bool((st["cache_len"].numpy() == S).all())
+    if verbose:
+        print({k: (round(v["rel_max"], 5), round(v["cos"], 6)) if isinstance(v, dict) else v for k, v in res.items()})
+    return res
+
+
+def close_bf16(gpu, ref) -> bool:
+    """For a tensor the block stores in bf16: every element within the block
+    tolerance (2e-2 of the reference rms) plus one bf16 unit in the last place
+    of the element (rounding of the two sides may land on neighbouring bf16
+    values), and cosine >= 0.9995."""
+    g = np.asarray(gpu, dtype=np.float64)
+    o = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(o * o))
+    ok = np.abs(g - o) <= TOL_REL_MAX * rms + 2.0 ** -7 * np.abs(o)
+    return bool(ok.all()) and cosine(g, o) >= TOL_COS
+
+
+def assert_block_ok(res):
+    assert res["router_mismatch"] == 0, res
+    lo = res["layer_output"]
+    assert lo["rel_max"] <= TOL_REL_MAX and lo["cos"] >= TOL_COS, lo

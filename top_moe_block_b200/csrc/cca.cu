@@ -1,0 +1,219 @@
+// CCA attention inputs: causal conv over q||k, the CCA mean residual,
+// qk_norm with the key temperature, partial RoPE, the value heads with their
+// delayed half, and the writes into the KV cache / conv_state / prev_hs.
+//
+// As the nnterp "zaya" page states it ("Queries and keys are convolved,
+// normed to sqrt(head_dim) and the keys scaled"):
+//   y[t,c]  = w[c,0] u[t-2,c] + w[c,1] u[t-1,c] + w[c,2] u[t,c] + b[c]   (u = q||k pre-conv)
+//   q_h    += (u_q[h] + u_k[g(h)]) / 2;   k_g += mean over h served by g of that
+//   q, k    -> x * sqrt(d) / max(|x|, eps);   k *= temp[g]
+//   RoPE on dims [0, rot): pairs (i, i + rot/2), angle = fp32(pos * inv_freq[i])
+//   v_g     = [v_current(t)[g*d/2 .. ] || v_delayed(t-1)[g*d/2 .. ]]
+// conv_state [B,C,2] and prev_hs [B,H] carry the two previous tokens' pre-conv
+// channels and the previous token's attention-norm output (ZAYA1-8B-JANGTQ2
+// README, "Architecture Summary").
+//
+// One CTA per token; warp w < n_q handles query head w, the next n_kv warps
+// the key heads, the last n_kv warps the value heads; each lane owns d/32
+// consecutive dims, so the head norm is a warp reduction and the RoPE pair
+// exchange a shuffle.  HBM-bound: ~3 KB read and ~3 KB written per token.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace zaya {
+
+namespace {
+
+template <int D>
+struct Pre {
+  // pre-conv value of channel c at token offset o (0: t, 1: t-1, 2: t-2)
+  const __nv_bfloat16* qkv;
+  size_t ld;
+  const __nv_bfloat16* conv_state;  // decode history [C, 2]
+  int tok, s, decode;
+  const int* mask;
+  bool real0, real1, real2;
+
+  __device__ __forceinline__ float at(int c, int o) const {
+    if (o == 0) return real0 ? bf2f(qkv[(size_t)tok * ld + c]) : 0.f;
+    if (decode) return bf2f(conv_state[(size_t)c * 2 + (o == 2 ? 0 : 1)]);
+    const bool r = (o == 1) ? real1 : real2;
+    return r ? bf2f(qkv[(size_t)(tok - o) * ld + c]) : 0.f;
+  }
+};
+
+template <int D>
+__device__ __forceinline__ void rope_apply(float (&y)[D / 32], int lane, int pos, int rot, float theta) {
+  constexpr int DPL = D / 32;
+  if (rot <= 0) return;
+  const int half = rot / 2;
+  const int off = half / DPL;  // lane distance between the two dims of a pair
+  const float posf = (float)pos;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    const int j = lane * DPL + i;
+    const bool lo = j < half;
+    const bool in_rot = j < rot;
+    int src = lo ? lane + off : lane - off;
+    if (!in_rot) src = lane;
+    const float partner = __shfl_sync(0xffffffffu, y[i], src);
+    if (in_rot) {
+      const int f = lo ? j : j - half;
+      const float inv_freq = (float)(1.0 / pow((double)theta, (double)(2 * f) / (double)rot));
+      const float ang = posf * inv_freq;
+      float sn, cs;
+      sincosf(ang, &sn, &cs);
+      y[i] = lo ? (y[i] * cs - partner * sn) : (y[i] * cs + partner * sn);
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
+  constexpr int DPL = D / 32;
+  const int tok = blockIdx.x;
+  const int b = p.decode ? tok : tok / p.S;
+  const int s = p.decode ? 0 : tok % p.S;
+  const int warp = warp_id(), lane = lane_id();
+  const int nq = p.n_q, nkv = p.n_kv, rep = nq / nkv;
+  const int C = (nq + nkv) * D;
+  const auto* qkv = static_cast<const __nv_bfloat16*>(p.qkv);
+  const size_t ld = (size_t)p.n_qkv;
+
+  const int pos = p.decode ? p.cache_len[b] : s;
+  if (pos < 0 || pos >= p.cache_cap) {
+    if (warp == 0 && lane == 0) set_status(p.status, ZAYA_ERR_DEVICE_RANGE);
+    return;
+  }
+  Pre<D> pre;
+  pre.qkv = qkv;
+  pre.ld = ld;
+  pre.conv_state = static_cast<const __nv_bfloat16*>(p.conv_state) + (size_t)b * C * 2;
+  pre.tok = tok;
+  pre.s = s;
+  pre.decode = p.decode;
+  pre.mask = p.mask;
+  pre.real0 = p.decode || !p.mask || p.mask[tok] != 0;
+  pre.real1 = !p.decode && s >= 1 && (!p.mask || p.mask[tok - 1] != 0);
+  pre.real2 = !p.decode && s >= 2 && (!p.mask || p.mask[tok - 2] != 0);
+  const bool last = p.decode || s == p.S - 1;
+  auto* cstate = static_cast<__nv_bfloat16*>(p.conv_state) + (size_t)b * C * 2;
+  const float sqrt_d = sqrtf((float)D);
+
+  if (warp < nq + nkv) {
+    // ------------------------------------------------ query head / key head
+    const bool is_q = warp < nq;
+    const int head = is_q ? warp : warp - nq;
+    const int g = is_q ? warp / rep : head;
+    float y[DPL];
+    float u0[DPL], u1[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const int j = lane * DPL + i;
+      const int c = (is_q ? head * D : nq * D + head * D) + j;
+      const float a0 = pre.at(c, 0), a1 = pre.at(c, 1), a2 = pre.at(c, 2);
+      u0[i] = a0;
+      u1[i] = a1;
+      float acc = __ldg(p.conv_b + c);
+      acc = fmaf(__ldg(p.conv_w + 3 * c + 0), a2, acc);
+      acc = fmaf(__ldg(p.conv_w + 3 * c + 1), a1, acc);
+      acc = fmaf(__ldg(p.conv_w + 3 * c + 2), a0, acc);
+      if (p.cca_res) {
+        const float kpre = pre.at(nq * D + g * D + j, 0);
+        if (is_q) {
+          acc += 0.5f * (a0 + kpre);
+        } else {
+          float qs = 0.f;
+          for (int h = g * rep; h < (g + 1) * rep; ++h) qs += pre.at(h * D + j, 0);
+          acc += 0.5f * (qs / (float)rep + kpre);
+        }
+      }
+      y[i] = acc;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) ss += y[i] * y[i];
+    ss = warp_sum(ss);
+    float scl = sqrt_d / fmaxf(sqrtf(ss), p.eps);
+    if (!is_q) scl *= __ldg(p.k_temp + g);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) y[i] *= scl;
+    rope_apply<D>(y, lane, pos, p.rot, p.theta);
+
+    __nv_bfloat16* dst;
+    if (is_q) {
+      const int Sq = p.decode ? 1 : p.S;
+      const size_t off = (((size_t)b * nq + head) * Sq + (p.decode ? 0 : s)) * D + lane * DPL;
+      dst = static_cast<__nv_bfloat16*>(p.q_out) + off;
+      if (p.tap_q) {
+        __nv_bfloat16* t = static_cast<__nv_bfloat16*>(p.tap_q) + off;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) t[i] = f2bf(y[i]);
+      }
+    } else {
+      dst = static_cast<__nv_bfloat16*>(p.k_cache) + (((size_t)b * nkv + head) * p.cache_cap + pos) * D + lane * DPL;
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) dst[i] = f2bf(y[i]);
+
+    if (last) {  // conv_state <- pre-conv channels of tokens t-1, t
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const int c = (is_q ? head * D : nq * D + head * D) + lane * DPL + i;
+        cstate[(size_t)c * 2 + 0] = f2bf(u1[i]);
+        cstate[(size_t)c * 2 + 1] = f2bf(u0[i]);
+      }
+    }
+  } else if (warp < nq + 2 * nkv) {
+    // ------------------------------------------------ value head
+    const int g = warp - nq - nkv;
+    const int vc0 = nq * D + nkv * D;
+    const int vd0 = vc0 + nkv * (D / 2);
+    __nv_bfloat16* dst =
+        static_cast<__nv_bfloat16*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + pos) * D + lane * DPL;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const int j = lane * DPL + i;
+      float v;
+      if (j < D / 2) {
+        v = pre.real0 ? bf2f(qkv[(size_t)tok * ld + vc0 + g * (D / 2) + j]) : 0.f;
+      } else {
+        const int col = vd0 + g * (D / 2) + (j - D / 2);
+        if (!p.v_delayed) {
+          v = pre.real0 ? bf2f(qkv[(size_t)tok * ld + col]) : 0.f;
+        } else if (p.decode) {
+          v = bf2f(qkv[(size_t)(p.B + b) * ld + col]);  // projection of prev_hs
+        } else {
+          v = pre.real1 ? bf2f(qkv[(size_t)(tok - 1) * ld + col]) : 0.f;
+        }
+      }
+      dst[i] = f2bf(v);
+    }
+    if (last && g == 0) {  // prev_hs <- attention_norm_output of this token
+      const uint2* src = reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.a_in) + (size_t)tok * p.H);
+      uint2* ph = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.prev_hs) + (size_t)b * p.H);
+      for (int c = lane; c < p.H / 4; c += 32) ph[c] = src[c];
+      if (!p.decode && lane == 0) p.cache_len[b] = p.S;
+    }
+  }
+}
+
+}  // namespace
+
+int launch_cca(const CcaParams& p, cudaStream_t st) {
+  const int tokens = p.decode ? p.B : p.B * p.S;
+  if (tokens <= 0) return ZAYA_OK;
+  const int threads = 32 * (p.n_q + 2 * p.n_kv);
+  if (threads > 1024) return ZAYA_ERR_UNSUPPORTED;
+  if (p.d == 128)
+    cca_kernel<128><<<tokens, threads, 0, st>>>(p);
+  else if (p.d == 64)
+    cca_kernel<64><<<tokens, threads, 0, st>>>(p);
+  else
+    return ZAYA_ERR_UNSUPPORTED;
+  return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
+}
+
+}  // namespace zaya

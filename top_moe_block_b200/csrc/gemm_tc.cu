@@ -1,0 +1,391 @@
+// tcgen05 GEMM for the ZAYA1 block's dense contractions (sm_100a).
+//
+// C[M, N] = A[M, K] * B[N, K]^T with bf16 operands and fp32 accumulation in
+// tensor memory.  One persistent CTA per SM walks 128 x BN output tiles:
+//   warp 0      TMA producer: 128x64 A and BNx64 B tiles into a STAGES-deep
+//               shared-memory ring (128-byte swizzle), one mbarrier per slot;
+//   warp 1      one elected thread issues tcgen05.mma (M=128, N=BN, K=16) into
+//               one of two TMEM accumulators and commits slot releases;
+//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator (each warp
+//               owns the 32 TMEM lanes its warp index allows), the fused
+//               epilogue, global stores; then the accumulator is handed back,
+//               so the epilogue of tile i overlaps the main loop of tile i+1.
+// Grouped mode (the experts): A rows are the tokens permuted by expert, B is
+// the stacked expert weights; the tile list is derived on the device from
+// the per-expert row offsets, so no host synchronisation is needed.
+//
+// Epilogues (what the block needs right after each contraction):
+//   STORE_BF16   q/k/v projections, lm_head logits
+//   MERGE_ATTN   o_proj, then merge 1 of the zaya page ("The block, in
+//                order"): attention_output = bf16((o + hb) * hs);
+//                h = attention_output + (x + rb) * rs written over x
+//   ROUTER_DOWN  router down_proj + bias + previous state * router_states_scale
+//   SWIGLU       expert gate/up: act = bf16(silu(gate) * up)
+//   MERGE_MLP    expert down: y = w_t * acc; mlp_output = bf16((y + hb) * hs);
+//                out = mlp_output + (h + rb) * rs, scattered to token t's row
+#include <stdio.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace zaya {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int A_STAGE_BYTES = BM * BK * 2;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int B_STAGE_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);  // ~192 KB ring
+  static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct TileInfo {
+  int m0;      // first A row
+  int m_end;   // A rows of this tile's group end here (exclusive)
+  int n0;      // first output column
+  int b_row;   // first B row (gate rows for SWIGLU)
+  int b_row2;  // SWIGLU: first up row
+};
+
+template <int EPI, int BN_OUT>
+__device__ __forceinline__ int total_tiles(const GemmParams& p) {
+  const int nt = p.N / BN_OUT;
+  if (!p.grouped) return ((p.M + BM - 1) / BM) * nt;
+  return p.mt_start[p.n_groups] * nt;
+}
+
+template <int EPI, int BN_OUT>
+__device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
+  TileInfo ti;
+  const int nt = p.N / BN_OUT;
+  if (!p.grouped) {
+    const int mt = (p.M + BM - 1) / BM;
+    ti.m0 = (t % mt) * BM;
+    ti.n0 = (t / mt) * BN_OUT;
+    ti.m_end = p.M;
+    ti.b_row = ti.n0;
+    ti.b_row2 = ti.n0;
+  } else {
+    int e = 0;
+    while (e + 1 < p.n_groups && p.mt_start[e + 1] * nt <= t) ++e;
+    const int local = t - p.mt_start[e] * nt;
+    const int mte = p.mt_start[e + 1] - p.mt_start[e];
+    ti.m0 = p.group_off[e] + (local % mte) * BM;
+    ti.m_end = p.group_off[e + 1];
+    ti.n0 = (local / mte) * BN_OUT;
+    ti.b_row = e * p.b_rows_per_group + ti.n0;
+    ti.b_row2 = e * p.b_rows_per_group + (p.b_rows_per_group >> 1) + ti.n0;
+  }
+  return ti;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+// Epilogue of one row (this thread) x 32 consecutive columns.
+template <int EPI>
+__device__ __forceinline__ void epilogue32(const GemmParams& p, int row, int col, const uint32_t (&r)[32],
+                                           const uint32_t (&r2)[32]) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  if constexpr (EPI == EPI_STORE_BF16 || EPI == EPI_SWIGLU) {
+    if constexpr (EPI == EPI_SWIGLU) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = silu_f(v[j]) * __uint_as_float(r2[j]);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.ldo + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 u;
+      u.x = pack_bf2(v[8 * q + 0], v[8 * q + 1]);
+      u.y = pack_bf2(v[8 * q + 2], v[8 * q + 3]);
+      u.z = pack_bf2(v[8 * q + 4], v[8 * q + 5]);
+      u.w = pack_bf2(v[8 * q + 6], v[8 * q + 7]);
+      dst[q] = u;
+    }
+  } else if constexpr (EPI == EPI_ROUTER_DOWN) {
+    float* dst = static_cast<float*>(p.out) + (size_t)row * p.ldo + col;
+    const float* prev = p.prev ? p.prev + (size_t)row * p.N + col : nullptr;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 o;
+      float* op = &o.x;
+      float4 pv = prev ? *reinterpret_cast<const float4*>(prev + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float* pp = &pv.x;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = col + 4 * q + j;
+        float x = v[4 * q + j] + __ldg(p.bias + c);
+        if (prev) x = fmaf(pp[j], __ldg(p.prev_scale + c), x);
+        op[j] = x;
+      }
+      reinterpret_cast<float4*>(dst)[q] = o;
+    }
+  } else {  // MERGE_ATTN / MERGE_MLP
+    int token = row;
+    float wt = 1.0f;
+    if constexpr (EPI == EPI_MERGE_MLP) {
+      token = p.perm[row];
+      wt = p.row_w[token];
+    }
+    const int N = p.N;
+    float* srow = p.stream + (size_t)token * N + col;
+    __nv_bfloat16* tap = p.tap_bf16 ? static_cast<__nv_bfloat16*>(p.tap_bf16) + (size_t)token * N + col : nullptr;
+    float* tapf = p.tap_f32 ? p.tap_f32 + (size_t)token * N + col : nullptr;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 x4 = reinterpret_cast<const float4*>(srow)[q];
+      float* xp = &x4.x;
+      float cb[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = col + 4 * q + j;
+        const float hb = __ldg(p.merge + c), hs = __ldg(p.merge + N + c);
+        const float rb = __ldg(p.merge + 2 * N + c), rs = __ldg(p.merge + 3 * N + c);
+        const float contrib = round_bf((v[4 * q + j] * wt + hb) * hs);
+        cb[j] = contrib;
+        xp[j] = fmaf(xp[j] + rb, rs, contrib);
+      }
+      reinterpret_cast<float4*>(srow)[q] = x4;
+      if (tapf) reinterpret_cast<float4*>(tapf)[q] = x4;
+      if (tap) {
+        uint2 u;
+        u.x = pack_bf2(cb[0], cb[1]);
+        u.y = pack_bf2(cb[2], cb[3]);
+        reinterpret_cast<uint2*>(tap)[q] = u;
+      }
+    }
+  }
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+  using C = GemmCfg<BN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int BN_OUT = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    fence_barrier_init();
+    fence_proxy_async();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int k_blocks = p.K / BK;
+  const int ntiles = total_tiles<EPI, BN_OUT>(p);
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const TileInfo ti = tile_info<EPI, BN_OUT>(p, t);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) goto producer_done;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * BK, ti.m0);
+          uint8_t* b_dst = sB + stage * C::B_STAGE_BYTES;
+          if constexpr (EPI == EPI_SWIGLU) {
+            tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
+            tma_load_2d(b_dst + (BN / 2) * BK * 2, &tmB, &full[stage], kb * BK, ti.b_row2);
+          } else {
+            tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * C::B_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), IDESC,
+                        (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5
+    const int q = warp & 3;  // TMEM lanes [32q, 32q+32) are reachable from this warp
+    int local = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      const TileInfo ti = tile_info<EPI, BN_OUT>(p, t);
+      if (!mbar_wait(&tfull[acc], acc_phase, p.status)) break;
+      tc_fence_after();
+      const int row = ti.m0 + q * 32 + lane;
+      const bool valid = row < ti.m_end;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN_OUT; c += 32) {
+        uint32_t r[32], r2[32];
+        tmem_ld32(tbase + c, r);
+        if constexpr (EPI == EPI_SWIGLU) tmem_ld32(tbase + BN / 2 + c, r2);
+        tmem_ld_wait();
+        if (valid) epilogue32<EPI>(p, row, ti.n0 + c, r, r2);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+template <int BN, int EPI>
+int launch_impl(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, int ntiles_hint, int num_sms,
+                cudaStream_t st) {
+  using C = GemmCfg<BN>;
+  auto kern = gemm_tc_kernel<BN, EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return ZAYA_ERR_CUDA;
+    attr_set = true;
+  }
+  int grid = ntiles_hint < num_sms ? ntiles_hint : num_sms;
+  if (grid < 1) grid = 1;
+  kern<<<grid, 192, C::SMEM_BYTES, st>>>(ma, mb, p);
+  return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
+}
+
+}  // namespace
+
+int make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return ZAYA_ERR_CUDA;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (cols * 2) % 16) return ZAYA_ERR_MISALIGNED;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ZAYA_OK : ZAYA_ERR_CUDA;
+}
+
+int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b_rows, const GemmParams& p,
+                int num_sms, cudaStream_t st) {
+  if (p.K % BK != 0 || p.K <= 0) return ZAYA_ERR_UNSUPPORTED;
+  const int bn_out = (epi == EPI_SWIGLU) ? bn / 2 : bn;
+  if (p.N % bn_out != 0) return ZAYA_ERR_UNSUPPORTED;
+  if (a_rows <= 0) return ZAYA_OK;
+  CUtensorMap ma, mb;
+  int rc = make_tmap_bf16(&ma, A, (uint64_t)a_rows, (uint64_t)p.K, BM);
+  if (rc) return rc;
+  rc = make_tmap_bf16(&mb, B, (uint64_t)b_rows, (uint64_t)p.K, epi == EPI_SWIGLU ? bn / 2 : bn);
+  if (rc) return rc;
+  const int nt = p.N / bn_out;
+  int hint = p.grouped ? num_sms : ((p.M + BM - 1) / BM) * nt;
+#define ZAYA_GEMM_CASE(BNV, EPIV) \
+  if (bn == BNV && epi == EPIV) return launch_impl<BNV, EPIV>(ma, mb, p, hint, num_sms, st);
+  ZAYA_GEMM_CASE(256, EPI_STORE_BF16)
+  ZAYA_GEMM_CASE(128, EPI_STORE_BF16)
+  ZAYA_GEMM_CASE(64, EPI_STORE_BF16)
+  ZAYA_GEMM_CASE(256, EPI_MERGE_ATTN)
+  ZAYA_GEMM_CASE(128, EPI_MERGE_ATTN)
+  ZAYA_GEMM_CASE(64, EPI_MERGE_ATTN)
+  ZAYA_GEMM_CASE(128, EPI_ROUTER_DOWN)
+  ZAYA_GEMM_CASE(64, EPI_ROUTER_DOWN)
+  ZAYA_GEMM_CASE(32, EPI_ROUTER_DOWN)
+  ZAYA_GEMM_CASE(32 * 8, EPI_SWIGLU)
+  ZAYA_GEMM_CASE(256, EPI_MERGE_MLP)
+  ZAYA_GEMM_CASE(128, EPI_MERGE_MLP)
+  ZAYA_GEMM_CASE(64, EPI_MERGE_MLP)
+#undef ZAYA_GEMM_CASE
+  return ZAYA_ERR_UNSUPPORTED;
+}
+
+}  // namespace zaya

@@ -1,0 +1,148 @@
+// Internal launchers of the ZAYA1 block kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace zaya {
+
+// ------------------------------------------------------------------ GEMM
+enum EpiKind {
+  EPI_STORE_BF16 = 0,   // out[m, n] = bf16(acc)
+  EPI_MERGE_ATTN = 1,   // o_proj + merge 1, stream updated in place
+  EPI_ROUTER_DOWN = 2,  // out[m, n] = acc + bias[n] (+ prev[m, n] * scale[n]) in fp32
+  EPI_SWIGLU = 3,       // grouped: act = bf16(silu(gate) * up)
+  EPI_MERGE_MLP = 4     // grouped: expert down + weight + merge 2, scattered to token rows
+};
+
+struct GemmParams {
+  int M, N, K;               // C[M, N] = A[M, K] * B[N, K]^T (N = output columns)
+  int grouped;               // expert-grouped A rows / B row blocks
+  const int* group_off;      // [E+1] first A row of each expert (grouped)
+  const int* mt_start;       // [E+1] prefix of per-expert 128-row tile counts (grouped)
+  int n_groups;              // E
+  int b_rows_per_group;      // rows of B per expert (2I or H)
+  int* status;
+  void* out;                 // STORE_BF16 / SWIGLU: bf16 [rows, ldo]; ROUTER_DOWN: fp32 [M, ldo]
+  int ldo;
+  float* stream;             // MERGE_*: fp32 [tokens, N]
+  const float* merge;        // MERGE_*: fp32 [4, N] hb, hs, rb, rs
+  const float* bias;         // ROUTER_DOWN [N]
+  const float* prev;         // ROUTER_DOWN [M, N] or null
+  const float* prev_scale;   // ROUTER_DOWN [N]
+  const int* perm;           // MERGE_MLP: permuted row -> token
+  const float* row_w;        // MERGE_MLP: per-token expert weight
+  void* tap_bf16;            // MERGE_*: optional bf16 [tokens, N] contribution tap
+  float* tap_f32;            // MERGE_ATTN: optional fp32 [tokens, N] layer_mid tap
+};
+
+// Encodes a 2-D bf16 tensor map (rows x cols, row-major) with a box of
+// box_rows x 64 and the 128-byte swizzle.  Returns 0 on success.
+int make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
+// Launches the tcgen05 GEMM; bn = 64, 128 or 256 (SWIGLU: 128 output
+// columns per tile, 256 MMA columns).  A and B maps are built inside.
+int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b_rows, const GemmParams& p,
+                int num_sms, cudaStream_t st);
+
+// ------------------------------------------------------------------ norms
+// out[m] = bf16(w * xb * rsqrt(mean(xb^2) + eps)), xb = bf16(x[m * row_mul +
+// row_add]); extra rows [M, M+n_copy) of out are a copy of copy_src (decode:
+// prev_hs, whose projection gives the delayed values).
+int launch_rmsnorm(const float* x, int row_mul, int row_add, const void* w, void* out, void* tap, int M, int H,
+                   float eps, const void* copy_src, int n_copy, cudaStream_t st);
+int launch_embed(const int* ids, const void* table, float* stream, int M, int H, int vocab, float mult,
+                 float shift, int* status, cudaStream_t st);
+
+// ------------------------------------------------------------------ CCA attention input
+struct CcaParams {
+  const void* qkv;        // bf16 [rows, n_qkv]
+  int n_qkv;
+  const float* conv_w;    // [C, 3]
+  const float* conv_b;    // [C]
+  const float* k_temp;    // [n_kv]
+  const int* mask;        // prefill [B, S] or null
+  void* q_out;            // bf16 [B, n_q, S, d]
+  void* tap_q;            // optional copy of q_out
+  void* k_cache;
+  void* v_cache;
+  int cache_cap;
+  int* cache_len;         // [B]
+  void* conv_state;       // bf16 [B, C, 2]
+  void* prev_hs;          // bf16 [B, H]
+  const void* a_in;       // bf16 [rows, H] (prev_hs source)
+  int B, S, H, n_q, n_kv, d, rot;
+  int cca_res, v_delayed;
+  float theta, eps;
+  int decode;             // 1: one token per sequence, history from conv_state
+  int* status;
+};
+int launch_cca(const CcaParams& p, cudaStream_t st);
+
+// ------------------------------------------------------------------ attention
+struct AttnParams {
+  const void* q;          // bf16 [B, n_q, S, d]
+  const void* k_cache;    // bf16 [B, n_kv, cap, d]
+  const void* v_cache;
+  const int* mask;        // [B, S] or null
+  void* out;              // bf16 premix [B*S, n_q*d]
+  int B, S, cap, n_q, n_kv, d, window;
+  float scale;
+};
+int launch_attn_prefill(const AttnParams& p, cudaStream_t st);
+
+struct DecodeAttnParams {
+  const void* q;          // bf16 [B, n_q, d]
+  const void* k_cache;
+  const void* v_cache;
+  const int* cache_len;   // [B]: position of the new token (already in the cache)
+  void* out;              // bf16 premix [B, n_q*d]
+  float* part;            // workspace partials
+  int B, cap, n_q, n_kv, d, window, n_chunks;
+  float scale;
+};
+size_t decode_attn_ws_bytes(int B, int n_q, int d, int window);
+int launch_attn_decode(const DecodeAttnParams& p, cudaStream_t st);
+
+// ------------------------------------------------------------------ router / MoE dispatch
+struct RouterParams {
+  const float* r;         // [M, R] router state (down_proj output)
+  const float* norm_w;
+  const float* fc1_w; const float* fc1_b;
+  const float* fc2_w; const float* fc2_b;
+  const float* out_w;     // [E+1, R]
+  const float* balancing; // [E+1]
+  const int* mask;        // [M] token validity or null
+  float* logits;          // [M, E+1]
+  int* cls;               // [M] 0..E (E = skip)
+  int* idx;               // optional [M]
+  float* w;               // [M]
+  float* w_tap;           // optional [M]
+  int M, R, E;
+  float eps;
+};
+int launch_router(const RouterParams& p, cudaStream_t st);
+
+// Stable counting sort of tokens by class: pos[t] = permuted row of token t,
+// perm[row] = token; group_off[E+1]; mt_start[E+1] (128-row tiles).
+int launch_permute(const int* cls, int M, int E, int* group_off, int* mt_start, int* pos, int* perm, int* status,
+                   cudaStream_t st);
+
+// Copies m_in rows of routed tokens into their permuted rows; writes the
+// merge-2 output of skipped (and padding) tokens; decode: cache_len += 1.
+struct DispatchParams {
+  const int* cls; const int* pos;
+  const void* m_in;       // bf16 [M, H]
+  void* x_perm;           // bf16 [M, H]
+  float* stream;          // [M, H] in: layer_mid; skip rows -> layer_output
+  const float* merge_m;   // [4, H]
+  void* tap_mlp_out;      // optional bf16 [M, H]
+  int* cache_len_inc;     // optional [M] (decode)
+  int M, H, E;
+};
+int launch_dispatch(const DispatchParams& p, cudaStream_t st);
+
+int num_sms_current();
+
+}  // namespace zaya

@@ -1,0 +1,115 @@
+// RMSNorm of the fp32 stream and the embedding gather.
+//
+// A block norm casts the fp32 stream to its weight's dtype (bf16) and norms
+// it (nnterp "zaya" page, "The stream is float32 whatever the load"):
+//   out = bf16(w * xb / sqrt(mean(xb^2) + eps)),  xb = bf16(x).
+// One warp per row, float4 loads, the row kept in registers; HBM-bound
+// (4 bytes read + 2 bytes written per element).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace zaya {
+
+namespace {
+
+template <int CHUNKS>  // H = CHUNKS * 128
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, int row_mul, int row_add,
+                                                      const __nv_bfloat16* __restrict__ w,
+                                                      __nv_bfloat16* __restrict__ out, __nv_bfloat16* __restrict__ tap,
+                                                      int M, float eps, const __nv_bfloat16* __restrict__ copy_src,
+                                                      int n_copy) {
+  constexpr int H = CHUNKS * 128;
+  const int row = blockIdx.x * 8 + warp_id();
+  const int lane = lane_id();
+  if (row >= M + n_copy) return;
+  if (row >= M) {  // verbatim copy rows (decode: prev_hs feeds the delayed values)
+    const uint2* src = reinterpret_cast<const uint2*>(copy_src + (size_t)(row - M) * H);
+    uint2* dst = reinterpret_cast<uint2*>(out + (size_t)row * H);
+#pragma unroll
+    for (int c = 0; c < CHUNKS; ++c) dst[c * 32 + lane] = src[c * 32 + lane];
+    return;
+  }
+  const int src_row = row * row_mul + row_add;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)src_row * H);
+  float v[CHUNKS * 4];
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < CHUNKS; ++c) {
+    float4 t = xr[c * 32 + lane];
+    v[4 * c + 0] = round_bf(t.x);
+    v[4 * c + 1] = round_bf(t.y);
+    v[4 * c + 2] = round_bf(t.z);
+    v[4 * c + 3] = round_bf(t.w);
+    ss += v[4 * c] * v[4 * c] + v[4 * c + 1] * v[4 * c + 1] + v[4 * c + 2] * v[4 * c + 2] +
+          v[4 * c + 3] * v[4 * c + 3];
+  }
+  ss = warp_sum(ss);
+  const float inv = rsqrtf(ss / (float)H + eps);
+  const uint2* wr = reinterpret_cast<const uint2*>(w);
+  uint2* orow = reinterpret_cast<uint2*>(out + (size_t)row * H);
+  uint2* trow = tap ? reinterpret_cast<uint2*>(tap + (size_t)row * H) : nullptr;
+#pragma unroll
+  for (int c = 0; c < CHUNKS; ++c) {
+    const uint2 wu = wr[c * 32 + lane];
+    const float2 w01 = unpack_bf2(wu.x), w23 = unpack_bf2(wu.y);
+    uint2 o;
+    o.x = pack_bf2(w01.x * (v[4 * c] * inv), w01.y * (v[4 * c + 1] * inv));
+    o.y = pack_bf2(w23.x * (v[4 * c + 2] * inv), w23.y * (v[4 * c + 3] * inv));
+    orow[c * 32 + lane] = o;
+    if (trow) trow[c * 32 + lane] = o;
+  }
+}
+
+// stream[m] = fp32((E[id] + shift) * mult); one warp per row.
+__global__ void __launch_bounds__(256) embed_kernel(const int* __restrict__ ids, const __nv_bfloat16* __restrict__ table,
+                                                    float* __restrict__ stream, int M, int H, int vocab, float mult,
+                                                    float shift, int* status) {
+  const int row = blockIdx.x * 8 + warp_id();
+  const int lane = lane_id();
+  if (row >= M) return;
+  const int id = ids[row];
+  float4* dst = reinterpret_cast<float4*>(stream + (size_t)row * H);
+  if (id < 0 || id >= vocab) {
+    if (lane == 0) set_status(status, ZAYA_ERR_DEVICE_RANGE);
+    for (int c = lane; c < H / 4; c += 32) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const uint2* src = reinterpret_cast<const uint2*>(table + (size_t)id * H);
+  for (int c = lane; c < H / 4; c += 32) {
+    const uint2 u = src[c];
+    const float2 a = unpack_bf2(u.x), b = unpack_bf2(u.y);
+    dst[c] = make_float4((a.x + shift) * mult, (a.y + shift) * mult, (b.x + shift) * mult, (b.y + shift) * mult);
+  }
+}
+
+}  // namespace
+
+int launch_rmsnorm(const float* x, int row_mul, int row_add, const void* w, void* out, void* tap, int M, int H,
+                   float eps, const void* copy_src, int n_copy, cudaStream_t st) {
+  const int rows = M + n_copy;
+  if (rows <= 0) return ZAYA_OK;
+  const dim3 grid((rows + 7) / 8);
+  const auto* wb = static_cast<const __nv_bfloat16*>(w);
+  auto* ob = static_cast<__nv_bfloat16*>(out);
+  auto* tb = static_cast<__nv_bfloat16*>(tap);
+  const auto* cs = static_cast<const __nv_bfloat16*>(copy_src);
+  switch (H / 128) {
+    case 2: rmsnorm_kernel<2><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 4: rmsnorm_kernel<4><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 8: rmsnorm_kernel<8><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 16: rmsnorm_kernel<16><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 32: rmsnorm_kernel<32><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    default: return ZAYA_ERR_UNSUPPORTED;
+  }
+  return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
+}
+
+int launch_embed(const int* ids, const void* table, float* stream, int M, int H, int vocab, float mult, float shift,
+                 int* status, cudaStream_t st) {
+  if (M <= 0) return ZAYA_OK;
+  embed_kernel<<<(M + 7) / 8, 256, 0, st>>>(ids, static_cast<const __nv_bfloat16*>(table), stream, M, H, vocab, mult,
+                                            shift, status);
+  return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
+}
+
+}  // namespace zaya
