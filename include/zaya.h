@@ -184,6 +184,35 @@ int zaya_block_decode(const zaya_config* cfg, const zaya_block_weights* w, int32
                       const zaya_block_state* state, const zaya_taps* taps,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* zaya_block_decode without a caller-supplied workspace.  The paper has no
+ * counterpart: this is a calling convention of the library.
+ *
+ * For callers that cannot allocate device memory where they run a decode
+ * step -- for example a serving runtime that has handed all device memory to
+ * its own pools and forbids further allocations, or a plain C host program
+ * with no device allocator of its own -- and so cannot provide the workspace
+ * zaya_block_decode takes.  Arguments and results are those of
+ * zaya_block_decode; inputs and outputs are still the caller's buffers.
+ *
+ * Scratch: a fixed 8 MiB array in the library's own device memory (held on
+ * every GPU that loads the library until the process exits), enough for a
+ * full-width decode step (hidden 2048, 16 experts x 2048) of up to 64
+ * sequences.  A call whose zaya_workspace_size(cfg, ZAYA_DECODE, B, 1)
+ * exceeds 8 MiB returns ZAYA_ERR_WORKSPACE without launching anything.  No
+ * cudaMalloc, cudaFree or other allocating call is made.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps the previous call's
+ *    contents; the call clears the device status word it needs at zero.
+ *    Calls that overlap on the GPU (other streams, other threads) race on
+ *    the array and corrupt each other: serialise them.
+ *  - Device-side faults are recorded in the array's status word, which no
+ *    entry point returns. */
+int zaya_block_decode_noalloc(const zaya_config* cfg, const zaya_block_weights* w, int32_t block_idx, int32_t B,
+                              float* hidden, const float* router_state_in, float* router_state_out,
+                              const zaya_block_state* state, const zaya_taps* taps, void* stream);
+
 /* The whole stack: embedding -> n_blocks blocks (router state chained on the
  * device) -> final norm -> tied lm_head (zaya page, "Printout" and "The
  * readout and the tokenizer": logits = lm_head(norm(stream)), no cap).

@@ -17,7 +17,8 @@ from ._abi import (ZAYA_DECODE, ZAYA_OK, ZAYA_PREFILL, zaya_block_state,  # noqa
                    zaya_block_weights, zaya_config, zaya_taps)
 
 __all__ = ["make_config", "make_weights", "make_state", "make_taps", "zaya_workspace_size",
-           "zaya_stack_workspace_size", "zaya_block_prefill", "zaya_block_decode", "zaya_stack_forward",
+           "zaya_stack_workspace_size", "zaya_block_prefill", "zaya_block_decode", "zaya_block_decode_noalloc",
+           "zaya_stack_forward",
            "zaya_device_status", "zaya_status_string", "zaya_abi_version", "zaya_profile_enable",
            "zaya_profile_reset", "zaya_profile_read", "zaya_launch_count", "ZayaError", "ZAYA_PREFILL",
            "ZAYA_DECODE"]
@@ -122,6 +123,16 @@ def zaya_block_decode(cfg, weights, block_idx, B, hidden, router_state_in, route
         C.byref(cfg), C.byref(weights), block_idx, B, _ptr(hidden), _ptr(router_state_in), _ptr(router_state_out),
         C.byref(state), _ref(taps), _ptr(workspace), ws_bytes, _stream_ptr(stream))
     return _check(rc, "zaya_block_decode", check)
+
+
+def zaya_block_decode_noalloc(cfg, weights, block_idx, B, hidden, router_state_in, router_state_out, state,
+                              taps=None, stream=None, check=True) -> int:
+    """zaya_block_decode with the library's own fixed scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    rc = _abi.lib().zaya_block_decode_noalloc(
+        C.byref(cfg), C.byref(weights), block_idx, B, _ptr(hidden), _ptr(router_state_in), _ptr(router_state_out),
+        C.byref(state), _ref(taps), _stream_ptr(stream))
+    return _check(rc, "zaya_block_decode_noalloc", check)
 
 
 def zaya_stack_forward(cfg, blocks, embed, final_norm_w, mode, B, S, ids, attn_mask, states, logits,

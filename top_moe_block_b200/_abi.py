@@ -73,6 +73,9 @@ def lib() -> C.CDLL:
         L.zaya_block_decode.argtypes = [P(zaya_config), P(zaya_block_weights), i32, i32, vp, vp, vp,
                                         P(zaya_block_state), P(zaya_taps), vp, sz, vp]
         L.zaya_block_decode.restype = C.c_int
+        L.zaya_block_decode_noalloc.argtypes = [P(zaya_config), P(zaya_block_weights), i32, i32, vp, vp, vp,
+                                                P(zaya_block_state), P(zaya_taps), vp]
+        L.zaya_block_decode_noalloc.restype = C.c_int
         L.zaya_stack_forward.argtypes = [P(zaya_config), i32, P(zaya_block_weights), vp, vp, i32, i32, i32, vp, vp,
                                          P(zaya_block_state), vp, i32, vp, sz, vp]
         L.zaya_stack_forward.restype = C.c_int

@@ -557,3 +557,49 @@ int zaya_device_status(void* workspace, void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ decode without a caller workspace
+// Scratch for zaya_block_decode_noalloc, in the library's own device memory:
+// every GPU that loads this library holds these bytes until the process exits.
+namespace {
+constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code cannot use the symbol itself: on the host it names a
+// host-side stand-in, not device memory).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZAYA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ZAYA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ZAYA_OK;
+}
+}  // namespace
+
+extern "C" int zaya_block_decode_noalloc(const zaya_config* cfg, const zaya_block_weights* w, int32_t block_idx,
+                                         int32_t B, float* hidden, const float* router_state_in,
+                                         float* router_state_out, const zaya_block_state* state,
+                                         const zaya_taps* taps, void* stream) {
+  if (check_config(cfg) != ZAYA_OK) return check_config(cfg);
+  if (B <= 0) return ZAYA_ERR_INVALID_ARG;
+  const size_t need = zaya_workspace_size(cfg, ZAYA_DECODE, B, 1);
+  if (need == 0) return ZAYA_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) return ZAYA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  ZAYA_TRY(noalloc_scratch(&scratch));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The scratch keeps the previous call's contents; only the status word must start at zero.
+  if (cudaMemsetAsync(scratch, 0, 256, st) != cudaSuccess) return ZAYA_ERR_CUDA;
+  return zaya_block_decode(cfg, w, block_idx, B, hidden, router_state_in, router_state_out, state, taps, scratch,
+                           kNoAllocScratchBytes, stream);
+}
