@@ -344,7 +344,7 @@ def run_ours(args, world, rank, local):
 
 
 def kernel_source_sha(name):
-    files = {"attention": "attn_prefill.cu", "experts_gate_up": "gemm_tc.cu", "experts_down_merge": "gemm_tc.cu",
+    files = {"attention": "attn_tc.cu", "experts_gate_up": "gemm_tc.cu", "experts_down_merge": "gemm_tc.cu",
              "qkv_gemm": "gemm_tc.cu", "o_proj_merge": "gemm_tc.cu", "router_down": "gemm_tc.cu",
              "router_mlp": "router.cu", "permute": "router.cu", "dispatch": "router.cu", "cca": "cca.cu",
              "rmsnorm_attn": "norm.cu", "rmsnorm_mlp": "norm.cu"}

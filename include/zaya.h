@@ -239,11 +239,12 @@ const char* zaya_status_string(int code);
 
 /* Stage timing for measurement (no counterpart on the pages).  When enabled,
  * a CUDA event is recorded on the caller's stream before and after every
- * kernel launch of the entry points above; zaya_profile_read synchronises
- * those events and returns, per stage name (static strings such as
- * "attention", "experts_gate_up"), the accumulated milliseconds and kernel
- * launches since the last reset.  Returns the number of stages, of which
- * at most max_stages are written.  Off by default. */
+ * stage (one or two kernel launches) of the entry points above;
+ * zaya_profile_read synchronises those events and returns, per stage name
+ * (static strings such as "attention", "experts_gate_up"), the accumulated
+ * milliseconds and the number of times the stage ran since the last reset.
+ * Returns the number of stages, of which at most max_stages are written.
+ * Off by default. */
 void zaya_profile_enable(int on);
 void zaya_profile_reset(void);
 int zaya_profile_read(int32_t max_stages, const char** names, double* total_ms, int64_t* launches);

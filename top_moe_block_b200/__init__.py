@@ -161,7 +161,7 @@ def zaya_profile_reset() -> None:
 
 
 def zaya_profile_read(max_stages: int = 64) -> dict:
-    """{stage name: (total milliseconds, kernel launches)} since the last reset."""
+    """{stage name: (total milliseconds, stage calls)} since the last reset."""
     names = (C.c_char_p * max_stages)()
     ms = (C.c_double * max_stages)()
     n_l = (C.c_int64 * max_stages)()

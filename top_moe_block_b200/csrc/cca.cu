@@ -13,10 +13,11 @@
 // channels and the previous token's attention-norm output (ZAYA1-8B-JANGTQ2
 // README, "Architecture Summary").
 //
-// One CTA per token; warp w < n_q handles query head w, the next n_kv warps
-// the key heads, the last n_kv warps the value heads; each lane owns d/32
-// consecutive dims, so the head norm is a warp reduction and the RoPE pair
-// exchange a shuffle.  HBM-bound: ~3 KB read and ~3 KB written per token.
+// Each lane owns d/32 consecutive dims of a head, so the head norm is a warp
+// reduction and the RoPE pair exchange a shuffle.  Prefill: a CTA covers 16
+// consecutive tokens with their pre-conv rows staged in shared memory.
+// Decode: a CTA per sequence.  HBM-bound: ~3 KB read and ~3 KB written per
+// token.
 #include <math.h>
 
 #include "common.cuh"
@@ -44,6 +45,19 @@ struct Pre {
   }
 };
 
+// DPL consecutive bf16 written as one 4- or 8-byte store.
+template <int DPL>
+__device__ __forceinline__ void store_bf(__nv_bfloat16* dst, const float (&y)[DPL]) {
+  if constexpr (DPL == 4) {
+    uint2 u;
+    u.x = pack_bf2(y[0], y[1]);
+    u.y = pack_bf2(y[2], y[3]);
+    *reinterpret_cast<uint2*>(dst) = u;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf2(y[0], y[1]);
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void rope_apply(float (&y)[D / 32], int lane, int pos, int rot, float theta) {
   constexpr int DPL = D / 32;
@@ -70,6 +84,8 @@ __device__ __forceinline__ void rope_apply(float (&y)[D / 32], int lane, int pos
   }
 }
 
+// Decode (one token per sequence, history from conv_state) -- and the
+// general per-token form: CTA = one token, one warp per head.
 template <int D>
 __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
   constexpr int DPL = D / 32;
@@ -200,13 +216,180 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
   }
 }
 
+
+// Prefill: CTA = kTok consecutive tokens of one sequence.  The pre-conv rows
+// t0-2 .. t0+kTok-1 (all q/k/v projection columns, padding rows zeroed) are
+// staged once in shared memory, so every conv tap, the CCA residual and the
+// delayed value half read shared memory; RoPE cos/sin are tabled once per
+// (token, frequency) and shared by all heads.
+constexpr int kTok = 16;
+
+template <int D>
+__global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
+  constexpr int DPL = D / 32;
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int nq = p.n_q, nkv = p.n_kv, rep = nq / nkv;
+  const int C = (nq + nkv) * D;
+  const int ld = p.n_qkv;
+  const int b = blockIdx.y;
+  const int s0 = blockIdx.x * kTok;
+  const int half = p.rot / 2;
+  auto* u = reinterpret_cast<__nv_bfloat16*>(sm);                              // [kTok + 2][ld]
+  float* inv_f = reinterpret_cast<float*>(sm + (size_t)(kTok + 2) * ld * 2);   // [half]
+  float2* cs = reinterpret_cast<float2*>(inv_f + 64);                          // [kTok][half]
+  const auto* qkv = static_cast<const __nv_bfloat16*>(p.qkv);
+  const size_t row0 = (size_t)b * p.S;
+
+  // stage rows s0-2 .. s0+kTok-1 with cp.async (16-byte vectors, all issued before
+  // one wait; zero-filled outside the sequence and at padding)
+  const int vec_per_row = ld / 8;
+  for (int i = threadIdx.x; i < (kTok + 2) * vec_per_row; i += blockDim.x) {
+    const int r = i / vec_per_row, c = i % vec_per_row;
+    const int s = s0 - 2 + r;
+    const bool valid = s >= 0 && s < p.S && (!p.mask || p.mask[row0 + s] != 0);
+    const __nv_bfloat16* src = qkv + (row0 + (valid ? s : 0)) * ld + c * 8;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(u + (size_t)r * ld + c * 8)),
+                 "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int f = threadIdx.x; f < half; f += blockDim.x)
+    inv_f[f] = (float)(1.0 / pow((double)p.theta, (double)(2 * f) / (double)p.rot));
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  for (int i = threadIdx.x; i < kTok * half; i += blockDim.x) {
+    const int tt = i / half, f = i % half;
+    float sn, c;
+    sincosf((float)(s0 + tt) * inv_f[f], &sn, &c);
+    cs[i] = make_float2(c, sn);
+  }
+  __syncthreads();
+
+  const int warp = warp_id(), lane = lane_id();
+  const int n_heads = nq + 2 * nkv;
+  const float sqrt_d = sqrtf((float)D);
+  for (int task = warp; task < kTok * n_heads; task += blockDim.x / 32) {
+    const int tt = task / n_heads, head = task % n_heads;
+    const int s = s0 + tt;
+    if (s >= p.S) continue;
+    const __nv_bfloat16* ut = u + (size_t)(tt + 2) * ld;   // token t
+    const __nv_bfloat16* u1 = ut - ld;                      // t - 1
+    const __nv_bfloat16* u2 = ut - 2 * ld;                  // t - 2
+    if (head < nq + nkv) {
+      const bool is_q = head < nq;
+      const int hh = is_q ? head : head - nq;
+      const int g = is_q ? head / rep : hh;
+      const int cbase = (is_q ? hh * D : nq * D + hh * D) + lane * DPL;
+      float y[DPL], a0[DPL], a1[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const int c = cbase + i;
+        a0[i] = bf2f(ut[c]);
+        a1[i] = bf2f(u1[c]);
+        const float a2 = bf2f(u2[c]);
+        float acc = __ldg(p.conv_b + c);
+        acc = fmaf(__ldg(p.conv_w + 3 * c + 0), a2, acc);
+        acc = fmaf(__ldg(p.conv_w + 3 * c + 1), a1[i], acc);
+        acc = fmaf(__ldg(p.conv_w + 3 * c + 2), a0[i], acc);
+        if (p.cca_res) {
+          const int j = lane * DPL + i;
+          const float kpre = bf2f(ut[nq * D + g * D + j]);
+          if (is_q) {
+            acc += 0.5f * (a0[i] + kpre);
+          } else {
+            float qs = 0.f;
+            for (int h2 = g * rep; h2 < (g + 1) * rep; ++h2) qs += bf2f(ut[h2 * D + j]);
+            acc += 0.5f * (qs / (float)rep + kpre);
+          }
+        }
+        y[i] = acc;
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) ss += y[i] * y[i];
+      ss = warp_sum(ss);
+      float scl = sqrt_d / fmaxf(sqrtf(ss), p.eps);
+      if (!is_q) scl *= __ldg(p.k_temp + g);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) y[i] *= scl;
+      if (half > 0) {   // rotate-half over dims [0, rot)
+        const int off = half / DPL;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) {
+          const int j = lane * DPL + i;
+          const bool lo = j < half, in_rot = j < p.rot;
+          const int src = in_rot ? (lo ? lane + off : lane - off) : lane;
+          const float partner = __shfl_sync(0xffffffffu, y[i], src);
+          if (in_rot) {
+            const float2 e = cs[tt * half + (lo ? j : j - half)];
+            y[i] = lo ? (y[i] * e.x - partner * e.y) : (y[i] * e.x + partner * e.y);
+          }
+        }
+      }
+      __nv_bfloat16* dst;
+      if (is_q) {
+        const size_t off = (((size_t)b * nq + hh) * p.S + s) * D + lane * DPL;
+        dst = static_cast<__nv_bfloat16*>(p.q_out) + off;
+        if (p.tap_q) store_bf<DPL>(static_cast<__nv_bfloat16*>(p.tap_q) + off, y);
+      } else {
+        dst = static_cast<__nv_bfloat16*>(p.k_cache) + (((size_t)b * nkv + hh) * p.cache_cap + s) * D + lane * DPL;
+      }
+      store_bf<DPL>(dst, y);
+      if (s == p.S - 1) {   // conv_state <- pre-conv channels of tokens S-2, S-1
+        auto* cst = static_cast<__nv_bfloat16*>(p.conv_state) + (size_t)b * C * 2;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) {
+          cst[(size_t)(cbase + i) * 2 + 0] = f2bf(a1[i]);
+          cst[(size_t)(cbase + i) * 2 + 1] = f2bf(a0[i]);
+        }
+      }
+    } else {
+      const int g = head - nq - nkv;
+      const int vc0 = nq * D + nkv * D;
+      const int vd0 = vc0 + nkv * (D / 2);
+      __nv_bfloat16* dst =
+          static_cast<__nv_bfloat16*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + s) * D + lane * DPL;
+      float vv[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const int j = lane * DPL + i;
+        if (j < D / 2)
+          vv[i] = bf2f(ut[vc0 + g * (D / 2) + j]);
+        else
+          vv[i] = bf2f((p.v_delayed ? u1 : ut)[vd0 + g * (D / 2) + (j - D / 2)]);
+      }
+      store_bf<DPL>(dst, vv);
+      if (s == p.S - 1 && g == 0) {   // prev_hs <- attention_norm_output of token S-1
+        const uint2* src = reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.a_in) + (row0 + s) * p.H);
+        uint2* ph = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.prev_hs) + (size_t)b * p.H);
+        for (int c = lane; c < p.H / 4; c += 32) ph[c] = src[c];
+        if (lane == 0) p.cache_len[b] = p.S;
+      }
+    }
+  }
+}
+
 }  // namespace
 
 int launch_cca(const CcaParams& p, cudaStream_t st) {
   const int tokens = p.decode ? p.B : p.B * p.S;
   if (tokens <= 0) return ZAYA_OK;
   const int threads = 32 * (p.n_q + 2 * p.n_kv);
-  if (threads > 1024) return ZAYA_ERR_UNSUPPORTED;
+  if (threads > 1024 || p.rot / 2 > 64 || p.n_qkv % 8) return ZAYA_ERR_UNSUPPORTED;
+  if (!p.decode) {
+    const size_t smem = (size_t)(kTok + 2) * p.n_qkv * 2 + 64 * 4 + (size_t)kTok * (p.rot / 2) * 8;
+    const dim3 grid((p.S + kTok - 1) / kTok, p.B);
+    if (p.d == 128) {
+      cudaFuncSetAttribute(cca_prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cca_prefill_kernel<128><<<grid, 512, smem, st>>>(p);
+    } else if (p.d == 64) {
+      cudaFuncSetAttribute(cca_prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cca_prefill_kernel<64><<<grid, 512, smem, st>>>(p);
+    } else {
+      return ZAYA_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
+  }
   if (p.d == 128)
     cca_kernel<128><<<tokens, threads, 0, st>>>(p);
   else if (p.d == 64)

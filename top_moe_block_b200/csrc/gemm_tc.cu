@@ -6,10 +6,14 @@
 //               shared-memory ring (128-byte swizzle), one mbarrier per slot;
 //   warp 1      one elected thread issues tcgen05.mma (M=128, N=BN, K=16) into
 //               one of two TMEM accumulators and commits slot releases;
-//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator (each warp
-//               owns the 32 TMEM lanes its warp index allows), the fused
-//               epilogue, global stores; then the accumulator is handed back,
-//               so the epilogue of tile i overlaps the main loop of tile i+1.
+//   warps 2..   epilogue (4 warps; 8 for the merge epilogues, two per TMEM
+//               lane quarter splitting the columns): tcgen05.ld of the finished
+//               accumulator (each warp reads the 32 TMEM lanes its warp index
+//               allows), the fused epilogue, global stores; then the
+//               accumulator is handed back, so the epilogue of tile i overlaps
+//               the main loop of tile i+1.
+// The producer also pulls B (weight) boxes into L2 eight k-blocks ahead of
+// their loads, so the ring's loads wait on L2 rather than on HBM.
 // Grouped mode (the experts): A rows are the tokens permuted by expert, B is
 // the stacked expert weights; the tile list is derived on the device from
 // the per-expert row offsets, so no host synchronisation is needed.
@@ -20,6 +24,8 @@
 //                order"): attention_output = bf16((o + hb) * hs);
 //                h = attention_output + (x + rb) * rs written over x
 //   ROUTER_DOWN  router down_proj + bias + previous state * router_states_scale
+//   STORE_F32    fp32 partial sums of a split-K product (router down_proj: the
+//                router kernel adds the slabs in a fixed order)
 //   SWIGLU       expert gate/up: act = bf16(silu(gate) * up)
 //   MERGE_MLP    expert down: y = w_t * acc; mlp_output = bf16((y + hb) * hs);
 //                out = mlp_output + (h + rb) * rs, scattered to token t's row
@@ -36,16 +42,26 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 
+template <int EPI>
+__host__ __device__ constexpr int epi_warps() { return (EPI == EPI_MERGE_ATTN || EPI == EPI_MERGE_MLP) ? 8 : 4; }
+template <int EPI>
+__host__ __device__ constexpr bool is_merge() { return EPI == EPI_MERGE_ATTN || EPI == EPI_MERGE_MLP; }
+constexpr int kPrefetchAhead = 8;  // k-blocks of B pulled into L2 ahead of their TMA load
+
 template <int BN>
 struct GemmCfg {
   static constexpr int B_STAGE_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);  // ~192 KB ring
   static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int PARAM_BYTES = 2 * 4 * BN * 4;  // merge epilogues: [2 tiles][hb,hs,rb,rs][BN] fp32
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + PARAM_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
 struct TileInfo {
+  int kb0;     // first k-block of this tile's K slab
+  int nkb;     // k-blocks in the slab
+  int split;   // slab index (STORE_F32)
   int m0;      // first A row
   int m_end;   // A rows of this tile's group end here (exclusive)
   int n0;      // first output column
@@ -56,7 +72,8 @@ struct TileInfo {
 template <int EPI, int BN_OUT>
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
   const int nt = p.N / BN_OUT;
-  if (!p.grouped) return ((p.M + BM - 1) / BM) * nt;
+  const int ks = p.k_splits > 1 ? p.k_splits : 1;
+  if (!p.grouped) return ((p.M + BM - 1) / BM) * nt * ks;
   return p.mt_start[p.n_groups] * nt;
 }
 
@@ -64,10 +81,17 @@ template <int EPI, int BN_OUT>
 __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
   TileInfo ti;
   const int nt = p.N / BN_OUT;
+  const int ks = p.k_splits > 1 ? p.k_splits : 1;
+  ti.nkb = p.K / BK / ks;
+  ti.split = 0;
+  ti.kb0 = 0;
   if (!p.grouped) {
     const int mt = (p.M + BM - 1) / BM;
     ti.m0 = (t % mt) * BM;
-    ti.n0 = (t / mt) * BN_OUT;
+    const int rest = t / mt;
+    ti.split = rest % ks;
+    ti.kb0 = ti.split * ti.nkb;
+    ti.n0 = (rest / ks) * BN_OUT;
     ti.m_end = p.M;
     ti.b_row = ti.n0;
     ti.b_row2 = ti.n0;
@@ -89,8 +113,8 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)
 
 // Epilogue of one row (this thread) x 32 consecutive columns.
 template <int EPI>
-__device__ __forceinline__ void epilogue32(const GemmParams& p, int row, int col, const uint32_t (&r)[32],
-                                           const uint32_t (&r2)[32]) {
+__device__ __forceinline__ void epilogue32(const GemmParams& p, int row, int col, int split, const uint32_t (&r)[32],
+                                           const uint32_t (&r2)[32], const float* prm, int prm_ld) {
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -109,6 +133,10 @@ __device__ __forceinline__ void epilogue32(const GemmParams& p, int row, int col
       u.w = pack_bf2(v[8 * q + 6], v[8 * q + 7]);
       dst[q] = u;
     }
+  } else if constexpr (EPI == EPI_STORE_F32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + ((size_t)split * p.M + row) * p.ldo + col);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
   } else if constexpr (EPI == EPI_ROUTER_DOWN) {
     float* dst = static_cast<float*>(p.out) + (size_t)row * p.ldo + col;
     const float* prev = p.prev ? p.prev + (size_t)row * p.N + col : nullptr;
@@ -138,19 +166,27 @@ __device__ __forceinline__ void epilogue32(const GemmParams& p, int row, int col
     float* srow = p.stream + (size_t)token * N + col;
     __nv_bfloat16* tap = p.tap_bf16 ? static_cast<__nv_bfloat16*>(p.tap_bf16) + (size_t)token * N + col : nullptr;
     float* tapf = p.tap_f32 ? p.tap_f32 + (size_t)token * N + col : nullptr;
+    float4 xs[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) xs[q] = reinterpret_cast<const float4*>(srow)[q];   // all loads in flight first
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      float4 x4 = reinterpret_cast<const float4*>(srow)[q];
+      float4 x4 = xs[q];
       float* xp = &x4.x;
+      const float4 hb4 = *reinterpret_cast<const float4*>(prm + 4 * q);
+      const float4 hs4 = *reinterpret_cast<const float4*>(prm + prm_ld + 4 * q);
+      const float4 rb4 = *reinterpret_cast<const float4*>(prm + 2 * prm_ld + 4 * q);
+      const float4 rs4 = *reinterpret_cast<const float4*>(prm + 3 * prm_ld + 4 * q);
+      const float* hbp = &hb4.x;
+      const float* hsp = &hs4.x;
+      const float* rbp = &rb4.x;
+      const float* rsp = &rs4.x;
       float cb[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int c = col + 4 * q + j;
-        const float hb = __ldg(p.merge + c), hs = __ldg(p.merge + N + c);
-        const float rb = __ldg(p.merge + 2 * N + c), rs = __ldg(p.merge + 3 * N + c);
-        const float contrib = round_bf((v[4 * q + j] * wt + hb) * hs);
+        const float contrib = round_bf((v[4 * q + j] * wt + hbp[j]) * hsp[j]);
         cb[j] = contrib;
-        xp[j] = fmaf(xp[j] + rb, rs, contrib);
+        xp[j] = fmaf(xp[j] + rbp[j], rsp[j], contrib);
       }
       reinterpret_cast<float4*>(srow)[q] = x4;
       if (tapf) reinterpret_cast<float4*>(tapf)[q] = x4;
@@ -165,7 +201,7 @@ __device__ __forceinline__ void epilogue32(const GemmParams& p, int row, int col
 }
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
   using C = GemmCfg<BN>;
@@ -177,7 +213,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_STAGE_BYTES);
+  float* sPrm = reinterpret_cast<float*>(sB + STAGES * C::B_STAGE_BYTES);   // merge params [2][4][BN_OUT]
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sPrm) + C::PARAM_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -193,7 +230,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], epi_warps<EPI>());
     }
     fence_barrier_init();
     fence_proxy_async();
@@ -206,7 +243,6 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int k_blocks = p.K / BK;
   const int ntiles = total_tiles<EPI, BN_OUT>(p);
 
   if (warp == 0) {
@@ -216,7 +252,16 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
         const TileInfo ti = tile_info<EPI, BN_OUT>(p, t);
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        const int kb_end = ti.kb0 + ti.nkb;
+        for (int kb = ti.kb0; kb < ti.kb0 + kPrefetchAhead && kb < kb_end; ++kb) {
+          tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row);
+          if constexpr (EPI == EPI_SWIGLU) tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row2);
+        }
+        for (int kb = ti.kb0; kb < kb_end; ++kb) {
+          if (kb + kPrefetchAhead < kb_end) {
+            tma_prefetch_l2_2d(&tmB, (kb + kPrefetchAhead) * BK, ti.b_row);
+            if constexpr (EPI == EPI_SWIGLU) tma_prefetch_l2_2d(&tmB, (kb + kPrefetchAhead) * BK, ti.b_row2);
+          }
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) goto producer_done;
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
           tma_load_2d(sA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * BK, ti.m0);
@@ -247,8 +292,9 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
+        const int nkb = tile_info<EPI, BN_OUT>(p, t).nkb;
         bool ok = true;
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.status)) {
             ok = false;
             break;
@@ -272,25 +318,47 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5
-    const int q = warp & 3;  // TMEM lanes [32q, 32q+32) are reachable from this warp
+    // ---------------- epilogue warps 2 .. 2+EW-1
+    constexpr int EW = epi_warps<EPI>();
+    const int q = warp & 3;              // TMEM lanes [32q, 32q+32) are reachable from this warp
+    const int part = (warp - 2) >> 2;    // column interleave among the warps sharing a lane quarter
+    const int et = threadIdx.x - 64;     // epilogue thread index
     int local = 0;
+    bool aborted = false;   // a wait ran out: keep walking the tiles (barrier partners) without waiting
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const TileInfo ti = tile_info<EPI, BN_OUT>(p, t);
-      if (!mbar_wait(&tfull[acc], acc_phase, p.status)) break;
+      float* prm = sPrm + acc * 4 * BN_OUT;
+      if constexpr (is_merge<EPI>()) {
+        // this tile's merge parameters (hb, hs, rb, rs for its columns) into shared memory
+        for (int i = et; i < 4 * BN_OUT; i += EW * 32) {
+          const int r = i / BN_OUT, c = i % BN_OUT;
+          prm[i] = __ldg(p.merge + (size_t)r * p.N + ti.n0 + c);
+        }
+        // pull this thread's stream segment into L2 while the main loop runs
+        const int prow = ti.m0 + q * 32 + lane;
+        if (part == 0 && prow < ti.m_end) {
+          const int token = (EPI == EPI_MERGE_MLP) ? p.perm[prow] : prow;
+          const char* base = reinterpret_cast<const char*>(p.stream + (size_t)token * p.N + ti.n0);
+#pragma unroll
+          for (int off = 0; off < BN_OUT * 4; off += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + off));
+        }
+        named_barrier_sync(1, EW * 32);
+      }
+      if (!aborted && !mbar_wait(&tfull[acc], acc_phase, p.status)) aborted = true;
+      if (aborted) continue;
       tc_fence_after();
       const int row = ti.m0 + q * 32 + lane;
       const bool valid = row < ti.m_end;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
 #pragma unroll 1
-      for (int c = 0; c < BN_OUT; c += 32) {
+      for (int c = part * 32; c < BN_OUT; c += 32 * (EW / 4)) {
         uint32_t r[32], r2[32];
         tmem_ld32(tbase + c, r);
         if constexpr (EPI == EPI_SWIGLU) tmem_ld32(tbase + BN / 2 + c, r2);
         tmem_ld_wait();
-        if (valid) epilogue32<EPI>(p, row, ti.n0 + c, r, r2);
+        if (valid) epilogue32<EPI>(p, row, ti.n0 + c, ti.split, r, r2, prm + c, BN_OUT);
       }
       tc_fence_before();
       __syncwarp();
@@ -336,7 +404,7 @@ int launch_impl(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& 
   }
   int grid = ntiles_hint < num_sms ? ntiles_hint : num_sms;
   if (grid < 1) grid = 1;
-  kern<<<grid, 192, C::SMEM_BYTES, st>>>(ma, mb, p);
+  kern<<<grid, 64 + 32 * epi_warps<EPI>(), C::SMEM_BYTES, st>>>(ma, mb, p);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 
@@ -359,6 +427,8 @@ int make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t co
 int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b_rows, const GemmParams& p,
                 int num_sms, cudaStream_t st) {
   if (p.K % BK != 0 || p.K <= 0) return ZAYA_ERR_UNSUPPORTED;
+  const int ks = p.k_splits > 1 ? p.k_splits : 1;
+  if ((p.K / BK) % ks != 0 || (ks > 1 && (p.grouped || epi != EPI_STORE_F32))) return ZAYA_ERR_UNSUPPORTED;
   const int bn_out = (epi == EPI_SWIGLU) ? bn / 2 : bn;
   if (p.N % bn_out != 0) return ZAYA_ERR_UNSUPPORTED;
   if (a_rows <= 0) return ZAYA_OK;
@@ -368,7 +438,7 @@ int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b
   rc = make_tmap_bf16(&mb, B, (uint64_t)b_rows, (uint64_t)p.K, epi == EPI_SWIGLU ? bn / 2 : bn);
   if (rc) return rc;
   const int nt = p.N / bn_out;
-  int hint = p.grouped ? num_sms : ((p.M + BM - 1) / BM) * nt;
+  int hint = p.grouped ? num_sms : ((p.M + BM - 1) / BM) * nt * ks;
 #define ZAYA_GEMM_CASE(BNV, EPIV) \
   if (bn == BNV && epi == EPIV) return launch_impl<BNV, EPIV>(ma, mb, p, hint, num_sms, st);
   ZAYA_GEMM_CASE(256, EPI_STORE_BF16)
@@ -380,6 +450,10 @@ int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b
   ZAYA_GEMM_CASE(128, EPI_ROUTER_DOWN)
   ZAYA_GEMM_CASE(64, EPI_ROUTER_DOWN)
   ZAYA_GEMM_CASE(32, EPI_ROUTER_DOWN)
+  ZAYA_GEMM_CASE(256, EPI_STORE_F32)
+  ZAYA_GEMM_CASE(128, EPI_STORE_F32)
+  ZAYA_GEMM_CASE(64, EPI_STORE_F32)
+  ZAYA_GEMM_CASE(32, EPI_STORE_F32)
   ZAYA_GEMM_CASE(32 * 8, EPI_SWIGLU)
   ZAYA_GEMM_CASE(256, EPI_MERGE_MLP)
   ZAYA_GEMM_CASE(128, EPI_MERGE_MLP)

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,18 +14,21 @@ enum EpiKind {
   EPI_MERGE_ATTN = 1,   // o_proj + merge 1, stream updated in place
   EPI_ROUTER_DOWN = 2,  // out[m, n] = acc + bias[n] (+ prev[m, n] * scale[n]) in fp32
   EPI_SWIGLU = 3,       // grouped: act = bf16(silu(gate) * up)
-  EPI_MERGE_MLP = 4     // grouped: expert down + weight + merge 2, scattered to token rows
+  EPI_MERGE_MLP = 4,    // grouped: expert down + weight + merge 2, scattered to token rows
+  EPI_STORE_F32 = 5     // out[split][m, n] = acc (fp32 partial sums of a split-K product)
 };
 
 struct GemmParams {
   int M, N, K;               // C[M, N] = A[M, K] * B[N, K]^T (N = output columns)
+  int k_splits;              // dense STORE_F32 only: K split into this many slabs (0 or 1: none)
   int grouped;               // expert-grouped A rows / B row blocks
   const int* group_off;      // [E+1] first A row of each expert (grouped)
   const int* mt_start;       // [E+1] prefix of per-expert 128-row tile counts (grouped)
   int n_groups;              // E
   int b_rows_per_group;      // rows of B per expert (2I or H)
   int* status;
-  void* out;                 // STORE_BF16 / SWIGLU: bf16 [rows, ldo]; ROUTER_DOWN: fp32 [M, ldo]
+  void* out;                 // STORE_BF16 / SWIGLU: bf16 [rows, ldo]; ROUTER_DOWN: fp32 [M, ldo];
+                             // STORE_F32: fp32 [k_splits, M, ldo]
   int ldo;
   float* stream;             // MERGE_*: fp32 [tokens, N]
   const float* merge;        // MERGE_*: fp32 [4, N] hb, hs, rb, rs
@@ -45,6 +49,16 @@ int make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t co
 // columns per tile, 256 MMA columns).  A and B maps are built inside.
 int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b_rows, const GemmParams& p,
                 int num_sms, cudaStream_t st);
+
+// K slabs for the router down-projection of M rows (a power of two, at most
+// 8 and K/64): enough 128-row x slab tiles to fill the GPU while the fp32
+// partial slabs stay small.  Deterministic in M.
+inline int router_down_splits(int M, int K) {
+  const int mt = (M + 127) / 128;
+  int ks = 1;
+  while (ks * 2 <= 8 && ks * 2 <= K / 64 && mt * ks * 2 <= 148) ks *= 2;
+  return ks;
+}
 
 // ------------------------------------------------------------------ norms
 // out[m] = bf16(w * xb * rsqrt(mean(xb^2) + eps)), xb = bf16(x[m * row_mul +
@@ -90,7 +104,7 @@ struct AttnParams {
   int B, S, cap, n_q, n_kv, d, window;
   float scale;
 };
-int launch_attn_prefill(const AttnParams& p, cudaStream_t st);
+int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st);
 
 struct DecodeAttnParams {
   const void* q;          // bf16 [B, n_q, d]
@@ -107,10 +121,16 @@ int launch_attn_decode(const DecodeAttnParams& p, cudaStream_t st);
 
 // ------------------------------------------------------------------ router / MoE dispatch
 struct RouterParams {
-  const float* r;         // [M, R] router state (down_proj output)
+  const float* part;      // [n_splits, M, R] partial sums of m_in . W_down^T (split over K)
+  int n_splits;
+  const float* bias;      // [R] down_proj bias
+  const float* prev;      // [M, R] previous block's router state, or null (block 0)
+  const float* prev_scale;// [R] router_states_scale
+  float* r_out;           // [M, R] router state out (= router_state_out)
   const float* norm_w;
   const float* fc1_w; const float* fc1_b;
   const float* fc2_w; const float* fc2_b;
+  __nv_bfloat16* wsplit;  // workspace [2 layers][hi|lo][R][R] bf16: fc1/fc2 split for the tensor cores
   const float* out_w;     // [E+1, R]
   const float* balancing; // [E+1]
   const int* mask;        // [M] token validity or null

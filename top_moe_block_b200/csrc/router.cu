@@ -7,9 +7,12 @@
 // out_proj(gelu(fc2(gelu(fc1(rmsnorm(r)))))) over E + 1 classes, the last
 // being skip; p = softmax(logits) in fp32; class = argmax(p +
 // balancing_biases), the lowest index on exact ties; weight = p[class] (not
-// renormalised); skip -> (index 0, weight 0).  Runs in fp32 on CUDA cores:
-// 16 tokens per CTA, each 256x256 layer as a register-tiled product whose
-// weight slab is staged transposed in shared memory.
+// renormalised); skip -> (index 0, weight 0).  The choice is taken on fp32
+// scores, so the logits must carry fp32 accuracy: fc1 and fc2 run on tensor
+// cores with both operands split into bf16 hi + lo parts (three products
+// hi.hi + hi.lo + lo.hi, fp32 accumulation: ~16 significant bits per product,
+// about fp32's error after the 256-term sums); norm, GELU, out_proj and the
+// softmax run in fp32 on CUDA cores.  32 tokens per CTA.
 #include <math.h>
 
 #include "common.cuh"
@@ -19,97 +22,218 @@ namespace zaya {
 
 namespace {
 
-constexpr int kTM = 16;     // tokens per router CTA
-constexpr int kKC = 32;     // k-chunk of a weight slab
+constexpr int kTM = 32;          // tokens per router CTA
+constexpr int kThreads = 256;    // 8 warps: warp w -> rows 16*(w&1) .., outputs (w>>1)*R/4 ..
 constexpr int kRMax = 256;
+constexpr int kZS = kRMax + 8;   // row stride (floats) of the fp32 activation tiles: conflict-free float2 reads
 
 __device__ __forceinline__ float gelu_exact(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
-// out[tt][j] = gelu(sum_k in[tt][k] * W[j][k] + bias[j]) for tt < kTM, j < R.
-__device__ __forceinline__ void dense_gelu(const float* __restrict__ in, float* __restrict__ out,
-                                           const float* __restrict__ W, const float* __restrict__ bias, float* wt,
-                                           int R) {
-  const int j = threadIdx.x;
-  float acc[kTM];
+// fp32 -> (hi, lo) bf16 with hi + lo equal to x to about 16 significant bits.
+__device__ __forceinline__ void split_bf(float x, float& hi, float& lo) {
+  hi = round_bf(x);
+  lo = x - hi;
+}
+
+template <int R>
+struct RouterShape {
+  static constexpr int KCH = R < 64 ? R : 64;       // k columns per staged weight chunk
+  static constexpr int WS = KCH + 8;                // bf16 row stride of a chunk: conflict-free ldmatrix
+  static constexpr int CHUNK = R * WS;              // bf16 elements of one (hi or lo) chunk
+  static constexpr int NTW = R / 32;                // 8-wide n-tiles per warp
+  static constexpr size_t SMEM = sizeof(float) * 2 * kTM * kZS + sizeof(__nv_bfloat16) * 2 * 2 * CHUNK;
+};
+
+// Stage columns [kc, kc+KCH) of the split weight (hi and lo, [R][R] bf16) into a padded chunk.
+template <int R>
+__device__ __forceinline__ void stage_chunk(__nv_bfloat16* dst, const __nv_bfloat16* __restrict__ whi,
+                                            const __nv_bfloat16* __restrict__ wlo, int kc) {
+  using Sh = RouterShape<R>;
+  constexpr int V = Sh::KCH / 8;   // 16-byte vectors per row
+  for (int i = threadIdx.x; i < 2 * R * V; i += kThreads) {
+    const int part = i / (R * V), rem = i % (R * V);
+    const int row = rem / V, c = rem % V;
+    const __nv_bfloat16* src = (part ? wlo : whi) + (size_t)row * R + kc + c * 8;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + part * Sh::CHUNK + row * Sh::WS + c * 8)),
+                 "l"(src)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// out[t][j] = gelu(sum_k in[t][k] W[j][k] + bias[j]) for the CTA's 32 tokens, on
+// tensor cores (mma.sync m16n8k16) with both operands split into bf16 hi + lo:
+// in.W ~= in_hi.W_hi + in_hi.W_lo + in_lo.W_hi, fp32 accumulation.
+template <int R>
+__device__ __forceinline__ void dense_gelu_tc(const float* in, float* out, const __nv_bfloat16* __restrict__ whi,
+                                              const __nv_bfloat16* __restrict__ wlo, const float* __restrict__ bias,
+                                              __nv_bfloat16* wring) {
+  using Sh = RouterShape<R>;
+  const int warp = warp_id(), lane = lane_id();
+  const int rg = warp & 1, ng = warp >> 1;
+  const int g = lane >> 2, t = lane & 3;
+  const int nbase = ng * (R / 4);
+  float acc[Sh::NTW][4];
 #pragma unroll
-  for (int t = 0; t < kTM; ++t) acc[t] = 0.f;
-  for (int kc = 0; kc < R; kc += kKC) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < R * kKC; i += blockDim.x) {
-      const int jj = i / kKC, k = i % kKC;
-      wt[k * (kRMax + 1) + jj] = __ldg(W + (size_t)jj * R + kc + k);
+  for (int j = 0; j < Sh::NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  constexpr int nch = R / Sh::KCH;
+  stage_chunk<R>(wring, whi, wlo, 0);
+  for (int c = 0; c < nch; ++c) {
+    if (c + 1 < nch) {
+      stage_chunk<R>(wring + ((c + 1) & 1) * 2 * Sh::CHUNK, whi, wlo, (c + 1) * Sh::KCH);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
-    if (j < R) {
-#pragma unroll 4
-      for (int k = 0; k < kKC; k += 4) {
-        const float w0 = wt[(k + 0) * (kRMax + 1) + j], w1 = wt[(k + 1) * (kRMax + 1) + j];
-        const float w2 = wt[(k + 2) * (kRMax + 1) + j], w3 = wt[(k + 3) * (kRMax + 1) + j];
+    const __nv_bfloat16* wh = wring + (c & 1) * 2 * Sh::CHUNK;
+    const __nv_bfloat16* wl = wh + Sh::CHUNK;
 #pragma unroll
-        for (int t = 0; t < kTM; ++t) {
-          const float4 x = *reinterpret_cast<const float4*>(in + t * kRMax + kc + k);
-          acc[t] = fmaf(x.x, w0, fmaf(x.y, w1, fmaf(x.z, w2, fmaf(x.w, w3, acc[t]))));
+    for (int ks = 0; ks < Sh::KCH / 16; ++ks) {
+      const int c0 = c * Sh::KCH + ks * 16 + 2 * t;
+      const int r0 = rg * 16 + g;
+      const float2 v00 = *reinterpret_cast<const float2*>(in + r0 * kZS + c0);
+      const float2 v10 = *reinterpret_cast<const float2*>(in + (r0 + 8) * kZS + c0);
+      const float2 v01 = *reinterpret_cast<const float2*>(in + r0 * kZS + c0 + 8);
+      const float2 v11 = *reinterpret_cast<const float2*>(in + (r0 + 8) * kZS + c0 + 8);
+      float h[8], l[8];
+      split_bf(v00.x, h[0], l[0]); split_bf(v00.y, h[1], l[1]);
+      split_bf(v10.x, h[2], l[2]); split_bf(v10.y, h[3], l[3]);
+      split_bf(v01.x, h[4], l[4]); split_bf(v01.y, h[5], l[5]);
+      split_bf(v11.x, h[6], l[6]); split_bf(v11.y, h[7], l[7]);
+      const uint32_t ah[4] = {pack_bf2(h[0], h[1]), pack_bf2(h[2], h[3]), pack_bf2(h[4], h[5]), pack_bf2(h[6], h[7])};
+      const uint32_t al[4] = {pack_bf2(l[0], l[1]), pack_bf2(l[2], l[3]), pack_bf2(l[4], l[5]), pack_bf2(l[6], l[7])};
+      const int m = lane >> 3;
+#pragma unroll
+      for (int j = 0; j < Sh::NTW; j += 2) {
+        if (j + 1 < Sh::NTW) {
+          const int row = nbase + j * 8 + (m >> 1) * 8 + (lane & 7);
+          const int col = ks * 16 + (m & 1) * 8;
+          uint32_t bh0, bh1, bh2, bh3, bl0, bl1, bl2, bl3;
+          ldsm_x4(smem_u32(wh + row * Sh::WS + col), bh0, bh1, bh2, bh3);
+          ldsm_x4(smem_u32(wl + row * Sh::WS + col), bl0, bl1, bl2, bl3);
+          mma16816(acc[j], ah, bh0, bh1);
+          mma16816(acc[j], ah, bl0, bl1);
+          mma16816(acc[j], al, bh0, bh1);
+          mma16816(acc[j + 1], ah, bh2, bh3);
+          mma16816(acc[j + 1], ah, bl2, bl3);
+          mma16816(acc[j + 1], al, bh2, bh3);
+        } else {   // a single n-tile left: b fragments read directly (two bf16 per 32-bit word)
+          const int row = nbase + j * 8 + g;
+          const int col = ks * 16 + 2 * t;
+          const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(wh + row * Sh::WS + col);
+          const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(wh + row * Sh::WS + col + 8);
+          const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(wl + row * Sh::WS + col);
+          const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(wl + row * Sh::WS + col + 8);
+          mma16816(acc[j], ah, bh0, bh1);
+          mma16816(acc[j], ah, bl0, bl1);
+          mma16816(acc[j], al, bh0, bh1);
         }
       }
     }
+    __syncthreads();
   }
-  if (j < R) {
-    const float bj = __ldg(bias + j);
+  const int r0 = rg * 16 + g;
 #pragma unroll
-    for (int t = 0; t < kTM; ++t) out[t * kRMax + j] = gelu_exact(acc[t] + bj);
+  for (int j = 0; j < Sh::NTW; ++j) {
+    const int n = nbase + j * 8 + 2 * t;
+    const float b0 = __ldg(bias + n), b1 = __ldg(bias + n + 1);
+    *reinterpret_cast<float2*>(out + r0 * kZS + n) = make_float2(gelu_exact(acc[j][0] + b0), gelu_exact(acc[j][1] + b1));
+    *reinterpret_cast<float2*>(out + (r0 + 8) * kZS + n) =
+        make_float2(gelu_exact(acc[j][2] + b0), gelu_exact(acc[j][3] + b1));
   }
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(256) router_kernel(const RouterParams p) {
+// fc1 / fc2 weights (fp32 [R][R]) -> bf16 hi and lo parts: wsplit = [layer][hi|lo][R][R].
+__global__ void router_split_kernel(const float* __restrict__ fc1, const float* __restrict__ fc2,
+                                    __nv_bfloat16* __restrict__ wsplit, int R) {
+  const int n = R * R;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < 2 * n; i += gridDim.x * blockDim.x) {
+    const int layer = i / n, e = i % n;
+    const float x = (layer ? fc2 : fc1)[e];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    wsplit[(size_t)layer * 2 * n + e] = hi;
+    wsplit[(size_t)layer * 2 * n + n + e] = __float2bfloat16_rn(x - __bfloat162float(hi));
+  }
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams p) {
+  using Sh = RouterShape<R>;
   extern __shared__ __align__(16) float sm[];
-  float* z = sm;                         // [kTM][kRMax]
-  float* g = z + kTM * kRMax;            // [kTM][kRMax]
-  float* wt = g + kTM * kRMax;           // [kKC][kRMax + 1]
-  float* lg = wt + kKC * (kRMax + 1);    // [kTM][E+1]
-  const int R = p.R, E1 = p.E + 1;
+  float* z = sm;                                                              // [kTM][kZS]
+  float* g = z + kTM * kZS;                                                   // [kTM][kZS]
+  __nv_bfloat16* wring = reinterpret_cast<__nv_bfloat16*>(g + kTM * kZS);     // [2 stages][hi|lo][R][WS]
+  const int E1 = p.E + 1;
   const int t0 = blockIdx.x * kTM;
   const int warp = warp_id(), lane = lane_id();
 
-  for (int i = threadIdx.x; i < kTM * R; i += blockDim.x) {
-    const int tt = i / R, k = i % R;
-    z[tt * kRMax + k] = (t0 + tt < p.M) ? p.r[(size_t)(t0 + tt) * R + k] : 0.f;
+  // router state r = down_proj partial sums (fixed order) + bias (+ previous state * scale);
+  // float4 per thread, every load of a group issued before the adds.
+  {
+    constexpr int R4 = R / 4;
+#pragma unroll 2
+    for (int i = threadIdx.x; i < kTM * R4; i += kThreads) {
+      const int tt = i / R4, k4 = i % R4, t = t0 + tt;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < p.M) {
+        const float4* pp = reinterpret_cast<const float4*>(p.part) + (size_t)t * R4 + k4;
+        const size_t slab = (size_t)p.M * R4;
+        const int ns = p.n_splits;
+        float4 a[8];
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp) a[sp] = (sp < ns) ? pp[sp * slab] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 8; sp < ns; ++sp) {   // more than 8 slabs (small M): folded in order
+          const float4 x = pp[sp * slab];
+          a[7].x += x.x; a[7].y += x.y; a[7].z += x.z; a[7].w += x.w;
+        }
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp) { v.x += a[sp].x; v.y += a[sp].y; v.z += a[sp].z; v.w += a[sp].w; }
+        const float4 bb = __ldg(reinterpret_cast<const float4*>(p.bias) + k4);
+        v.x += bb.x; v.y += bb.y; v.z += bb.z; v.w += bb.w;
+        if (p.prev) {
+          const float4 pv = reinterpret_cast<const float4*>(p.prev)[(size_t)t * R4 + k4];
+          const float4 sc = __ldg(reinterpret_cast<const float4*>(p.prev_scale) + k4);
+          v.x = fmaf(pv.x, sc.x, v.x); v.y = fmaf(pv.y, sc.y, v.y);
+          v.z = fmaf(pv.z, sc.z, v.z); v.w = fmaf(pv.w, sc.w, v.w);
+        }
+        reinterpret_cast<float4*>(p.r_out)[(size_t)t * R4 + k4] = v;
+      }
+      *reinterpret_cast<float4*>(z + tt * kZS + k4 * 4) = v;
+    }
   }
   __syncthreads();
-  for (int tt = warp; tt < kTM; tt += 8) {   // router_mlp.norm (RMSNorm over R)
+  for (int tt = warp; tt < kTM; tt += kThreads / 32) {   // router_mlp.norm (RMSNorm over R)
     float ss = 0.f;
-    for (int k = lane; k < R; k += 32) ss += z[tt * kRMax + k] * z[tt * kRMax + k];
+    for (int k = lane; k < R; k += 32) ss += z[tt * kZS + k] * z[tt * kZS + k];
     ss = warp_sum(ss);
     const float inv = rsqrtf(ss / (float)R + p.eps);
-    for (int k = lane; k < R; k += 32) z[tt * kRMax + k] = __ldg(p.norm_w + k) * (z[tt * kRMax + k] * inv);
-  }
-  dense_gelu(z, g, p.fc1_w, p.fc1_b, wt, R);
-  dense_gelu(g, z, p.fc2_w, p.fc2_b, wt, R);
-  for (int i = threadIdx.x; i < kTM * E1; i += blockDim.x) {   // out_proj (no bias)
-    const int tt = i / E1, c = i % E1;
-    const float* wr = p.out_w + (size_t)c * R;
-    float a = 0.f;
-    for (int k = 0; k < R; k += 4) {
-      const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + k));
-      const float4 x4 = *reinterpret_cast<const float4*>(z + tt * kRMax + k);
-      a = fmaf(x4.x, w4.x, fmaf(x4.y, w4.y, fmaf(x4.z, w4.z, fmaf(x4.w, w4.w, a))));
-    }
-    lg[tt * E1 + c] = a;
+    for (int k = lane; k < R; k += 32) z[tt * kZS + k] = __ldg(p.norm_w + k) * (z[tt * kZS + k] * inv);
   }
   __syncthreads();
-  for (int tt = warp; tt < kTM; tt += 8) {   // softmax, balancing, top-1, skip
+  const size_t n = (size_t)R * R;
+  dense_gelu_tc<R>(z, g, p.wsplit, p.wsplit + n, p.fc1_b, wring);
+  dense_gelu_tc<R>(g, z, p.wsplit + 2 * n, p.wsplit + 3 * n, p.fc2_b, wring);
+  // out_proj (no bias, fp32 on CUDA cores) and the choice, one warp per token
+  for (int tt = warp; tt < kTM; tt += kThreads / 32) {
     const int t = t0 + tt;
     if (t >= p.M) continue;
-    float l[3], s[3], e[3];
-    float mx = -INFINITY;
+    float zr[R / 32];
 #pragma unroll
-    for (int u = 0; u < 3; ++u) {
-      const int c = lane + 32 * u;
-      l[u] = c < E1 ? lg[tt * E1 + c] : -INFINITY;
-      mx = fmaxf(mx, l[u]);
+    for (int j = 0; j < R / 32; ++j) zr[j] = z[tt * kZS + lane + 32 * j];
+    float l[3] = {-INFINITY, -INFINITY, -INFINITY};
+    for (int c = 0; c < E1; ++c) {
+      const float* wr = p.out_w + (size_t)c * R;
+      float a = 0.f;
+#pragma unroll
+      for (int j = 0; j < R / 32; ++j) a = fmaf(zr[j], __ldg(wr + lane + 32 * j), a);
+      a = warp_sum(a);
+      if ((c & 31) == lane) l[c >> 5] = a;
     }
+    float mx = fmaxf(fmaxf(l[0], l[1]), l[2]);
     mx = warp_max(mx);
-    float sum = 0.f;
+    float e[3], sum = 0.f;
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
       e[u] = (lane + 32 * u < E1) ? expf(l[u] - mx) : 0.f;
@@ -123,9 +247,9 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterParams p) {
       const int c = lane + 32 * u;
       if (c < E1) {
         const float pc = e[u] / sum;
-        s[u] = pc + __ldg(p.balancing + c);
-        if (s[u] > best) {
-          best = s[u];
+        const float sc = pc + __ldg(p.balancing + c);
+        if (sc > best) {
+          best = sc;
           bc = c;
           bestp = pc;
         }
@@ -154,6 +278,15 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterParams p) {
       if (p.w_tap) p.w_tap[t] = w;
     }
   }
+}
+
+template <int R>
+int launch_router_r(const RouterParams& p, cudaStream_t st) {
+  using Sh = RouterShape<R>;
+  router_split_kernel<<<64, 256, 0, st>>>(p.fc1_w, p.fc2_w, p.wsplit, R);
+  cudaFuncSetAttribute(router_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::SMEM);
+  router_kernel<R><<<(p.M + kTM - 1) / kTM, kThreads, Sh::SMEM, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 
 // Stable counting sort by class, one CTA of 32 warps; warp w owns a
@@ -252,9 +385,22 @@ __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
   const int H = p.H;
   const int c = p.cls[t];
   if (c >= 0 && c < p.E) {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * H);
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)p.pos[t] * H);
-    for (int i = lane; i < H / 8; i += 32) dst[i] = src[i];
+    const uint4* __restrict__ src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * H);
+    uint4* __restrict__ dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)p.pos[t] * H);
+    const int n = H / 8;   // 16-byte vectors per row
+    for (int base = 0; base < n; base += 32 * 4) {   // four loads in flight per lane before the stores
+      uint4 v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = base + lane + 32 * k;
+        if (i < n) v[k] = src[i];
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = base + lane + 32 * k;
+        if (i < n) dst[i] = v[k];
+      }
+    }
   } else {
     // skip: no expert runs; mlp_output = bf16(hb * hs), out = mlp_output + (h + rb) * rs
     float4* s4 = reinterpret_cast<float4*>(p.stream + (size_t)t * H);
@@ -286,15 +432,14 @@ __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
 
 int launch_router(const RouterParams& p, cudaStream_t st) {
   if (p.M <= 0) return ZAYA_OK;
-  if (p.R > kRMax || p.R % 32 || p.E + 1 > 96) return ZAYA_ERR_UNSUPPORTED;
-  const size_t smem = sizeof(float) * (2 * kTM * kRMax + kKC * (kRMax + 1) + kTM * (p.E + 1));
-  static bool set = false;
-  if (!set) {
-    cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-    set = true;
+  if (p.E + 1 > 96 || p.n_splits < 1 || !p.wsplit) return ZAYA_ERR_UNSUPPORTED;
+  switch (p.R) {
+    case 32: return launch_router_r<32>(p, st);
+    case 64: return launch_router_r<64>(p, st);
+    case 128: return launch_router_r<128>(p, st);
+    case 256: return launch_router_r<256>(p, st);
+    default: return ZAYA_ERR_UNSUPPORTED;
   }
-  router_kernel<<<(p.M + kTM - 1) / kTM, 256, smem, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 
 int launch_permute(const int* cls, int M, int E, int* group_off, int* mt_start, int* pos, int* perm, int* status,

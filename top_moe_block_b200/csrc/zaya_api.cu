@@ -145,7 +145,8 @@ int check_weights(const zaya_block_weights* w) {
 }
 
 struct Ws {
-  size_t status, a_in, qkv, q, premix, m_in, logits, cls, w, pos, perm, group_off, mt_start, xperm, act, part, total;
+  size_t status, a_in, qkv, q, premix, m_in, logits, cls, w, pos, perm, group_off, mt_start, xperm, act, part, rpart,
+      wsplit, total;
 };
 
 Ws plan(const zaya_config& c, int mode, int B, int S) {
@@ -170,6 +171,8 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.xperm = o; o += up(M * d.H * 2);
   w.act = o; o += up(M * d.I * 2);
   w.part = o; o += up(mode == ZAYA_DECODE ? decode_attn_ws_bytes(B, d.nq, d.d, c.window) : 0);
+  w.rpart = o; o += up((size_t)router_down_splits((int)M, d.H) * M * d.R * 4);
+  w.wsplit = o; o += up((size_t)4 * d.R * d.R * 2);
   w.total = o;
   return w;
 }
@@ -179,17 +182,26 @@ inline T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
 }
 
-// Largest tile width whose tile count still fills the GPU, else the smallest.
-int pick_bn(int M, int N, const int* cands, int n, int sms) {
-  int last = 0;
+// Tile width with the least per-SM work: waves(BN) x BN, where waves is the
+// number of rounds of tiles over the SMs; ties go to the wider tile (less
+// operand traffic per FLOP).  m_tiles is the number of 128-row tiles.
+int pick_bn_tiles(long m_tiles, int N, const int* cands, int n, int sms) {
+  int best = 0;
+  long best_cost = 0;
   for (int i = 0; i < n; ++i) {
     const int bn = cands[i];
     if (N % bn) continue;
-    last = bn;
-    const long tiles = (long)((M + 127) / 128) * (N / bn);
-    if (tiles >= sms) return bn;
+    const long tiles = m_tiles * (N / bn);
+    const long cost = ((tiles + sms - 1) / sms) * bn;
+    if (!best || cost < best_cost) {
+      best = bn;
+      best_cost = cost;
+    }
   }
-  return last;
+  return best;
+}
+int pick_bn(int M, int N, const int* cands, int n, int sms) {
+  return pick_bn_tiles((M + 127) / 128, N, cands, n, sms);
 }
 
 #define ZAYA_TRY(x)            \
@@ -218,28 +230,30 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
   void* m_in = at<void>(ws, L.m_in);
   ZAYA_STAGE("rmsnorm_mlp", 1, launch_rmsnorm(hidden, 1, 0, w->ln2_w, m_in, taps ? taps->mlp_norm_output : nullptr,
                                               M, d.H, c.rms_eps, nullptr, 0, st));
-  {  // router down_proj (+ carried state)
-    GemmParams p{};
-    p.M = M; p.N = d.R; p.K = d.H; p.status = status;
-    p.out = rout; p.ldo = d.R; p.bias = w->router_down_b;
-    p.prev = (block_idx > 0) ? rin : nullptr;
-    p.prev_scale = w->router_state_scale;
-    const int c3[] = {128, 64, 32};
-    const int bn = pick_bn(M, d.R, c3, 3, sms);
-    ZAYA_STAGE("router_down", 1, launch_gemm(EPI_ROUTER_DOWN, bn, m_in, M, w->router_down_w, d.R, p, sms, st));
-  }
   int* cls = at<int>(ws, L.cls);
   float* wgt = at<float>(ws, L.w);
-  {
+  float* rpart = at<float>(ws, L.rpart);
+  const int ks = router_down_splits(M, d.H);
+  {  // router down_proj as fp32 partial sums over K slabs
+    GemmParams p{};
+    p.M = M; p.N = d.R; p.K = d.H; p.k_splits = ks; p.status = status;
+    p.out = rpart; p.ldo = d.R;
+    const int bn = (d.R % 256 == 0) ? 256 : (d.R % 128 == 0) ? 128 : (d.R % 64 == 0) ? 64 : 32;
+    ZAYA_STAGE("router_down", 1, launch_gemm(EPI_STORE_F32, bn, m_in, M, w->router_down_w, d.R, p, sms, st));
+  }
+  {  // router state (slab sum + bias + carried state), router MLP, scoring, top-1
     RouterParams p{};
-    p.r = rout; p.norm_w = w->router_norm_w;
+    p.part = rpart; p.n_splits = ks; p.bias = w->router_down_b;
+    p.prev = (block_idx > 0) ? rin : nullptr; p.prev_scale = w->router_state_scale; p.r_out = rout;
+    p.norm_w = w->router_norm_w;
     p.fc1_w = w->fc1_w; p.fc1_b = w->fc1_b; p.fc2_w = w->fc2_w; p.fc2_b = w->fc2_b;
+    p.wsplit = at<__nv_bfloat16>(ws, L.wsplit);
     p.out_w = w->out_w; p.balancing = w->balancing; p.mask = attn_mask;
     p.logits = (taps && taps->router_logits) ? taps->router_logits : at<float>(ws, L.logits);
     p.cls = cls; p.idx = taps ? taps->expert_indices : nullptr; p.w = wgt;
     p.w_tap = taps ? taps->expert_weights : nullptr;
     p.M = M; p.R = d.R; p.E = d.E; p.eps = c.rms_eps;
-    ZAYA_STAGE("router_mlp", 1, launch_router(p, st));
+    ZAYA_STAGE("router_mlp", 2, launch_router(p, st));
   }
   int* group_off = at<int>(ws, L.group_off);
   int* mt_start = at<int>(ws, L.mt_start);
@@ -269,7 +283,8 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.n_groups = d.E; p.b_rows_per_group = d.H; p.status = status;
     p.stream = hidden; p.merge = w->merge_m; p.perm = perm; p.row_w = wgt;
     p.tap_bf16 = taps ? taps->mlp_output : nullptr;
-    const int bn = (M >= 2048 && d.H % 256 == 0) ? 256 : 128;
+    const int c2[] = {256, 128};
+    const int bn = pick_bn_tiles((M + 127) / 128 + d.E / 2, d.H, c2, 2, sms);
     ZAYA_STAGE("experts_down_merge", 1, launch_gemm(EPI_MERGE_MLP, bn, act, M, w->w_down, d.E * d.H, p, sms, st));
   }
   return ZAYA_OK;
@@ -328,7 +343,7 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     p.out = at<void>(ws, L.premix);
     p.B = B; p.S = S; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = c.window;
     p.scale = d.scale;
-    ZAYA_STAGE("attention", 1, launch_attn_prefill(p, st));
+    ZAYA_STAGE("attention", 1, launch_attn_prefill_tc(p, status, st));
   }
   return block_tail(c, d, w, block_idx, M, hidden, rin, rout, taps, ws, L, nullptr, mask, sms, st);
 }
@@ -530,7 +545,7 @@ int zaya_profile_read(int32_t max_stages, const char** names, double* total_ms, 
       acc = &g_prof_acc.back();
     }
     acc->ms += ms;
-    acc->launches += r.kernels;
+    acc->launches += 1;   // stage calls (a stage may launch more than one kernel)
     g_prof_pool.push_back(r.a);
     g_prof_pool.push_back(r.b);
   }
