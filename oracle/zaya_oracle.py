@@ -383,6 +383,46 @@ def block_prefill(cfg, W, x, attn_mask=None, router_state_in=None, block_idx=Non
     return out
 
 
+def block_prefill_rows(cfg, W, x, r0, r1, router_state_in=None, block_idx=None, force_cls=None):
+    """The block outputs of rows [r0, r1) of one unpadded sequence, computed
+    from only the tokens those rows depend on: keys back to r0 - window + 1
+    and two more tokens of conv history.  Positions are the rows' own, so the
+    result is the full prefill's at those rows (up to summation order).
+    x [S,H]; router_state_in [S,R] or None; force_cls [r1-r0] or None.
+    Returns taps of the rows (no decode state)."""
+    x = as64(x)
+    bidx = cfg.block_idx if block_idx is None else block_idx
+    d, nq = cfg.head_dim, cfg.n_q
+    lo = max(0, r0 - cfg.window + 1)     # first key any of the rows sees
+    t0 = max(0, lo - 3)                  # plus the conv / delayed-value history
+    seg = x[t0:r1]
+    a_in = block_norm(seg, as64(W["ln1_w"]), cfg.rms_eps)
+    proj = round_bf16(a_in @ as64(W["w_qkv"]).T)
+    q_pre, k_pre, vc, vd = _split_proj(cfg, proj)
+    pos = np.arange(t0, r1)
+    q, k, u = _qk(cfg, W, q_pre, k_pre, np.zeros((2, cfg.qk_channels)), pos)
+    vd_prev = np.concatenate([np.zeros((1, cfg.v_half)), vd[:-1]], axis=0)
+    if not cfg.v_delayed:
+        vd_prev = vd
+    v = round_bf16(_values(cfg, vc, vd_prev))
+    k = round_bf16(k)
+    # rows whose conv / delayed-value history starts before t0 were computed with zeros
+    # there: they are keys only if >= lo, and lo >= t0 + 2 whenever t0 > 0
+    kl = lo - t0
+    qi = np.arange(r0, r1) - t0
+    o = attention(q[qi], k[kl:], v[kl:], np.arange(r0, r1), np.arange(lo, r1), np.ones(r1 - lo, dtype=bool),
+                  cfg.window, cfg.scale)
+    premix = o.reshape(r1 - r0, nq * d)
+    attn_o = premix @ as64(W["w_o"]).T
+    attn_out, h = merge(attn_o, x[r0:r1], as64(W["merge_a"]))
+    rin = None if router_state_in is None else as64(router_state_in)[r0:r1]
+    mt = _mlp_half(cfg, W, h, rin, bidx, np.ones(r1 - r0, dtype=bool), force_cls)
+    out = dict(attention_norm_output=a_in[r0 - t0:], attention_premix=premix, attention_output=attn_out,
+               layer_mid=h, layer_input=x[r0:r1], attention_keys=k[r0 - t0:], attention_values=v[r0 - t0:])
+    out.update(mt)
+    return out
+
+
 def block_decode(cfg, W, x, state, router_state_in=None, block_idx=None, force_cls=None):
     """One new token per sequence through a block with a cache.
 

@@ -1,0 +1,207 @@
+"""GPU parity of the whole stack (embedding -> blocks -> final norm -> tied
+lm_head) through zaya_stack_forward, against the CPU oracle.
+
+The stack's logits are compared with the oracle's head applied to the final
+stream obtained by running the same blocks one at a time through the C ABI
+(each block teacher-forced against the oracle on its own GPU input).  Long
+workloads are checked on sampled blocks, sequences and rows."""
+import numpy as np
+import pytest
+import torch
+
+from synthetic import (gen_block_weights, gen_decode_state, gen_prefill_inputs, gen_stack_weights_extra,
+                       gen_token_ids, get_config)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from top_moe_block_b200 import build
+    build.build()
+
+
+def _embed_stream(cfg, embed, ids):
+    """The stream entering block 0, computed with the same single fp32
+    operations the embedding kernel performs ((e + shift) * mult)."""
+    e = embed[ids.long()].float()
+    return (e + cfg.emb_shift) * torch.tensor(cfg.emb_mult, dtype=torch.float32)
+
+
+def _check_logits(gpu_logits, ref_logits):
+    from tests import harness as Hn
+    g = gpu_logits.float().cpu().numpy()
+    assert Hn.rel_max(g, ref_logits) <= Hn.TOL_REL_MAX and Hn.cosine(g, ref_logits) >= Hn.TOL_COS, (
+        Hn.rel_max(g, ref_logits), Hn.cosine(g, ref_logits))
+
+
+def test_tiny_stack_prefill():
+    import top_moe_block_b200 as ZB
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config("tiny").with_(n_blocks=3, block_idx=0, batch=2, seq=50)
+    B, S, V = cfg.batch, cfg.seq, cfg.vocab
+    blocks = [gen_block_weights(cfg, block=i) for i in range(cfg.n_blocks)]
+    bd = [Hn.dev_weights(w) for w in blocks]
+    extra = gen_stack_weights_extra(cfg)
+    ed = Hn.dev_weights(extra)
+    ids = gen_token_ids(cfg).cuda()
+    states = [Hn.new_state(cfg, B, S) for _ in blocks]
+    c = ZB.make_config(cfg)
+    logits = torch.empty(B, S, V, dtype=torch.bfloat16, device="cuda")
+    ws = Hn.workspace(ZB.zaya_stack_workspace_size(c, ZB.ZAYA_PREFILL, B, S))
+    ZB.zaya_stack_forward(c, [ZB.make_weights(w) for w in bd], ed["embed"], ed["final_norm_w"], ZB.ZAYA_PREFILL,
+                          B, S, ids, None, [ZB.make_state(s) for s in states], logits, 0, ws)
+    assert ZB.zaya_device_status(ws) == 0
+    # the same blocks one at a time, each teacher-forced against the oracle
+    x = _embed_stream(cfg, ed["embed"], ids)
+    te, x_or = Z.embed(cfg, extra["embed"], ids.cpu().numpy())
+    np.testing.assert_array_equal(x.cpu().numpy(), x_or)
+    r = None
+    for i, W in enumerate(blocks):
+        out = Hn.gpu_prefill(cfg, bd[i], x, None, r, block_idx=i)
+        inp = {"x": x.cpu(), "attn_mask": None, "router_state_in": None if r is None else r.cpu()}
+        res = Hn.check_prefill_block(cfg, W, inp, out, block_idx=i, verbose=False)
+        Hn.assert_block_ok(res)
+        x, r = out["layer_output"], out["router_state"]
+    _, ref = Z.lm_head(cfg, extra["embed"], extra["final_norm_w"], Z.as64(x))
+    _check_logits(logits, ref)
+    # the stack's own state equals the composed run's
+    np.testing.assert_array_equal(states[-1]["cache_len"].cpu().numpy(), S)
+
+
+def test_tiny_stack_decode_after_prefill():
+    """prefill(S) through the stack, then one decode step through the stack;
+    the decode logits against the oracle's decode of the GPU's states."""
+    import top_moe_block_b200 as ZB
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config("tiny").with_(n_blocks=2, block_idx=0, batch=3, seq=40)
+    B, S, V = cfg.batch, cfg.seq, cfg.vocab
+    blocks = [gen_block_weights(cfg, block=i) for i in range(cfg.n_blocks)]
+    bd = [Hn.dev_weights(w) for w in blocks]
+    extra = gen_stack_weights_extra(cfg)
+    ed = Hn.dev_weights(extra)
+    ids = gen_token_ids(cfg.with_(seq=S + 1)).cuda()
+    states = [Hn.new_state(cfg, B, S + 4) for _ in blocks]
+    c = ZB.make_config(cfg)
+    ws = Hn.workspace(ZB.zaya_stack_workspace_size(c, ZB.ZAYA_PREFILL, B, S))
+    lp = torch.empty(B, V, dtype=torch.bfloat16, device="cuda")
+    ZB.zaya_stack_forward(c, [ZB.make_weights(w) for w in bd], ed["embed"], ed["final_norm_w"], ZB.ZAYA_PREFILL,
+                          B, S, ids[:, :S].contiguous(), None, [ZB.make_state(s) for s in states], lp, 1, ws)
+    host_states = [{k: v.cpu().clone() for k, v in s.items()} for s in states]
+    wsd = Hn.workspace(ZB.zaya_stack_workspace_size(c, ZB.ZAYA_DECODE, B, 1))
+    ld = torch.empty(B, V, dtype=torch.bfloat16, device="cuda")
+    ZB.zaya_stack_forward(c, [ZB.make_weights(w) for w in bd], ed["embed"], ed["final_norm_w"], ZB.ZAYA_DECODE,
+                          B, 1, ids[:, S].contiguous(), None, [ZB.make_state(s) for s in states], ld, 0, wsd)
+    assert ZB.zaya_device_status(wsd) == 0
+    # oracle decode, block by block, on the GPU's prefill states and the GPU's own
+    # block inputs (recomputed one block at a time through the C ABI)
+    dec_states = [{k: v.clone() for k, v in s.items()} for s in host_states]
+    x = _embed_stream(cfg, ed["embed"], ids[:, S])
+    r = None
+    for i, W in enumerate(blocks):
+        st = {k: v.cuda() for k, v in dec_states[i].items()}
+        out = Hn.gpu_decode(cfg, bd[i], x, st, r, block_idx=i)
+        g_cls = Hn.gpu_classes(cfg, out)
+        ref = Z.block_decode(cfg, W, x.cpu(), dec_states[i], None if r is None else r.cpu(), block_idx=i,
+                             force_cls=g_cls)
+        lo = Hn.report("layer_output", out["layer_output"].numpy(), ref["layer_output"])
+        assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, (i, lo)
+        x, r = out["layer_output"].cuda(), out["router_state"].cuda()
+    _, ref_logits = Z.lm_head(cfg, extra["embed"], extra["final_norm_w"], Z.as64(x))
+    _check_logits(ld, ref_logits)
+    assert int(states[0]["cache_len"][0]) == S + 1
+
+
+def test_decode_stack_b64_40_blocks():
+    """The decode workload: B64, 40 full-width blocks, 8192 cached tokens per
+    sequence, window 4096, vocab 262144.  Blocks 0, 1 and 39 are checked
+    against the oracle on 4 of the 64 sequences; the logits on those rows."""
+    import top_moe_block_b200 as ZB
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config("decode_stack_b64")
+    B, V, L = cfg.batch, cfg.vocab, cfg.cache_prior
+    cap = L + 8
+    dev = "cuda"
+    blocks_d = [gen_block_weights(cfg, block=i, device=dev) for i in range(cfg.n_blocks)]
+    extra_d = gen_stack_weights_extra(cfg, device=dev)
+    ids = gen_token_ids(cfg)[:, 0].contiguous().to(dev)
+    states = [gen_decode_state(cfg, i, cap, device=dev) for i in range(cfg.n_blocks)]
+    pre = [{k: v.clone() for k, v in s.items()} for s in states]
+    c = ZB.make_config(cfg)
+    ws = Hn.workspace(ZB.zaya_stack_workspace_size(c, ZB.ZAYA_DECODE, B, 1))
+    logits = torch.empty(B, V, dtype=torch.bfloat16, device=dev)
+    ZB.zaya_stack_forward(c, [ZB.make_weights(w) for w in blocks_d], extra_d["embed"], extra_d["final_norm_w"],
+                          ZB.ZAYA_DECODE, B, 1, ids, None, [ZB.make_state(s) for s in states], logits, 0, ws)
+    assert ZB.zaya_device_status(ws) == 0
+    assert (states[0]["cache_len"] == L + 1).all()
+    rows = [0, 17, 40, 63]
+    x = _embed_stream(cfg, extra_d["embed"], ids)
+    r = None
+    for i in range(cfg.n_blocks):
+        st = pre[i]
+        if i in (0, 1, cfg.n_blocks - 1):
+            host = {k: v[rows].cpu() for k, v in st.items()}
+        out = Hn.gpu_decode(cfg, blocks_d[i], x, st, r, block_idx=i)
+        if i in (0, 1, cfg.n_blocks - 1):
+            W = {k: v.cpu() for k, v in blocks_d[i].items()}
+            g_cls = Hn.gpu_classes(cfg, out)[rows]
+            ref = Z.block_decode(cfg, W, x[rows].cpu(), host, None if r is None else r[rows].cpu(), block_idx=i,
+                                 force_cls=g_cls)
+            lo = Hn.report("layer_output", out["layer_output"][rows].numpy(), ref["layer_output"])
+            assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, (i, lo)
+            t_cls, gap, _, _ = Hn.router_teacher_forced(cfg, W, out["mlp_norm_output"][rows],
+                                                        None if r is None else r[rows].cpu(), i)
+            assert ((t_cls == g_cls) | (gap < Hn.NEAR_TIE)).all(), i
+        x, r = out["layer_output"].to(dev), out["router_state"].to(dev)
+    emb = extra_d["embed"].cpu()
+    _, ref_logits = Z.lm_head(cfg, emb, extra_d["final_norm_w"].cpu(), Z.as64(x[rows]))
+    _check_logits(logits[rows], ref_logits)
+
+
+def test_prefill_stack_32k_sampled():
+    """The long-prefill workload: B1 x S32768 through 40 full-width blocks,
+    window 4096, vocab 262144, logits at every position.  Blocks 0 and 39 are
+    checked against the oracle on sampled rows (the last 48 positions and the
+    window edge 4094..4098), the logits on sampled positions."""
+    import top_moe_block_b200 as ZB
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config("prefill_stack_32k")
+    B, S, V = cfg.batch, cfg.seq, cfg.vocab
+    dev = "cuda"
+    blocks_d = [gen_block_weights(cfg, block=i, device=dev) for i in range(cfg.n_blocks)]
+    extra_d = gen_stack_weights_extra(cfg, device=dev)
+    ids = gen_token_ids(cfg).to(dev)
+    states = [Hn.new_state(cfg, B, S) for _ in range(cfg.n_blocks)]
+    c = ZB.make_config(cfg)
+    ws = Hn.workspace(ZB.zaya_stack_workspace_size(c, ZB.ZAYA_PREFILL, B, S), poison=False)
+    logits = torch.empty(B, S, V, dtype=torch.bfloat16, device=dev)
+    ZB.zaya_stack_forward(c, [ZB.make_weights(w) for w in blocks_d], extra_d["embed"], extra_d["final_norm_w"],
+                          ZB.ZAYA_PREFILL, B, S, ids, None, [ZB.make_state(s) for s in states], logits, 0, ws)
+    assert ZB.zaya_device_status(ws) == 0
+    del states
+    ranges = [(S - 48, S), (4094, 4099)]
+    x = _embed_stream(cfg, extra_d["embed"], ids)
+    r = None
+    for i in range(cfg.n_blocks):
+        out = Hn.gpu_prefill(cfg, blocks_d[i], x, None, r, block_idx=i, taps=(i in (0, cfg.n_blocks - 1)))
+        if i in (0, cfg.n_blocks - 1):
+            W = {k: v.cpu() for k, v in blocks_d[i].items()}
+            g_all = Hn.gpu_classes(cfg, out)
+            for r0, r1 in ranges:
+                ref = Z.block_prefill_rows(cfg, W, x[0].cpu(), r0, r1, None if r is None else r[0].cpu(),
+                                           block_idx=i, force_cls=g_all[r0:r1])
+                lo = Hn.report("layer_output", out["layer_output"][0, r0:r1].numpy(), ref["layer_output"])
+                assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, (i, r0, lo)
+        x = out["layer_output"].to(dev)
+        r = out["router_state"].to(dev)
+        del out
+    rows = [0, 4095, 4096, S - 1]
+    emb = extra_d["embed"].cpu()
+    _, ref_logits = Z.lm_head(cfg, emb, extra_d["final_norm_w"].cpu(), Z.as64(x[0, rows]))
+    _check_logits(logits[0, rows], ref_logits)

@@ -415,3 +415,20 @@ def test_stack_with_silent_sublayers():
         x = Z.round_f32((x + a[2]) * a[3])
         x = Z.round_f32((x + m[2]) * m[3])
     np.testing.assert_array_equal(out["final_stream"], x)
+
+
+def test_prefill_rows_equals_full_prefill():
+    """The windowed evaluation of a row range (used for long sequences)
+    equals the full prefill at those rows, including ranges whose window and
+    conv history start mid-sequence."""
+    cfg = get_config("tiny").with_(seq=120, window=20)
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    full = Z.block_prefill(cfg, W, inp["x"], None, inp["router_state_in"])
+    for r0, r1 in ((0, 5), (30, 47), (100, 120), (21, 22)):
+        part = Z.block_prefill_rows(cfg, W, inp["x"][0], r0, r1, inp["router_state_in"][0])
+        for key in ("layer_output", "router_state", "attention_premix", "mlp_output"):
+            np.testing.assert_allclose(part[key], full[key][0, r0:r1], rtol=1e-9, atol=1e-9, err_msg=key)
+        np.testing.assert_array_equal(part["expert_cls"], full["expert_cls"][0, r0:r1])
+        np.testing.assert_allclose(part["attention_keys"].transpose(1, 0, 2),
+                                   full["attention_keys"][0][:, r0:r1], rtol=1e-9, atol=1e-9)

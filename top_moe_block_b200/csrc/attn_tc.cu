@@ -197,7 +197,8 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(&s_full[buf], (j >> 1) & 1, status)) {
+      // every wait that guards a .sync.aligned TMEM access is made warp-uniform
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (j >> 1) & 1, status))) {
         ok = false;
         break;
       }
@@ -227,16 +228,20 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[buf]);   // S is in registers: the buffer may be refilled
       const float m_new = fmaxf(m_used, tmax);
-      if (m_new > m_used + kRescaleLog2) {   // also the first finite max
-        if (j > 0 && m_used != -INFINITY) {
+      // Move the running max when it grew by more than 2^8 -- for the whole warp
+      // at once, since the O rescale below is a warp-wide TMEM access.  Each
+      // lane scales its own row by exp2(m_used - m_new) <= 1, so the result is
+      // exact whichever lanes asked.
+      if (__any_sync(0xffffffffu, m_new > m_used + kRescaleLog2)) {
+        const bool finite_new = m_new != -INFINITY;
+        const float f = (m_used == -INFINITY || !finite_new) ? 1.f : exp2f(m_used - m_new);
+        if (j > 0 && __any_sync(0xffffffffu, m_used != -INFINITY)) {
           // O holds tiles < j: wait for PV(j-1), then scale it in TMEM
-          if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const float f = exp2f(m_used - m_new);
-          l *= f;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -248,7 +253,8 @@ __global__ void __launch_bounds__(192, 1)
           }
           tmem_st_wait();
         }
-        m_used = m_new;
+        l *= f;
+        if (finite_new) m_used = m_new;
       }
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
       uint32_t pk[32];
@@ -261,7 +267,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       if (j >= 2) {   // P buffer `buf` was read by PV(j-2)
-        if (!mbar_wait(&pv_done[buf], ((j - 2) >> 1) & 1, status)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[buf], ((j - 2) >> 1) & 1, status))) {
           ok = false;
           break;
         }
@@ -275,7 +281,8 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[buf]);
     }
-    if (ok && n_tiles > 0 && mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, status)) {
+    if (ok && n_tiles > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, status))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int ld = p.n_q * D;

@@ -346,7 +346,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         }
         named_barrier_sync(1, EW * 32);
       }
-      if (!aborted && !mbar_wait(&tfull[acc], acc_phase, p.status)) aborted = true;
+      // warp-uniform: the TMEM loads below are .sync.aligned
+      if (!aborted && !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, p.status))) aborted = true;
       if (aborted) continue;
       tc_fence_after();
       const int row = ti.m0 + q * 32 + lane;
