@@ -28,9 +28,11 @@
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream); nothing synchronises the host.
  *  - Row-major layouts; bf16 = IEEE bfloat16, fp32 = IEEE float.
- *  - Every bf16 matrix operand (weights and activations) must start on a
- *    16-byte boundary (ZAYA_ERR_MISALIGNED otherwise); every pointer must be
- *    non-NULL unless stated otherwise (ZAYA_ERR_INVALID_ARG).
+ *  - Every weight matrix and vector of zaya_block_weights except k_temp,
+ *    the router MLP biases and norm weight, and balancing, and every bf16
+ *    activation, must start on a 16-byte boundary (ZAYA_ERR_MISALIGNED
+ *    otherwise); every pointer must be non-NULL unless stated otherwise
+ *    (ZAYA_ERR_INVALID_ARG).
  *  - Return value: ZAYA_OK (0) or a ZAYA_ERR_* code; argument errors are
  *    detected on the host before anything is launched.  Faults found on the
  *    device (a bounded wait that ran out, an index out of range) are written

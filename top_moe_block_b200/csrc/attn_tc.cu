@@ -6,15 +6,17 @@
 // key j is not padding (nnterp "zaya" page: grouped-query eager softmax
 // attention).  A query with no visible key outputs 0.
 //
-// CTA = 128 queries of one (sequence, head), 6 warps:
-//   warp 0     TMA: the Q tile once, then K and V tiles of 64 keys into two
-//              3-slot rings (128-byte swizzle, 64-wide d atoms);
-//   warp 1     one thread issues tcgen05.mma: S = Q K^T into one of two TMEM
-//              buffers (64 fp32 columns each), then O += P V into a TMEM
-//              accumulator (P from one of two shared-memory buffers, V as an
-//              MN-major operand); S of tile j+1 is computed while the
-//              softmax works on tile j;
-//   warps 2-5  softmax, one thread per query row (its TMEM lane): row max
+// CTA = 128 queries of two query heads that share a kv head, 10 warps:
+//   warp 0     TMA: both heads' Q tiles once, then K and V tiles of 64 keys
+//              into two 3-slot rings (128-byte swizzle, 64-wide d atoms),
+//              shared by the two heads;
+//   warp 1     one thread issues tcgen05.mma: per head, S = Q K^T into one of
+//              two TMEM buffers (64 fp32 columns each), then O += P V into the
+//              head's TMEM accumulator (P from one of two shared-memory
+//              buffers, V as an MN-major operand); S of tile j+1 is computed
+//              while the softmax works on tile j;
+//   warps 2-9  softmax, a warpgroup per head, one thread per query row (its
+//              TMEM lane): row max
 //              and sum are thread-local; P is written to shared memory in
 //              the swizzled K-major layout the MMA reads.  The running
 //              max is only moved (and O rescaled in TMEM) when it grows by
@@ -33,6 +35,7 @@ namespace {
 
 constexpr int kQT = 128;  // queries per CTA
 constexpr int kKT = 64;   // keys per tile
+constexpr int kHPC = 2;   // query heads per CTA (sharing one kv head)
 constexpr int kRing = 3;  // K and V ring depth
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -41,13 +44,14 @@ struct AttnTc {
   static constexpr int SUB = D / 64;               // 64-wide swizzle atoms along d
   static constexpr int Q_ATOM = kQT * 128;         // [128 rows][64] bf16 atom: 16 KB
   static constexpr int KV_ATOM = kKT * 128;        // [64 rows][64] bf16 atom: 8 KB
-  static constexpr int Q_BYTES = SUB * Q_ATOM;
+  static constexpr int Q_BYTES = SUB * Q_ATOM;     // one head's Q tile
   static constexpr int KV_BYTES = SUB * KV_ATOM;   // one K (or V) tile
   static constexpr int P_BYTES = kQT * kKT * 2;    // [128 queries][64 keys]: one 16 KB atom
-  static constexpr int SMEM_USED = 1024 + Q_BYTES + 2 * kRing * KV_BYTES + 2 * P_BYTES + 256;
+  static constexpr int SMEM_USED = 1024 + kHPC * Q_BYTES + 2 * kRing * KV_BYTES + kHPC * 2 * P_BYTES + 512;
   // at least 120 KB so a second CTA never shares the SM (and its TMEM)
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-  static constexpr uint32_t TMEM_COLS = 256;       // S0 [0,64), S1 [64,128), O [128, 128+D)
+  static constexpr uint32_t TMEM_COLS = 512;       // per head: S0 [0,64), S1 [64,128), O [128, 128+D)
+  static constexpr uint32_t HEAD_COLS = 256;
   static constexpr uint32_t O_COL = 2 * kKT;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, kKT);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32_bmn(128, D);
@@ -66,31 +70,31 @@ __device__ __forceinline__ bool key_visible(int q, int key, int window, int S, c
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams p, int* status) {
   using C = AttnTc<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::Q_BYTES;                // [kRing] K tiles
+  uint8_t* sQ = smem;                           // [kHPC] Q tiles
+  uint8_t* sK = sQ + kHPC * C::Q_BYTES;         // [kRing] K tiles
   uint8_t* sV = sK + kRing * C::KV_BYTES;       // [kRing] V tiles
-  uint8_t* sP = sV + kRing * C::KV_BYTES;       // [2] P tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
+  uint8_t* sP = sV + kRing * C::KV_BYTES;       // [kHPC][2] P tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kHPC * 2 * C::P_BYTES);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;                  // [kRing]
   uint64_t* k_empty = k_full + kRing;           // [kRing]
   uint64_t* v_full = k_empty + kRing;           // [kRing]
   uint64_t* v_empty = v_full + kRing;           // [kRing]
-  uint64_t* s_full = v_empty + kRing;           // [2]
-  uint64_t* s_free = s_full + 2;                // [2]
-  uint64_t* p_full = s_free + 2;                // [2]
-  uint64_t* pv_done = p_full + 2;               // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
+  uint64_t* s_full = v_empty + kRing;           // [kHPC][2]
+  uint64_t* s_free = s_full + 2 * kHPC;         // [kHPC][2]
+  uint64_t* p_full = s_free + 2 * kHPC;         // [kHPC][2]
+  uint64_t* pv_done = p_full + 2 * kHPC;        // [kHPC][2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2 * kHPC);
 
   const int qb = gridDim.x - 1 - blockIdx.x;   // heaviest (latest) query tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int g = h / (p.n_q / p.n_kv);
+  const int h0 = blockIdx.y * kHPC, b = blockIdx.z;
+  const int g = h0 / (p.n_q / p.n_kv);
   const int m0 = qb * kQT;
   const int S = p.S;
   const int lo = max(0, m0 - p.window + 1);
@@ -107,7 +111,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2 * kHPC; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
       mbar_init(&p_full[i], 4);
@@ -126,13 +130,17 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer: Q once, then K(j) and V(j) into their rings
+    // ---------------- TMA producer: both heads' Q once, then K(j) and V(j) into their rings
     if (elect_one()) {
-      const int q_row = (b * p.n_q + h) * S + m0;
       const int kv_row = (b * p.n_kv + g) * p.cap + n_begin;
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+      mbar_arrive_expect_tx(q_full, kHPC * C::Q_BYTES);
 #pragma unroll
-      for (int s = 0; s < C::SUB; ++s) tma_load_2d(sQ + s * C::Q_ATOM, &tmQ, q_full, s * 64, q_row);
+      for (int x = 0; x < kHPC; ++x) {
+        const int q_row = (b * p.n_q + h0 + x) * S + m0;
+#pragma unroll
+        for (int s = 0; s < C::SUB; ++s)
+          tma_load_2d(sQ + x * C::Q_BYTES + s * C::Q_ATOM, &tmQ, q_full, s * 64, q_row);
+      }
       for (int j = 0; j < n_tiles; ++j) {
         const int slot = j % kRing;
         const uint32_t par = ((j / kRing) & 1) ^ 1u;
@@ -149,22 +157,27 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: for each key tile, S = Q K^T of both heads, then P V of both
     if (elect_one()) {
       bool ok = mbar_wait(q_full, 0, status);
       auto issue_qk = [&](int j) -> bool {
         const int slot = j % kRing, buf = j & 1;
         if (!mbar_wait(&k_full[slot], (j / kRing) & 1, status)) return false;
-        if (!mbar_wait(&s_free[buf], ((j >> 1) & 1) ^ 1u, status)) return false;
-        tc_fence_after();
-        const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK + slot * C::KV_BYTES);
+        const uint32_t ka = smem_u32(sK + slot * C::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;
-          tc_mma_bf16(tmem_base + buf * kKT, smem_desc_sw128(qa + (kk >> 2) * C::Q_ATOM + koff, 16, 1024),
-                      smem_desc_sw128(ka + (kk >> 2) * C::KV_ATOM + koff, 16, 1024), C::IDESC_QK, kk > 0 ? 1u : 0u);
+        for (int x = 0; x < kHPC; ++x) {
+          if (!mbar_wait(&s_free[x * 2 + buf], ((j >> 1) & 1) ^ 1u, status)) return false;
+          tc_fence_after();
+          const uint32_t qa = smem_u32(sQ + x * C::Q_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk & 3) * 32;
+            tc_mma_bf16(tmem_base + x * C::HEAD_COLS + buf * kKT,
+                        smem_desc_sw128(qa + (kk >> 2) * C::Q_ATOM + koff, 16, 1024),
+                        smem_desc_sw128(ka + (kk >> 2) * C::KV_ATOM + koff, 16, 1024), C::IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[x * 2 + buf]);
         }
-        tc_commit(&s_full[buf]);
         tc_commit(&k_empty[slot]);
         return true;
       };
@@ -172,25 +185,38 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = 0; ok && j < n_tiles; ++j) {
         if (j + 1 < n_tiles && !issue_qk(j + 1)) break;
         const int slot = j % kRing, buf = j & 1;
-        if (!mbar_wait(&p_full[buf], (j >> 1) & 1, status)) break;
         if (!mbar_wait(&v_full[slot], (j / kRing) & 1, status)) break;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(sP + buf * C::P_BYTES), va = smem_u32(sV + slot * C::KV_BYTES);
+        const uint32_t va = smem_u32(sV + slot * C::KV_BYTES);
+        for (int x = 0; ok && x < kHPC; ++x) {
+          if (!mbar_wait(&p_full[x * 2 + buf], (j >> 1) & 1, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pa = smem_u32(sP + (x * 2 + buf) * C::P_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < kKT / 16; ++kk) {
-          tc_mma_bf16(tmem_base + C::O_COL, smem_desc_sw128(pa + kk * 32, 16, 1024),
-                      smem_desc_sw128(va + kk * 2048, C::KV_ATOM, 1024), C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kKT / 16; ++kk) {
+            tc_mma_bf16(tmem_base + x * C::HEAD_COLS + C::O_COL, smem_desc_sw128(pa + kk * 32, 16, 1024),
+                        smem_desc_sw128(va + kk * 2048, C::KV_ATOM, 1024), C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&pv_done[x * 2 + buf]);
         }
-        tc_commit(&pv_done[buf]);
+        if (!ok) break;
         tc_commit(&v_empty[slot]);
       }
     }
   } else {
-    // ---------------- softmax: one thread per query row
+    // ---------------- softmax: warpgroup x handles head h0 + x, one thread per query row
+    const int x = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int q = m0 + row;
-    const uint32_t tl = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t tl = tmem_base + x * C::HEAD_COLS + ((uint32_t)(quarter * 32) << 16);
+    uint64_t* my_s_full = s_full + x * 2;
+    uint64_t* my_s_free = s_free + x * 2;
+    uint64_t* my_p_full = p_full + x * 2;
+    uint64_t* my_pv_done = pv_done + x * 2;
+    uint8_t* my_p = sP + x * 2 * C::P_BYTES;
     const int* mask = p.mask ? p.mask + (size_t)b * S : nullptr;
     const float sl2 = p.scale * 1.4426950408889634f;
     float m_used = -INFINITY, l = 0.f;
@@ -198,7 +224,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int j = 0; j < n_tiles; ++j) {
       const int buf = j & 1;
       // every wait that guards a .sync.aligned TMEM access is made warp-uniform
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (j >> 1) & 1, status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&my_s_full[buf], (j >> 1) & 1, status))) {
         ok = false;
         break;
       }
@@ -216,8 +242,8 @@ __global__ void __launch_bounds__(192, 1)
       } else {
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          const float x = __uint_as_float(r[i >> 5][i & 31]) * sl2;
-          v[i] = key_visible(q, key0 + i, p.window, S, mask) ? x : -INFINITY;
+          const float xv = __uint_as_float(r[i >> 5][i & 31]) * sl2;
+          v[i] = key_visible(q, key0 + i, p.window, S, mask) ? xv : -INFINITY;
         }
       }
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
@@ -226,7 +252,7 @@ __global__ void __launch_bounds__(192, 1)
       const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[buf]);   // S is in registers: the buffer may be refilled
+      if (lane == 0) mbar_arrive(&my_s_free[buf]);   // S is in registers: the buffer may be refilled
       const float m_new = fmaxf(m_used, tmax);
       // Move the running max when it grew by more than 2^8 -- for the whole warp
       // at once, since the O rescale below is a warp-wide TMEM access.  Each
@@ -237,7 +263,7 @@ __global__ void __launch_bounds__(192, 1)
         const float f = (m_used == -INFINITY || !finite_new) ? 1.f : exp2f(m_used - m_new);
         if (j > 0 && __any_sync(0xffffffffu, m_used != -INFINITY)) {
           // O holds tiles < j: wait for PV(j-1), then scale it in TMEM
-          if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&my_pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status))) {
             ok = false;
             break;
           }
@@ -267,26 +293,26 @@ __global__ void __launch_bounds__(192, 1)
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       if (j >= 2) {   // P buffer `buf` was read by PV(j-2)
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[buf], ((j - 2) >> 1) & 1, status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&my_pv_done[buf], ((j - 2) >> 1) & 1, status))) {
           ok = false;
           break;
         }
       }
-      uint8_t* prow = sP + buf * C::P_BYTES + row * 128;
+      uint8_t* prow = my_p + buf * C::P_BYTES + row * 128;
 #pragma unroll
       for (int u = 0; u < 8; ++u)
         *reinterpret_cast<uint4*>(prow + ((u ^ (row & 7)) << 4)) =
             make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       fence_proxy_async();   // P's generic-proxy stores -> visible to the tensor core
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[buf]);
+      if (lane == 0) mbar_arrive(&my_p_full[buf]);
     }
     if (ok && n_tiles > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, status))) {
+        __all_sync(0xffffffffu, mbar_wait(&my_pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, status))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int ld = p.n_q * D;
-      auto* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * S + q) * ld + h * D;
+      auto* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * S + q) * ld + (h0 + x) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -295,12 +321,12 @@ __global__ void __launch_bounds__(192, 1)
         if (q < S) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            uint4 v;
-            v.x = pack_bf2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
-            v.y = pack_bf2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
-            v.z = pack_bf2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
-            v.w = pack_bf2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
-            reinterpret_cast<uint4*>(out + c * 32)[u] = v;
+            uint4 vv;
+            vv.x = pack_bf2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
+            vv.y = pack_bf2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
+            vv.z = pack_bf2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
+            vv.w = pack_bf2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
+            reinterpret_cast<uint4*>(out + c * 32)[u] = vv;
           }
         }
       }
@@ -326,7 +352,8 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
   if (!rc) rc = make_tmap_bf16(&mk, p.k_cache, (uint64_t)p.B * p.n_kv * p.cap, (uint64_t)p.d, kKT);
   if (!rc) rc = make_tmap_bf16(&mv, p.v_cache, (uint64_t)p.B * p.n_kv * p.cap, (uint64_t)p.d, kKT);
   if (rc) return rc;
-  const dim3 grid((p.S + kQT - 1) / kQT, p.n_q, p.B);
+  if (p.n_q % kHPC || (p.n_q / p.n_kv) % kHPC) return ZAYA_ERR_UNSUPPORTED;
+  const dim3 grid((p.S + kQT - 1) / kQT, p.n_q / kHPC, p.B);
   if (p.d == 128) {
     auto kern = attn_tc_kernel<128>;
     static bool set = false;
@@ -334,7 +361,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTc<128>::SMEM);
       set = true;
     }
-    kern<<<grid, 192, AttnTc<128>::SMEM, st>>>(mq, mk, mv, p, status);
+    kern<<<grid, 64 + 32 * 4 * kHPC, AttnTc<128>::SMEM, st>>>(mq, mk, mv, p, status);
   } else {
     auto kern = attn_tc_kernel<64>;
     static bool set = false;
@@ -342,7 +369,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTc<64>::SMEM);
       set = true;
     }
-    kern<<<grid, 192, AttnTc<64>::SMEM, st>>>(mq, mk, mv, p, status);
+    kern<<<grid, 64 + 32 * 4 * kHPC, AttnTc<64>::SMEM, st>>>(mq, mk, mv, p, status);
   }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }

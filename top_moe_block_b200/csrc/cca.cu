@@ -45,6 +45,36 @@ struct Pre {
   }
 };
 
+// DPL consecutive bf16 (4- or 8-byte aligned) read as one load.
+template <int DPL>
+__device__ __forceinline__ void load_bf(const __nv_bfloat16* src, float (&y)[DPL]) {
+  if constexpr (DPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(src);
+    const float2 a = unpack_bf2(u.x), b = unpack_bf2(u.y);
+    y[0] = a.x; y[1] = a.y; y[2] = b.x; y[3] = b.y;
+  } else {
+    const float2 a = unpack_bf2(*reinterpret_cast<const uint32_t*>(src));
+    y[0] = a.x; y[1] = a.y;
+  }
+}
+// N consecutive fp32 (16-byte aligned when N % 4 == 0) through the read-only path.
+template <int N>
+__device__ __forceinline__ void load_f(const float* __restrict__ src, float (&y)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(src) + i);
+      y[4 * i] = v.x; y[4 * i + 1] = v.y; y[4 * i + 2] = v.z; y[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const float2 v = __ldg(reinterpret_cast<const float2*>(src) + i);
+      y[2 * i] = v.x; y[2 * i + 1] = v.y;
+    }
+  }
+}
+
 // DPL consecutive bf16 written as one 4- or 8-byte store.
 template <int DPL>
 __device__ __forceinline__ void store_bf(__nv_bfloat16* dst, const float (&y)[DPL]) {
@@ -59,7 +89,7 @@ __device__ __forceinline__ void store_bf(__nv_bfloat16* dst, const float (&y)[DP
 }
 
 template <int D>
-__device__ __forceinline__ void rope_apply(float (&y)[D / 32], int lane, int pos, int rot, float theta) {
+__device__ __forceinline__ void rope_apply(float (&y)[D / 32], int lane, int pos, int rot, const float* inv_freq_tab) {
   constexpr int DPL = D / 32;
   if (rot <= 0) return;
   const int half = rot / 2;
@@ -75,7 +105,7 @@ __device__ __forceinline__ void rope_apply(float (&y)[D / 32], int lane, int pos
     const float partner = __shfl_sync(0xffffffffu, y[i], src);
     if (in_rot) {
       const int f = lo ? j : j - half;
-      const float inv_freq = (float)(1.0 / pow((double)theta, (double)(2 * f) / (double)rot));
+      const float inv_freq = inv_freq_tab[f];
       const float ang = posf * inv_freq;
       float sn, cs;
       sincosf(ang, &sn, &cs);
@@ -156,7 +186,7 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
     if (!is_q) scl *= __ldg(p.k_temp + g);
 #pragma unroll
     for (int i = 0; i < DPL; ++i) y[i] *= scl;
-    rope_apply<D>(y, lane, pos, p.rot, p.theta);
+    rope_apply<D>(y, lane, pos, p.rot, p.inv_freq);
 
     __nv_bfloat16* dst;
     if (is_q) {
@@ -253,8 +283,7 @@ __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
                  : "memory");
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
-  for (int f = threadIdx.x; f < half; f += blockDim.x)
-    inv_f[f] = (float)(1.0 / pow((double)p.theta, (double)(2 * f) / (double)p.rot));
+  for (int f = threadIdx.x; f < half; f += blockDim.x) inv_f[f] = p.inv_freq[f];
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
   for (int i = threadIdx.x; i < kTok * half; i += blockDim.x) {
@@ -280,29 +309,39 @@ __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
       const int hh = is_q ? head : head - nq;
       const int g = is_q ? head / rep : hh;
       const int cbase = (is_q ? hh * D : nq * D + hh * D) + lane * DPL;
-      float y[DPL], a0[DPL], a1[DPL];
+      float y[DPL], a0[DPL], a1[DPL], a2[DPL], w[3 * DPL], bias[DPL];
+      load_bf<DPL>(ut + cbase, a0);
+      load_bf<DPL>(u1 + cbase, a1);
+      load_bf<DPL>(u2 + cbase, a2);
+      load_f<3 * DPL>(p.conv_w + 3 * cbase, w);
+      load_f<DPL>(p.conv_b + cbase, bias);
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
-        const int c = cbase + i;
-        a0[i] = bf2f(ut[c]);
-        a1[i] = bf2f(u1[c]);
-        const float a2 = bf2f(u2[c]);
-        float acc = __ldg(p.conv_b + c);
-        acc = fmaf(__ldg(p.conv_w + 3 * c + 0), a2, acc);
-        acc = fmaf(__ldg(p.conv_w + 3 * c + 1), a1[i], acc);
-        acc = fmaf(__ldg(p.conv_w + 3 * c + 2), a0[i], acc);
-        if (p.cca_res) {
-          const int j = lane * DPL + i;
-          const float kpre = bf2f(ut[nq * D + g * D + j]);
-          if (is_q) {
-            acc += 0.5f * (a0[i] + kpre);
-          } else {
-            float qs = 0.f;
-            for (int h2 = g * rep; h2 < (g + 1) * rep; ++h2) qs += bf2f(ut[h2 * D + j]);
-            acc += 0.5f * (qs / (float)rep + kpre);
-          }
-        }
+        float acc = bias[i];
+        acc = fmaf(w[3 * i + 0], a2[i], acc);
+        acc = fmaf(w[3 * i + 1], a1[i], acc);
+        acc = fmaf(w[3 * i + 2], a0[i], acc);
         y[i] = acc;
+      }
+      if (p.cca_res) {
+        float kpre[DPL];
+        load_bf<DPL>(ut + nq * D + g * D + lane * DPL, kpre);
+        if (is_q) {
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) y[i] += 0.5f * (a0[i] + kpre[i]);
+        } else {
+          float qs[DPL];
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) qs[i] = 0.f;
+          for (int h2 = g * rep; h2 < (g + 1) * rep; ++h2) {
+            float qh[DPL];
+            load_bf<DPL>(ut + h2 * D + lane * DPL, qh);
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) qs[i] += qh[i];
+          }
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) y[i] += 0.5f * (qs[i] / (float)rep + kpre[i]);
+        }
       }
       float ss = 0.f;
 #pragma unroll
@@ -350,14 +389,11 @@ __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
       __nv_bfloat16* dst =
           static_cast<__nv_bfloat16*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + s) * D + lane * DPL;
       float vv[DPL];
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) {
-        const int j = lane * DPL + i;
-        if (j < D / 2)
-          vv[i] = bf2f(ut[vc0 + g * (D / 2) + j]);
-        else
-          vv[i] = bf2f((p.v_delayed ? u1 : ut)[vd0 + g * (D / 2) + (j - D / 2)]);
-      }
+      const int j0 = lane * DPL;   // DPL consecutive dims lie in one half of the head
+      if (j0 < D / 2)
+        load_bf<DPL>(ut + vc0 + g * (D / 2) + j0, vv);
+      else
+        load_bf<DPL>((p.v_delayed ? u1 : ut) + vd0 + g * (D / 2) + (j0 - D / 2), vv);
       store_bf<DPL>(dst, vv);
       if (s == p.S - 1 && g == 0) {   // prev_hs <- attention_norm_output of token S-1
         const uint2* src = reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.a_in) + (row0 + s) * p.H);

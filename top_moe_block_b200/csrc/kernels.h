@@ -91,6 +91,7 @@ struct CcaParams {
   float theta, eps;
   int decode;             // 1: one token per sequence, history from conv_state
   int* status;
+  float inv_freq[64];     // RoPE inverse frequencies theta^(-2i/rot), i < rot/2 (fp32)
 };
 int launch_cca(const CcaParams& p, cudaStream_t st);
 

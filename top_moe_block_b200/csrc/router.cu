@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   // float4 per thread, every load of a group issued before the adds.
   {
     constexpr int R4 = R / 4;
-#pragma unroll 2
+#pragma unroll
     for (int i = threadIdx.x; i < kTM * R4; i += kThreads) {
       const int tt = i / R4, k4 = i % R4, t = t0 + tt;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -215,7 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   const size_t n = (size_t)R * R;
   dense_gelu_tc<R>(z, g, p.wsplit, p.wsplit + n, p.fc1_b, wring);
   dense_gelu_tc<R>(g, z, p.wsplit + 2 * n, p.wsplit + 3 * n, p.fc2_b, wring);
-  // out_proj (no bias, fp32 on CUDA cores) and the choice, one warp per token
+  // out_proj (no bias, fp32 on CUDA cores) and the choice, one warp per token;
+  // out_w is staged in shared memory (the weight ring is free now).
+  float* ow = reinterpret_cast<float*>(wring);
+  for (int i = threadIdx.x; i < E1 * R / 4; i += kThreads)
+    reinterpret_cast<float4*>(ow)[i] = __ldg(reinterpret_cast<const float4*>(p.out_w) + i);
+  __syncthreads();
   for (int tt = warp; tt < kTM; tt += kThreads / 32) {
     const int t = t0 + tt;
     if (t >= p.M) continue;
@@ -223,13 +228,25 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
 #pragma unroll
     for (int j = 0; j < R / 32; ++j) zr[j] = z[tt * kZS + lane + 32 * j];
     float l[3] = {-INFINITY, -INFINITY, -INFINITY};
-    for (int c = 0; c < E1; ++c) {
-      const float* wr = p.out_w + (size_t)c * R;
-      float a = 0.f;
+    for (int c0 = 0; c0 < E1; c0 += 4) {   // four classes per round: independent chains
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < R / 32; ++j) a = fmaf(zr[j], __ldg(wr + lane + 32 * j), a);
-      a = warp_sum(a);
-      if ((c & 31) == lane) l[c >> 5] = a;
+      for (int u = 0; u < 4; ++u) {
+        if (c0 + u < E1) {
+          const float* wr = ow + (c0 + u) * R;
+#pragma unroll
+          for (int j = 0; j < R / 32; ++j) a[u] = fmaf(zr[j], wr[lane + 32 * j], a[u]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] += __shfl_xor_sync(0xffffffffu, a[u], o);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u;
+        if (c < E1 && (c & 31) == lane) l[c >> 5] = a[u];
+      }
     }
     float mx = fmaxf(fmaxf(l[0], l[1]), l[2]);
     mx = warp_max(mx);
@@ -378,54 +395,46 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ c
   }
 }
 
+// One thread per 16-byte chunk (8 columns) of a token row: routed tokens copy
+// the chunk of m_in to their permuted row; skipped (and padding) tokens
+// write merge 2 with a zero routed output for those 8 columns.
 __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
-  const int t = blockIdx.x * 8 + warp_id();
-  const int lane = lane_id();
-  if (t >= p.M) return;
-  const int H = p.H;
+  const int per_row = p.H / 8;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)p.M * per_row) return;
+  const int t = (int)(i / per_row), ch = (int)(i % per_row);
   const int c = p.cls[t];
   if (c >= 0 && c < p.E) {
-    const uint4* __restrict__ src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * H);
-    uint4* __restrict__ dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)p.pos[t] * H);
-    const int n = H / 8;   // 16-byte vectors per row
-    for (int base = 0; base < n; base += 32 * 4) {   // four loads in flight per lane before the stores
-      uint4 v[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int i = base + lane + 32 * k;
-        if (i < n) v[k] = src[i];
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int i = base + lane + 32 * k;
-        if (i < n) dst[i] = v[k];
-      }
-    }
+    const uint4 v = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * p.H)[ch];
+    reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)p.pos[t] * p.H)[ch] = v;
   } else {
     // skip: no expert runs; mlp_output = bf16(hb * hs), out = mlp_output + (h + rb) * rs
-    float4* s4 = reinterpret_cast<float4*>(p.stream + (size_t)t * H);
-    __nv_bfloat16* tap = p.tap_mlp_out ? static_cast<__nv_bfloat16*>(p.tap_mlp_out) + (size_t)t * H : nullptr;
-    for (int i = lane; i < H / 4; i += 32) {
-      float4 x = s4[i];
+    const int H = p.H;
+    float4* s4 = reinterpret_cast<float4*>(p.stream + (size_t)t * H + ch * 8);
+    float cb[8];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float4 x = s4[h];
       float* xp = &x.x;
-      float cb[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int col = 4 * i + j;
+        const int col = ch * 8 + 4 * h + j;
         const float contrib = round_bf(__ldg(p.merge_m + col) * __ldg(p.merge_m + H + col));
-        cb[j] = contrib;
+        cb[4 * h + j] = contrib;
         xp[j] = fmaf(xp[j] + __ldg(p.merge_m + 2 * H + col), __ldg(p.merge_m + 3 * H + col), contrib);
       }
-      s4[i] = x;
-      if (tap) {
-        uint2 u;
-        u.x = pack_bf2(cb[0], cb[1]);
-        u.y = pack_bf2(cb[2], cb[3]);
-        reinterpret_cast<uint2*>(tap)[i] = u;
-      }
+      s4[h] = x;
+    }
+    if (p.tap_mlp_out) {
+      uint4 u;
+      u.x = pack_bf2(cb[0], cb[1]);
+      u.y = pack_bf2(cb[2], cb[3]);
+      u.z = pack_bf2(cb[4], cb[5]);
+      u.w = pack_bf2(cb[6], cb[7]);
+      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.tap_mlp_out) + (size_t)t * H)[ch] = u;
     }
   }
-  if (p.cache_len_inc && lane == 0) p.cache_len_inc[t] += 1;
+  if (p.cache_len_inc && ch == 0) p.cache_len_inc[t] += 1;
 }
 
 }  // namespace
@@ -451,7 +460,9 @@ int launch_permute(const int* cls, int M, int E, int* group_off, int* mt_start, 
 
 int launch_dispatch(const DispatchParams& p, cudaStream_t st) {
   if (p.M <= 0) return ZAYA_OK;
-  dispatch_kernel<<<(p.M + 7) / 8, 256, 0, st>>>(p);
+  if (p.H % 8) return ZAYA_ERR_UNSUPPORTED;
+  const long n = (long)p.M * (p.H / 8);
+  dispatch_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 

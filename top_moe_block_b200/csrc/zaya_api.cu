@@ -138,7 +138,8 @@ int check_weights(const zaya_block_weights* w) {
   for (const void* p : ptrs)
     if (!p) return ZAYA_ERR_INVALID_ARG;
   const void* mats[] = {w->ln1_w, w->ln2_w, w->w_qkv, w->w_o, w->router_down_w, w->w_gate_up, w->w_down,
-                        w->merge_a, w->merge_m, w->out_w, w->fc1_w, w->fc2_w};
+                        w->merge_a, w->merge_m, w->out_w, w->fc1_w, w->fc2_w, w->conv_w, w->conv_b,
+                        w->router_down_b, w->router_state_scale};
   for (const void* p : mats)
     if (!a16(p)) return ZAYA_ERR_MISALIGNED;
   return ZAYA_OK;
@@ -202,6 +203,12 @@ int pick_bn_tiles(long m_tiles, int N, const int* cands, int n, int sms) {
 }
 int pick_bn(int M, int N, const int* cands, int n, int sms) {
   return pick_bn_tiles((M + 127) / 128, N, cands, n, sms);
+}
+
+// RoPE inverse frequencies theta^(-2i/rot) rounded to fp32 (Llama's rotary
+// keeps them in fp32), computed once per call on the host.
+void fill_inv_freq(float* out, int rot, float theta) {
+  for (int i = 0; i < 64; ++i) out[i] = (2 * i < rot) ? (float)(1.0 / pow((double)theta, (double)(2 * i) / rot)) : 0.f;
 }
 
 #define ZAYA_TRY(x)            \
@@ -335,6 +342,7 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     p.B = B; p.S = S; p.H = d.H; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.rot = c.rot_dim;
     p.cca_res = c.cca_mean_residual; p.v_delayed = c.v_delayed; p.theta = c.rope_theta; p.eps = c.qk_norm_eps;
     p.decode = 0; p.status = status;
+    fill_inv_freq(p.inv_freq, c.rot_dim, c.rope_theta);
     ZAYA_STAGE("cca", 1, launch_cca(p, st));
   }
   {
@@ -387,6 +395,7 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
     p.B = B; p.S = 1; p.H = d.H; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.rot = c.rot_dim;
     p.cca_res = c.cca_mean_residual; p.v_delayed = c.v_delayed; p.theta = c.rope_theta; p.eps = c.qk_norm_eps;
     p.decode = 1; p.status = status;
+    fill_inv_freq(p.inv_freq, c.rot_dim, c.rope_theta);
     ZAYA_STAGE("cca", 1, launch_cca(p, st));
   }
   {
