@@ -119,7 +119,8 @@ typedef struct zaya_block_weights {
 
 /* One block's decode state (in/out, caller-owned). */
 typedef struct zaya_block_state {
-  void* k_cache;        /* bf16 [B, n_kv, cache_cap, d]: keys after norm, temp and RoPE */
+  void* k_cache;        /* bf16 [B, n_kv, cache_cap, d]: keys after norm, temp and RoPE
+                           (this and the three state buffers below: 16-byte aligned) */
   void* v_cache;        /* bf16 [B, n_kv, cache_cap, d] */
   int32_t cache_cap;    /* positions per sequence the caches hold */
   int32_t* cache_len;   /* device int32 [B]: prefill writes S; decode appends at cache_len[b]
@@ -139,7 +140,7 @@ typedef struct zaya_taps {
   float* layer_mid;          /* fp32 [M, H] */
   void* mlp_norm_output;     /* bf16 [M, H] */
   void* mlp_output;          /* bf16 [M, H]: (routed + hb) * hs */
-  void* attention_queries;   /* bf16 [B, n_q, S, d] (prefill) / [B, n_q, d] (decode) */
+  void* attention_queries;   /* bf16 [B, n_q, S, d] (prefill) / [B, n_q, d] (decode); 16-byte aligned */
 } zaya_taps;
 
 /* Bytes of device workspace a call needs: mode ZAYA_PREFILL with (B, S), or

@@ -405,6 +405,197 @@ __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
   }
 }
 
+// Prefill, streaming form: a thread owns 8 consecutive channels of one q/k
+// head (the d/8 threads of a head are adjacent lanes, so the head norm and the
+// RoPE pair exchange are shuffles inside that lane group) and walks the CTA's
+// kStream tokens in order, with its conv taps and bias in registers and the
+// two previous pre-conv values carried from step to step.  Value heads: d/8
+// threads per kv head copy the current / delayed halves.  Needs rot % 16 == 0
+// (a thread's 8 dims are all inside or all outside the rotated range).
+constexpr int kStream = 16;
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&y)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(src);
+  const float2 a = unpack_bf2(v.x), b = unpack_bf2(v.y), c = unpack_bf2(v.z), d = unpack_bf2(v.w);
+  y[0] = a.x; y[1] = a.y; y[2] = b.x; y[3] = b.y; y[4] = c.x; y[5] = c.y; y[6] = d.x; y[7] = d.y;
+}
+__device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
+  return make_uint4(pack_bf2(y[0], y[1]), pack_bf2(y[2], y[3]), pack_bf2(y[4], y[5]), pack_bf2(y[6], y[7]));
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__ CcaParams p) {
+  constexpr int LPH = D / 8;   // threads per head
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int nq = p.n_q, nkv = p.n_kv, rep = nq / nkv;
+  const int C = (nq + nkv) * D;
+  const int ld = p.n_qkv;
+  const int b = blockIdx.y;
+  const int s0 = blockIdx.x * kStream;
+  const int half = p.rot / 2;
+  auto* u = reinterpret_cast<__nv_bfloat16*>(sm);                                 // [kStream + 2][ld]
+  float2* cs = reinterpret_cast<float2*>(sm + (size_t)(kStream + 2) * ld * 2);    // [kStream][half]
+  const auto* qkv = static_cast<const __nv_bfloat16*>(p.qkv);
+  const size_t row0 = (size_t)b * p.S;
+
+  // rows s0-2 .. s0+kStream-1 (zero outside the sequence and at padding), one cp.async wait
+  const int vec_per_row = ld / 8;
+  for (int i = threadIdx.x; i < (kStream + 2) * vec_per_row; i += blockDim.x) {
+    const int r = i / vec_per_row, c = i % vec_per_row;
+    const int s = s0 - 2 + r;
+    const bool valid = s >= 0 && s < p.S && (!p.mask || p.mask[row0 + s] != 0);
+    const __nv_bfloat16* src = qkv + (row0 + (valid ? s : 0)) * ld + c * 8;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(u + (size_t)r * ld + c * 8)),
+                 "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int i = threadIdx.x; i < kStream * half; i += blockDim.x) {
+    const int tt = i / half, f = i % half;
+    float sn, c;
+    sincosf((float)(s0 + tt) * p.inv_freq[f], &sn, &c);
+    cs[i] = make_float2(c, sn);
+  }
+  const int tid = threadIdx.x, lane = lane_id();
+  const int n_qk = (nq + nkv) * LPH;
+  // conv taps / bias of this thread's channels, loaded under the staging
+  float w0[8], w1[8], w2[8], bb[8];
+  const int head = tid / LPH, l = tid % LPH;
+  const int cb = head * D + l * 8;
+  if (tid < n_qk) {
+    const float4* wp = reinterpret_cast<const float4*>(p.conv_w + 3 * cb);
+    float wv[24];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+      const float4 v = __ldg(wp + i);
+      wv[4 * i] = v.x; wv[4 * i + 1] = v.y; wv[4 * i + 2] = v.z; wv[4 * i + 3] = v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { w0[i] = wv[3 * i]; w1[i] = wv[3 * i + 1]; w2[i] = wv[3 * i + 2]; }
+    const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.conv_b + cb));
+    const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.conv_b + cb) + 1);
+    bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w; bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+
+  if (tid < n_qk) {
+    const bool is_q = head < nq;
+    const int hh = is_q ? head : head - nq;
+    const int g = is_q ? head / rep : hh;
+    const unsigned gmask = ((1u << LPH) - 1u) << (lane & ~(LPH - 1));   // this head's lanes
+    const float scl0 = sqrtf((float)D) * (is_q ? 1.f : __ldg(p.k_temp + g));
+    const int j0 = l * 8;
+    const bool in_rot = j0 < p.rot, lo = j0 < half;
+    const int src_lane = in_rot ? (lo ? lane + half / 8 : lane - half / 8) : lane;
+    const int f0 = lo ? j0 : j0 - half;
+    const int kcb = nq * D + g * D + l * 8;   // the group's key channels (query residual)
+    float x2[8], x1[8];
+    load8(u + cb, x2);
+    load8(u + ld + cb, x1);
+    __nv_bfloat16* dst = is_q ? static_cast<__nv_bfloat16*>(p.q_out) + (((size_t)b * nq + hh) * p.S + s0) * D + j0
+                              : static_cast<__nv_bfloat16*>(p.k_cache) + (((size_t)b * nkv + hh) * p.cache_cap + s0) * D + j0;
+    __nv_bfloat16* tap = (is_q && p.tap_q)
+                             ? static_cast<__nv_bfloat16*>(p.tap_q) + (((size_t)b * nq + hh) * p.S + s0) * D + j0
+                             : nullptr;
+#pragma unroll 2
+    for (int tt = 0; tt < kStream; ++tt) {
+      const int s = s0 + tt;
+      if (s >= p.S) break;   // uniform over the head's lanes
+      const __nv_bfloat16* row = u + (size_t)(tt + 2) * ld;
+      float x0[8], y[8];
+      load8(row + cb, x0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float acc = bb[i];
+        acc = fmaf(w0[i], x2[i], acc);
+        acc = fmaf(w1[i], x1[i], acc);
+        acc = fmaf(w2[i], x0[i], acc);
+        y[i] = acc;
+      }
+      if (p.cca_res) {
+        if (is_q) {
+          float kp[8];
+          load8(row + kcb, kp);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[i] += 0.5f * (x0[i] + kp[i]);
+        } else {
+          float qs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          for (int h2 = g * rep; h2 < (g + 1) * rep; ++h2) {
+            float qh[8];
+            load8(row + h2 * D + l * 8, qh);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qs[i] += qh[i];
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[i] += 0.5f * (qs[i] / (float)rep + x0[i]);
+        }
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(y[i], y[i], ss);
+#pragma unroll
+      for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gmask, ss, o);
+      const float scl = scl0 / fmaxf(sqrtf(ss), p.eps);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[i] *= scl;
+      if (half > 0) {   // rotate-half over dims [0, rot)
+        float pt[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pt[i] = __shfl_sync(gmask, y[i], src_lane);
+        if (in_rot) {
+          const float4* e4 = reinterpret_cast<const float4*>(cs + tt * half + f0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 e = e4[i];   // (cos, sin) of dims 2i and 2i + 1
+            if (lo) {
+              y[2 * i] = y[2 * i] * e.x - pt[2 * i] * e.y;
+              y[2 * i + 1] = y[2 * i + 1] * e.z - pt[2 * i + 1] * e.w;
+            } else {
+              y[2 * i] = y[2 * i] * e.x + pt[2 * i] * e.y;
+              y[2 * i + 1] = y[2 * i + 1] * e.z + pt[2 * i + 1] * e.w;
+            }
+          }
+        }
+      }
+      const uint4 o = pack8(y);
+      *reinterpret_cast<uint4*>(dst + (size_t)tt * D) = o;
+      if (tap) *reinterpret_cast<uint4*>(tap + (size_t)tt * D) = o;
+      if (s == p.S - 1) {   // conv_state <- pre-conv channels of tokens S-2, S-1
+        auto* cst = static_cast<__nv_bfloat16*>(p.conv_state) + (size_t)b * C * 2 + (size_t)cb * 2;
+        uint4 c0, c1;
+        c0.x = pack_bf2(x1[0], x0[0]); c0.y = pack_bf2(x1[1], x0[1]);
+        c0.z = pack_bf2(x1[2], x0[2]); c0.w = pack_bf2(x1[3], x0[3]);
+        c1.x = pack_bf2(x1[4], x0[4]); c1.y = pack_bf2(x1[5], x0[5]);
+        c1.z = pack_bf2(x1[6], x0[6]); c1.w = pack_bf2(x1[7], x0[7]);
+        reinterpret_cast<uint4*>(cst)[0] = c0;
+        reinterpret_cast<uint4*>(cst)[1] = c1;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { x2[i] = x1[i]; x1[i] = x0[i]; }
+    }
+  } else if (tid < n_qk + nkv * LPH) {
+    const int vt = tid - n_qk, g = vt / LPH, j0 = (vt % LPH) * 8;
+    const int vc0 = nq * D + nkv * D;          // current halves
+    const int vd0 = vc0 + nkv * (D / 2);       // delayed halves (from token t-1)
+    auto* dst = static_cast<__nv_bfloat16*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + s0) * D + j0;
+    for (int tt = 0; tt < kStream; ++tt) {
+      const int s = s0 + tt;
+      if (s >= p.S) break;
+      const __nv_bfloat16* row = u + (size_t)(tt + 2) * ld;
+      const __nv_bfloat16* src = (j0 < D / 2) ? row + vc0 + g * (D / 2) + j0
+                                              : (p.v_delayed ? row - ld : row) + vd0 + g * (D / 2) + (j0 - D / 2);
+      *reinterpret_cast<uint4*>(dst + (size_t)tt * D) = *reinterpret_cast<const uint4*>(src);
+      if (s == p.S - 1 && g == 0) {   // prev_hs <- attention_norm_output of token S-1
+        const uint4* hs = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.a_in) + (row0 + s) * p.H);
+        uint4* ph = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.prev_hs) + (size_t)b * p.H);
+        for (int c = vt; c < p.H / 8; c += LPH) ph[c] = hs[c];
+        if (vt == 0) p.cache_len[b] = p.S;
+      }
+    }
+  }
+}
+
 }  // namespace
 
 int launch_cca(const CcaParams& p, cudaStream_t st) {
@@ -412,6 +603,22 @@ int launch_cca(const CcaParams& p, cudaStream_t st) {
   if (tokens <= 0) return ZAYA_OK;
   const int threads = 32 * (p.n_q + 2 * p.n_kv);
   if (threads > 1024 || p.rot / 2 > 64 || p.n_qkv % 8) return ZAYA_ERR_UNSUPPORTED;
+  if (!p.decode && (p.d == 128 || p.d == 64) && p.rot % 16 == 0 && p.H % 8 == 0) {
+    const int lph = p.d / 8;
+    const int nthr = ((p.n_q + 2 * p.n_kv) * lph + 31) / 32 * 32;
+    const size_t smem = (size_t)(kStream + 2) * p.n_qkv * 2 + (size_t)kStream * (p.rot / 2) * 8;
+    if (nthr <= 256 && smem <= 227 * 1024) {
+      const dim3 grid((p.S + kStream - 1) / kStream, p.B);
+      if (p.d == 128) {
+        cudaFuncSetAttribute(cca_stream_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cca_stream_kernel<128><<<grid, nthr, smem, st>>>(p);
+      } else {
+        cudaFuncSetAttribute(cca_stream_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cca_stream_kernel<64><<<grid, nthr, smem, st>>>(p);
+      }
+      return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
+    }
+  }
   if (!p.decode) {
     const size_t smem = (size_t)(kTok + 2) * p.n_qkv * 2 + 64 * 4 + (size_t)kTok * (p.rot / 2) * 8;
     const dim3 grid((p.S + kTok - 1) / kTok, p.B);

@@ -48,14 +48,22 @@ template <int EPI>
 __host__ __device__ constexpr bool is_merge() { return EPI == EPI_MERGE_ATTN || EPI == EPI_MERGE_MLP; }
 constexpr int kPrefetchAhead = 8;  // k-blocks of B pulled into L2 ahead of their TMA load
 
-template <int BN>
+constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA (227 KB)
+
+template <int BN, int EPI>
 struct GemmCfg {
   static constexpr int B_STAGE_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);  // ~192 KB ring
   static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
   static constexpr int PARAM_BYTES = 2 * 4 * BN * 4;  // merge epilogues: [2 tiles][hb,hs,rb,rs][BN] fp32
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + PARAM_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  // merge epilogues: a 32 x 32 fp32 transpose buffer per epilogue warp
+  static constexpr int T_BYTES = is_merge<EPI>() ? epi_warps<EPI>() * 32 * 32 * 4 : 0;
+  static constexpr int FIXED = PARAM_BYTES + T_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int DEF_STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);  // ~192 KB ring
+  static constexpr int FIT_STAGES = (kSmemLimit - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = DEF_STAGES < FIT_STAGES ? DEF_STAGES : FIT_STAGES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED;
+  static_assert(STAGES >= 3, "ring too shallow");
 };
 
 struct TileInfo {
@@ -200,11 +208,82 @@ __device__ __forceinline__ void epilogue32(const GemmParams& p, int row, int col
   }
 }
 
+// Merge epilogue of a warp's 32 rows x 32 columns, coalesced: the accumulator
+// rows (one per lane, as tcgen05.ld delivers them) go through a 32 x 32 fp32
+// shared-memory transpose (16-byte chunks XOR-swizzled by row), then each
+// step covers 4 rows x 128 contiguous bytes of the fp32 stream; all eight
+// steps' stream loads are issued before the first use.
+template <int EPI>
+__device__ __forceinline__ void merge_chunk(const GemmParams& p, int row0, int m_end, int col,
+                                            const uint32_t (&r)[32], float* T, const float* prm, int prm_ld) {
+  const int lane = lane_id();
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<float4*>(T + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+        make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]),
+                    __uint_as_float(r[4 * j + 3]));
+  __syncwarp();
+  const int jj = lane & 7, rsub = lane >> 3;
+  const int N = p.N;
+  int tok[8];
+  float wt[8];
+  float4 xs[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int grow = row0 + 4 * i + rsub;
+    tok[i] = -1;
+    if (grow < m_end) tok[i] = (EPI == EPI_MERGE_MLP) ? p.perm[grow] : grow;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    wt[i] = 1.0f;
+    xs[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tok[i] >= 0) {
+      if constexpr (EPI == EPI_MERGE_MLP) wt[i] = p.row_w[tok[i]];
+      xs[i] = *reinterpret_cast<const float4*>(p.stream + (size_t)tok[i] * N + col + 4 * jj);
+    }
+  }
+  const float4 hb4 = *reinterpret_cast<const float4*>(prm + 4 * jj);
+  const float4 hs4 = *reinterpret_cast<const float4*>(prm + prm_ld + 4 * jj);
+  const float4 rb4 = *reinterpret_cast<const float4*>(prm + 2 * prm_ld + 4 * jj);
+  const float4 rs4 = *reinterpret_cast<const float4*>(prm + 3 * prm_ld + 4 * jj);
+  const float* hbp = &hb4.x;
+  const float* hsp = &hs4.x;
+  const float* rbp = &rb4.x;
+  const float* rsp = &rs4.x;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (tok[i] < 0) continue;
+    const int rr = 4 * i + rsub;
+    const float4 a4 = *reinterpret_cast<const float4*>(T + rr * 32 + ((jj ^ (rr & 7)) << 2));
+    const float* ap = &a4.x;
+    float4 x4 = xs[i];
+    float* xp = &x4.x;
+    float cb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float contrib = round_bf((ap[j] * wt[i] + hbp[j]) * hsp[j]);
+      cb[j] = contrib;
+      xp[j] = fmaf(xp[j] + rbp[j], rsp[j], contrib);
+    }
+    const size_t off = (size_t)tok[i] * N + col + 4 * jj;
+    *reinterpret_cast<float4*>(p.stream + off) = x4;
+    if (p.tap_f32) *reinterpret_cast<float4*>(p.tap_f32 + off) = x4;
+    if (p.tap_bf16) {
+      uint2 u;
+      u.x = pack_bf2(cb[0], cb[1]);
+      u.y = pack_bf2(cb[2], cb[3]);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.tap_bf16) + off) = u;
+    }
+  }
+  __syncwarp();
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, EPI>;
   constexpr int STAGES = C::STAGES;
   constexpr int BN_OUT = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
@@ -214,7 +293,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
   float* sPrm = reinterpret_cast<float*>(sB + STAGES * C::B_STAGE_BYTES);   // merge params [2][4][BN_OUT]
-  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sPrm) + C::PARAM_BYTES);
+  float* sT = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sPrm) + C::PARAM_BYTES);   // [EW][32][32]
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sT) + C::T_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -359,7 +439,10 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         tmem_ld32(tbase + c, r);
         if constexpr (EPI == EPI_SWIGLU) tmem_ld32(tbase + BN / 2 + c, r2);
         tmem_ld_wait();
-        if (valid) epilogue32<EPI>(p, row, ti.n0 + c, ti.split, r, r2, prm + c, BN_OUT);
+        if constexpr (is_merge<EPI>())
+          merge_chunk<EPI>(p, ti.m0 + q * 32, ti.m_end, ti.n0 + c, r, sT + (warp - 2) * 1024, prm + c, BN_OUT);
+        else if (valid)
+          epilogue32<EPI>(p, row, ti.n0 + c, ti.split, r, r2, prm + c, BN_OUT);
       }
       tc_fence_before();
       __syncwarp();
@@ -395,7 +478,7 @@ EncodeTiledFn get_encode_fn() {
 template <int BN, int EPI>
 int launch_impl(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, int ntiles_hint, int num_sms,
                 cudaStream_t st) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, EPI>;
   auto kern = gemm_tc_kernel<BN, EPI>;
   static bool attr_set = false;
   if (!attr_set) {

@@ -23,9 +23,10 @@ namespace zaya {
 namespace {
 
 constexpr int kTM = 32;          // tokens per router CTA
-constexpr int kThreads = 256;    // 8 warps: warp w -> rows 16*(w&1) .., outputs (w>>1)*R/4 ..
+constexpr int kThreads = 512;    // 16 warps: warp w -> rows 16*(w&1) .., output group w>>1
 constexpr int kRMax = 256;
-constexpr int kZS = kRMax + 8;   // row stride (floats) of the fp32 activation tiles: conflict-free float2 reads
+constexpr int kZS = kRMax + 8;   // row stride (floats) of the fp32 activation tile
+constexpr int kAS = kRMax + 8;   // row stride (bf16) of the hi / lo operand tiles: conflict-free ldmatrix
 
 __device__ __forceinline__ float gelu_exact(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
@@ -40,8 +41,10 @@ struct RouterShape {
   static constexpr int KCH = R < 64 ? R : 64;       // k columns per staged weight chunk
   static constexpr int WS = KCH + 8;                // bf16 row stride of a chunk: conflict-free ldmatrix
   static constexpr int CHUNK = R * WS;              // bf16 elements of one (hi or lo) chunk
-  static constexpr int NTW = R / 32;                // 8-wide n-tiles per warp
-  static constexpr size_t SMEM = sizeof(float) * 2 * kTM * kZS + sizeof(__nv_bfloat16) * 2 * 2 * CHUNK;
+  static constexpr int NG = R / 8 < 8 ? R / 8 : 8;  // output groups (warp pairs)
+  static constexpr int NTW = R / (8 * NG);          // 8-wide n-tiles per warp
+  static constexpr size_t SMEM = sizeof(float) * kTM * kZS + sizeof(__nv_bfloat16) * 2 * kTM * kAS +
+                                 sizeof(__nv_bfloat16) * 2 * 2 * CHUNK;
 };
 
 // Stage columns [kc, kc+KCH) of the split weight (hi and lo, [R][R] bf16) into a padded chunk.
@@ -61,88 +64,88 @@ __device__ __forceinline__ void stage_chunk(__nv_bfloat16* dst, const __nv_bfloa
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// out[t][j] = gelu(sum_k in[t][k] W[j][k] + bias[j]) for the CTA's 32 tokens, on
+// acc[t][j] += sum_{k in chunk c} a[t][k] W[j][k] for the CTA's 32 tokens, on
 // tensor cores (mma.sync m16n8k16) with both operands split into bf16 hi + lo:
-// in.W ~= in_hi.W_hi + in_hi.W_lo + in_lo.W_hi, fp32 accumulation.
+// a.W ~= a_hi.W_hi + a_hi.W_lo + a_lo.W_hi, fp32 accumulation.  ah / al are the
+// activation's hi / lo tiles ([32][kAS]); wh / wl the staged weight chunk.
 template <int R>
-__device__ __forceinline__ void dense_gelu_tc(const float* in, float* out, const __nv_bfloat16* __restrict__ whi,
-                                              const __nv_bfloat16* __restrict__ wlo, const float* __restrict__ bias,
-                                              __nv_bfloat16* wring) {
+__device__ __forceinline__ void mlp_chunk(const __nv_bfloat16* ah_t, const __nv_bfloat16* al_t, float (*acc)[4],
+                                          const __nv_bfloat16* wh, const __nv_bfloat16* wl, int c) {
   using Sh = RouterShape<R>;
   const int warp = warp_id(), lane = lane_id();
   const int rg = warp & 1, ng = warp >> 1;
+  if (ng >= Sh::NG) return;
   const int g = lane >> 2, t = lane & 3;
-  const int nbase = ng * (R / 4);
-  float acc[Sh::NTW][4];
+  const int nbase = ng * (R / Sh::NG);
+  const int arow = rg * 16 + (lane & 15);
+  const int m = lane >> 3;
 #pragma unroll
-  for (int j = 0; j < Sh::NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  constexpr int nch = R / Sh::KCH;
-  stage_chunk<R>(wring, whi, wlo, 0);
-  for (int c = 0; c < nch; ++c) {
-    if (c + 1 < nch) {
-      stage_chunk<R>(wring + ((c + 1) & 1) * 2 * Sh::CHUNK, whi, wlo, (c + 1) * Sh::KCH);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    }
-    __syncthreads();
-    const __nv_bfloat16* wh = wring + (c & 1) * 2 * Sh::CHUNK;
-    const __nv_bfloat16* wl = wh + Sh::CHUNK;
+  for (int ks = 0; ks < Sh::KCH / 16; ++ks) {
+    const int acol = c * Sh::KCH + ks * 16 + (lane >> 4) * 8;
+    uint32_t ah[4], al[4];
+    ldsm_x4(smem_u32(ah_t + arow * kAS + acol), ah[0], ah[1], ah[2], ah[3]);
+    ldsm_x4(smem_u32(al_t + arow * kAS + acol), al[0], al[1], al[2], al[3]);
 #pragma unroll
-    for (int ks = 0; ks < Sh::KCH / 16; ++ks) {
-      const int c0 = c * Sh::KCH + ks * 16 + 2 * t;
-      const int r0 = rg * 16 + g;
-      const float2 v00 = *reinterpret_cast<const float2*>(in + r0 * kZS + c0);
-      const float2 v10 = *reinterpret_cast<const float2*>(in + (r0 + 8) * kZS + c0);
-      const float2 v01 = *reinterpret_cast<const float2*>(in + r0 * kZS + c0 + 8);
-      const float2 v11 = *reinterpret_cast<const float2*>(in + (r0 + 8) * kZS + c0 + 8);
-      float h[8], l[8];
-      split_bf(v00.x, h[0], l[0]); split_bf(v00.y, h[1], l[1]);
-      split_bf(v10.x, h[2], l[2]); split_bf(v10.y, h[3], l[3]);
-      split_bf(v01.x, h[4], l[4]); split_bf(v01.y, h[5], l[5]);
-      split_bf(v11.x, h[6], l[6]); split_bf(v11.y, h[7], l[7]);
-      const uint32_t ah[4] = {pack_bf2(h[0], h[1]), pack_bf2(h[2], h[3]), pack_bf2(h[4], h[5]), pack_bf2(h[6], h[7])};
-      const uint32_t al[4] = {pack_bf2(l[0], l[1]), pack_bf2(l[2], l[3]), pack_bf2(l[4], l[5]), pack_bf2(l[6], l[7])};
-      const int m = lane >> 3;
-#pragma unroll
-      for (int j = 0; j < Sh::NTW; j += 2) {
-        if (j + 1 < Sh::NTW) {
-          const int row = nbase + j * 8 + (m >> 1) * 8 + (lane & 7);
-          const int col = ks * 16 + (m & 1) * 8;
-          uint32_t bh0, bh1, bh2, bh3, bl0, bl1, bl2, bl3;
-          ldsm_x4(smem_u32(wh + row * Sh::WS + col), bh0, bh1, bh2, bh3);
-          ldsm_x4(smem_u32(wl + row * Sh::WS + col), bl0, bl1, bl2, bl3);
-          mma16816(acc[j], ah, bh0, bh1);
-          mma16816(acc[j], ah, bl0, bl1);
-          mma16816(acc[j], al, bh0, bh1);
-          mma16816(acc[j + 1], ah, bh2, bh3);
-          mma16816(acc[j + 1], ah, bl2, bl3);
-          mma16816(acc[j + 1], al, bh2, bh3);
-        } else {   // a single n-tile left: b fragments read directly (two bf16 per 32-bit word)
-          const int row = nbase + j * 8 + g;
-          const int col = ks * 16 + 2 * t;
-          const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(wh + row * Sh::WS + col);
-          const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(wh + row * Sh::WS + col + 8);
-          const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(wl + row * Sh::WS + col);
-          const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(wl + row * Sh::WS + col + 8);
-          mma16816(acc[j], ah, bh0, bh1);
-          mma16816(acc[j], ah, bl0, bl1);
-          mma16816(acc[j], al, bh0, bh1);
-        }
+    for (int j = 0; j < Sh::NTW; j += 2) {
+      if (j + 1 < Sh::NTW) {
+        const int row = nbase + j * 8 + (m >> 1) * 8 + (lane & 7);
+        const int col = ks * 16 + (m & 1) * 8;
+        uint32_t bh0, bh1, bh2, bh3, bl0, bl1, bl2, bl3;
+        ldsm_x4(smem_u32(wh + row * Sh::WS + col), bh0, bh1, bh2, bh3);
+        ldsm_x4(smem_u32(wl + row * Sh::WS + col), bl0, bl1, bl2, bl3);
+        mma16816(acc[j], ah, bh0, bh1);
+        mma16816(acc[j + 1], ah, bh2, bh3);
+        mma16816(acc[j], ah, bl0, bl1);
+        mma16816(acc[j + 1], ah, bl2, bl3);
+        mma16816(acc[j], al, bh0, bh1);
+        mma16816(acc[j + 1], al, bh2, bh3);
+      } else {   // a single n-tile left: b fragments read directly (two bf16 per 32-bit word)
+        const int row = nbase + j * 8 + g;
+        const int col = ks * 16 + 2 * t;
+        const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(wh + row * Sh::WS + col);
+        const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(wh + row * Sh::WS + col + 8);
+        const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(wl + row * Sh::WS + col);
+        const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(wl + row * Sh::WS + col + 8);
+        mma16816(acc[j], ah, bh0, bh1);
+        mma16816(acc[j], ah, bl0, bl1);
+        mma16816(acc[j], al, bh0, bh1);
       }
     }
-    __syncthreads();
   }
-  const int r0 = rg * 16 + g;
+}
+
+// v = gelu(acc + bias) for this thread's outputs; written either as the next
+// layer's hi / lo operand tiles or as fp32.  acc is cleared.
+template <int R>
+__device__ __forceinline__ void mlp_epilogue(float (*acc)[4], const float2* bias, __nv_bfloat16* oh,
+                                             __nv_bfloat16* ol, float* of) {
+  using Sh = RouterShape<R>;
+  const int warp = warp_id(), lane = lane_id();
+  if ((warp >> 1) >= Sh::NG) return;
+  const int r0 = (warp & 1) * 16 + (lane >> 2);
+  const int nbase = (warp >> 1) * (R / Sh::NG);
 #pragma unroll
   for (int j = 0; j < Sh::NTW; ++j) {
-    const int n = nbase + j * 8 + 2 * t;
-    const float b0 = __ldg(bias + n), b1 = __ldg(bias + n + 1);
-    *reinterpret_cast<float2*>(out + r0 * kZS + n) = make_float2(gelu_exact(acc[j][0] + b0), gelu_exact(acc[j][1] + b1));
-    *reinterpret_cast<float2*>(out + (r0 + 8) * kZS + n) =
-        make_float2(gelu_exact(acc[j][2] + b0), gelu_exact(acc[j][3] + b1));
+    const int n = nbase + j * 8 + 2 * (lane & 3);
+    float v[4];
+    v[0] = gelu_exact(acc[j][0] + bias[j].x);
+    v[1] = gelu_exact(acc[j][1] + bias[j].y);
+    v[2] = gelu_exact(acc[j][2] + bias[j].x);
+    v[3] = gelu_exact(acc[j][3] + bias[j].y);
+    if (of) {
+      *reinterpret_cast<float2*>(of + r0 * kZS + n) = make_float2(v[0], v[1]);
+      *reinterpret_cast<float2*>(of + (r0 + 8) * kZS + n) = make_float2(v[2], v[3]);
+    } else {
+      float h[4], l[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) split_bf(v[i], h[i], l[i]);
+      *reinterpret_cast<uint32_t*>(oh + r0 * kAS + n) = pack_bf2(h[0], h[1]);
+      *reinterpret_cast<uint32_t*>(oh + (r0 + 8) * kAS + n) = pack_bf2(h[2], h[3]);
+      *reinterpret_cast<uint32_t*>(ol + r0 * kAS + n) = pack_bf2(l[0], l[1]);
+      *reinterpret_cast<uint32_t*>(ol + (r0 + 8) * kAS + n) = pack_bf2(l[2], l[3]);
+    }
+    acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
   }
-  __syncthreads();
 }
 
 // fc1 / fc2 weights (fp32 [R][R]) -> bf16 hi and lo parts: wsplit = [layer][hi|lo][R][R].
@@ -161,66 +164,145 @@ __global__ void router_split_kernel(const float* __restrict__ fc1, const float* 
 template <int R>
 __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams p) {
   using Sh = RouterShape<R>;
+  constexpr int nch = R / Sh::KCH;
   extern __shared__ __align__(16) float sm[];
-  float* z = sm;                                                              // [kTM][kZS]
-  float* g = z + kTM * kZS;                                                   // [kTM][kZS]
-  __nv_bfloat16* wring = reinterpret_cast<__nv_bfloat16*>(g + kTM * kZS);     // [2 stages][hi|lo][R][WS]
+  float* z = sm;                                                                // fp32 [kTM][kZS]
+  __nv_bfloat16* zh = reinterpret_cast<__nv_bfloat16*>(z + kTM * kZS);          // bf16 hi [kTM][kAS]
+  __nv_bfloat16* zl = zh + kTM * kAS;                                           // bf16 lo [kTM][kAS]
+  __nv_bfloat16* wring = zl + kTM * kAS;                                        // [2 stages][hi|lo][R][WS]
   const int E1 = p.E + 1;
   const int t0 = blockIdx.x * kTM;
   const int warp = warp_id(), lane = lane_id();
+  const size_t n = (size_t)R * R;
+  // weight chunk q of the fc1 -> fc2 sequence into ring stage q & 1 (one cp.async group)
+  auto stage_w = [&](int q) {
+    const __nv_bfloat16* whi = p.wsplit + (size_t)(q / nch) * 2 * n;
+    stage_chunk<R>(wring + (q & 1) * 2 * Sh::CHUNK, whi, whi + n, (q % nch) * Sh::KCH);
+  };
+  stage_w(0);   // the first fc1 chunk streams in under the state assembly
 
-  // router state r = down_proj partial sums (fixed order) + bias (+ previous state * scale);
-  // float4 per thread, every load of a group issued before the adds.
+  // router state r = down_proj partial sums (in slab order) + bias (+ previous
+  // state * scale).  Each thread owns kPos float4 positions; the loads of two
+  // slabs for all of them are issued before any add.
   {
     constexpr int R4 = R / 4;
+    constexpr int kPos = (kTM * R4 + kThreads - 1) / kThreads;
+    const size_t slab = (size_t)p.M * R4;
+    const int ns = p.n_splits;
+    const float4* part = reinterpret_cast<const float4*>(p.part);
+    float4 v[kPos];
+    size_t off[kPos];
+    bool live[kPos], here[kPos];
 #pragma unroll
-    for (int i = threadIdx.x; i < kTM * R4; i += kThreads) {
+    for (int u = 0; u < kPos; ++u) {
+      const int i = threadIdx.x + u * kThreads;
       const int tt = i / R4, k4 = i % R4, t = t0 + tt;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t < p.M) {
-        const float4* pp = reinterpret_cast<const float4*>(p.part) + (size_t)t * R4 + k4;
-        const size_t slab = (size_t)p.M * R4;
-        const int ns = p.n_splits;
-        float4 a[8];
+      here[u] = i < kTM * R4;
+      live[u] = here[u] && t < p.M;
+      off[u] = (size_t)(live[u] ? t : 0) * R4 + k4;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int sp = 0; sp < ns; sp += 2) {
+      float4 a0[kPos], a1[kPos];
 #pragma unroll
-        for (int sp = 0; sp < 8; ++sp) a[sp] = (sp < ns) ? pp[sp * slab] : make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp = 8; sp < ns; ++sp) {   // more than 8 slabs (small M): folded in order
-          const float4 x = pp[sp * slab];
-          a[7].x += x.x; a[7].y += x.y; a[7].z += x.z; a[7].w += x.w;
-        }
-#pragma unroll
-        for (int sp = 0; sp < 8; ++sp) { v.x += a[sp].x; v.y += a[sp].y; v.z += a[sp].z; v.w += a[sp].w; }
-        const float4 bb = __ldg(reinterpret_cast<const float4*>(p.bias) + k4);
-        v.x += bb.x; v.y += bb.y; v.z += bb.z; v.w += bb.w;
-        if (p.prev) {
-          const float4 pv = reinterpret_cast<const float4*>(p.prev)[(size_t)t * R4 + k4];
-          const float4 sc = __ldg(reinterpret_cast<const float4*>(p.prev_scale) + k4);
-          v.x = fmaf(pv.x, sc.x, v.x); v.y = fmaf(pv.y, sc.y, v.y);
-          v.z = fmaf(pv.z, sc.z, v.z); v.w = fmaf(pv.w, sc.w, v.w);
-        }
-        reinterpret_cast<float4*>(p.r_out)[(size_t)t * R4 + k4] = v;
+      for (int u = 0; u < kPos; ++u) {
+        a0[u] = part[sp * slab + off[u]];
+        a1[u] = (sp + 1 < ns) ? part[(sp + 1) * slab + off[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      *reinterpret_cast<float4*>(z + tt * kZS + k4 * 4) = v;
+#pragma unroll
+      for (int u = 0; u < kPos; ++u) {
+        v[u].x += a0[u].x; v[u].y += a0[u].y; v[u].z += a0[u].z; v[u].w += a0[u].w;
+        v[u].x += a1[u].x; v[u].y += a1[u].y; v[u].z += a1[u].z; v[u].w += a1[u].w;
+      }
+    }
+    float4 pv[kPos];
+    if (p.prev) {
+#pragma unroll
+      for (int u = 0; u < kPos; ++u) pv[u] = reinterpret_cast<const float4*>(p.prev)[off[u]];
+    }
+#pragma unroll
+    for (int u = 0; u < kPos; ++u) {
+      const int i = threadIdx.x + u * kThreads;
+      const int tt = i / R4, k4 = i % R4;
+      if (!here[u]) continue;
+      const float4 bb = __ldg(reinterpret_cast<const float4*>(p.bias) + k4);
+      v[u].x += bb.x; v[u].y += bb.y; v[u].z += bb.z; v[u].w += bb.w;
+      if (p.prev) {
+        const float4 sc = __ldg(reinterpret_cast<const float4*>(p.prev_scale) + k4);
+        v[u].x = fmaf(pv[u].x, sc.x, v[u].x); v[u].y = fmaf(pv[u].y, sc.y, v[u].y);
+        v[u].z = fmaf(pv[u].z, sc.z, v[u].z); v[u].w = fmaf(pv[u].w, sc.w, v[u].w);
+      }
+      if (!live[u]) v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      else reinterpret_cast<float4*>(p.r_out)[off[u]] = v[u];
+      *reinterpret_cast<float4*>(z + tt * kZS + k4 * 4) = v[u];
+    }
+  }
+  // fc1 / fc2 bias pairs of this thread's outputs, loaded once
+  float2 b1[Sh::NTW], b2[Sh::NTW];
+  if ((warp >> 1) < Sh::NG) {
+    const int nbase = (warp >> 1) * (R / Sh::NG) + 2 * (lane & 3);
+#pragma unroll
+    for (int j = 0; j < Sh::NTW; ++j) {
+      b1[j] = make_float2(__ldg(p.fc1_b + nbase + j * 8), __ldg(p.fc1_b + nbase + j * 8 + 1));
+      b2[j] = make_float2(__ldg(p.fc2_b + nbase + j * 8), __ldg(p.fc2_b + nbase + j * 8 + 1));
     }
   }
   __syncthreads();
-  for (int tt = warp; tt < kTM; tt += kThreads / 32) {   // router_mlp.norm (RMSNorm over R)
-    float ss = 0.f;
-    for (int k = lane; k < R; k += 32) ss += z[tt * kZS + k] * z[tt * kZS + k];
-    ss = warp_sum(ss);
-    const float inv = rsqrtf(ss / (float)R + p.eps);
-    for (int k = lane; k < R; k += 32) z[tt * kZS + k] = __ldg(p.norm_w + k) * (z[tt * kZS + k] * inv);
+  {  // router_mlp.norm (RMSNorm over R), one warp per token -> fc1's hi / lo operand
+    float nw[R / 32];
+#pragma unroll
+    for (int j = 0; j < R / 32; ++j) nw[j] = __ldg(p.norm_w + lane + 32 * j);
+    for (int tt = warp; tt < kTM; tt += kThreads / 32) {
+      float zr[R / 32], ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < R / 32; ++j) {
+        zr[j] = z[tt * kZS + lane + 32 * j];
+        ss += zr[j] * zr[j];
+      }
+      ss = warp_sum(ss);
+      const float inv = rsqrtf(ss / (float)R + p.eps);
+#pragma unroll
+      for (int j = 0; j < R / 32; ++j) {
+        float h, l;
+        split_bf(nw[j] * (zr[j] * inv), h, l);
+        zh[tt * kAS + lane + 32 * j] = __float2bfloat16_rn(h);
+        zl[tt * kAS + lane + 32 * j] = __float2bfloat16_rn(l);
+      }
+    }
   }
+  // fc1 then fc2 (GELU after each): 2 * nch weight chunks through a two-stage
+  // ring, chunk q + 1 in flight while chunk q is multiplied; out_w follows the
+  // last chunk into the stage that chunk leaves free (or its own region).
+  const bool ow_in_ring = (size_t)E1 * R * sizeof(float) <= 2 * Sh::CHUNK * sizeof(__nv_bfloat16);
+  float* ow = ow_in_ring ? reinterpret_cast<float*>(wring + ((2 * nch) & 1) * 2 * Sh::CHUNK)
+                         : reinterpret_cast<float*>(wring + 4 * Sh::CHUNK);
+  float acc[Sh::NTW][4];
+#pragma unroll
+  for (int j = 0; j < Sh::NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  for (int q = 0; q < 2 * nch; ++q) {
+    if (q + 1 < 2 * nch) {
+      stage_w(q + 1);
+    } else {
+      for (int i = threadIdx.x; i < E1 * R / 4; i += kThreads)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(ow + 4 * i)), "l"(p.out_w + 4 * i)
+                     : "memory");
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncthreads();
+    const __nv_bfloat16* wh = wring + (q & 1) * 2 * Sh::CHUNK;
+    mlp_chunk<R>(zh, zl, acc, wh, wh + Sh::CHUNK, q % nch);
+    if (q == nch - 1) {   // fc1 done: its GELU output becomes fc2's operand (in place)
+      __syncthreads();
+      mlp_epilogue<R>(acc, b1, zh, zl, nullptr);
+    } else if (q == 2 * nch - 1) {
+      mlp_epilogue<R>(acc, b2, nullptr, nullptr, z);
+    }
+    __syncthreads();
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  const size_t n = (size_t)R * R;
-  dense_gelu_tc<R>(z, g, p.wsplit, p.wsplit + n, p.fc1_b, wring);
-  dense_gelu_tc<R>(g, z, p.wsplit + 2 * n, p.wsplit + 3 * n, p.fc2_b, wring);
-  // out_proj (no bias, fp32 on CUDA cores) and the choice, one warp per token;
-  // out_w is staged in shared memory (the weight ring is free now).
-  float* ow = reinterpret_cast<float*>(wring);
-  for (int i = threadIdx.x; i < E1 * R / 4; i += kThreads)
-    reinterpret_cast<float4*>(ow)[i] = __ldg(reinterpret_cast<const float4*>(p.out_w) + i);
-  __syncthreads();
+  // out_proj (no bias, fp32 on CUDA cores) and the choice, one warp per token
   for (int tt = warp; tt < kTM; tt += kThreads / 32) {
     const int t = t0 + tt;
     if (t >= p.M) continue;
@@ -301,8 +383,11 @@ template <int R>
 int launch_router_r(const RouterParams& p, cudaStream_t st) {
   using Sh = RouterShape<R>;
   router_split_kernel<<<64, 256, 0, st>>>(p.fc1_w, p.fc2_w, p.wsplit, R);
-  cudaFuncSetAttribute(router_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::SMEM);
-  router_kernel<R><<<(p.M + kTM - 1) / kTM, kThreads, Sh::SMEM, st>>>(p);
+  const size_t ow_bytes = (size_t)(p.E + 1) * R * sizeof(float);
+  const size_t smem = Sh::SMEM + (ow_bytes <= 2 * Sh::CHUNK * sizeof(__nv_bfloat16) ? 0 : ow_bytes);
+  if (smem > 227 * 1024) return ZAYA_ERR_UNSUPPORTED;
+  cudaFuncSetAttribute(router_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  router_kernel<R><<<(p.M + kTM - 1) / kTM, kThreads, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 

@@ -186,20 +186,22 @@ inline T* at(void* base, size_t off) {
 // Tile width with the least per-SM work: waves(BN) x BN, where waves is the
 // number of rounds of tiles over the SMs; ties go to the wider tile (less
 // operand traffic per FLOP).  m_tiles is the number of 128-row tiles.
+// Tile width for a persistent GEMM.  128-wide tiles measured fastest for the
+// block's prefill contractions (q/k/v, o_proj + merge, expert down + merge:
+// against 256 they trade a little operand reuse for a deeper TMA ring, twice
+// the tiles to balance and half the exposed epilogue); when 128-wide tiles
+// do not give every SM a tile (decode-sized M), the narrowest candidate does
+// the most to spread the weight stream over the SMs.
 int pick_bn_tiles(long m_tiles, int N, const int* cands, int n, int sms) {
-  int best = 0;
-  long best_cost = 0;
+  bool has128 = false;
+  int narrow = 0;
   for (int i = 0; i < n; ++i) {
-    const int bn = cands[i];
-    if (N % bn) continue;
-    const long tiles = m_tiles * (N / bn);
-    const long cost = ((tiles + sms - 1) / sms) * bn;
-    if (!best || cost < best_cost) {
-      best = bn;
-      best_cost = cost;
-    }
+    if (N % cands[i]) continue;
+    if (cands[i] == 128) has128 = true;
+    if (!narrow || cands[i] < narrow) narrow = cands[i];
   }
-  return best;
+  if (has128 && m_tiles * (N / 128) >= sms) return 128;
+  return narrow;
 }
 int pick_bn(int M, int N, const int* cands, int n, int sms) {
   return pick_bn_tiles((M + 127) / 128, N, cands, n, sms);
@@ -300,7 +302,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
 int check_state(const zaya_block_state* s, int need_cap) {
   if (!s || !s->k_cache || !s->v_cache || !s->cache_len || !s->conv_state || !s->prev_hs) return ZAYA_ERR_INVALID_ARG;
   if (s->cache_cap < need_cap) return ZAYA_ERR_INVALID_ARG;
-  if (!a16(s->k_cache) || !a16(s->v_cache)) return ZAYA_ERR_MISALIGNED;
+  if (!a16(s->k_cache) || !a16(s->v_cache) || !a16(s->conv_state) || !a16(s->prev_hs)) return ZAYA_ERR_MISALIGNED;
   return ZAYA_OK;
 }
 
@@ -313,6 +315,7 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
   if (block_idx < 0 || (block_idx > 0 && !rin) || rin == rout) return ZAYA_ERR_INVALID_ARG;
   ZAYA_TRY(check_state(state, S));
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) || !a16(hidden) || !a16(rout)) return ZAYA_ERR_MISALIGNED;
+  if (taps && taps->attention_queries && !a16(taps->attention_queries)) return ZAYA_ERR_MISALIGNED;
   const zaya_config& c = *cfg;
   const Derived d = derive(c);
   const Ws L = plan(c, ZAYA_PREFILL, B, S);
@@ -365,6 +368,7 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
   if (block_idx < 0 || (block_idx > 0 && !rin) || rin == rout) return ZAYA_ERR_INVALID_ARG;
   ZAYA_TRY(check_state(state, 1));
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) || !a16(hidden) || !a16(rout)) return ZAYA_ERR_MISALIGNED;
+  if (taps && taps->attention_queries && !a16(taps->attention_queries)) return ZAYA_ERR_MISALIGNED;
   const zaya_config& c = *cfg;
   const Derived d = derive(c);
   const Ws L = plan(c, ZAYA_DECODE, B, 1);
