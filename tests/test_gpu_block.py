@@ -54,6 +54,18 @@ def test_tiny_padding():
     Hn.assert_block_ok(res)
 
 
+def test_tiny_split_kv_attention():
+    """Long causal rows against a short launch: the attention cuts the longest
+    row tiles into key chunks and merges their partials (B2 x S1000, window
+    1024, a ragged last tile and left padding)."""
+    from tests import harness as Hn
+    cfg = get_config("tiny").with_(batch=2, seq=1000, window=1024, pad_max=100)
+    res = _run_prefill(cfg)
+    Hn.assert_block_ok(res)
+    for key in ("attention_queries", "attention_output"):
+        assert res[key]["bf16_ok"], (key, res[key])
+
+
 def test_full_prefill_4k():
     """Full-width block, B1 x S4096 (the benchmark workload)."""
     from tests import harness as Hn

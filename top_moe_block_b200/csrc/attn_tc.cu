@@ -24,6 +24,16 @@
 // Only key tiles that intersect the window are visited; per-element masks
 // only on tiles that straddle the diagonal, the window edge, the sequence
 // end or a padding mask.
+// Balance: causal rows differ in length (row tile i of a short sequence sees
+// i+1 key tiles), so when the longest row tile holds more key tiles than an
+// SM's share of the whole launch, row tiles are cut into key chunks of at
+// most that share.  The host lists the (row tile, chunk, head pair,
+// sequence) items longest first; a chunk writes its unnormalised O with its
+// running max and sum (fp32), and the last chunk of a row tile to finish
+// (a per-row-tile counter) merges all chunks in chunk order:
+// O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c, M = max_c m_c.
+#include <algorithm>
+#include <vector>
 #include <math.h>
 
 #include "common.cuh"
@@ -38,6 +48,92 @@ constexpr int kKT = 64;   // keys per tile
 constexpr int kHPC = 2;   // query heads per CTA (sharing one kv head)
 constexpr int kRing = 3;  // K and V ring depth
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kMaxItems = 512;   // split-plan items carried in the kernel parameters
+constexpr int kPlanSms = 148;    // the SM count the split plan balances over
+constexpr int kMinChunk = 8;     // fewest key tiles in a chunk
+
+struct AttnItems {
+  int n_items;   // 0: grid (row tiles, head pairs, sequences), no row tile split
+  float* po;     // partial O, per slot [kHPC][d][kQT] fp32 (row index fastest)
+  float* pml;    // per slot [kHPC][2][kQT] fp32: running max (log2 units), running sum
+  int* ctr;      // per split (row tile, head pair, sequence): chunks finished
+  uint4 it[kMaxItems];   // {rt | c << 16 | nc << 24, b | hp << 16, first slot of the group, counter}
+};
+
+// Key tiles of row tile rt (the same arithmetic as the kernel's).
+inline int host_row_tiles(int rt, int S, int window) {
+  const int m0 = rt * kQT;
+  const int lo = std::max(0, m0 - window + 1);
+  const int n_begin = (lo / kKT) * kKT;
+  const int n_end = std::min(S, m0 + kQT);
+  return (n_end - n_begin + kKT - 1) / kKT;
+}
+
+// The split plan: fills `items` (when non-null) and the slot / counter counts.
+// Returns false when no row tile is split.
+bool plan_split(int B, int S, int window, int n_hp, AttnItems* items, int* n_slots, int* n_ctr) {
+  *n_slots = 0;
+  *n_ctr = 0;
+  if (items) items->n_items = 0;
+  const int n_rt = (S + kQT - 1) / kQT;
+  long total = 0;
+  int maxnt = 0;
+  for (int rt = 0; rt < n_rt; ++rt) {
+    const int nt = host_row_tiles(rt, S, window);
+    total += nt;
+    maxnt = std::max(maxnt, nt);
+  }
+  total *= (long)B * n_hp;
+  const double share = (double)total / kPlanSms;
+  if (maxnt <= share) return false;
+  // chunks of about one SM's share: the in-order CTA dispatch then pairs the
+  // first round's long items with the second round's short ones
+  for (int L = std::max(kMinChunk, (int)(share + 0.999)); L < maxnt; L *= 2) {
+    long n_items = 0, slots = 0, ctrs = 0;
+    bool fits = true;
+    for (int rt = 0; rt < n_rt && fits; ++rt) {
+      const int nc = (host_row_tiles(rt, S, window) + L - 1) / L;
+      if (nc > 255) fits = false;
+      n_items += (long)nc * n_hp * B;
+      if (nc > 1) {
+        slots += (long)nc * n_hp * B;
+        ctrs += (long)n_hp * B;
+      }
+    }
+    if (!fits || n_items > kMaxItems || B > 0xffff || n_hp > 0xffff || n_rt > 0xffff) continue;
+    *n_slots = (int)slots;
+    *n_ctr = (int)ctrs;
+    if (items) {
+      struct It { int size; uint4 v; };
+      std::vector<It> v;
+      int slot = 0, ctr = 0;
+      for (int rt = n_rt - 1; rt >= 0; --rt) {
+        const int nt = host_row_tiles(rt, S, window);
+        const int nc = (nt + L - 1) / L;
+        for (int hp = 0; hp < n_hp; ++hp)
+          for (int b = 0; b < B; ++b) {
+            const int s0 = slot, c0 = ctr;
+            if (nc > 1) {
+              slot += nc;
+              ++ctr;
+            }
+            for (int c = 0; c < nc; ++c) {
+              const int size = (c + 1) * nt / nc - c * nt / nc;
+              v.push_back({size, make_uint4((uint32_t)rt | ((uint32_t)c << 16) | ((uint32_t)nc << 24),
+                                            (uint32_t)b | ((uint32_t)hp << 16), (uint32_t)s0, (uint32_t)c0)});
+            }
+          }
+      }
+      std::stable_sort(v.begin(), v.end(), [](const It& a, const It& b) { return a.size > b.size; });
+      items->n_items = (int)v.size();
+      for (size_t i = 0; i < v.size(); ++i) items->it[i] = v[i].v;
+    }
+    return true;
+  }
+  return false;
+}
+
+size_t slot_bytes(int d) { return (size_t)kHPC * d * kQT * 4 + (size_t)kHPC * 2 * kQT * 4; }
 
 template <int D>
 struct AttnTc {
@@ -72,7 +168,8 @@ __device__ __forceinline__ bool key_visible(int q, int key, int window, int S, c
 template <int D>
 __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const AttnParams p, int* status) {
+                   const __grid_constant__ CUtensorMap tmV, const AttnParams p,
+                   const __grid_constant__ AttnItems items, int* status) {
   using C = AttnTc<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -91,16 +188,34 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
   uint64_t* p_full = s_free + 2 * kHPC;         // [kHPC][2]
   uint64_t* pv_done = p_full + 2 * kHPC;        // [kHPC][2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2 * kHPC);
+  int* s_last = reinterpret_cast<int*>(tmem_slot + 1);
 
-  const int qb = gridDim.x - 1 - blockIdx.x;   // heaviest (latest) query tiles first
-  const int h0 = blockIdx.y * kHPC, b = blockIdx.z;
+  // this CTA's item: a row tile of two heads, or one key chunk of it
+  int qb, hp, b, chunk = 0, n_chunks = 1, slot0 = 0, ctr = 0;
+  if (items.n_items) {
+    const uint4 it = items.it[blockIdx.x];
+    qb = (int)(it.x & 0xffff);
+    chunk = (int)((it.x >> 16) & 0xff);
+    n_chunks = (int)(it.x >> 24);
+    b = (int)(it.y & 0xffff);
+    hp = (int)(it.y >> 16);
+    slot0 = (int)it.z;
+    ctr = (int)it.w;
+  } else {
+    qb = gridDim.x - 1 - blockIdx.x;   // heaviest (latest) query tiles first
+    hp = blockIdx.y;
+    b = blockIdx.z;
+  }
+  const int h0 = hp * kHPC;
   const int g = h0 / (p.n_q / p.n_kv);
   const int m0 = qb * kQT;
   const int S = p.S;
   const int lo = max(0, m0 - p.window + 1);
   const int n_begin = (lo / kKT) * kKT;
   const int n_end = min(S, m0 + kQT);
-  const int n_tiles = (n_end - n_begin + kKT - 1) / kKT;
+  const int n_row_tiles = (n_end - n_begin + kKT - 1) / kKT;
+  const int t_begin = chunk * n_row_tiles / n_chunks;
+  const int n_tiles = (chunk + 1) * n_row_tiles / n_chunks - t_begin;   // key tiles of this item
   const int warp = warp_id(), lane = lane_id();
 
   if (warp == 0 && lane == 0) {
@@ -132,7 +247,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
   if (warp == 0) {
     // ---------------- TMA producer: both heads' Q once, then K(j) and V(j) into their rings
     if (elect_one()) {
-      const int kv_row = (b * p.n_kv + g) * p.cap + n_begin;
+      const int kv_row = (b * p.n_kv + g) * p.cap + n_begin + t_begin * kKT;
       mbar_arrive_expect_tx(q_full, kHPC * C::Q_BYTES);
 #pragma unroll
       for (int x = 0; x < kHPC; ++x) {
@@ -229,7 +344,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
         break;
       }
       tc_fence_after();
-      const int key0 = n_begin + j * kKT;
+      const int key0 = n_begin + (t_begin + j) * kKT;
       const bool full_vis = !mask && key0 + kKT - 1 <= m0 && (m0 + kQT - 1 - key0) < p.window && key0 + kKT <= S;
       uint32_t r[2][32];
       tmem_ld32(tl + buf * kKT, r[0]);
@@ -307,27 +422,87 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&my_p_full[buf]);
     }
-    if (ok && n_tiles > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&my_pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, status))) {
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int ld = p.n_q * D;
-      auto* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * S + q) * ld + (h0 + x) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tl + C::O_COL + c * 32, o);
-        tmem_ld_wait();
-        if (q < S) {
+    const bool have = ok && n_tiles > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&my_pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, status));
+    const int ld = p.n_q * D;
+    auto* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * S + q) * ld + (h0 + x) * D;
+    // this row's 32 output columns [c, c + 32), scaled, as bf16
+    auto store32 = [&](int c, const float* v, float sc) {
+      if (q >= S) return;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 vv;
-            vv.x = pack_bf2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
-            vv.y = pack_bf2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
-            vv.z = pack_bf2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
-            vv.w = pack_bf2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
-            reinterpret_cast<uint4*>(out + c * 32)[u] = vv;
+      for (int u = 0; u < 4; ++u) {
+        uint4 vv;
+        vv.x = pack_bf2(v[8 * u + 0] * sc, v[8 * u + 1] * sc);
+        vv.y = pack_bf2(v[8 * u + 2] * sc, v[8 * u + 3] * sc);
+        vv.z = pack_bf2(v[8 * u + 4] * sc, v[8 * u + 5] * sc);
+        vv.w = pack_bf2(v[8 * u + 6] * sc, v[8 * u + 7] * sc);
+        reinterpret_cast<uint4*>(out + c)[u] = vv;
+      }
+    };
+    if (n_chunks == 1) {
+      if (have) {
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tl + C::O_COL + c * 32, o);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]);
+          store32(c * 32, v, inv);
+        }
+      }
+    } else {
+      // unnormalised partial of this key chunk: O transposed (row fastest, so a
+      // warp's stores are contiguous), running max and sum
+      float* po = items.po + ((size_t)(slot0 + chunk) * kHPC + x) * D * kQT;
+      float* pml = items.pml + ((size_t)(slot0 + chunk) * kHPC + x) * 2 * kQT;
+      if (have) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tl + C::O_COL + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) po[(size_t)(c * 32 + i) * kQT + row] = __uint_as_float(o[i]);
+        }
+        pml[row] = m_used;
+        pml[kQT + row] = l;
+      }
+      __threadfence();
+      named_barrier_sync(1, 32 * 4 * kHPC);
+      if (warp == 2 && lane == 0) *s_last = (atomicAdd(items.ctr + ctr, 1) == n_chunks - 1);
+      named_barrier_sync(1, 32 * 4 * kHPC);
+      if (*s_last) {   // every chunk of this row tile is written: merge in chunk order
+        __threadfence();
+        auto ml = [&](int cc, int which) {
+          return __ldcg(items.pml + ((size_t)(slot0 + cc) * kHPC + x) * 2 * kQT + which * kQT + row);
+        };
+        float M = -INFINITY;
+        for (int cc = 0; cc < n_chunks; ++cc) M = fmaxf(M, ml(cc, 0));
+        float Ls = 0.f;
+        for (int cc = 0; cc < n_chunks; ++cc) {
+          const float mc = ml(cc, 0);
+          if (mc != -INFINITY) Ls += exp2f(mc - M) * ml(cc, 1);
+        }
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float acc[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+          for (int cc = 0; cc < n_chunks; ++cc) {
+            const float mc = ml(cc, 0);
+            if (mc == -INFINITY) continue;
+            const float w = exp2f(mc - M);
+            const float* pc = items.po + ((size_t)(slot0 + cc) * kHPC + x) * D * kQT + (size_t)c * 32 * kQT + row;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, __ldcg(pc + (size_t)i * kQT), acc[i]);
           }
+          store32(c * 32, acc, inv);
         }
       }
     }
@@ -344,16 +519,38 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
 
 }  // namespace
 
+size_t attn_prefill_ws_bytes(int B, int S, int window, int n_q, int n_kv, int d) {
+  if (B <= 0 || S <= 0 || n_q % kHPC) return 0;
+  int n_slots = 0, n_ctr = 0;
+  if (!plan_split(B, S, window, n_q / kHPC, nullptr, &n_slots, &n_ctr)) return 0;
+  return (size_t)n_slots * slot_bytes(d) + (size_t)n_ctr * 4;
+}
+
 int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
   if (p.B <= 0 || p.S <= 0) return ZAYA_OK;
   if (p.d != 128 && p.d != 64) return ZAYA_ERR_UNSUPPORTED;
+  if (p.n_q % kHPC || (p.n_q / p.n_kv) % kHPC) return ZAYA_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
   int rc = make_tmap_bf16(&mq, p.q, (uint64_t)p.B * p.n_q * p.S, (uint64_t)p.d, 128);
   if (!rc) rc = make_tmap_bf16(&mk, p.k_cache, (uint64_t)p.B * p.n_kv * p.cap, (uint64_t)p.d, kKT);
   if (!rc) rc = make_tmap_bf16(&mv, p.v_cache, (uint64_t)p.B * p.n_kv * p.cap, (uint64_t)p.d, kKT);
   if (rc) return rc;
-  if (p.n_q % kHPC || (p.n_q / p.n_kv) % kHPC) return ZAYA_ERR_UNSUPPORTED;
-  const dim3 grid((p.S + kQT - 1) / kQT, p.n_q / kHPC, p.B);
+  AttnItems items;   // the kernel's item parameter (8 KB, copied at launch)
+  int n_slots = 0, n_ctr = 0;
+  dim3 grid((p.S + kQT - 1) / kQT, p.n_q / kHPC, p.B);
+  if (plan_split(p.B, p.S, p.window, p.n_q / kHPC, &items, &n_slots, &n_ctr)) {
+    const size_t need = (size_t)n_slots * slot_bytes(p.d) + (size_t)n_ctr * 4;
+    if (!p.part || p.part_bytes < need) return ZAYA_ERR_WORKSPACE;
+    items.po = static_cast<float*>(p.part);
+    items.pml = items.po + (size_t)n_slots * kHPC * p.d * kQT;
+    items.ctr = reinterpret_cast<int*>(items.pml + (size_t)n_slots * kHPC * 2 * kQT);
+    if (cudaMemsetAsync(items.ctr, 0, (size_t)n_ctr * 4, st) != cudaSuccess) return ZAYA_ERR_CUDA;
+    grid = dim3(items.n_items, 1, 1);
+  } else {
+    items.n_items = 0;
+    items.po = items.pml = nullptr;
+    items.ctr = nullptr;
+  }
   if (p.d == 128) {
     auto kern = attn_tc_kernel<128>;
     static bool set = false;
@@ -361,7 +558,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTc<128>::SMEM);
       set = true;
     }
-    kern<<<grid, 64 + 32 * 4 * kHPC, AttnTc<128>::SMEM, st>>>(mq, mk, mv, p, status);
+    kern<<<grid, 64 + 32 * 4 * kHPC, AttnTc<128>::SMEM, st>>>(mq, mk, mv, p, items, status);
   } else {
     auto kern = attn_tc_kernel<64>;
     static bool set = false;
@@ -369,7 +566,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTc<64>::SMEM);
       set = true;
     }
-    kern<<<grid, 64 + 32 * 4 * kHPC, AttnTc<64>::SMEM, st>>>(mq, mk, mv, p, status);
+    kern<<<grid, 64 + 32 * 4 * kHPC, AttnTc<64>::SMEM, st>>>(mq, mk, mv, p, items, status);
   }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }

@@ -104,7 +104,11 @@ struct AttnParams {
   void* out;              // bf16 premix [B*S, n_q*d]
   int B, S, cap, n_q, n_kv, d, window;
   float scale;
+  void* part;             // split-KV partials + merge counters (attn_prefill_ws_bytes)
+  size_t part_bytes;
 };
+// Workspace bytes of the split-KV plan for these sizes (0 when no row tile is split).
+size_t attn_prefill_ws_bytes(int B, int S, int window, int n_q, int n_kv, int d);
 int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st);
 
 struct DecodeAttnParams {

@@ -171,7 +171,8 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.mt_start = o; o += up((size_t)(d.E + 2) * 4);
   w.xperm = o; o += up(M * d.H * 2);
   w.act = o; o += up(M * d.I * 2);
-  w.part = o; o += up(mode == ZAYA_DECODE ? decode_attn_ws_bytes(B, d.nq, d.d, c.window) : 0);
+  w.part = o; o += up(mode == ZAYA_DECODE ? decode_attn_ws_bytes(B, d.nq, d.d, c.window)
+                                           : attn_prefill_ws_bytes(B, S, c.window, d.nq, d.nkv, d.d));
   w.rpart = o; o += up((size_t)router_down_splits((int)M, d.H) * M * d.R * 4);
   w.wsplit = o; o += up((size_t)4 * d.R * d.R * 2);
   w.total = o;
@@ -183,9 +184,6 @@ inline T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
 }
 
-// Tile width with the least per-SM work: waves(BN) x BN, where waves is the
-// number of rounds of tiles over the SMs; ties go to the wider tile (less
-// operand traffic per FLOP).  m_tiles is the number of 128-row tiles.
 // Tile width for a persistent GEMM.  128-wide tiles measured fastest for the
 // block's prefill contractions (q/k/v, o_proj + merge, expert down + merge:
 // against 256 they trade a little operand reuse for a deeper TMA ring, twice
@@ -354,6 +352,8 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     p.out = at<void>(ws, L.premix);
     p.B = B; p.S = S; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = c.window;
     p.scale = d.scale;
+    p.part = at<void>(ws, L.part);
+    p.part_bytes = attn_prefill_ws_bytes(B, S, c.window, d.nq, d.nkv, d.d);
     ZAYA_STAGE("attention", 1, launch_attn_prefill_tc(p, status, st));
   }
   return block_tail(c, d, w, block_idx, M, hidden, rin, rout, taps, ws, L, nullptr, mask, sms, st);
