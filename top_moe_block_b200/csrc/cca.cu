@@ -407,12 +407,15 @@ __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
 
 // Prefill, streaming form: a thread owns 8 consecutive channels of one q/k
 // head (the d/8 threads of a head are adjacent lanes, so the head norm and the
-// RoPE pair exchange are shuffles inside that lane group) and walks the CTA's
-// kStream tokens in order, with its conv taps and bias in registers and the
-// two previous pre-conv values carried from step to step.  Value heads: d/8
-// threads per kv head copy the current / delayed halves.  Needs rot % 16 == 0
-// (a thread's 8 dims are all inside or all outside the rotated range).
-constexpr int kStream = 16;
+// RoPE pair exchange are shuffles inside that lane group) and walks kPerGroup
+// consecutive tokens, with its conv taps and bias in registers and the two
+// previous pre-conv values carried from step to step; kGroups such thread
+// groups split the CTA's kStream staged tokens.  Value heads: d/8 threads per
+// kv head copy the current / delayed halves.  Needs rot % 16 == 0 (a thread's
+// 8 dims are all inside or all outside the rotated range).
+constexpr int kGroups = 4;
+constexpr int kPerGroup = 7;
+constexpr int kStream = kGroups * kPerGroup;   // 28 tokens: S = 4096 fills the 148 SMs in one round
 
 __device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&y)[8]) {
   const uint4 v = *reinterpret_cast<const uint4*>(src);
@@ -424,7 +427,7 @@ __device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__ CcaParams p) {
+__global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constant__ CcaParams p) {
   constexpr int LPH = D / 8;   // threads per head
   extern __shared__ __align__(16) uint8_t sm[];
   const int nq = p.n_q, nkv = p.n_kv, rep = nq / nkv;
@@ -435,6 +438,7 @@ __global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__
   const int half = p.rot / 2;
   auto* u = reinterpret_cast<__nv_bfloat16*>(sm);                                 // [kStream + 2][ld]
   float2* cs = reinterpret_cast<float2*>(sm + (size_t)(kStream + 2) * ld * 2);    // [kStream][half]
+  float* cbias = reinterpret_cast<float*>(cs + kStream * half);                    // [C]
   const auto* qkv = static_cast<const __nv_bfloat16*>(p.qkv);
   const size_t row0 = (size_t)b * p.S;
 
@@ -456,12 +460,17 @@ __global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__
     sincosf((float)(s0 + tt) * p.inv_freq[f], &sn, &c);
     cs[i] = make_float2(c, sn);
   }
-  const int tid = threadIdx.x, lane = lane_id();
+  const int gthreads = blockDim.x / kGroups;              // a multiple of 32
+  const int grp = threadIdx.x / gthreads, tid = threadIdx.x % gthreads, lane = lane_id();
+  const int tt0 = grp * kPerGroup;                        // this group's first token
   const int n_qk = (nq + nkv) * LPH;
   // conv taps / bias of this thread's channels, loaded under the staging
-  float w0[8], w1[8], w2[8], bb[8];
+  float w0[8], w1[8], w2[8];
   const int head = tid / LPH, l = tid % LPH;
   const int cb = head * D + l * 8;
+  if (grp == 0)   // conv bias of the q||k channels, shared by the groups
+    for (int i = tid; i < C / 4; i += gthreads)
+      reinterpret_cast<float4*>(cbias)[i] = __ldg(reinterpret_cast<const float4*>(p.conv_b) + i);
   if (tid < n_qk) {
     const float4* wp = reinterpret_cast<const float4*>(p.conv_w + 3 * cb);
     float wv[24];
@@ -472,9 +481,6 @@ __global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) { w0[i] = wv[3 * i]; w1[i] = wv[3 * i + 1]; w2[i] = wv[3 * i + 2]; }
-    const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.conv_b + cb));
-    const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.conv_b + cb) + 1);
-    bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w; bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
@@ -485,26 +491,31 @@ __global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__
     const int g = is_q ? head / rep : hh;
     const unsigned gmask = ((1u << LPH) - 1u) << (lane & ~(LPH - 1));   // this head's lanes
     const float scl0 = sqrtf((float)D) * (is_q ? 1.f : __ldg(p.k_temp + g));
+    const float inv_rep = 1.0f / (float)rep;
+    const float eps2 = p.eps * p.eps, inv_eps = 1.0f / p.eps;
     const int j0 = l * 8;
     const bool in_rot = j0 < p.rot, lo = j0 < half;
     const int src_lane = in_rot ? (lo ? lane + half / 8 : lane - half / 8) : lane;
     const int f0 = lo ? j0 : j0 - half;
     const int kcb = nq * D + g * D + l * 8;   // the group's key channels (query residual)
     float x2[8], x1[8];
-    load8(u + cb, x2);
-    load8(u + ld + cb, x1);
+    load8(u + (size_t)tt0 * ld + cb, x2);
+    load8(u + (size_t)(tt0 + 1) * ld + cb, x1);
     __nv_bfloat16* dst = is_q ? static_cast<__nv_bfloat16*>(p.q_out) + (((size_t)b * nq + hh) * p.S + s0) * D + j0
                               : static_cast<__nv_bfloat16*>(p.k_cache) + (((size_t)b * nkv + hh) * p.cache_cap + s0) * D + j0;
     __nv_bfloat16* tap = (is_q && p.tap_q)
                              ? static_cast<__nv_bfloat16*>(p.tap_q) + (((size_t)b * nq + hh) * p.S + s0) * D + j0
                              : nullptr;
-#pragma unroll 2
-    for (int tt = 0; tt < kStream; ++tt) {
+#pragma unroll 1
+    for (int tt = tt0; tt < tt0 + kPerGroup; ++tt) {
       const int s = s0 + tt;
       if (s >= p.S) break;   // uniform over the head's lanes
       const __nv_bfloat16* row = u + (size_t)(tt + 2) * ld;
       float x0[8], y[8];
       load8(row + cb, x0);
+      const float4 bb0 = reinterpret_cast<const float4*>(cbias + cb)[0];
+      const float4 bb1 = reinterpret_cast<const float4*>(cbias + cb)[1];
+      const float bb[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float acc = bb[i];
@@ -528,7 +539,7 @@ __global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__
             for (int i = 0; i < 8; ++i) qs[i] += qh[i];
           }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) y[i] += 0.5f * (qs[i] / (float)rep + x0[i]);
+          for (int i = 0; i < 8; ++i) y[i] += 0.5f * (qs[i] * inv_rep + x0[i]);
         }
       }
       float ss = 0.f;
@@ -536,25 +547,21 @@ __global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__
       for (int i = 0; i < 8; ++i) ss = fmaf(y[i], y[i], ss);
 #pragma unroll
       for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gmask, ss, o);
-      const float scl = scl0 / fmaxf(sqrtf(ss), p.eps);
+      const float scl = scl0 * (ss > eps2 ? rsqrtf(ss) : inv_eps);   // sqrt(d) / max(|y|, eps)
 #pragma unroll
       for (int i = 0; i < 8; ++i) y[i] *= scl;
       if (half > 0) {   // rotate-half over dims [0, rot)
-        float pt[8];
+        // pair by pair: both lanes of a pair read each other's value before either writes
+        const float4* e4 = reinterpret_cast<const float4*>(cs + tt * half + (in_rot ? f0 : 0));
+        const float sgn = lo ? -1.f : 1.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) pt[i] = __shfl_sync(gmask, y[i], src_lane);
-        if (in_rot) {
-          const float4* e4 = reinterpret_cast<const float4*>(cs + tt * half + f0);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4; ++i) {
+          const float pa = __shfl_sync(gmask, y[2 * i], src_lane);
+          const float pb = __shfl_sync(gmask, y[2 * i + 1], src_lane);
+          if (in_rot) {
             const float4 e = e4[i];   // (cos, sin) of dims 2i and 2i + 1
-            if (lo) {
-              y[2 * i] = y[2 * i] * e.x - pt[2 * i] * e.y;
-              y[2 * i + 1] = y[2 * i + 1] * e.z - pt[2 * i + 1] * e.w;
-            } else {
-              y[2 * i] = y[2 * i] * e.x + pt[2 * i] * e.y;
-              y[2 * i + 1] = y[2 * i + 1] * e.z + pt[2 * i + 1] * e.w;
-            }
+            y[2 * i] = fmaf(sgn * pa, e.y, y[2 * i] * e.x);
+            y[2 * i + 1] = fmaf(sgn * pb, e.w, y[2 * i + 1] * e.z);
           }
         }
       }
@@ -579,7 +586,7 @@ __global__ void __launch_bounds__(256) cca_stream_kernel(const __grid_constant__
     const int vc0 = nq * D + nkv * D;          // current halves
     const int vd0 = vc0 + nkv * (D / 2);       // delayed halves (from token t-1)
     auto* dst = static_cast<__nv_bfloat16*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + s0) * D + j0;
-    for (int tt = 0; tt < kStream; ++tt) {
+    for (int tt = tt0; tt < tt0 + kPerGroup; ++tt) {
       const int s = s0 + tt;
       if (s >= p.S) break;
       const __nv_bfloat16* row = u + (size_t)(tt + 2) * ld;
@@ -605,9 +612,10 @@ int launch_cca(const CcaParams& p, cudaStream_t st) {
   if (threads > 1024 || p.rot / 2 > 64 || p.n_qkv % 8) return ZAYA_ERR_UNSUPPORTED;
   if (!p.decode && (p.d == 128 || p.d == 64) && p.rot % 16 == 0 && p.H % 8 == 0) {
     const int lph = p.d / 8;
-    const int nthr = ((p.n_q + 2 * p.n_kv) * lph + 31) / 32 * 32;
-    const size_t smem = (size_t)(kStream + 2) * p.n_qkv * 2 + (size_t)kStream * (p.rot / 2) * 8;
-    if (nthr <= 256 && smem <= 227 * 1024) {
+    const int nthr = kGroups * (((p.n_q + 2 * p.n_kv) * lph + 31) / 32 * 32);
+    const size_t smem = (size_t)(kStream + 2) * p.n_qkv * 2 + (size_t)kStream * (p.rot / 2) * 8 +
+                        (size_t)(p.n_q + p.n_kv) * p.d * 4;
+    if (nthr <= 768 && smem <= 227 * 1024) {
       const dim3 grid((p.S + kStream - 1) / kStream, p.B);
       if (p.d == 128) {
         cudaFuncSetAttribute(cca_stream_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -50,16 +50,16 @@ constexpr int kPrefetchAhead = 8;  // k-blocks of B pulled into L2 ahead of thei
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA (227 KB)
 
-template <int BN, int EPI>
+template <int BN, int EPI, int CG = 1>
 struct GemmCfg {
-  static constexpr int B_STAGE_BYTES = BN * BK * 2;
+  static constexpr int B_STAGE_BYTES = BN / CG * BK * 2;   // a CTA pair splits B's columns
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
-  static constexpr int PARAM_BYTES = 2 * 4 * BN * 4;  // merge epilogues: [2 tiles][hb,hs,rb,rs][BN] fp32
+  static constexpr int PARAM_BYTES = is_merge<EPI>() ? 2 * 4 * BN * 4 : 0;  // merge: [2 tiles][hb,hs,rb,rs][BN] fp32
   // merge epilogues: a 32 x 32 fp32 transpose buffer per epilogue warp
   static constexpr int T_BYTES = is_merge<EPI>() ? epi_warps<EPI>() * 32 * 32 * 4 : 0;
   static constexpr int FIXED = PARAM_BYTES + T_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static constexpr int DEF_STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);  // ~192 KB ring
+  static constexpr int DEF_STAGES = (STAGE_BYTES >= 49152) ? 4 : (STAGE_BYTES >= 32768 ? 6 : 8);  // ~192 KB ring
   static constexpr int FIT_STAGES = (kSmemLimit - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = DEF_STAGES < FIT_STAGES ? DEF_STAGES : FIT_STAGES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED;
@@ -77,15 +77,15 @@ struct TileInfo {
   int b_row2;  // SWIGLU: first up row
 };
 
-template <int EPI, int BN_OUT>
+template <int EPI, int BN_OUT, int TM>   // TM: output rows per tile (128, or 256 for a CTA pair)
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
   const int nt = p.N / BN_OUT;
   const int ks = p.k_splits > 1 ? p.k_splits : 1;
-  if (!p.grouped) return ((p.M + BM - 1) / BM) * nt * ks;
-  return p.mt_start[p.n_groups] * nt;
+  if (!p.grouped) return ((p.M + TM - 1) / TM) * nt * ks;
+  return p.mt_start[p.n_groups] * nt;   // mt_start counts TM-row tiles
 }
 
-template <int EPI, int BN_OUT>
+template <int EPI, int BN_OUT, int TM>
 __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
   TileInfo ti;
   const int nt = p.N / BN_OUT;
@@ -94,8 +94,8 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
   ti.split = 0;
   ti.kb0 = 0;
   if (!p.grouped) {
-    const int mt = (p.M + BM - 1) / BM;
-    ti.m0 = (t % mt) * BM;
+    const int mt = (p.M + TM - 1) / TM;
+    ti.m0 = (t % mt) * TM;
     const int rest = t / mt;
     ti.split = rest % ks;
     ti.kb0 = ti.split * ti.nkb;
@@ -108,7 +108,7 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
     while (e + 1 < p.n_groups && p.mt_start[e + 1] * nt <= t) ++e;
     const int local = t - p.mt_start[e] * nt;
     const int mte = p.mt_start[e + 1] - p.mt_start[e];
-    ti.m0 = p.group_off[e] + (local % mte) * BM;
+    ti.m0 = p.group_off[e] + (local % mte) * TM;
     ti.m_end = p.group_off[e + 1];
     ti.n0 = (local / mte) * BN_OUT;
     ti.b_row = e * p.b_rows_per_group + ti.n0;
@@ -279,14 +279,24 @@ __device__ __forceinline__ void merge_chunk(const GemmParams& p, int row0, int m
   __syncwarp();
 }
 
-template <int BN, int EPI>
+// CG = 1: one CTA per SM, 128 x BN tiles.  CG = 2: clusters of two CTAs
+// (cta_group::2), 256 x BN tiles: CTA rank r loads A rows [m0 + 128r, +128)
+// and its half of B's BN rows (SWIGLU: rank 0 the gate rows, rank 1 the up
+// rows), both completing on the rank-0 CTA's `full` barrier, whose producer
+// alone arms it with both CTAs' bytes; rank 0's MMA thread issues M = 256
+// MMAs and its commits arrive on the `empty` / `tfull` barriers of both CTAs;
+// each CTA's epilogue reads its own 128 accumulator rows and releases the
+// accumulator on rank 0's `tempty`.
+template <int BN, int EPI, int CG>
 __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
-  using C = GemmCfg<BN, EPI>;
+  using C = GemmCfg<BN, EPI, CG>;
   constexpr int STAGES = C::STAGES;
   constexpr int BN_OUT = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+  constexpr int TM = BM * CG;   // output rows per tile
+  constexpr uint32_t IDESC = idesc_bf16_f32(TM, BN);
+  constexpr int EW = epi_warps<EPI>();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -302,6 +312,9 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+  const int unit = (CG == 2) ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;   // tile walker index
+  const int n_units = (CG == 2) ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -310,47 +323,66 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], epi_warps<EPI>());
+      mbar_init(&tempty[a], CG * EW);
     }
     fence_barrier_init();
     fence_proxy_async();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (CG == 2) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    else tmem_alloc(tmem_slot, C::TMEM_COLS);
+  }
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if constexpr (CG == 2) cluster_sync_all();   // both CTAs' barriers and TMEM are ready
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int ntiles = total_tiles<EPI, BN_OUT>(p);
+  const int ntiles = total_tiles<EPI, BN_OUT, TM>(p);
 
   if (warp == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer (each CTA loads its own A rows and B half)
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        const TileInfo ti = tile_info<EPI, BN_OUT>(p, t);
+      for (int t = unit; t < ntiles; t += n_units) {
+        const TileInfo ti = tile_info<EPI, BN_OUT, TM>(p, t);
+        // this CTA's B rows: CG = 1 all BN rows (SWIGLU: gate then up); CG = 2 its half
+        const int b_first = (CG == 1) ? ti.b_row
+                            : (EPI == EPI_SWIGLU) ? (rank == 0 ? ti.b_row : ti.b_row2)
+                                                  : ti.b_row + (int)rank * (BN / 2);
         const int kb_end = ti.kb0 + ti.nkb;
-        for (int kb = ti.kb0; kb < ti.kb0 + kPrefetchAhead && kb < kb_end; ++kb) {
-          tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row);
-          if constexpr (EPI == EPI_SWIGLU) tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row2);
-        }
-        for (int kb = ti.kb0; kb < kb_end; ++kb) {
-          if (kb + kPrefetchAhead < kb_end) {
-            tma_prefetch_l2_2d(&tmB, (kb + kPrefetchAhead) * BK, ti.b_row);
-            if constexpr (EPI == EPI_SWIGLU) tma_prefetch_l2_2d(&tmB, (kb + kPrefetchAhead) * BK, ti.b_row2);
-          }
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) goto producer_done;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * BK, ti.m0);
-          uint8_t* b_dst = sB + stage * C::B_STAGE_BYTES;
-          if constexpr (EPI == EPI_SWIGLU) {
-            tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
-            tma_load_2d(b_dst + (BN / 2) * BK * 2, &tmB, &full[stage], kb * BK, ti.b_row2);
+        auto prefetch_b = [&](int kb) {
+          if constexpr (EPI == EPI_SWIGLU && CG == 1) {
+            tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row);
+            tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row2);
           } else {
-            tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
+            tma_prefetch_l2_2d(&tmB, kb * BK, b_first);
+          }
+        };
+        for (int kb = ti.kb0; kb < ti.kb0 + kPrefetchAhead && kb < kb_end; ++kb) prefetch_b(kb);
+        for (int kb = ti.kb0; kb < kb_end; ++kb) {
+          if (kb + kPrefetchAhead < kb_end) prefetch_b(kb + kPrefetchAhead);
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) goto producer_done;
+          uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
+          uint8_t* b_dst = sB + stage * C::B_STAGE_BYTES;
+          if constexpr (CG == 2) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);   // both CTAs' bytes
+            const uint32_t bar = mapa_shared(&full[stage], 0);
+            tma_load_2d_pair(a_dst, &tmA, bar, kb * BK, ti.m0 + (int)rank * BM);
+            tma_load_2d_pair(b_dst, &tmB, bar, kb * BK, b_first);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+            tma_load_2d(a_dst, &tmA, &full[stage], kb * BK, ti.m0);
+            if constexpr (EPI == EPI_SWIGLU) {
+              tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
+              tma_load_2d(b_dst + (BN / 2) * BK * 2, &tmB, &full[stage], kb * BK, ti.b_row2);
+            } else {
+              tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
+            }
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -361,18 +393,18 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     producer_done:;
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (elect_one()) {
+    // ---------------- MMA issuer (rank 0 of a pair issues for both CTAs)
+    if (rank == 0 && elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+      for (int t = unit; t < ntiles; t += n_units, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        const int nkb = tile_info<EPI, BN_OUT>(p, t).nkb;
+        const int nkb = tile_info<EPI, BN_OUT, TM>(p, t).nkb;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.status)) {
@@ -384,31 +416,37 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
           const uint32_t b_addr = smem_u32(sB + stage * C::B_STAGE_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), IDESC,
-                        (kb | k) != 0 ? 1u : 0u);
+            if constexpr (CG == 2)
+              tc_mma_bf16_pair(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), IDESC,
+                               (kb | k) != 0 ? 1u : 0u);
+            else
+              tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), IDESC,
+                          (kb | k) != 0 ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          if constexpr (CG == 2) tc_commit_pair(&empty[stage], 3);
+          else tc_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(&tfull[acc]);
+        if constexpr (CG == 2) tc_commit_pair(&tfull[acc], 3);
+        else tc_commit(&tfull[acc]);
       }
     }
   } else {
-    // ---------------- epilogue warps 2 .. 2+EW-1
-    constexpr int EW = epi_warps<EPI>();
+    // ---------------- epilogue warps 2 .. 2+EW-1 (this CTA's 128 accumulator rows)
     const int q = warp & 3;              // TMEM lanes [32q, 32q+32) are reachable from this warp
     const int part = (warp - 2) >> 2;    // column interleave among the warps sharing a lane quarter
     const int et = threadIdx.x - 64;     // epilogue thread index
+    const int row_off = (int)rank * BM;  // this CTA's first row inside the tile
     int local = 0;
     bool aborted = false;   // a wait ran out: keep walking the tiles (barrier partners) without waiting
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+    for (int t = unit; t < ntiles; t += n_units, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      const TileInfo ti = tile_info<EPI, BN_OUT>(p, t);
+      const TileInfo ti = tile_info<EPI, BN_OUT, TM>(p, t);
       float* prm = sPrm + acc * 4 * BN_OUT;
       if constexpr (is_merge<EPI>()) {
         // this tile's merge parameters (hb, hs, rb, rs for its columns) into shared memory
@@ -417,7 +455,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
           prm[i] = __ldg(p.merge + (size_t)r * p.N + ti.n0 + c);
         }
         // pull this thread's stream segment into L2 while the main loop runs
-        const int prow = ti.m0 + q * 32 + lane;
+        const int prow = ti.m0 + row_off + q * 32 + lane;
         if (part == 0 && prow < ti.m_end) {
           const int token = (EPI == EPI_MERGE_MLP) ? p.perm[prow] : prow;
           const char* base = reinterpret_cast<const char*>(p.stream + (size_t)token * p.N + ti.n0);
@@ -430,7 +468,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
       if (!aborted && !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, p.status))) aborted = true;
       if (aborted) continue;
       tc_fence_after();
-      const int row = ti.m0 + q * 32 + lane;
+      const int row = ti.m0 + row_off + q * 32 + lane;
       const bool valid = row < ti.m_end;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
 #pragma unroll 1
@@ -440,22 +478,28 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         if constexpr (EPI == EPI_SWIGLU) tmem_ld32(tbase + BN / 2 + c, r2);
         tmem_ld_wait();
         if constexpr (is_merge<EPI>())
-          merge_chunk<EPI>(p, ti.m0 + q * 32, ti.m_end, ti.n0 + c, r, sT + (warp - 2) * 1024, prm + c, BN_OUT);
+          merge_chunk<EPI>(p, ti.m0 + row_off + q * 32, ti.m_end, ti.n0 + c, r, sT + (warp - 2) * 1024, prm + c,
+                           BN_OUT);
         else if (valid)
           epilogue32<EPI>(p, row, ti.n0 + c, ti.split, r, r2, prm + c, BN_OUT);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if constexpr (CG == 2) mbar_arrive_cluster(mapa_shared(&tempty[acc], 0));
+        else mbar_arrive(&tempty[acc]);
+      }
     }
   }
 
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();   // no CTA leaves while its peer may still touch it
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (CG == 2) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -475,20 +519,54 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int CG>
 int launch_impl(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, int ntiles_hint, int num_sms,
                 cudaStream_t st) {
-  using C = GemmCfg<BN, EPI>;
-  auto kern = gemm_tc_kernel<BN, EPI>;
+  using C = GemmCfg<BN, EPI, CG>;
+  auto kern = gemm_tc_kernel<BN, EPI, CG>;
   static bool attr_set = false;
+  static int max_pairs = 0;   // co-resident CTA pairs (CG = 2)
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return ZAYA_ERR_CUDA;
     attr_set = true;
+    if (CG == 2) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * (num_sms / 2));
+      cfg.blockDim = dim3(64 + 32 * epi_warps<EPI>());
+      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return ZAYA_ERR_CUDA;
+      max_pairs = n;
+    }
   }
-  int grid = ntiles_hint < num_sms ? ntiles_hint : num_sms;
-  if (grid < 1) grid = 1;
-  kern<<<grid, 64 + 32 * epi_warps<EPI>(), C::SMEM_BYTES, st>>>(ma, mb, p);
+  const int max_units = (CG == 2) ? max_pairs : num_sms;
+  int units = ntiles_hint < max_units ? ntiles_hint : max_units;
+  if (units < 1) units = 1;
+  if constexpr (CG == 1) {
+    kern<<<units, 64 + 32 * epi_warps<EPI>(), C::SMEM_BYTES, st>>>(ma, mb, p);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * units);
+    cfg.blockDim = dim3(64 + 32 * epi_warps<EPI>());
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ma, mb, p) != cudaSuccess) return ZAYA_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 
@@ -516,15 +594,21 @@ int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b
   const int bn_out = (epi == EPI_SWIGLU) ? bn / 2 : bn;
   if (p.N % bn_out != 0) return ZAYA_ERR_UNSUPPORTED;
   if (a_rows <= 0) return ZAYA_OK;
+  const int cg = p.pair ? 2 : 1;
+  if (cg == 2 && bn != 256 && bn != 128) return ZAYA_ERR_UNSUPPORTED;
   CUtensorMap ma, mb;
   int rc = make_tmap_bf16(&ma, A, (uint64_t)a_rows, (uint64_t)p.K, BM);
   if (rc) return rc;
-  rc = make_tmap_bf16(&mb, B, (uint64_t)b_rows, (uint64_t)p.K, epi == EPI_SWIGLU ? bn / 2 : bn);
+  // B box: a CTA pair splits the tile's B rows in two; SWIGLU loads gate and up rows as two boxes
+  rc = make_tmap_bf16(&mb, B, (uint64_t)b_rows, (uint64_t)p.K, (epi == EPI_SWIGLU || cg == 2) ? bn / 2 : bn);
   if (rc) return rc;
   const int nt = p.N / bn_out;
-  int hint = p.grouped ? num_sms : ((p.M + BM - 1) / BM) * nt * ks;
-#define ZAYA_GEMM_CASE(BNV, EPIV) \
-  if (bn == BNV && epi == EPIV) return launch_impl<BNV, EPIV>(ma, mb, p, hint, num_sms, st);
+  const int tm = BM * cg;
+  int hint = p.grouped ? num_sms : ((p.M + tm - 1) / tm) * nt * ks;
+#define ZAYA_GEMM_CASE(BNV, EPIV)                                                  \
+  if (bn == BNV && epi == EPIV)                                                    \
+    return cg == 2 ? launch_impl<BNV, EPIV, 2>(ma, mb, p, hint, num_sms, st)       \
+                   : launch_impl<BNV, EPIV, 1>(ma, mb, p, hint, num_sms, st);
   ZAYA_GEMM_CASE(256, EPI_STORE_BF16)
   ZAYA_GEMM_CASE(128, EPI_STORE_BF16)
   ZAYA_GEMM_CASE(64, EPI_STORE_BF16)

@@ -23,7 +23,8 @@ struct GemmParams {
   int k_splits;              // dense STORE_F32 only: K split into this many slabs (0 or 1: none)
   int grouped;               // expert-grouped A rows / B row blocks
   const int* group_off;      // [E+1] first A row of each expert (grouped)
-  const int* mt_start;       // [E+1] prefix of per-expert 128-row tile counts (grouped)
+  const int* mt_start;       // [E+1] prefix of per-expert tile counts (grouped; 128-row tiles, 256 with pair)
+  int pair;                  // 1: CTA-pair kernel (cta_group::2), 256-row tiles; bn 128 or 256
   int n_groups;              // E
   int b_rows_per_group;      // rows of B per expert (2I or H)
   int* status;
@@ -150,9 +151,9 @@ struct RouterParams {
 int launch_router(const RouterParams& p, cudaStream_t st);
 
 // Stable counting sort of tokens by class: pos[t] = permuted row of token t,
-// perm[row] = token; group_off[E+1]; mt_start[E+1] (128-row tiles).
-int launch_permute(const int* cls, int M, int E, int* group_off, int* mt_start, int* pos, int* perm, int* status,
-                   cudaStream_t st);
+// perm[row] = token; group_off[E+1]; mt_start[E+1] (tile_rows-row tiles).
+int launch_permute(const int* cls, int M, int E, int tile_rows, int* group_off, int* mt_start, int* pos, int* perm,
+                   int* status, cudaStream_t st);
 
 // Copies m_in rows of routed tokens into their permuted rows; writes the
 // merge-2 output of skipped (and padding) tokens; decode: cache_len += 1.

@@ -3,7 +3,10 @@
 // A block norm casts the fp32 stream to its weight's dtype (bf16) and norms
 // it (nnterp "zaya" page, "The stream is float32 whatever the load"):
 //   out = bf16(w * xb / sqrt(mean(xb^2) + eps)),  xb = bf16(x).
-// One warp per row, float4 loads, the row kept in registers; HBM-bound
+// One warp per row, float4 loads in groups; the row is read twice (sum of
+// squares, then the output) so that no thread keeps it in registers and four
+// 8-warp CTAs fit an SM (a 4096-row launch is one round); the second read is
+// served from cache.  The weight is staged in shared memory.  HBM-bound
 // (4 bytes read + 2 bytes written per element).
 #include "common.cuh"
 #include "kernels.h"
@@ -13,14 +16,19 @@ namespace zaya {
 namespace {
 
 template <int CHUNKS>  // H = CHUNKS * 128
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, int row_mul, int row_add,
-                                                      const __nv_bfloat16* __restrict__ w,
-                                                      __nv_bfloat16* __restrict__ out, __nv_bfloat16* __restrict__ tap,
-                                                      int M, float eps, const __nv_bfloat16* __restrict__ copy_src,
-                                                      int n_copy) {
+__global__ void __launch_bounds__(256, 4) rmsnorm_kernel(const float* __restrict__ x, int row_mul, int row_add,
+                                                         const __nv_bfloat16* __restrict__ w,
+                                                         __nv_bfloat16* __restrict__ out,
+                                                         __nv_bfloat16* __restrict__ tap, int M, float eps,
+                                                         const __nv_bfloat16* __restrict__ copy_src, int n_copy) {
   constexpr int H = CHUNKS * 128;
+  constexpr int G = CHUNKS < 8 ? CHUNKS : 8;   // float4 loads in flight per group
+  __shared__ __align__(16) __nv_bfloat16 ws[H];   // the norm weight, staged once per CTA
   const int row = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
+  for (int i = threadIdx.x; i < H / 8; i += blockDim.x)
+    reinterpret_cast<uint4*>(ws)[i] = __ldg(reinterpret_cast<const uint4*>(w) + i);
+  __syncthreads();
   if (row >= M + n_copy) return;
   if (row >= M) {  // verbatim copy rows (decode: prev_hs feeds the delayed values)
     const uint2* src = reinterpret_cast<const uint2*>(copy_src + (size_t)(row - M) * H);
@@ -31,32 +39,40 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
   }
   const int src_row = row * row_mul + row_add;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)src_row * H);
-  float v[CHUNKS * 4];
+  // pass 1: sum of squares of bf16(x); pass 2 reads the row again (now in L2 /
+  // L1), so no thread holds the row in registers
   float ss = 0.f;
+#pragma unroll 1
+  for (int c0 = 0; c0 < CHUNKS; c0 += G) {
+    float4 t[G];
 #pragma unroll
-  for (int c = 0; c < CHUNKS; ++c) {
-    float4 t = xr[c * 32 + lane];
-    v[4 * c + 0] = round_bf(t.x);
-    v[4 * c + 1] = round_bf(t.y);
-    v[4 * c + 2] = round_bf(t.z);
-    v[4 * c + 3] = round_bf(t.w);
-    ss += v[4 * c] * v[4 * c] + v[4 * c + 1] * v[4 * c + 1] + v[4 * c + 2] * v[4 * c + 2] +
-          v[4 * c + 3] * v[4 * c + 3];
+    for (int c = 0; c < G; ++c) t[c] = xr[(c0 + c) * 32 + lane];
+#pragma unroll
+    for (int c = 0; c < G; ++c) {
+      const float a0 = round_bf(t[c].x), a1 = round_bf(t[c].y), a2 = round_bf(t[c].z), a3 = round_bf(t[c].w);
+      ss += a0 * a0 + a1 * a1 + a2 * a2 + a3 * a3;
+    }
   }
   ss = warp_sum(ss);
   const float inv = rsqrtf(ss / (float)H + eps);
-  const uint2* wr = reinterpret_cast<const uint2*>(w);
+  const uint2* wr = reinterpret_cast<const uint2*>(ws);
   uint2* orow = reinterpret_cast<uint2*>(out + (size_t)row * H);
   uint2* trow = tap ? reinterpret_cast<uint2*>(tap + (size_t)row * H) : nullptr;
+#pragma unroll 1
+  for (int c0 = 0; c0 < CHUNKS; c0 += G) {
+    float4 t[G];
 #pragma unroll
-  for (int c = 0; c < CHUNKS; ++c) {
-    const uint2 wu = wr[c * 32 + lane];
-    const float2 w01 = unpack_bf2(wu.x), w23 = unpack_bf2(wu.y);
-    uint2 o;
-    o.x = pack_bf2(w01.x * (v[4 * c] * inv), w01.y * (v[4 * c + 1] * inv));
-    o.y = pack_bf2(w23.x * (v[4 * c + 2] * inv), w23.y * (v[4 * c + 3] * inv));
-    orow[c * 32 + lane] = o;
-    if (trow) trow[c * 32 + lane] = o;
+    for (int c = 0; c < G; ++c) t[c] = xr[(c0 + c) * 32 + lane];
+#pragma unroll
+    for (int c = 0; c < G; ++c) {
+      const uint2 wu = wr[(c0 + c) * 32 + lane];
+      const float2 w01 = unpack_bf2(wu.x), w23 = unpack_bf2(wu.y);
+      uint2 o;
+      o.x = pack_bf2(w01.x * (round_bf(t[c].x) * inv), w01.y * (round_bf(t[c].y) * inv));
+      o.y = pack_bf2(w23.x * (round_bf(t[c].z) * inv), w23.y * (round_bf(t[c].w) * inv));
+      orow[(c0 + c) * 32 + lane] = o;
+      if (trow) trow[(c0 + c) * 32 + lane] = o;
+    }
   }
 }
 

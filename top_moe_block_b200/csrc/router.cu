@@ -148,17 +148,20 @@ __device__ __forceinline__ void mlp_epilogue(float (*acc)[4], const float2* bias
   }
 }
 
-// fc1 / fc2 weights (fp32 [R][R]) -> bf16 hi and lo parts: wsplit = [layer][hi|lo][R][R].
-__global__ void router_split_kernel(const float* __restrict__ fc1, const float* __restrict__ fc2,
-                                    __nv_bfloat16* __restrict__ wsplit, int R) {
-  const int n = R * R;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < 2 * n; i += gridDim.x * blockDim.x) {
-    const int layer = i / n, e = i % n;
-    const float x = (layer ? fc2 : fc1)[e];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    wsplit[(size_t)layer * 2 * n + e] = hi;
-    wsplit[(size_t)layer * 2 * n + n + e] = __float2bfloat16_rn(x - __bfloat162float(hi));
-  }
+// fc1 / fc2 weights (fp32 [R][R]) -> bf16 hi and lo parts: wsplit = [layer][hi|lo][R][R];
+// four elements per thread.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ fc1, const float* __restrict__ fc2,
+                                                           __nv_bfloat16* __restrict__ wsplit, int R) {
+  const int n4 = R * R / 4;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 2 * n4) return;
+  const int layer = i / n4, e4 = i % n4;
+  const float4 x = __ldg(reinterpret_cast<const float4*>(layer ? fc2 : fc1) + e4);
+  const float hx = round_bf(x.x), hy = round_bf(x.y), hz = round_bf(x.z), hw = round_bf(x.w);
+  __nv_bfloat16* base = wsplit + (size_t)layer * 2 * R * R;
+  reinterpret_cast<uint2*>(base)[e4] = make_uint2(pack_bf2(hx, hy), pack_bf2(hz, hw));
+  reinterpret_cast<uint2*>(base + R * R)[e4] =
+      make_uint2(pack_bf2(x.x - hx, x.y - hy), pack_bf2(x.z - hz, x.w - hw));
 }
 
 template <int R>
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
 template <int R>
 int launch_router_r(const RouterParams& p, cudaStream_t st) {
   using Sh = RouterShape<R>;
-  router_split_kernel<<<64, 256, 0, st>>>(p.fc1_w, p.fc2_w, p.wsplit, R);
+  router_split_kernel<<<(2 * R * R / 4 + 255) / 256, 256, 0, st>>>(p.fc1_w, p.fc2_w, p.wsplit, R);
   const size_t ow_bytes = (size_t)(p.E + 1) * R * sizeof(float);
   const size_t smem = Sh::SMEM + (ow_bytes <= 2 * Sh::CHUNK * sizeof(__nv_bfloat16) ? 0 : ow_bytes);
   if (smem > 227 * 1024) return ZAYA_ERR_UNSUPPORTED;
@@ -392,9 +395,23 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
 }
 
 // Stable counting sort by class, one CTA of 32 warps; warp w owns a
-// contiguous token range, so token order is kept inside every class.
-__global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ cls, int M, int E, int* group_off,
-                                                       int* mt_start, int* pos, int* perm, int* status) {
+// contiguous token range, so token order is kept inside every class.  Pass 1
+// counts per (warp, class); after the scans, pass 2 replays the same warp-local
+// ranking from the scanned offsets.  Each pass loads the next 32 classes
+// before it ranks the current ones.
+__device__ __forceinline__ int load_cls(const int* __restrict__ cls, int t, int end, int E, int* status) {
+  if (t >= end) return -1;
+  int c = cls[t];
+  if (c < 0 || c > E) {
+    set_status(status, ZAYA_ERR_DEVICE_RANGE);
+    c = E;
+  }
+  return c;
+}
+
+__global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ cls, int M, int E, int tile_rows,
+                                                       int* group_off, int* mt_start, int* pos, int* perm,
+                                                       int* status) {
   __shared__ int cnt[32][66];
   __shared__ int cls_base[66];
   const int warp = warp_id(), lane = lane_id();
@@ -404,24 +421,18 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ c
   const int per = ((M + 31) / 32 + 31) / 32 * 32;
   const int begin = warp * per, end = min(M, begin + per);
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = begin; base < end; base += 32) {
-    const int t = base + lane;
-    int c = -1;
-    if (t < end) {
-      c = cls[t];
-      if (c < 0 || c > E) {
-        set_status(status, ZAYA_ERR_DEVICE_RANGE);
-        c = E;
-      }
+  {
+    int c_next = load_cls(cls, begin + lane, end, E, status);
+    for (int base = begin; base < end; base += 32) {
+      const int c = c_next;
+      c_next = load_cls(cls, base + 32 + lane, end, E, status);
+      const unsigned same = __match_any_sync(0xffffffffu, c);
+      const int leader = __ffs(same) - 1;
+      const int before = (c >= 0) ? cnt[warp][c] : 0;
+      __syncwarp();
+      if (c >= 0 && lane == leader) cnt[warp][c] = before + __popc(same);
+      __syncwarp();
     }
-    const unsigned same = __match_any_sync(0xffffffffu, c);
-    const int rank = __popc(same & lt_mask);
-    const int leader = __ffs(same) - 1;
-    const int before = (c >= 0) ? cnt[warp][c] : 0;
-    __syncwarp();
-    if (c >= 0 && lane == leader) cnt[warp][c] = before + __popc(same);
-    __syncwarp();
-    if (t < end) pos[t] = before + rank;
   }
   __syncthreads();
   // exclusive scan of cnt over (class-major, warp-minor)
@@ -442,7 +453,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ c
     for (int c0 = 0; c0 < E1; c0 += 32) {
       const int c = c0 + lane;
       const int tot = c < E1 ? cls_base[c] : 0;
-      const int tiles = (c < E) ? (tot + 127) / 128 : 0;
+      const int tiles = (c < E) ? (tot + tile_rows - 1) / tile_rows : 0;
       int inc = tot, tinc = tiles;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -468,58 +479,86 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ c
     }
   }
   __syncthreads();
-  for (int base = begin; base < end; base += 32) {
-    const int t = base + lane;
-    if (t < end) {
-      int c = cls[t];
-      if (c < 0 || c > E) c = E;
-      const int ps = cls_base[c] + cnt[warp][c] + pos[t];
-      pos[t] = ps;
-      perm[ps] = t;
+  for (int c = lane; c < E1; c += 32) cnt[warp][c] += cls_base[c];   // this warp's first row in class c
+  __syncwarp();
+  {
+    int c_next = load_cls(cls, begin + lane, end, E, nullptr);
+    for (int base = begin; base < end; base += 32) {
+      const int t = base + lane;
+      const int c = c_next;
+      c_next = load_cls(cls, base + 32 + lane, end, E, nullptr);
+      const unsigned same = __match_any_sync(0xffffffffu, c);
+      const int rank = __popc(same & lt_mask);
+      const int leader = __ffs(same) - 1;
+      const int first = (c >= 0) ? cnt[warp][c] : 0;
+      __syncwarp();
+      if (c >= 0 && lane == leader) cnt[warp][c] = first + __popc(same);
+      __syncwarp();
+      if (t < end) {
+        const int ps = first + rank;
+        pos[t] = ps;
+        perm[ps] = t;
+      }
     }
   }
 }
 
-// One thread per 16-byte chunk (8 columns) of a token row: routed tokens copy
-// the chunk of m_in to their permuted row; skipped (and padding) tokens
-// write merge 2 with a zero routed output for those 8 columns.
+// One warp per token row: routed tokens copy their m_in row to the permuted
+// row (all eight 16-byte loads of a lane in flight at once); skipped (and
+// padding) tokens write merge 2 with a zero routed output.
 __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
-  const int per_row = p.H / 8;
-  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (long)p.M * per_row) return;
-  const int t = (int)(i / per_row), ch = (int)(i % per_row);
+  const int t = blockIdx.x * 8 + warp_id();
+  const int lane = lane_id();
+  if (t >= p.M) return;
+  const int H = p.H;
+  const int per_row = H / 8;   // 16-byte chunks
   const int c = p.cls[t];
   if (c >= 0 && c < p.E) {
-    const uint4 v = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * p.H)[ch];
-    reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)p.pos[t] * p.H)[ch] = v;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * H);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)p.pos[t] * H);
+    constexpr int kV = 8;
+    for (int c0 = 0; c0 < per_row; c0 += 32 * kV) {
+      uint4 v[kV];
+#pragma unroll
+      for (int k = 0; k < kV; ++k) {
+        const int ch = c0 + k * 32 + lane;
+        if (ch < per_row) v[k] = src[ch];
+      }
+#pragma unroll
+      for (int k = 0; k < kV; ++k) {
+        const int ch = c0 + k * 32 + lane;
+        if (ch < per_row) dst[ch] = v[k];
+      }
+    }
   } else {
     // skip: no expert runs; mlp_output = bf16(hb * hs), out = mlp_output + (h + rb) * rs
-    const int H = p.H;
-    float4* s4 = reinterpret_cast<float4*>(p.stream + (size_t)t * H + ch * 8);
-    float cb[8];
+    for (int ch = lane; ch < per_row; ch += 32) {
+      float4* s4 = reinterpret_cast<float4*>(p.stream + (size_t)t * H + ch * 8);
+      float cb[8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float4 x = s4[h];
-      float* xp = &x.x;
+      for (int h = 0; h < 2; ++h) {
+        float4 x = s4[h];
+        float* xp = &x.x;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int col = ch * 8 + 4 * h + j;
-        const float contrib = round_bf(__ldg(p.merge_m + col) * __ldg(p.merge_m + H + col));
-        cb[4 * h + j] = contrib;
-        xp[j] = fmaf(xp[j] + __ldg(p.merge_m + 2 * H + col), __ldg(p.merge_m + 3 * H + col), contrib);
+        for (int j = 0; j < 4; ++j) {
+          const int col = ch * 8 + 4 * h + j;
+          const float contrib = round_bf(__ldg(p.merge_m + col) * __ldg(p.merge_m + H + col));
+          cb[4 * h + j] = contrib;
+          xp[j] = fmaf(xp[j] + __ldg(p.merge_m + 2 * H + col), __ldg(p.merge_m + 3 * H + col), contrib);
+        }
+        s4[h] = x;
       }
-      s4[h] = x;
-    }
-    if (p.tap_mlp_out) {
-      uint4 u;
-      u.x = pack_bf2(cb[0], cb[1]);
-      u.y = pack_bf2(cb[2], cb[3]);
-      u.z = pack_bf2(cb[4], cb[5]);
-      u.w = pack_bf2(cb[6], cb[7]);
-      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.tap_mlp_out) + (size_t)t * H)[ch] = u;
+      if (p.tap_mlp_out) {
+        uint4 u;
+        u.x = pack_bf2(cb[0], cb[1]);
+        u.y = pack_bf2(cb[2], cb[3]);
+        u.z = pack_bf2(cb[4], cb[5]);
+        u.w = pack_bf2(cb[6], cb[7]);
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.tap_mlp_out) + (size_t)t * H)[ch] = u;
+      }
     }
   }
-  if (p.cache_len_inc && ch == 0) p.cache_len_inc[t] += 1;
+  if (p.cache_len_inc && lane == 0) p.cache_len_inc[t] += 1;
 }
 
 }  // namespace
@@ -536,18 +575,17 @@ int launch_router(const RouterParams& p, cudaStream_t st) {
   }
 }
 
-int launch_permute(const int* cls, int M, int E, int* group_off, int* mt_start, int* pos, int* perm, int* status,
-                   cudaStream_t st) {
-  if (E + 1 > 65) return ZAYA_ERR_UNSUPPORTED;
-  permute_kernel<<<1, 1024, 0, st>>>(cls, M, E, group_off, mt_start, pos, perm, status);
+int launch_permute(const int* cls, int M, int E, int tile_rows, int* group_off, int* mt_start, int* pos, int* perm,
+                   int* status, cudaStream_t st) {
+  if (E + 1 > 65 || tile_rows <= 0) return ZAYA_ERR_UNSUPPORTED;
+  permute_kernel<<<1, 1024, 0, st>>>(cls, M, E, tile_rows, group_off, mt_start, pos, perm, status);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 
 int launch_dispatch(const DispatchParams& p, cudaStream_t st) {
   if (p.M <= 0) return ZAYA_OK;
   if (p.H % 8) return ZAYA_ERR_UNSUPPORTED;
-  const long n = (long)p.M * (p.H / 8);
-  dispatch_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+  dispatch_kernel<<<(unsigned)((p.M + 7) / 8), 256, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 

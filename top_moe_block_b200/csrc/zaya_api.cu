@@ -190,6 +190,8 @@ inline T* at(void* base, size_t off) {
 // the tiles to balance and half the exposed epilogue); when 128-wide tiles
 // do not give every SM a tile (decode-sized M), the narrowest candidate does
 // the most to spread the weight stream over the SMs.
+constexpr int kPairMinRows = 1024;   // rows from which the expert GEMMs use CTA pairs
+
 int pick_bn_tiles(long m_tiles, int N, const int* cands, int n, int sms) {
   bool has128 = false;
   int narrow = 0;
@@ -266,7 +268,9 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
   int* mt_start = at<int>(ws, L.mt_start);
   int* pos = at<int>(ws, L.pos);
   int* perm = at<int>(ws, L.perm);
-  ZAYA_STAGE("permute", 1, launch_permute(cls, M, d.E, group_off, mt_start, pos, perm, status, st));
+  // expert GEMMs of prefill-sized batches run on CTA pairs (256-row tiles)
+  const int pair = M >= kPairMinRows ? 1 : 0;
+  ZAYA_STAGE("permute", 1, launch_permute(cls, M, d.E, pair ? 256 : 128, group_off, mt_start, pos, perm, status, st));
   void* xperm = at<void>(ws, L.xperm);
   {
     DispatchParams p{};
@@ -280,18 +284,18 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
   {  // experts: gate/up + SwiGLU
     GemmParams p{};
     p.M = M; p.N = d.I; p.K = d.H; p.grouped = 1; p.group_off = group_off; p.mt_start = mt_start;
-    p.n_groups = d.E; p.b_rows_per_group = 2 * d.I; p.status = status;
+    p.n_groups = d.E; p.b_rows_per_group = 2 * d.I; p.status = status; p.pair = pair;
     p.out = act; p.ldo = d.I;
     ZAYA_STAGE("experts_gate_up", 1, launch_gemm(EPI_SWIGLU, 256, xperm, M, w->w_gate_up, d.E * 2 * d.I, p, sms, st));
   }
   {  // experts: down + weight + merge 2, scattered back to token rows
     GemmParams p{};
     p.M = M; p.N = d.H; p.K = d.I; p.grouped = 1; p.group_off = group_off; p.mt_start = mt_start;
-    p.n_groups = d.E; p.b_rows_per_group = d.H; p.status = status;
+    p.n_groups = d.E; p.b_rows_per_group = d.H; p.status = status; p.pair = pair;
     p.stream = hidden; p.merge = w->merge_m; p.perm = perm; p.row_w = wgt;
     p.tap_bf16 = taps ? taps->mlp_output : nullptr;
     const int c2[] = {256, 128};
-    const int bn = pick_bn_tiles((M + 127) / 128 + d.E / 2, d.H, c2, 2, sms);
+    const int bn = pair ? (d.H % 256 == 0 ? 256 : 128) : pick_bn_tiles((M + 127) / 128 + d.E / 2, d.H, c2, 2, sms);
     ZAYA_STAGE("experts_down_merge", 1, launch_gemm(EPI_MERGE_MLP, bn, act, M, w->w_down, d.E * d.H, p, sms, st));
   }
   return ZAYA_OK;
