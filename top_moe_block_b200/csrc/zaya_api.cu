@@ -190,7 +190,8 @@ inline T* at(void* base, size_t off) {
 // the tiles to balance and half the exposed epilogue); when 128-wide tiles
 // do not give every SM a tile (decode-sized M), the narrowest candidate does
 // the most to spread the weight stream over the SMs.
-constexpr int kPairMinRows = 1024;   // rows from which the expert GEMMs use CTA pairs
+constexpr int kPairMinRows = 1024;   // rows from which the GEMMs use CTA pairs (cta_group::2)
+constexpr int kPairDenseBn = 128;    // tile width of the CTA-pair dense GEMMs (256 x 128 tiles)
 
 int pick_bn_tiles(long m_tiles, int N, const int* cands, int n, int sms) {
   bool has128 = false;
@@ -233,7 +234,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.tap_bf16 = taps ? taps->attention_output : nullptr;
     p.tap_f32 = taps ? taps->layer_mid : nullptr;
     const int c3[] = {256, 128, 64};
-    const int bn = pick_bn(M, d.H, c3, 3, sms);
+    const int bn = pick_bn(M, d.H, c3, 3, sms);   // single-CTA tiles measured faster here than pairs
     ZAYA_STAGE("o_proj_merge", 1, launch_gemm(EPI_MERGE_ATTN, bn, at<void>(ws, L.premix), M, w->w_o, d.H, p, sms, st));
   }
   void* m_in = at<void>(ws, L.m_in);
@@ -334,7 +335,8 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     GemmParams p{};
     p.M = M; p.N = d.n_qkv; p.K = d.H; p.status = status; p.out = qkv; p.ldo = d.n_qkv;
     const int c3[] = {256, 128, 64};
-    const int bn = pick_bn(M, d.n_qkv, c3, 3, sms);
+    p.pair = (M >= kPairMinRows && d.n_qkv % kPairDenseBn == 0) ? 1 : 0;
+    const int bn = p.pair ? kPairDenseBn : pick_bn(M, d.n_qkv, c3, 3, sms);
     if (!bn) return ZAYA_ERR_UNSUPPORTED;
     ZAYA_STAGE("qkv_gemm", 1, launch_gemm(EPI_STORE_BF16, bn, a_in, M, w->w_qkv, d.n_qkv, p, sms, st));
   }
