@@ -8,19 +8,23 @@
 //
 // CTA = 128 queries of two query heads that share a kv head, 10 warps:
 //   warp 0     TMA: both heads' Q tiles once, then K and V tiles of 64 keys
-//              into two 3-slot rings (128-byte swizzle, 64-wide d atoms),
-//              shared by the two heads;
-//   warp 1     one thread issues tcgen05.mma: per head, S = Q K^T into one of
-//              two TMEM buffers (64 fp32 columns each), then O += P V into the
-//              head's TMEM accumulator (P from one of two shared-memory
-//              buffers, V as an MN-major operand); S of tile j+1 is computed
-//              while the softmax works on tile j;
+//              into a 3-slot and a 2-slot ring (128-byte swizzle, 64-wide d
+//              atoms), shared by the two heads;
+//   warp 1     one thread issues tcgen05.mma: per head, S(j) = Q K^T into one
+//              of two S buffers in tensor memory; once the softmax has written
+//              P(j) over it, O += P V with P read straight from tensor memory
+//              (A operand in TMEM) and V from shared memory as an MN-major
+//              operand, then S(j+2) into the same buffer: S runs two tiles
+//              ahead of the softmax and the two heads alternate;
 //   warps 2-9  softmax, a warpgroup per head, one thread per query row (its
-//              TMEM lane): row max
-//              and sum are thread-local; P is written to shared memory in
-//              the swizzled K-major layout the MMA reads.  The running
-//              max is only moved (and O rescaled in TMEM) when it grows by
-//              more than 2^8, which keeps P <= 256 and the result exact.
+//              TMEM lane): row max and sum are thread-local; P goes back into
+//              the S columns as bf16 pairs (tcgen05.st).  The running max is
+//              only moved (and O rescaled in TMEM) when it grows by more than
+//              2^8, which keeps P <= 256 and the result exact.
+// Shared memory carries only Q, K and V (P never leaves tensor memory): a
+// version with P staged in shared memory was measured to be limited by
+// shared-memory bandwidth, and one with a single S buffer per head by the
+// serial S -> softmax -> PV -> S chain.
 // Only key tiles that intersect the window are visited; per-element masks
 // only on tiles that straddle the diagonal, the window edge, the sequence
 // end or a padding mask.
@@ -46,11 +50,12 @@ namespace {
 constexpr int kQT = 128;  // queries per CTA
 constexpr int kKT = 64;   // keys per tile
 constexpr int kHPC = 2;   // query heads per CTA (sharing one kv head)
-constexpr int kRing = 3;  // K and V ring depth
+constexpr int kRing = 3;  // K ring depth (S runs two tiles ahead)
+constexpr int kRingV = 2; // V ring depth
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kMaxItems = 512;   // split-plan items carried in the kernel parameters
 constexpr int kPlanSms = 148;    // the SM count the split plan balances over
-constexpr int kMinChunk = 8;     // fewest key tiles in a chunk
+constexpr int kMinChunk = 4;     // fewest key tiles in a chunk
 
 struct AttnItems {
   int n_items;   // 0: grid (row tiles, head pairs, sequences), no row tile split
@@ -139,18 +144,18 @@ template <int D>
 struct AttnTc {
   static constexpr int SUB = D / 64;               // 64-wide swizzle atoms along d
   static constexpr int Q_ATOM = kQT * 128;         // [128 rows][64] bf16 atom: 16 KB
-  static constexpr int KV_ATOM = kKT * 128;        // [64 rows][64] bf16 atom: 8 KB
+  static constexpr int KV_ATOM = kKT * 128;        // [64 keys][64] bf16 atom: 8 KB
   static constexpr int Q_BYTES = SUB * Q_ATOM;     // one head's Q tile
   static constexpr int KV_BYTES = SUB * KV_ATOM;   // one K (or V) tile
-  static constexpr int P_BYTES = kQT * kKT * 2;    // [128 queries][64 keys]: one 16 KB atom
-  static constexpr int SMEM_USED = 1024 + kHPC * Q_BYTES + 2 * kRing * KV_BYTES + kHPC * 2 * P_BYTES + 512;
+  static constexpr int SMEM_USED = 1024 + kHPC * Q_BYTES + (kRing + kRingV) * KV_BYTES + 512;
   // at least 120 KB so a second CTA never shares the SM (and its TMEM)
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-  static constexpr uint32_t TMEM_COLS = 512;       // per head: S0 [0,64), S1 [64,128), O [128, 128+D)
+  static constexpr uint32_t TMEM_COLS = 512;       // per head: S0 / P0 [0, 64), S1 / P1 [64, 128), O [128, 128 + D)
   static constexpr uint32_t HEAD_COLS = 256;
   static constexpr uint32_t O_COL = 2 * kKT;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, kKT);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32_bmn(128, D);
+  static_assert(kHPC * (2 * kKT + D) <= 512, "tensor memory");
 };
 
 // 2^x on the special-function unit (inputs <= 0 here; results below 2^-126
@@ -175,19 +180,17 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                           // [kHPC] Q tiles
   uint8_t* sK = sQ + kHPC * C::Q_BYTES;         // [kRing] K tiles
-  uint8_t* sV = sK + kRing * C::KV_BYTES;       // [kRing] V tiles
-  uint8_t* sP = sV + kRing * C::KV_BYTES;       // [kHPC][2] P tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kHPC * 2 * C::P_BYTES);
+  uint8_t* sV = sK + kRing * C::KV_BYTES;       // [kRingV] V tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kRingV * C::KV_BYTES);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;                  // [kRing]
   uint64_t* k_empty = k_full + kRing;           // [kRing]
-  uint64_t* v_full = k_empty + kRing;           // [kRing]
-  uint64_t* v_empty = v_full + kRing;           // [kRing]
-  uint64_t* s_full = v_empty + kRing;           // [kHPC][2]
-  uint64_t* s_free = s_full + 2 * kHPC;         // [kHPC][2]
-  uint64_t* p_full = s_free + 2 * kHPC;         // [kHPC][2]
-  uint64_t* pv_done = p_full + 2 * kHPC;        // [kHPC][2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2 * kHPC);
+  uint64_t* v_full = k_empty + kRing;           // [kRingV]
+  uint64_t* v_empty = v_full + kRingV;          // [kRingV]
+  uint64_t* s_full = v_empty + kRingV;          // [kHPC][2]: S(j) of the head is in S buffer j & 1
+  uint64_t* p_full = s_full + 2 * kHPC;         // [kHPC][2]: P(j) is in TMEM over S(j)
+  uint64_t* pv_done = p_full + 2 * kHPC;        // [kHPC]: O += P(j) V(j) complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + kHPC);
   int* s_last = reinterpret_cast<int*>(tmem_slot + 1);
 
   // this CTA's item: a row tile of two heads, or one key chunk of it
@@ -223,15 +226,16 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kRingV; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2 * kHPC; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
       mbar_init(&p_full[i], 4);
-      mbar_init(&pv_done[i], 1);
     }
+    for (int i = 0; i < kHPC; ++i) mbar_init(&pv_done[i], 1);
     fence_barrier_init();
     fence_proxy_async();
     prefetch_tmap(&tmQ);
@@ -264,60 +268,64 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
 #pragma unroll
         for (int s = 0; s < C::SUB; ++s)
           tma_load_2d(sK + slot * C::KV_BYTES + s * C::KV_ATOM, &tmK, &k_full[slot], s * 64, kv_row + j * kKT);
-        if (!mbar_wait(&v_empty[slot], par, status)) break;
-        mbar_arrive_expect_tx(&v_full[slot], C::KV_BYTES);
+        const int vslot = j % kRingV;
+        if (!mbar_wait(&v_empty[vslot], ((j / kRingV) & 1) ^ 1u, status)) break;
+        mbar_arrive_expect_tx(&v_full[vslot], C::KV_BYTES);
 #pragma unroll
         for (int s = 0; s < C::SUB; ++s)
-          tma_load_2d(sV + slot * C::KV_BYTES + s * C::KV_ATOM, &tmV, &v_full[slot], s * 64, kv_row + j * kKT);
+          tma_load_2d(sV + vslot * C::KV_BYTES + s * C::KV_ATOM, &tmV, &v_full[vslot], s * 64, kv_row + j * kKT);
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer: for each key tile, S = Q K^T of both heads, then P V of both
+    // ---------------- MMA issuer.  Per head: S(j) into S buffer j & 1; the
+    // softmax writes P(j) over it; O += P(j) V(j) with P read from tensor
+    // memory; then S(j+2) into the same buffer (the tensor pipe runs one
+    // thread's MMAs in issue order, so S(j+2) is written after P(j) is read).
+    // S runs two tiles ahead of the softmax, and the two heads alternate.
     if (elect_one()) {
       bool ok = mbar_wait(q_full, 0, status);
-      auto issue_qk = [&](int j) -> bool {
-        const int slot = j % kRing, buf = j & 1;
-        if (!mbar_wait(&k_full[slot], (j / kRing) & 1, status)) return false;
-        const uint32_t ka = smem_u32(sK + slot * C::KV_BYTES);
+      auto issue_qk = [&](int x, int j) {
+        const uint32_t ka = smem_u32(sK + (j % kRing) * C::KV_BYTES);
+        const uint32_t qa = smem_u32(sQ + x * C::Q_BYTES);
 #pragma unroll
-        for (int x = 0; x < kHPC; ++x) {
-          if (!mbar_wait(&s_free[x * 2 + buf], ((j >> 1) & 1) ^ 1u, status)) return false;
-          tc_fence_after();
-          const uint32_t qa = smem_u32(sQ + x * C::Q_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk & 3) * 32;
-            tc_mma_bf16(tmem_base + x * C::HEAD_COLS + buf * kKT,
-                        smem_desc_sw128(qa + (kk >> 2) * C::Q_ATOM + koff, 16, 1024),
-                        smem_desc_sw128(ka + (kk >> 2) * C::KV_ATOM + koff, 16, 1024), C::IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&s_full[x * 2 + buf]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          tc_mma_bf16(tmem_base + x * C::HEAD_COLS + (j & 1) * kKT,
+                      smem_desc_sw128(qa + (kk >> 2) * C::Q_ATOM + koff, 16, 1024),
+                      smem_desc_sw128(ka + (kk >> 2) * C::KV_ATOM + koff, 16, 1024), C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&k_empty[slot]);
-        return true;
+        tc_commit(&s_full[x * 2 + (j & 1)]);
       };
-      if (ok && n_tiles > 0) ok = issue_qk(0);
+      for (int j = 0; ok && j < 2 && j < n_tiles; ++j) {   // S(0), S(1)
+        ok = mbar_wait(&k_full[j], 0, status);
+        if (!ok) break;
+        tc_fence_after();
+        for (int x = 0; x < kHPC; ++x) issue_qk(x, j);
+        tc_commit(&k_empty[j]);
+      }
       for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_qk(j + 1)) break;
-        const int slot = j % kRing, buf = j & 1;
-        if (!mbar_wait(&v_full[slot], (j / kRing) & 1, status)) break;
-        const uint32_t va = smem_u32(sV + slot * C::KV_BYTES);
+        const int vslot = j % kRingV, nslot = (j + 2) % kRing;
+        const bool more = j + 2 < n_tiles;
+        if (more && !mbar_wait(&k_full[nslot], ((j + 2) / kRing) & 1, status)) break;
+        if (!mbar_wait(&v_full[vslot], (j / kRingV) & 1, status)) break;
+        const uint32_t va = smem_u32(sV + vslot * C::KV_BYTES);
         for (int x = 0; ok && x < kHPC; ++x) {
-          if (!mbar_wait(&p_full[x * 2 + buf], (j >> 1) & 1, status)) {
+          if (!mbar_wait(&p_full[x * 2 + (j & 1)], (j >> 1) & 1, status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t pa = smem_u32(sP + (x * 2 + buf) * C::P_BYTES);
+          const uint32_t pa = tmem_base + x * C::HEAD_COLS + (j & 1) * kKT;   // P(j): bf16 pairs over S(j)
 #pragma unroll
-          for (int kk = 0; kk < kKT / 16; ++kk) {
-            tc_mma_bf16(tmem_base + x * C::HEAD_COLS + C::O_COL, smem_desc_sw128(pa + kk * 32, 16, 1024),
-                        smem_desc_sw128(va + kk * 2048, C::KV_ATOM, 1024), C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(&pv_done[x * 2 + buf]);
+          for (int kk = 0; kk < kKT / 16; ++kk)
+            tc_mma_bf16_ts(tmem_base + x * C::HEAD_COLS + C::O_COL, pa + kk * 8,
+                           smem_desc_sw128(va + kk * 2048, C::KV_ATOM, 1024), C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&pv_done[x]);
+          if (more) issue_qk(x, j + 2);
         }
         if (!ok) break;
-        tc_commit(&v_empty[slot]);
+        tc_commit(&v_empty[vslot]);
+        if (more) tc_commit(&k_empty[nslot]);
       }
     }
   } else {
@@ -327,47 +335,40 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
     const int row = quarter * 32 + lane;
     const int q = m0 + row;
     const uint32_t tl = tmem_base + x * C::HEAD_COLS + ((uint32_t)(quarter * 32) << 16);
-    uint64_t* my_s_full = s_full + x * 2;
-    uint64_t* my_s_free = s_free + x * 2;
-    uint64_t* my_p_full = p_full + x * 2;
-    uint64_t* my_pv_done = pv_done + x * 2;
-    uint8_t* my_p = sP + x * 2 * C::P_BYTES;
     const int* mask = p.mask ? p.mask + (size_t)b * S : nullptr;
     const float sl2 = p.scale * 1.4426950408889634f;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const int buf = j & 1;
       // every wait that guards a .sync.aligned TMEM access is made warp-uniform
-      if (!__all_sync(0xffffffffu, mbar_wait(&my_s_full[buf], (j >> 1) & 1, status))) {
+      const int buf = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x * 2 + buf], (j >> 1) & 1, status))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int key0 = n_begin + (t_begin + j) * kKT;
       const bool full_vis = !mask && key0 + kKT - 1 <= m0 && (m0 + kQT - 1 - key0) < p.window && key0 + kKT <= S;
-      uint32_t r[2][32];
-      tmem_ld32(tl + buf * kKT, r[0]);
-      tmem_ld32(tl + buf * kKT + 32, r[1]);
+      uint32_t r[kKT];
+#pragma unroll
+      for (int c = 0; c < kKT / 32; ++c)
+        tmem_ld32(tl + buf * kKT + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
       tmem_ld_wait();
-      float v[2 * 32];
+      float* v = reinterpret_cast<float*>(r);
       if (full_vis) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i >> 5][i & 31]) * sl2;
+        for (int i = 0; i < kKT; ++i) v[i] = __uint_as_float(r[i]) * sl2;
       } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float xv = __uint_as_float(r[i >> 5][i & 31]) * sl2;
+        for (int i = 0; i < kKT; ++i) {
+          const float xv = __uint_as_float(r[i]) * sl2;
           v[i] = key_visible(q, key0 + i, p.window, S, mask) ? xv : -INFINITY;
         }
       }
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
-      for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], v[i]);
+      for (int i = 0; i < kKT; ++i) mx[i & 3] = fmaxf(mx[i & 3], v[i]);
       const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&my_s_free[buf]);   // S is in registers: the buffer may be refilled
       const float m_new = fmaxf(m_used, tmax);
       // Move the running max when it grew by more than 2^8 -- for the whole warp
       // at once, since the O rescale below is a warp-wide TMEM access.  Each
@@ -377,8 +378,8 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
         const bool finite_new = m_new != -INFINITY;
         const float f = (m_used == -INFINITY || !finite_new) ? 1.f : exp2f(m_used - m_new);
         if (j > 0 && __any_sync(0xffffffffu, m_used != -INFINITY)) {
-          // O holds tiles < j: wait for PV(j-1), then scale it in TMEM
-          if (!__all_sync(0xffffffffu, mbar_wait(&my_pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, status))) {
+          // O holds tiles < j: wait for PV(j-1), then scale O in TMEM
+          if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[x], (j - 1) & 1, status))) {
             ok = false;
             break;
           }
@@ -398,32 +399,27 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
         if (finite_new) m_used = m_new;
       }
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t pk[32];
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // P = 2^(v - base) as bf16 pairs, written over the first kKT/2 columns of S(j)
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        const float p0 = ex2_approx(v[i] - base), p1 = ex2_approx(v[i + 1] - base);
-        ls[(i >> 1) & 3] += p0 + p1;
-        pk[i >> 1] = pack_bf2(p0, p1);
+      for (int c = 0; c < kKT / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = ex2_approx(v[c * 32 + i] - base), p1 = ex2_approx(v[c * 32 + i + 1] - base);
+          ls[(i >> 1) & 3] += p0 + p1;
+          pk[i >> 1] = pack_bf2(p0, p1);
+        }
+        tmem_st16(tl + buf * kKT + c * 16, pk);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      if (j >= 2) {   // P buffer `buf` was read by PV(j-2)
-        if (!__all_sync(0xffffffffu, mbar_wait(&my_pv_done[buf], ((j - 2) >> 1) & 1, status))) {
-          ok = false;
-          break;
-        }
-      }
-      uint8_t* prow = my_p + buf * C::P_BYTES + row * 128;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<uint4*>(prow + ((u ^ (row & 7)) << 4)) =
-            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-      fence_proxy_async();   // P's generic-proxy stores -> visible to the tensor core
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&my_p_full[buf]);
+      if (lane == 0) mbar_arrive(&p_full[x * 2 + buf]);
     }
     const bool have = ok && n_tiles > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&my_pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, status));
+        __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (n_tiles - 1) & 1, status));
     const int ld = p.n_q * D;
     auto* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * S + q) * ld + (h0 + x) * D;
     // this row's 32 output columns [c, c + 32), scaled, as bf16
