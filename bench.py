@@ -83,7 +83,6 @@ def stage_work(cfg, routed_tokens, pairs):
         "rmsnorm_mlp": ("hbm", M * H * (4 + 2) + H * 2, "B"),
         "router_down": ("tensor", 2.0 * M * H * R, "FLOP"),
         "router_mlp": ("alu", 2.0 * M * (2 * R * R + R * E1), "FLOP"),
-        "permute": ("hbm", M * 4 * 3, "B"),
         "dispatch": ("hbm", routed_tokens * H * 2 * 2 + (M - routed_tokens) * H * 8, "B"),
         "experts_gate_up": ("tensor", 2.0 * routed_tokens * H * 2 * I, "FLOP"),
         "experts_down_merge": ("tensor", 2.0 * routed_tokens * I * H, "FLOP"),
@@ -346,7 +345,7 @@ def run_ours(args, world, rank, local):
 def kernel_source_sha(name):
     files = {"attention": "attn_tc.cu", "experts_gate_up": "gemm_tc.cu", "experts_down_merge": "gemm_tc.cu",
              "qkv_gemm": "gemm_tc.cu", "o_proj_merge": "gemm_tc.cu", "router_down": "gemm_tc.cu",
-             "router_mlp": "router.cu", "permute": "router.cu", "dispatch": "router.cu", "cca": "cca.cu",
+             "router_mlp": "router.cu", "dispatch": "router.cu", "cca": "cca.cu",
              "rmsnorm_attn": "norm.cu", "rmsnorm_mlp": "norm.cu"}
     f = files.get(name)
     if not f:

@@ -145,20 +145,25 @@ struct RouterParams {
   int* idx;               // optional [M]
   float* w;               // [M]
   float* w_tap;           // optional [M]
+  int* class_count;       // [E+1], zero on entry: tokens per class (atomic, one add per CTA and class)
+  int* slot;              // [M]: the token's place among its class's rows (order across CTAs unspecified)
   int M, R, E;
   float eps;
 };
 int launch_router(const RouterParams& p, cudaStream_t st);
 
-// Stable counting sort of tokens by class: pos[t] = permuted row of token t,
-// perm[row] = token; group_off[E+1]; mt_start[E+1] (tile_rows-row tiles).
-int launch_permute(const int* cls, int M, int E, int tile_rows, int* group_off, int* mt_start, int* pos, int* perm,
-                   int* status, cudaStream_t st);
 
 // Copies m_in rows of routed tokens into their permuted rows; writes the
 // merge-2 output of skipped (and padding) tokens; decode: cache_len += 1.
 struct DispatchParams {
-  const int* cls; const int* pos;
+  const int* cls;
+  const int* class_count; // [E+1] tokens per class (from the router)
+  const int* slot;        // [M] place of the token among its class's rows
+  int* pos;               // [M] out: permuted row of the token
+  int* perm;              // [M] out: token of each permuted row
+  int* group_off;         // [E+2] out: first permuted row of each class (written by CTA 0)
+  int* mt_start;          // [E+2] out: prefix of per-expert tile counts (tile_rows rows) (CTA 0)
+  int tile_rows;
   const void* m_in;       // bf16 [M, H]
   void* x_perm;           // bf16 [M, H]
   float* stream;          // [M, H] in: layer_mid; skip rows -> layer_output

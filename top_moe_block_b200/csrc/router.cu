@@ -1,6 +1,6 @@
-// Router MLP, scoring and top-1 choice with the skip class; the stable
-// token -> expert permutation; the dispatch of routed rows and the merge of
-// skipped rows.
+// Router MLP, scoring and top-1 choice with the skip class (each CTA also
+// reserves its tokens' places among their class's rows); the token -> expert
+// permutation with the dispatch of routed rows and the merge of skipped rows.
 //
 // Router (nnterp "zaya" page, "One expert per token, chosen beside a skip
 // class", and the ZayaRouterMLP printout): router_logits =
@@ -177,6 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   const int t0 = blockIdx.x * kTM;
   const int warp = warp_id(), lane = lane_id();
   const size_t n = (size_t)R * R;
+  __shared__ int s_cnt[96], s_cls[kTM], s_rank[kTM];   // per-class counts of this CTA's tokens
+  for (int c = threadIdx.x; c < 96; c += kThreads) s_cnt[c] = 0;
   // weight chunk q of the fc1 -> fc2 sequence into ring stage q & 1 (one cp.async group)
   auto stage_w = [&](int q) {
     const __nv_bfloat16* whi = p.wsplit + (size_t)(q / nch) * 2 * n;
@@ -378,8 +380,17 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
       p.w[t] = w;
       if (p.idx) p.idx[t] = skip ? 0 : cls;
       if (p.w_tap) p.w_tap[t] = w;
+      s_cls[tt] = cls;
+      s_rank[tt] = atomicAdd(&s_cnt[cls], 1);   // place among this CTA's tokens of the class
     }
   }
+  // one global add per class reserves this CTA's rows within the class
+  __syncthreads();
+  for (int c = threadIdx.x; c < E1; c += kThreads)
+    if (s_cnt[c]) s_cnt[c] = atomicAdd(p.class_count + c, s_cnt[c]);
+  __syncthreads();
+  for (int tt = threadIdx.x; tt < kTM; tt += kThreads)
+    if (t0 + tt < p.M) p.slot[t0 + tt] = s_cnt[s_cls[tt]] + s_rank[tt];
 }
 
 template <int R>
@@ -394,128 +405,68 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 
-// Stable counting sort by class, one CTA of 32 warps; warp w owns a
-// contiguous token range, so token order is kept inside every class.  Pass 1
-// counts per (warp, class); after the scans, pass 2 replays the same warp-local
-// ranking from the scanned offsets.  Each pass loads the next 32 classes
-// before it ranks the current ones.
-__device__ __forceinline__ int load_cls(const int* __restrict__ cls, int t, int end, int E, int* status) {
-  if (t >= end) return -1;
-  int c = cls[t];
-  if (c < 0 || c > E) {
-    set_status(status, ZAYA_ERR_DEVICE_RANGE);
-    c = E;
-  }
-  return c;
-}
-
-__global__ void __launch_bounds__(1024) permute_kernel(const int* __restrict__ cls, int M, int E, int tile_rows,
-                                                       int* group_off, int* mt_start, int* pos, int* perm,
-                                                       int* status) {
-  __shared__ int cnt[32][66];
-  __shared__ int cls_base[66];
-  const int warp = warp_id(), lane = lane_id();
-  const int E1 = E + 1;
-  for (int i = threadIdx.x; i < 32 * 66; i += blockDim.x) cnt[i / 66][i % 66] = 0;
-  __syncthreads();
-  const int per = ((M + 31) / 32 + 31) / 32 * 32;
-  const int begin = warp * per, end = min(M, begin + per);
-  const unsigned lt_mask = (1u << lane) - 1u;
-  {
-    int c_next = load_cls(cls, begin + lane, end, E, status);
-    for (int base = begin; base < end; base += 32) {
-      const int c = c_next;
-      c_next = load_cls(cls, base + 32 + lane, end, E, status);
-      const unsigned same = __match_any_sync(0xffffffffu, c);
-      const int leader = __ffs(same) - 1;
-      const int before = (c >= 0) ? cnt[warp][c] : 0;
-      __syncwarp();
-      if (c >= 0 && lane == leader) cnt[warp][c] = before + __popc(same);
-      __syncwarp();
-    }
-  }
-  __syncthreads();
-  // exclusive scan of cnt over (class-major, warp-minor)
-  for (int c = warp; c < E1; c += 32) {
-    int v = cnt[lane][c];
-    int inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += n;
-    }
-    cnt[lane][c] = inc - v;                              // offset of warp 'lane' inside class c
-    if (lane == 31) cls_base[c] = inc;                   // class total (scanned below)
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int carry = 0, tcarry = 0;
-    for (int c0 = 0; c0 < E1; c0 += 32) {
-      const int c = c0 + lane;
-      const int tot = c < E1 ? cls_base[c] : 0;
-      const int tiles = (c < E) ? (tot + tile_rows - 1) / tile_rows : 0;
-      int inc = tot, tinc = tiles;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, inc, o);
-        const int tn = __shfl_up_sync(0xffffffffu, tinc, o);
-        if (lane >= o) {
-          inc += n;
-          tinc += tn;
-        }
-      }
-      __syncwarp();
-      if (c < E1) {
-        cls_base[c] = carry + inc - tot;
-        group_off[c] = carry + inc - tot;
-        mt_start[c] = tcarry + tinc - tiles;
-      }
-      carry += __shfl_sync(0xffffffffu, inc, 31);
-      tcarry += __shfl_sync(0xffffffffu, tinc, 31);
-      __syncwarp();
-    }
-    if (lane == 0) {
-      mt_start[E1] = tcarry;   // unused entry past the skip class
-    }
-  }
-  __syncthreads();
-  for (int c = lane; c < E1; c += 32) cnt[warp][c] += cls_base[c];   // this warp's first row in class c
-  __syncwarp();
-  {
-    int c_next = load_cls(cls, begin + lane, end, E, nullptr);
-    for (int base = begin; base < end; base += 32) {
-      const int t = base + lane;
-      const int c = c_next;
-      c_next = load_cls(cls, base + 32 + lane, end, E, nullptr);
-      const unsigned same = __match_any_sync(0xffffffffu, c);
-      const int rank = __popc(same & lt_mask);
-      const int leader = __ffs(same) - 1;
-      const int first = (c >= 0) ? cnt[warp][c] : 0;
-      __syncwarp();
-      if (c >= 0 && lane == leader) cnt[warp][c] = first + __popc(same);
-      __syncwarp();
-      if (t < end) {
-        const int ps = first + rank;
-        pos[t] = ps;
-        perm[ps] = t;
-      }
-    }
-  }
-}
-
 // One warp per token row: routed tokens copy their m_in row to the permuted
 // row (all eight 16-byte loads of a lane in flight at once); skipped (and
 // padding) tokens write merge 2 with a zero routed output.
 __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
   const int t = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
+  const int E1 = p.E + 1;
+  // class offsets: exclusive prefix of the class counts (and, from CTA 0, the
+  // expert offsets and tile prefix the expert GEMMs read)
+  int cnt[3], tiles[3];
+#pragma unroll
+  for (int u = 0; u < 3; ++u) {
+    const int c = lane + 32 * u;
+    cnt[u] = c < E1 ? p.class_count[c] : 0;
+    tiles[u] = c < p.E ? (cnt[u] + p.tile_rows - 1) / p.tile_rows : 0;
+  }
+  int off[3], toff[3], carry = 0, tcarry = 0;
+#pragma unroll
+  for (int u = 0; u < 3; ++u) {
+    int inc = cnt[u], tinc = tiles[u];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, inc, o), b2 = __shfl_up_sync(0xffffffffu, tinc, o);
+      if (lane >= o) {
+        inc += a;
+        tinc += b2;
+      }
+    }
+    off[u] = carry + inc - cnt[u];
+    toff[u] = tcarry + tinc - tiles[u];
+    carry += __shfl_sync(0xffffffffu, inc, 31);
+    tcarry += __shfl_sync(0xffffffffu, tinc, 31);
+  }
+  if (blockIdx.x == 0 && warp_id() == 0) {
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+      const int c = lane + 32 * u;
+      if (c < E1) {
+        p.group_off[c] = off[u];
+        p.mt_start[c] = toff[u];
+      }
+    }
+    if (lane == 0) {
+      p.group_off[E1] = carry;
+      p.mt_start[E1] = tcarry;
+    }
+  }
   if (t >= p.M) return;
   const int H = p.H;
   const int per_row = H / 8;   // 16-byte chunks
-  const int c = p.cls[t];
-  if (c >= 0 && c < p.E) {
+  int c = p.cls[t];
+  if (c < 0 || c > p.E) c = p.E;
+  const int row = __shfl_sync(0xffffffffu, off[0], c & 31) * (c < 32) +
+                  __shfl_sync(0xffffffffu, off[1], c & 31) * (c >= 32 && c < 64) +
+                  __shfl_sync(0xffffffffu, off[2], c & 31) * (c >= 64) + p.slot[t];
+  if (lane == 0) {
+    p.pos[t] = row;
+    p.perm[row] = t;
+  }
+  if (c < p.E) {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * H);
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)p.pos[t] * H);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)row * H);
     constexpr int kV = 8;
     for (int c0 = 0; c0 < per_row; c0 += 32 * kV) {
       uint4 v[kV];
@@ -575,16 +526,9 @@ int launch_router(const RouterParams& p, cudaStream_t st) {
   }
 }
 
-int launch_permute(const int* cls, int M, int E, int tile_rows, int* group_off, int* mt_start, int* pos, int* perm,
-                   int* status, cudaStream_t st) {
-  if (E + 1 > 65 || tile_rows <= 0) return ZAYA_ERR_UNSUPPORTED;
-  permute_kernel<<<1, 1024, 0, st>>>(cls, M, E, tile_rows, group_off, mt_start, pos, perm, status);
-  return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
-}
-
 int launch_dispatch(const DispatchParams& p, cudaStream_t st) {
   if (p.M <= 0) return ZAYA_OK;
-  if (p.H % 8) return ZAYA_ERR_UNSUPPORTED;
+  if (p.H % 8 || p.E + 1 > 96 || p.tile_rows <= 0) return ZAYA_ERR_UNSUPPORTED;
   dispatch_kernel<<<(unsigned)((p.M + 7) / 8), 256, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }

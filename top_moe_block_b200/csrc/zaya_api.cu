@@ -147,7 +147,7 @@ int check_weights(const zaya_block_weights* w) {
 
 struct Ws {
   size_t status, a_in, qkv, q, premix, m_in, logits, cls, w, pos, perm, group_off, mt_start, xperm, act, part, rpart,
-      wsplit, total;
+      wsplit, slot, ccount, total;
 };
 
 Ws plan(const zaya_config& c, int mode, int B, int S) {
@@ -175,6 +175,8 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
                                            : attn_prefill_ws_bytes(B, S, c.window, d.nq, d.nkv, d.d));
   w.rpart = o; o += up((size_t)router_down_splits((int)M, d.H) * M * d.R * 4);
   w.wsplit = o; o += up((size_t)4 * d.R * d.R * 2);
+  w.slot = o; o += up(M * 4);
+  w.ccount = o; o += up((size_t)(d.E + 2) * 4);
   w.total = o;
   return w;
 }
@@ -263,6 +265,8 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.cls = cls; p.idx = taps ? taps->expert_indices : nullptr; p.w = wgt;
     p.w_tap = taps ? taps->expert_weights : nullptr;
     p.M = M; p.R = d.R; p.E = d.E; p.eps = c.rms_eps;
+    p.class_count = at<int>(ws, L.ccount); p.slot = at<int>(ws, L.slot);
+    if (cudaMemsetAsync(p.class_count, 0, (size_t)(d.E + 1) * 4, st) != cudaSuccess) return ZAYA_ERR_CUDA;
     ZAYA_STAGE("router_mlp", 2, launch_router(p, st));
   }
   int* group_off = at<int>(ws, L.group_off);
@@ -271,11 +275,12 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
   int* perm = at<int>(ws, L.perm);
   // expert GEMMs of prefill-sized batches run on CTA pairs (256-row tiles)
   const int pair = M >= kPairMinRows ? 1 : 0;
-  ZAYA_STAGE("permute", 1, launch_permute(cls, M, d.E, pair ? 256 : 128, group_off, mt_start, pos, perm, status, st));
   void* xperm = at<void>(ws, L.xperm);
-  {
+  {  // the token -> expert-row permutation, the copy of routed rows, merge 2 of skipped rows
     DispatchParams p{};
-    p.cls = cls; p.pos = pos; p.m_in = m_in; p.x_perm = xperm; p.stream = hidden; p.merge_m = w->merge_m;
+    p.cls = cls; p.class_count = at<int>(ws, L.ccount); p.slot = at<int>(ws, L.slot);
+    p.pos = pos; p.perm = perm; p.group_off = group_off; p.mt_start = mt_start; p.tile_rows = pair ? 256 : 128;
+    p.m_in = m_in; p.x_perm = xperm; p.stream = hidden; p.merge_m = w->merge_m;
     p.tap_mlp_out = taps ? taps->mlp_output : nullptr;
     p.cache_len_inc = cache_len_inc;
     p.M = M; p.H = d.H; p.E = d.E;
