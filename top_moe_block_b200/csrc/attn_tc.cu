@@ -31,7 +31,7 @@
 // Balance: causal rows differ in length (row tile i of a short sequence sees
 // i+1 key tiles), so when the longest row tile holds more key tiles than an
 // SM's share of the whole launch, row tiles are cut into key chunks of at
-// most that share.  The host lists the (row tile, chunk, head pair,
+// most two thirds of that share.  The host lists the (row tile, chunk, head pair,
 // sequence) items longest first; a chunk writes its unnormalised O with its
 // running max and sum (fp32), and the last chunk of a row tile to finish
 // (a per-row-tile counter) merges all chunks in chunk order:
@@ -91,9 +91,13 @@ bool plan_split(int B, int S, int window, int n_hp, AttnItems* items, int* n_slo
   total *= (long)B * n_hp;
   const double share = (double)total / kPlanSms;
   if (maxnt <= share) return false;
-  // chunks of about one SM's share: the in-order CTA dispatch then pairs the
-  // first round's long items with the second round's short ones
-  for (int L = std::max(kMinChunk, (int)(share + 0.999)); L < maxnt; L *= 2) {
+  // chunks of about two thirds of an SM's share: the in-order CTA dispatch
+  // then pairs the first round's long items with the later rounds' short
+  // ones.  Each item costs a pipeline fill and drain (Q load, first S, the O
+  // readout or partial write), so much shorter chunks lose more than the
+  // finer balance gains (measured at S = 4096: share/1.5 beat share, share/2
+  // and share/3).
+  for (int L = std::max(kMinChunk, (int)(share / 1.5 + 0.999)); L < maxnt; L *= 2) {
     long n_items = 0, slots = 0, ctrs = 0;
     bool fits = true;
     for (int rt = 0; rt < n_rt && fits; ++rt) {

@@ -408,9 +408,10 @@ __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
 // Prefill, streaming form: a thread owns 8 consecutive channels of one q/k
 // head (the d/8 threads of a head are adjacent lanes, so the head norm and the
 // RoPE pair exchange are shuffles inside that lane group) and walks kPerGroup
-// consecutive tokens, with its conv taps and bias in registers and the two
-// previous pre-conv values carried from step to step; kGroups such thread
-// groups split the CTA's kStream staged tokens.  Value heads: d/8 threads per
+// consecutive tokens, reading each token's three conv inputs (t-2, t-1, t)
+// and its taps and bias from shared memory (no values carried in registers:
+// 768 threads leave 85 registers a thread); kGroups such thread groups split
+// the CTA's kStream staged tokens.  Value heads: d/8 threads per
 // kv head copy the current / delayed halves.  Needs rot % 16 == 0 (a thread's
 // 8 dims are all inside or all outside the rotated range).
 constexpr int kGroups = 4;
@@ -439,13 +440,20 @@ __global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constan
   auto* u = reinterpret_cast<__nv_bfloat16*>(sm);                                 // [kStream + 2][ld]
   float2* cs = reinterpret_cast<float2*>(sm + (size_t)(kStream + 2) * ld * 2);    // [kStream][half]
   float* cbias = reinterpret_cast<float*>(cs + kStream * half);                    // [C]
+  float* cw = cbias + C;                                                           // [C][3] conv taps
   const auto* qkv = static_cast<const __nv_bfloat16*>(p.qkv);
   const size_t row0 = (size_t)b * p.S;
 
-  // rows s0-2 .. s0+kStream-1 (zero outside the sequence and at padding), one cp.async wait
+  // rows s0-2 .. s0+kStream-1 (zero outside the sequence and at padding), one
+  // cp.async wait; (row, 16-byte column) advance by blockDim.x vectors a step
   const int vec_per_row = ld / 8;
-  for (int i = threadIdx.x; i < (kStream + 2) * vec_per_row; i += blockDim.x) {
-    const int r = i / vec_per_row, c = i % vec_per_row;
+  const int dr = blockDim.x / vec_per_row, dc = blockDim.x % vec_per_row;
+  for (int r = threadIdx.x / vec_per_row, c = threadIdx.x % vec_per_row; r < kStream + 2; r += dr, c += dc) {
+    if (c >= vec_per_row) {
+      c -= vec_per_row;
+      ++r;
+      if (r >= kStream + 2) break;
+    }
     const int s = s0 - 2 + r;
     const bool valid = s >= 0 && s < p.S && (!p.mask || p.mask[row0 + s] != 0);
     const __nv_bfloat16* src = qkv + (row0 + (valid ? s : 0)) * ld + c * 8;
@@ -464,24 +472,15 @@ __global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constan
   const int grp = threadIdx.x / gthreads, tid = threadIdx.x % gthreads, lane = lane_id();
   const int tt0 = grp * kPerGroup;                        // this group's first token
   const int n_qk = (nq + nkv) * LPH;
-  // conv taps / bias of this thread's channels, loaded under the staging
-  float w0[8], w1[8], w2[8];
+  // conv bias and taps of the q||k channels into shared memory (read by every
+  // group each token, which keeps the token loop's registers below the cap
+  // of 768 threads per SM), loaded under the staging
   const int head = tid / LPH, l = tid % LPH;
   const int cb = head * D + l * 8;
-  if (grp == 0)   // conv bias of the q||k channels, shared by the groups
-    for (int i = tid; i < C / 4; i += gthreads)
-      reinterpret_cast<float4*>(cbias)[i] = __ldg(reinterpret_cast<const float4*>(p.conv_b) + i);
-  if (tid < n_qk) {
-    const float4* wp = reinterpret_cast<const float4*>(p.conv_w + 3 * cb);
-    float wv[24];
-#pragma unroll
-    for (int i = 0; i < 6; ++i) {
-      const float4 v = __ldg(wp + i);
-      wv[4 * i] = v.x; wv[4 * i + 1] = v.y; wv[4 * i + 2] = v.z; wv[4 * i + 3] = v.w;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { w0[i] = wv[3 * i]; w1[i] = wv[3 * i + 1]; w2[i] = wv[3 * i + 2]; }
-  }
+  for (int i = threadIdx.x; i < C / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(cbias)[i] = __ldg(reinterpret_cast<const float4*>(p.conv_b) + i);
+  for (int i = threadIdx.x; i < 3 * C / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(cw)[i] = __ldg(reinterpret_cast<const float4*>(p.conv_w) + i);
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
@@ -498,30 +497,36 @@ __global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constan
     const int src_lane = in_rot ? (lo ? lane + half / 8 : lane - half / 8) : lane;
     const int f0 = lo ? j0 : j0 - half;
     const int kcb = nq * D + g * D + l * 8;   // the group's key channels (query residual)
-    float x2[8], x1[8];
-    load8(u + (size_t)tt0 * ld + cb, x2);
-    load8(u + (size_t)(tt0 + 1) * ld + cb, x1);
+    const float4* wq = reinterpret_cast<const float4*>(cw + 3 * cb);   // taps (t-2, t-1, t) per channel
     __nv_bfloat16* dst = is_q ? static_cast<__nv_bfloat16*>(p.q_out) + (((size_t)b * nq + hh) * p.S + s0) * D + j0
                               : static_cast<__nv_bfloat16*>(p.k_cache) + (((size_t)b * nkv + hh) * p.cache_cap + s0) * D + j0;
     __nv_bfloat16* tap = (is_q && p.tap_q)
                              ? static_cast<__nv_bfloat16*>(p.tap_q) + (((size_t)b * nq + hh) * p.S + s0) * D + j0
                              : nullptr;
 #pragma unroll 1
-    for (int tt = tt0; tt < tt0 + kPerGroup; ++tt) {
+    for (int k = 0; k < kPerGroup; ++k) {
+      const int tt = tt0 + k;
       const int s = s0 + tt;
       if (s >= p.S) break;   // uniform over the head's lanes
       const __nv_bfloat16* row = u + (size_t)(tt + 2) * ld;
-      float x0[8], y[8];
+      float x2[8], x1[8], x0[8], y[8], wv[24];
+      load8(row - 2 * ld + cb, x2);
+      load8(row - ld + cb, x1);
       load8(row + cb, x0);
+#pragma unroll
+      for (int i = 0; i < 6; ++i) {
+        const float4 v = wq[i];
+        wv[4 * i] = v.x; wv[4 * i + 1] = v.y; wv[4 * i + 2] = v.z; wv[4 * i + 3] = v.w;
+      }
       const float4 bb0 = reinterpret_cast<const float4*>(cbias + cb)[0];
       const float4 bb1 = reinterpret_cast<const float4*>(cbias + cb)[1];
       const float bb[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float acc = bb[i];
-        acc = fmaf(w0[i], x2[i], acc);
-        acc = fmaf(w1[i], x1[i], acc);
-        acc = fmaf(w2[i], x0[i], acc);
+        acc = fmaf(wv[3 * i], x2[i], acc);
+        acc = fmaf(wv[3 * i + 1], x1[i], acc);
+        acc = fmaf(wv[3 * i + 2], x0[i], acc);
         y[i] = acc;
       }
       if (p.cca_res) {
@@ -578,8 +583,6 @@ __global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constan
         reinterpret_cast<uint4*>(cst)[0] = c0;
         reinterpret_cast<uint4*>(cst)[1] = c1;
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { x2[i] = x1[i]; x1[i] = x0[i]; }
     }
   } else if (tid < n_qk + nkv * LPH) {
     const int vt = tid - n_qk, g = vt / LPH, j0 = (vt % LPH) * 8;
@@ -614,7 +617,7 @@ int launch_cca(const CcaParams& p, cudaStream_t st) {
     const int lph = p.d / 8;
     const int nthr = kGroups * (((p.n_q + 2 * p.n_kv) * lph + 31) / 32 * 32);
     const size_t smem = (size_t)(kStream + 2) * p.n_qkv * 2 + (size_t)kStream * (p.rot / 2) * 8 +
-                        (size_t)(p.n_q + p.n_kv) * p.d * 4;
+                        (size_t)(p.n_q + p.n_kv) * p.d * 4 * 4;   // bias + three taps per q||k channel
     if (nthr <= 768 && smem <= 227 * 1024) {
       const dim3 grid((p.S + kStream - 1) / kStream, p.B);
       if (p.d == 128) {
