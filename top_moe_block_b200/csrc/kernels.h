@@ -147,6 +147,7 @@ struct RouterParams {
   float* w_tap;           // optional [M]
   int* class_count;       // [E+1], zero on entry: tokens per class (atomic, one add per CTA and class)
   int* slot;              // [M]: the token's place among its class's rows (order across CTAs unspecified)
+  int* status;            // device status word (a bounded wait that ran out records ZAYA_ERR_TIMEOUT)
   int M, R, E;
   float eps;
 };

@@ -15,6 +15,8 @@
 // softmax run in fp32 on CUDA cores.  32 tokens per CTA.
 #include <math.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -39,13 +41,27 @@ __device__ __forceinline__ void split_bf(float x, float& hi, float& lo) {
 template <int R>
 struct RouterShape {
   static constexpr int KCH = R < 64 ? R : 64;       // k columns per staged weight chunk
-  static constexpr int WS = KCH + 8;                // bf16 row stride of a chunk: conflict-free ldmatrix
+  // R >= 64: chunks arrive by TMA as [R rows][128 bytes] with the 128-byte
+  // swizzle (16-byte units XOR row & 7), which keeps ldmatrix conflict-free;
+  // R = 32: cp.async into rows padded to KCH + 8
+  static constexpr bool TMA = R >= 64;
+  static constexpr int WS = TMA ? KCH : KCH + 8;    // bf16 row stride of a chunk
   static constexpr int CHUNK = R * WS;              // bf16 elements of one (hi or lo) chunk
   static constexpr int NG = R / 8 < 8 ? R / 8 : 8;  // output groups (warp pairs)
   static constexpr int NTW = R / (8 * NG);          // 8-wide n-tiles per warp
-  static constexpr size_t SMEM = sizeof(float) * kTM * kZS + sizeof(__nv_bfloat16) * 2 * kTM * kAS +
-                                 sizeof(__nv_bfloat16) * 2 * 2 * CHUNK;
+  static constexpr size_t RING_OFF = sizeof(float) * kTM * kZS + sizeof(__nv_bfloat16) * 2 * kTM * kAS;
+  static constexpr size_t SMEM = RING_OFF + sizeof(__nv_bfloat16) * 2 * 2 * CHUNK + (TMA ? 1024 : 0);
 };
+
+// Byte offset of bf16 element (row, col) inside a staged weight chunk.
+template <int R>
+__device__ __forceinline__ uint32_t wofs(int row, int col) {
+  using Sh = RouterShape<R>;
+  if constexpr (Sh::TMA)
+    return (uint32_t)row * 128u + ((uint32_t)((col >> 3) ^ (row & 7)) << 4) + (uint32_t)(col & 7) * 2u;
+  else
+    return (uint32_t)(row * Sh::WS + col) * 2u;
+}
 
 // Stage columns [kc, kc+KCH) of the split weight (hi and lo, [R][R] bf16) into a padded chunk.
 template <int R>
@@ -91,8 +107,8 @@ __device__ __forceinline__ void mlp_chunk(const __nv_bfloat16* ah_t, const __nv_
         const int row = nbase + j * 8 + (m >> 1) * 8 + (lane & 7);
         const int col = ks * 16 + (m & 1) * 8;
         uint32_t bh0, bh1, bh2, bh3, bl0, bl1, bl2, bl3;
-        ldsm_x4(smem_u32(wh + row * Sh::WS + col), bh0, bh1, bh2, bh3);
-        ldsm_x4(smem_u32(wl + row * Sh::WS + col), bl0, bl1, bl2, bl3);
+        ldsm_x4(smem_u32(wh) + wofs<R>(row, col), bh0, bh1, bh2, bh3);
+        ldsm_x4(smem_u32(wl) + wofs<R>(row, col), bl0, bl1, bl2, bl3);
         mma16816(acc[j], ah, bh0, bh1);
         mma16816(acc[j + 1], ah, bh2, bh3);
         mma16816(acc[j], ah, bl0, bl1);
@@ -102,10 +118,12 @@ __device__ __forceinline__ void mlp_chunk(const __nv_bfloat16* ah_t, const __nv_
       } else {   // a single n-tile left: b fragments read directly (two bf16 per 32-bit word)
         const int row = nbase + j * 8 + g;
         const int col = ks * 16 + 2 * t;
-        const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(wh + row * Sh::WS + col);
-        const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(wh + row * Sh::WS + col + 8);
-        const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(wl + row * Sh::WS + col);
-        const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(wl + row * Sh::WS + col + 8);
+        const char* whb = reinterpret_cast<const char*>(wh);
+        const char* wlb = reinterpret_cast<const char*>(wl);
+        const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(whb + wofs<R>(row, col));
+        const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(whb + wofs<R>(row, col + 8));
+        const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(wlb + wofs<R>(row, col));
+        const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(wlb + wofs<R>(row, col + 8));
         mma16816(acc[j], ah, bh0, bh1);
         mma16816(acc[j], ah, bl0, bl1);
         mma16816(acc[j], al, bh0, bh1);
@@ -165,25 +183,50 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
 }
 
 template <int R>
-__global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams p) {
+__global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams p,
+                                                             const __grid_constant__ CUtensorMap tmW) {
   using Sh = RouterShape<R>;
   constexpr int nch = R / Sh::KCH;
   extern __shared__ __align__(16) float sm[];
   float* z = sm;                                                                // fp32 [kTM][kZS]
   __nv_bfloat16* zh = reinterpret_cast<__nv_bfloat16*>(z + kTM * kZS);          // bf16 hi [kTM][kAS]
   __nv_bfloat16* zl = zh + kTM * kAS;                                           // bf16 lo [kTM][kAS]
-  __nv_bfloat16* wring = zl + kTM * kAS;                                        // [2 stages][hi|lo][R][WS]
+  // [2 stages][hi|lo][R][WS]; 1024-byte aligned for the swizzled TMA chunks
+  __nv_bfloat16* wring = reinterpret_cast<__nv_bfloat16*>(
+      Sh::TMA ? (reinterpret_cast<uintptr_t>(zl + kTM * kAS) + 1023) & ~uintptr_t(1023)
+              : reinterpret_cast<uintptr_t>(zl + kTM * kAS));
+  __shared__ uint64_t wfull[2];   // TMA mode: chunk landed in ring stage s
   const int E1 = p.E + 1;
   const int t0 = blockIdx.x * kTM;
   const int warp = warp_id(), lane = lane_id();
   const size_t n = (size_t)R * R;
   __shared__ int s_cnt[96], s_cls[kTM], s_rank[kTM];   // per-class counts of this CTA's tokens
   for (int c = threadIdx.x; c < 96; c += kThreads) s_cnt[c] = 0;
-  // weight chunk q of the fc1 -> fc2 sequence into ring stage q & 1 (one cp.async group)
+  // weight chunk q of the fc1 -> fc2 sequence into ring stage q & 1: two TMA
+  // boxes (hi, lo) of [R rows][64 columns] on the stage's barrier, issued by
+  // thread 0; or (R = 32) one cp.async group of all threads
   auto stage_w = [&](int q) {
-    const __nv_bfloat16* whi = p.wsplit + (size_t)(q / nch) * 2 * n;
-    stage_chunk<R>(wring + (q & 1) * 2 * Sh::CHUNK, whi, whi + n, (q % nch) * Sh::KCH);
+    if constexpr (Sh::TMA) {
+      if (threadIdx.x == 0) {
+        uint64_t* bar = &wfull[q & 1];
+        mbar_arrive_expect_tx(bar, 2 * Sh::CHUNK * (uint32_t)sizeof(__nv_bfloat16));
+        const int row = (q / nch) * 2 * R;   // layer q / nch: hi rows, then lo rows
+        tma_load_2d(wring + (q & 1) * 2 * Sh::CHUNK, &tmW, bar, (q % nch) * Sh::KCH, row);
+        tma_load_2d(wring + (q & 1) * 2 * Sh::CHUNK + Sh::CHUNK, &tmW, bar, (q % nch) * Sh::KCH, row + R);
+      }
+    } else {
+      const __nv_bfloat16* whi = p.wsplit + (size_t)(q / nch) * 2 * n;
+      stage_chunk<R>(wring + (q & 1) * 2 * Sh::CHUNK, whi, whi + n, (q % nch) * Sh::KCH);
+    }
   };
+  if constexpr (Sh::TMA) {
+    if (threadIdx.x == 0) {
+      mbar_init(&wfull[0], 1);
+      mbar_init(&wfull[1], 1);
+      fence_barrier_init();
+      prefetch_tmap(&tmW);
+    }
+  }
   stage_w(0);   // the first fc1 chunk streams in under the state assembly
 
   // router state r = down_proj partial sums (in slab order) + bias (+ previous
@@ -284,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   float acc[Sh::NTW][4];
 #pragma unroll
   for (int j = 0; j < Sh::NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  bool ok = true;   // TMA mode: false once a chunk wait has run out (status set)
   for (int q = 0; q < 2 * nch; ++q) {
     if (q + 1 < 2 * nch) {
       stage_w(q + 1);
@@ -294,6 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
     asm volatile("cp.async.wait_group 1;" ::: "memory");
+    if constexpr (Sh::TMA) {   // every thread sees chunk q land (bounded wait)
+      if (ok && !mbar_wait(&wfull[q & 1], (uint32_t)(q >> 1) & 1u, p.status)) ok = false;
+    }
     __syncthreads();
     const __nv_bfloat16* wh = wring + (q & 1) * 2 * Sh::CHUNK;
     mlp_chunk<R>(zh, zl, acc, wh, wh + Sh::CHUNK, q % nch);
@@ -400,8 +447,15 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
   const size_t ow_bytes = (size_t)(p.E + 1) * R * sizeof(float);
   const size_t smem = Sh::SMEM + (ow_bytes <= 2 * Sh::CHUNK * sizeof(__nv_bfloat16) ? 0 : ow_bytes);
   if (smem > 227 * 1024) return ZAYA_ERR_UNSUPPORTED;
+  CUtensorMap mw;   // wsplit as [4R rows (layer, hi|lo, row)][R columns], boxes of R rows x 64 columns
+  memset(&mw, 0, sizeof(mw));
+  if constexpr (Sh::TMA) {
+    if (!p.status) return ZAYA_ERR_UNSUPPORTED;
+    const int rc = make_tmap_bf16(&mw, p.wsplit, (uint64_t)4 * R, (uint64_t)R, (uint32_t)R);
+    if (rc) return rc;
+  }
   cudaFuncSetAttribute(router_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  router_kernel<R><<<(p.M + kTM - 1) / kTM, kThreads, smem, st>>>(p);
+  router_kernel<R><<<(p.M + kTM - 1) / kTM, kThreads, smem, st>>>(p, mw);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 

@@ -265,7 +265,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.cls = cls; p.idx = taps ? taps->expert_indices : nullptr; p.w = wgt;
     p.w_tap = taps ? taps->expert_weights : nullptr;
     p.M = M; p.R = d.R; p.E = d.E; p.eps = c.rms_eps;
-    p.class_count = at<int>(ws, L.ccount); p.slot = at<int>(ws, L.slot);
+    p.class_count = at<int>(ws, L.ccount); p.slot = at<int>(ws, L.slot); p.status = status;
     if (cudaMemsetAsync(p.class_count, 0, (size_t)(d.E + 1) * 4, st) != cudaSuccess) return ZAYA_ERR_CUDA;
     ZAYA_STAGE("router_mlp", 2, launch_router(p, st));
   }
