@@ -136,7 +136,7 @@ struct RouterParams {
   const float* norm_w;
   const float* fc1_w; const float* fc1_b;
   const float* fc2_w; const float* fc2_b;
-  __nv_bfloat16* wsplit;  // workspace [2 layers][hi|lo][R][R] bf16: fc1/fc2 split for the tensor cores
+  __nv_bfloat16* wsplit;  // workspace bf16: [2 layers][hi|lo][R][R] (fc1, fc2), then [hi|lo][NP][R] (out_proj, E+1 rows padded to 8)
   const float* out_w;     // [E+1, R]
   const float* balancing; // [E+1]
   const int* mask;        // [M] token validity or null

@@ -8,11 +8,12 @@
 // being skip; p = softmax(logits) in fp32; class = argmax(p +
 // balancing_biases), the lowest index on exact ties; weight = p[class] (not
 // renormalised); skip -> (index 0, weight 0).  The choice is taken on fp32
-// scores, so the logits must carry fp32 accuracy: fc1 and fc2 run on tensor
-// cores with both operands split into bf16 hi + lo parts (three products
-// hi.hi + hi.lo + lo.hi, fp32 accumulation: ~16 significant bits per product,
-// about fp32's error after the 256-term sums); norm, GELU, out_proj and the
-// softmax run in fp32 on CUDA cores.  32 tokens per CTA.
+// scores, so the logits must carry fp32 accuracy: fc1, fc2 and out_proj run
+// on tensor cores with both operands split into bf16 hi + lo parts (three
+// products hi.hi + hi.lo + lo.hi, fp32 accumulation: ~16 significant bits per
+// product, about fp32's error after the 256-term sums); norm, GELU and the
+// softmax run in fp32 on CUDA cores.  32 tokens per CTA; the fc1 / fc2 weight
+// chunks arrive by TMA.
 #include <math.h>
 
 #include <cstring>
@@ -166,20 +167,38 @@ __device__ __forceinline__ void mlp_epilogue(float (*acc)[4], const float2* bias
   }
 }
 
+// Output classes padded to whole 8-wide MMA tiles.
+__host__ __device__ constexpr int router_np(int e1) { return (e1 + 7) / 8 * 8; }
+
 // fc1 / fc2 weights (fp32 [R][R]) -> bf16 hi and lo parts: wsplit = [layer][hi|lo][R][R];
+// then out_proj (fp32 [E1][R]) -> [hi|lo][NP][R] with zero rows from E1 on;
 // four elements per thread.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ fc1, const float* __restrict__ fc2,
+                                                           const float* __restrict__ out_w, int e1,
                                                            __nv_bfloat16* __restrict__ wsplit, int R) {
-  const int n4 = R * R / 4;
+  const int n4 = R * R / 4, r4 = R / 4, np = router_np(e1);
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= 2 * n4) return;
-  const int layer = i / n4, e4 = i % n4;
-  const float4 x = __ldg(reinterpret_cast<const float4*>(layer ? fc2 : fc1) + e4);
+  if (i >= 2 * n4 + np * r4) return;
+  float4 x;
+  __nv_bfloat16* hi;
+  __nv_bfloat16* lo;
+  int e4;
+  if (i < 2 * n4) {
+    const int layer = i / n4;
+    e4 = i % n4;
+    x = __ldg(reinterpret_cast<const float4*>(layer ? fc2 : fc1) + e4);
+    hi = wsplit + (size_t)layer * 2 * R * R;
+    lo = hi + R * R;
+  } else {
+    e4 = i - 2 * n4;
+    const int row = e4 / r4;
+    x = row < e1 ? __ldg(reinterpret_cast<const float4*>(out_w) + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    hi = wsplit + (size_t)4 * R * R;
+    lo = hi + (size_t)np * R;
+  }
   const float hx = round_bf(x.x), hy = round_bf(x.y), hz = round_bf(x.z), hw = round_bf(x.w);
-  __nv_bfloat16* base = wsplit + (size_t)layer * 2 * R * R;
-  reinterpret_cast<uint2*>(base)[e4] = make_uint2(pack_bf2(hx, hy), pack_bf2(hz, hw));
-  reinterpret_cast<uint2*>(base + R * R)[e4] =
-      make_uint2(pack_bf2(x.x - hx, x.y - hy), pack_bf2(x.z - hz, x.w - hw));
+  reinterpret_cast<uint2*>(hi)[e4] = make_uint2(pack_bf2(hx, hy), pack_bf2(hz, hw));
+  reinterpret_cast<uint2*>(lo)[e4] = make_uint2(pack_bf2(x.x - hx, x.y - hy), pack_bf2(x.z - hz, x.w - hw));
 }
 
 template <int R>
@@ -319,11 +338,13 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     }
   }
   // fc1 then fc2 (GELU after each): 2 * nch weight chunks through a two-stage
-  // ring, chunk q + 1 in flight while chunk q is multiplied; out_w follows the
-  // last chunk into the stage that chunk leaves free (or its own region).
-  const bool ow_in_ring = (size_t)E1 * R * sizeof(float) <= 2 * Sh::CHUNK * sizeof(__nv_bfloat16);
-  float* ow = ow_in_ring ? reinterpret_cast<float*>(wring + ((2 * nch) & 1) * 2 * Sh::CHUNK)
-                         : reinterpret_cast<float*>(wring + 4 * Sh::CHUNK);
+  // ring, chunk q + 1 in flight while chunk q is multiplied; the split out_proj
+  // weight ([hi|lo][NP][R + 8], padded rows) follows the last chunk into the
+  // stage that chunk leaves free (or its own region).
+  const int NP = router_np(E1);
+  constexpr int OWS = R + 8;
+  const bool ow_in_ring = (size_t)2 * NP * OWS <= (size_t)2 * Sh::CHUNK;
+  __nv_bfloat16* ow = ow_in_ring ? wring + ((2 * nch) & 1) * 2 * Sh::CHUNK : wring + 4 * Sh::CHUNK;
   float acc[Sh::NTW][4];
 #pragma unroll
   for (int j = 0; j < Sh::NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
@@ -332,9 +353,13 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     if (q + 1 < 2 * nch) {
       stage_w(q + 1);
     } else {
-      for (int i = threadIdx.x; i < E1 * R / 4; i += kThreads)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(ow + 4 * i)), "l"(p.out_w + 4 * i)
+      const __nv_bfloat16* ows = p.wsplit + (size_t)4 * R * R;   // [hi|lo][NP][R]
+      for (int i = threadIdx.x; i < 2 * NP * (R / 8); i += kThreads) {
+        const int row = i / (R / 8), c = i % (R / 8);   // row over hi rows then lo rows
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(ow + row * OWS + c * 8)),
+                     "l"(ows + (size_t)row * R + c * 8)
                      : "memory");
+      }
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
     asm volatile("cp.async.wait_group 1;" ::: "memory");
@@ -347,41 +372,52 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     if (q == nch - 1) {   // fc1 done: its GELU output becomes fc2's operand (in place)
       __syncthreads();
       mlp_epilogue<R>(acc, b1, zh, zl, nullptr);
-    } else if (q == 2 * nch - 1) {
-      mlp_epilogue<R>(acc, b2, nullptr, nullptr, z);
+    } else if (q == 2 * nch - 1) {   // fc2 done: its GELU output becomes out_proj's operand
+      __syncthreads();
+      mlp_epilogue<R>(acc, b2, zh, zl, nullptr);
     }
     __syncthreads();
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  // out_proj (no bias, fp32 on CUDA cores) and the choice, one warp per token
+  // out_proj (no bias) on tensor cores with the same hi / lo split: tile w < 2 * NP / 8
+  // (warps stride over them) is rows 16 * (w & 1) .. + 16 by classes 8 * (w >> 1) .. + 8
+  // over all of R; the logits go to shared memory (z, fp32 [kTM][kZS], free since
+  // fc2's epilogue)
+  for (int w = warp; w < 2 * (NP / 8); w += kThreads / 32) {
+    const int mt = w & 1, nt = w >> 1;
+    const int g = lane >> 2, tq = lane & 3;
+    const int arow = mt * 16 + (lane & 15);
+    const __nv_bfloat16* owh = ow + (nt * 8 + g) * OWS;
+    const __nv_bfloat16* owl = owh + NP * OWS;
+    float c4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int ks = 0; ks < R / 16; ++ks) {
+      const int acol = ks * 16 + (lane >> 4) * 8;
+      uint32_t ah[4], al[4];
+      ldsm_x4(smem_u32(zh + arow * kAS + acol), ah[0], ah[1], ah[2], ah[3]);
+      ldsm_x4(smem_u32(zl + arow * kAS + acol), al[0], al[1], al[2], al[3]);
+      const int col = ks * 16 + 2 * tq;
+      const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(owh + col);
+      const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(owh + col + 8);
+      const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(owl + col);
+      const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(owl + col + 8);
+      mma16816(c4, ah, bh0, bh1);
+      mma16816(c4, ah, bl0, bl1);
+      mma16816(c4, al, bh0, bh1);
+    }
+    const int r0 = mt * 16 + g, n0 = nt * 8 + 2 * tq;
+    *reinterpret_cast<float2*>(z + r0 * kZS + n0) = make_float2(c4[0], c4[1]);
+    *reinterpret_cast<float2*>(z + (r0 + 8) * kZS + n0) = make_float2(c4[2], c4[3]);
+  }
+  __syncthreads();
+  // softmax and the choice, one warp per token
   for (int tt = warp; tt < kTM; tt += kThreads / 32) {
     const int t = t0 + tt;
     if (t >= p.M) continue;
-    float zr[R / 32];
+    float l[3];
 #pragma unroll
-    for (int j = 0; j < R / 32; ++j) zr[j] = z[tt * kZS + lane + 32 * j];
-    float l[3] = {-INFINITY, -INFINITY, -INFINITY};
-    for (int c0 = 0; c0 < E1; c0 += 4) {   // four classes per round: independent chains
-      float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (c0 + u < E1) {
-          const float* wr = ow + (c0 + u) * R;
-#pragma unroll
-          for (int j = 0; j < R / 32; ++j) a[u] = fmaf(zr[j], wr[lane + 32 * j], a[u]);
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) a[u] += __shfl_xor_sync(0xffffffffu, a[u], o);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u;
-        if (c < E1 && (c & 31) == lane) l[c >> 5] = a[u];
-      }
-    }
+    for (int u = 0; u < 3; ++u) l[u] = (lane + 32 * u < E1) ? z[tt * kZS + lane + 32 * u] : -INFINITY;
     float mx = fmaxf(fmaxf(l[0], l[1]), l[2]);
     mx = warp_max(mx);
     float e[3], sum = 0.f;
@@ -443,9 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
 template <int R>
 int launch_router_r(const RouterParams& p, cudaStream_t st) {
   using Sh = RouterShape<R>;
-  router_split_kernel<<<(2 * R * R / 4 + 255) / 256, 256, 0, st>>>(p.fc1_w, p.fc2_w, p.wsplit, R);
-  const size_t ow_bytes = (size_t)(p.E + 1) * R * sizeof(float);
-  const size_t smem = Sh::SMEM + (ow_bytes <= 2 * Sh::CHUNK * sizeof(__nv_bfloat16) ? 0 : ow_bytes);
+  const int np = router_np(p.E + 1);
+  const int n_split = 2 * R * R / 4 + np * R / 4;
+  router_split_kernel<<<(n_split + 255) / 256, 256, 0, st>>>(p.fc1_w, p.fc2_w, p.out_w, p.E + 1, p.wsplit, R);
+  const size_t ow_elems = (size_t)2 * np * (R + 8);
+  const size_t smem = Sh::SMEM + (ow_elems <= (size_t)2 * Sh::CHUNK ? 0 : ow_elems * sizeof(__nv_bfloat16));
   if (smem > 227 * 1024) return ZAYA_ERR_UNSUPPORTED;
   CUtensorMap mw;   // wsplit as [4R rows (layer, hi|lo, row)][R columns], boxes of R rows x 64 columns
   memset(&mw, 0, sizeof(mw));

@@ -174,7 +174,7 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.part = o; o += up(mode == ZAYA_DECODE ? decode_attn_ws_bytes(B, d.nq, d.d, c.window)
                                            : attn_prefill_ws_bytes(B, S, c.window, d.nq, d.nkv, d.d));
   w.rpart = o; o += up((size_t)router_down_splits((int)M, d.H) * M * d.R * 4);
-  w.wsplit = o; o += up((size_t)4 * d.R * d.R * 2);
+  w.wsplit = o; o += up(((size_t)4 * d.R * d.R + (size_t)2 * ((d.E + 1 + 7) / 8 * 8) * d.R) * 2);   // fc1, fc2, out_proj hi / lo
   w.slot = o; o += up(M * 4);
   w.ccount = o; o += up((size_t)(d.E + 2) * 4);
   w.total = o;
