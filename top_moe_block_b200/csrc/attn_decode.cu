@@ -26,6 +26,7 @@ template <int D, int REP>
 __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams p) {
   constexpr int DPL = D / 32;
   constexpr int KPG = 32 / REP;  // keys per group: KPG * REP == 32 scores per warp step
+  griddep_begin();
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
   // A position outside the cache (already reported by the conv kernel) gives
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
 
 template <int D>
 __global__ void attn_decode_combine(const DecodeAttnParams p, int rep) {
+  griddep_begin();
   const int bh = blockIdx.x;
   const int b = bh / p.n_q, h = bh % p.n_q;
   const int g = h / rep, hh = h % rep;
@@ -206,8 +208,8 @@ int launch_attn_decode(const DecodeAttnParams& p, cudaStream_t st) {
   const dim3 grid(p.n_chunks, p.n_kv, p.B);
 #define ZAYA_DEC(DV, RV)                                                   \
   if (p.d == DV && rep == RV) {                                            \
-    attn_decode_kernel<DV, RV><<<grid, 32 * kWarps, 0, st>>>(p);           \
-    attn_decode_combine<DV><<<p.B * p.n_q, DV, 0, st>>>(p, RV);            \
+    launch_k(attn_decode_kernel<DV, RV>, grid, dim3(32 * kWarps), 0, st, nullptr, 0, p);          \
+    launch_k(attn_decode_combine<DV>, dim3(p.B * p.n_q), dim3(DV), 0, st, nullptr, 0, p, RV);   \
     return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;    \
   }
   ZAYA_DEC(128, 4)

@@ -251,6 +251,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_begin();   // the prologue above overlaps the previous kernel; global memory only from here
 
   if (warp == 0) {
     // ---------------- TMA producer: both heads' Q once, then K(j) and V(j) into their rings
@@ -558,7 +559,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTc<128>::SMEM);
       set = true;
     }
-    kern<<<grid, 64 + 32 * 4 * kHPC, AttnTc<128>::SMEM, st>>>(mq, mk, mv, p, items, status);
+    launch_k(kern, grid, dim3(64 + 32 * 4 * kHPC), AttnTc<128>::SMEM, st, nullptr, 0, mq, mk, mv, p, items, status);
   } else {
     auto kern = attn_tc_kernel<64>;
     static bool set = false;
@@ -566,7 +567,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTc<64>::SMEM);
       set = true;
     }
-    kern<<<grid, 64 + 32 * 4 * kHPC, AttnTc<64>::SMEM, st>>>(mq, mk, mv, p, items, status);
+    launch_k(kern, grid, dim3(64 + 32 * 4 * kHPC), AttnTc<64>::SMEM, st, nullptr, 0, mq, mk, mv, p, items, status);
   }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }

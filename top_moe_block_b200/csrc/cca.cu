@@ -119,6 +119,7 @@ __device__ __forceinline__ void rope_apply(float (&y)[D / 32], int lane, int pos
 template <int D>
 __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
   constexpr int DPL = D / 32;
+  griddep_begin();
   const int tok = blockIdx.x;
   const int b = p.decode ? tok : tok / p.S;
   const int s = p.decode ? 0 : tok % p.S;
@@ -257,6 +258,7 @@ constexpr int kTok = 16;
 template <int D>
 __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
   constexpr int DPL = D / 32;
+  griddep_begin();
   extern __shared__ __align__(16) uint8_t sm[];
   const int nq = p.n_q, nkv = p.n_kv, rep = nq / nkv;
   const int C = (nq + nkv) * D;
@@ -430,6 +432,7 @@ __device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
 template <int D>
 __global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constant__ CcaParams p) {
   constexpr int LPH = D / 8;   // threads per head
+  griddep_begin();
   extern __shared__ __align__(16) uint8_t sm[];
   const int nq = p.n_q, nkv = p.n_kv, rep = nq / nkv;
   const int C = (nq + nkv) * D;
@@ -622,10 +625,10 @@ int launch_cca(const CcaParams& p, cudaStream_t st) {
       const dim3 grid((p.S + kStream - 1) / kStream, p.B);
       if (p.d == 128) {
         cudaFuncSetAttribute(cca_stream_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        cca_stream_kernel<128><<<grid, nthr, smem, st>>>(p);
+        launch_k(cca_stream_kernel<128>, grid, dim3(nthr), smem, st, nullptr, 0, p);
       } else {
         cudaFuncSetAttribute(cca_stream_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        cca_stream_kernel<64><<<grid, nthr, smem, st>>>(p);
+        launch_k(cca_stream_kernel<64>, grid, dim3(nthr), smem, st, nullptr, 0, p);
       }
       return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
     }
@@ -635,19 +638,19 @@ int launch_cca(const CcaParams& p, cudaStream_t st) {
     const dim3 grid((p.S + kTok - 1) / kTok, p.B);
     if (p.d == 128) {
       cudaFuncSetAttribute(cca_prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      cca_prefill_kernel<128><<<grid, 512, smem, st>>>(p);
+      launch_k(cca_prefill_kernel<128>, grid, dim3(512), smem, st, nullptr, 0, p);
     } else if (p.d == 64) {
       cudaFuncSetAttribute(cca_prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      cca_prefill_kernel<64><<<grid, 512, smem, st>>>(p);
+      launch_k(cca_prefill_kernel<64>, grid, dim3(512), smem, st, nullptr, 0, p);
     } else {
       return ZAYA_ERR_UNSUPPORTED;
     }
     return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
   }
   if (p.d == 128)
-    cca_kernel<128><<<tokens, threads, 0, st>>>(p);
+    launch_k(cca_kernel<128>, dim3(tokens), dim3(threads), 0, st, nullptr, 0, p);
   else if (p.d == 64)
-    cca_kernel<64><<<tokens, threads, 0, st>>>(p);
+    launch_k(cca_kernel<64>, dim3(tokens), dim3(threads), 0, st, nullptr, 0, p);
   else
     return ZAYA_ERR_UNSUPPORTED;
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;

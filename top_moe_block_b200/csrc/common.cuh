@@ -37,6 +37,22 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation (launch_k) and starts with
+// griddep_begin(): it first waits until the previous kernel in the stream has
+// completed and its memory is visible (griddepcontrol.wait, before any global
+// read or write, so no kernel overtakes an older one that still reads a buffer
+// it writes), then lets the next kernel launch (griddepcontrol.launch_dependents).
+// The next kernel's launch and prologue (barrier init, TMEM allocation, smem
+// carve-out) then overlap this kernel's run and its tail.  The dependents of a
+// grid launch only once all of its CTAs have made the call, i.e. are resident,
+// so a waiting dependent never holds resources an unscheduled CTA of its
+// predecessor needs.
+__device__ __forceinline__ void griddep_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -337,6 +353,26 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
+}
+
+
+// Launch with programmatic stream serialisation (the kernel must begin with
+// griddep_begin()); extra launch attributes (a cluster shape) may be added.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            const cudaLaunchAttribute* extra, int n_extra, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[4];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  for (int i = 0; i < n_extra && i < 3; ++i) attr[1 + i] = extra[i];
+  cfg.attrs = attr;
+  cfg.numAttrs = 1 + (n_extra < 3 ? n_extra : 3);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
 
 }  // namespace zaya

@@ -340,6 +340,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_begin();   // the prologue above overlaps the previous kernel; global memory only from here
 
   const int ntiles = total_tiles<EPI, BN_OUT, TM>(p);
 
@@ -551,21 +552,18 @@ int launch_impl(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& 
   int units = ntiles_hint < max_units ? ntiles_hint : max_units;
   if (units < 1) units = 1;
   if constexpr (CG == 1) {
-    kern<<<units, 64 + 32 * epi_warps<EPI>(), C::SMEM_BYTES, st>>>(ma, mb, p);
+    if (launch_k(kern, dim3(units), dim3(64 + 32 * epi_warps<EPI>()), C::SMEM_BYTES, st, nullptr, 0, ma, mb, p) !=
+        cudaSuccess)
+      return ZAYA_ERR_CUDA;
   } else {
-    cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * units);
-    cfg.blockDim = dim3(64 + 32 * epi_warps<EPI>());
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, ma, mb, p) != cudaSuccess) return ZAYA_ERR_CUDA;
+    if (launch_k(kern, dim3(2 * units), dim3(64 + 32 * epi_warps<EPI>()), C::SMEM_BYTES, st, attr, 1, ma, mb, p) !=
+        cudaSuccess)
+      return ZAYA_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }

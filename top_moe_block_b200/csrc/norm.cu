@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(256, 4) rmsnorm_kernel(const float* __restrict
   constexpr int H = CHUNKS * 128;
   constexpr int G = CHUNKS < 8 ? CHUNKS : 8;   // float4 loads in flight per group
   __shared__ __align__(16) __nv_bfloat16 ws[H];   // the norm weight, staged once per CTA
+  griddep_begin();
   const int row = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   for (int i = threadIdx.x; i < H / 8; i += blockDim.x)
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(256, 4) rmsnorm_kernel(const float* __restrict
 __global__ void __launch_bounds__(256) embed_kernel(const int* __restrict__ ids, const __nv_bfloat16* __restrict__ table,
                                                     float* __restrict__ stream, int M, int H, int vocab, float mult,
                                                     float shift, int* status) {
+  griddep_begin();
   const int row = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   if (row >= M) return;
@@ -110,11 +112,11 @@ int launch_rmsnorm(const float* x, int row_mul, int row_add, const void* w, void
   auto* tb = static_cast<__nv_bfloat16*>(tap);
   const auto* cs = static_cast<const __nv_bfloat16*>(copy_src);
   switch (H / 128) {
-    case 2: rmsnorm_kernel<2><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
-    case 4: rmsnorm_kernel<4><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
-    case 8: rmsnorm_kernel<8><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
-    case 16: rmsnorm_kernel<16><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
-    case 32: rmsnorm_kernel<32><<<grid, 256, 0, st>>>(x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 2: launch_k(rmsnorm_kernel<2>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 4: launch_k(rmsnorm_kernel<4>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 8: launch_k(rmsnorm_kernel<8>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 16: launch_k(rmsnorm_kernel<16>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 32: launch_k(rmsnorm_kernel<32>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
     default: return ZAYA_ERR_UNSUPPORTED;
   }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
@@ -123,8 +125,8 @@ int launch_rmsnorm(const float* x, int row_mul, int row_add, const void* w, void
 int launch_embed(const int* ids, const void* table, float* stream, int M, int H, int vocab, float mult, float shift,
                  int* status, cudaStream_t st) {
   if (M <= 0) return ZAYA_OK;
-  embed_kernel<<<(M + 7) / 8, 256, 0, st>>>(ids, static_cast<const __nv_bfloat16*>(table), stream, M, H, vocab, mult,
-                                            shift, status);
+  launch_k(embed_kernel, dim3((M + 7) / 8), dim3(256), 0, st, nullptr, 0, ids,
+           static_cast<const __nv_bfloat16*>(table), stream, M, H, vocab, mult, shift, status);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 

@@ -176,6 +176,7 @@ __host__ __device__ constexpr int router_np(int e1) { return (e1 + 7) / 8 * 8; }
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ fc1, const float* __restrict__ fc2,
                                                            const float* __restrict__ out_w, int e1,
                                                            __nv_bfloat16* __restrict__ wsplit, int R) {
+  griddep_begin();
   const int n4 = R * R / 4, r4 = R / 4, np = router_np(e1);
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= 2 * n4 + np * r4) return;
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
                                                              const __grid_constant__ CUtensorMap tmW) {
   using Sh = RouterShape<R>;
   constexpr int nch = R / Sh::KCH;
+  griddep_begin();
   extern __shared__ __align__(16) float sm[];
   float* z = sm;                                                                // fp32 [kTM][kZS]
   __nv_bfloat16* zh = reinterpret_cast<__nv_bfloat16*>(z + kTM * kZS);          // bf16 hi [kTM][kAS]
@@ -481,7 +483,8 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
   using Sh = RouterShape<R>;
   const int np = router_np(p.E + 1);
   const int n_split = 2 * R * R / 4 + np * R / 4;
-  router_split_kernel<<<(n_split + 255) / 256, 256, 0, st>>>(p.fc1_w, p.fc2_w, p.out_w, p.E + 1, p.wsplit, R);
+  launch_k(router_split_kernel, dim3((n_split + 255) / 256), dim3(256), 0, st, nullptr, 0, p.fc1_w, p.fc2_w, p.out_w,
+           p.E + 1, p.wsplit, R);
   const size_t ow_elems = (size_t)2 * np * (R + 8);
   const size_t smem = Sh::SMEM + (ow_elems <= (size_t)2 * Sh::CHUNK ? 0 : ow_elems * sizeof(__nv_bfloat16));
   if (smem > 227 * 1024) return ZAYA_ERR_UNSUPPORTED;
@@ -493,7 +496,7 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
     if (rc) return rc;
   }
   cudaFuncSetAttribute(router_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  router_kernel<R><<<(p.M + kTM - 1) / kTM, kThreads, smem, st>>>(p, mw);
+  launch_k(router_kernel<R>, dim3((p.M + kTM - 1) / kTM), dim3(kThreads), smem, st, nullptr, 0, p, mw);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 
@@ -501,6 +504,7 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
 // row (all eight 16-byte loads of a lane in flight at once); skipped (and
 // padding) tokens write merge 2 with a zero routed output.
 __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
+  griddep_begin();
   const int t = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   const int E1 = p.E + 1;
@@ -621,7 +625,7 @@ int launch_router(const RouterParams& p, cudaStream_t st) {
 int launch_dispatch(const DispatchParams& p, cudaStream_t st) {
   if (p.M <= 0) return ZAYA_OK;
   if (p.H % 8 || p.E + 1 > 96 || p.tile_rows <= 0) return ZAYA_ERR_UNSUPPORTED;
-  dispatch_kernel<<<(unsigned)((p.M + 7) / 8), 256, 0, st>>>(p);
+  launch_k(dispatch_kernel, dim3((unsigned)((p.M + 7) / 8)), dim3(256), 0, st, nullptr, 0, p);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 
