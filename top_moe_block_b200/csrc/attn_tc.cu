@@ -527,6 +527,15 @@ size_t attn_prefill_ws_bytes(int B, int S, int window, int n_q, int n_kv, int d)
   return (size_t)n_slots * slot_bytes(d) + (size_t)n_ctr * 4;
 }
 
+int attn_prefill_ctr(int B, int S, int window, int n_q, int d, size_t* byte_off) {
+  *byte_off = 0;
+  if (B <= 0 || S <= 0 || n_q % kHPC) return 0;
+  int n_slots = 0, n_ctr = 0;
+  if (!plan_split(B, S, window, n_q / kHPC, nullptr, &n_slots, &n_ctr)) return 0;
+  *byte_off = (size_t)n_slots * slot_bytes(d);
+  return n_ctr;
+}
+
 int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
   if (p.B <= 0 || p.S <= 0) return ZAYA_OK;
   if (p.d != 128 && p.d != 64) return ZAYA_ERR_UNSUPPORTED;
@@ -545,7 +554,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
     items.po = static_cast<float*>(p.part);
     items.pml = items.po + (size_t)n_slots * kHPC * p.d * kQT;
     items.ctr = reinterpret_cast<int*>(items.pml + (size_t)n_slots * kHPC * 2 * kQT);
-    if (cudaMemsetAsync(items.ctr, 0, (size_t)n_ctr * 4, st) != cudaSuccess) return ZAYA_ERR_CUDA;
+    if (!p.ctr_cleared && cudaMemsetAsync(items.ctr, 0, (size_t)n_ctr * 4, st) != cudaSuccess) return ZAYA_ERR_CUDA;
     grid = dim3(items.n_items, 1, 1);
   } else {
     items.n_items = 0;

@@ -259,6 +259,8 @@ template <int D>
 __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
   constexpr int DPL = D / 32;
   griddep_begin();
+  if (p.zero_words && blockIdx.x == 0 && blockIdx.y == 0)   // the attention's merge counters
+    for (int i = threadIdx.x; i < p.n_zero_words; i += blockDim.x) p.zero_words[i] = 0;
   extern __shared__ __align__(16) uint8_t sm[];
   const int nq = p.n_q, nkv = p.n_kv, rep = nq / nkv;
   const int C = (nq + nkv) * D;
@@ -433,6 +435,8 @@ template <int D>
 __global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constant__ CcaParams p) {
   constexpr int LPH = D / 8;   // threads per head
   griddep_begin();
+  if (p.zero_words && blockIdx.x == 0 && blockIdx.y == 0)   // the attention's merge counters
+    for (int i = threadIdx.x; i < p.n_zero_words; i += blockDim.x) p.zero_words[i] = 0;
   extern __shared__ __align__(16) uint8_t sm[];
   const int nq = p.n_q, nkv = p.n_kv, rep = nq / nkv;
   const int C = (nq + nkv) * D;

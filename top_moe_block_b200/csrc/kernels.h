@@ -92,6 +92,8 @@ struct CcaParams {
   float theta, eps;
   int decode;             // 1: one token per sequence, history from conv_state
   int* status;
+  int* zero_words;        // prefill: words CTA 0 clears for the next kernel (attention's merge counters), or null
+  int n_zero_words;
   float inv_freq[64];     // RoPE inverse frequencies theta^(-2i/rot), i < rot/2 (fp32)
 };
 int launch_cca(const CcaParams& p, cudaStream_t st);
@@ -107,7 +109,11 @@ struct AttnParams {
   float scale;
   void* part;             // split-KV partials + merge counters (attn_prefill_ws_bytes)
   size_t part_bytes;
+  int ctr_cleared;        // 1: the merge counters (attn_prefill_ctr) were cleared by the previous kernel
 };
+// The merge counters inside `part` for these sizes: returns their count (0
+// without a split) and their byte offset; they must be zero at launch.
+int attn_prefill_ctr(int B, int S, int window, int n_q, int d, size_t* byte_off);
 // Workspace bytes of the split-KV plan for these sizes (0 when no row tile is split).
 size_t attn_prefill_ws_bytes(int B, int S, int window, int n_q, int n_kv, int d);
 int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st);
@@ -145,7 +151,7 @@ struct RouterParams {
   int* idx;               // optional [M]
   float* w;               // [M]
   float* w_tap;           // optional [M]
-  int* class_count;       // [E+1], zero on entry: tokens per class (atomic, one add per CTA and class)
+  int* class_count;       // [E+1] tokens per class (cleared by the launch, then one atomic add per CTA and class)
   int* slot;              // [M]: the token's place among its class's rows (order across CTAs unspecified)
   int* status;            // device status word (a bounded wait that ran out records ZAYA_ERR_TIMEOUT)
   int M, R, E;

@@ -172,11 +172,14 @@ __host__ __device__ constexpr int router_np(int e1) { return (e1 + 7) / 8 * 8; }
 
 // fc1 / fc2 weights (fp32 [R][R]) -> bf16 hi and lo parts: wsplit = [layer][hi|lo][R][R];
 // then out_proj (fp32 [E1][R]) -> [hi|lo][NP][R] with zero rows from E1 on;
-// four elements per thread.
+// four elements per thread.  Block 0 also clears the router's per-class counts
+// (a kernel, not a memset, keeps the launch chain programmatic).
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ fc1, const float* __restrict__ fc2,
                                                            const float* __restrict__ out_w, int e1,
-                                                           __nv_bfloat16* __restrict__ wsplit, int R) {
+                                                           __nv_bfloat16* __restrict__ wsplit, int R,
+                                                           int* __restrict__ class_count) {
   griddep_begin();
+  if (blockIdx.x == 0 && threadIdx.x < e1) class_count[threadIdx.x] = 0;
   const int n4 = R * R / 4, r4 = R / 4, np = router_np(e1);
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= 2 * n4 + np * r4) return;
@@ -484,7 +487,7 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
   const int np = router_np(p.E + 1);
   const int n_split = 2 * R * R / 4 + np * R / 4;
   launch_k(router_split_kernel, dim3((n_split + 255) / 256), dim3(256), 0, st, nullptr, 0, p.fc1_w, p.fc2_w, p.out_w,
-           p.E + 1, p.wsplit, R);
+           p.E + 1, p.wsplit, R, p.class_count);
   const size_t ow_elems = (size_t)2 * np * (R + 8);
   const size_t smem = Sh::SMEM + (ow_elems <= (size_t)2 * Sh::CHUNK ? 0 : ow_elems * sizeof(__nv_bfloat16));
   if (smem > 227 * 1024) return ZAYA_ERR_UNSUPPORTED;
@@ -612,7 +615,7 @@ __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
 
 int launch_router(const RouterParams& p, cudaStream_t st) {
   if (p.M <= 0) return ZAYA_OK;
-  if (p.E + 1 > 96 || p.n_splits < 1 || !p.wsplit) return ZAYA_ERR_UNSUPPORTED;
+  if (p.E + 1 > 96 || p.n_splits < 1 || !p.wsplit || !p.class_count) return ZAYA_ERR_UNSUPPORTED;
   switch (p.R) {
     case 32: return launch_router_r<32>(p, st);
     case 64: return launch_router_r<64>(p, st);

@@ -266,7 +266,6 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.w_tap = taps ? taps->expert_weights : nullptr;
     p.M = M; p.R = d.R; p.E = d.E; p.eps = c.rms_eps;
     p.class_count = at<int>(ws, L.ccount); p.slot = at<int>(ws, L.slot); p.status = status;
-    if (cudaMemsetAsync(p.class_count, 0, (size_t)(d.E + 1) * 4, st) != cudaSuccess) return ZAYA_ERR_CUDA;
     ZAYA_STAGE("router_mlp", 2, launch_router(p, st));
   }
   int* group_off = at<int>(ws, L.group_off);
@@ -354,11 +353,15 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     p.B = B; p.S = S; p.H = d.H; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.rot = c.rot_dim;
     p.cca_res = c.cca_mean_residual; p.v_delayed = c.v_delayed; p.theta = c.rope_theta; p.eps = c.qk_norm_eps;
     p.decode = 0; p.status = status;
+    size_t ctr_off = 0;   // the attention's split merge counters, cleared by this kernel
+    p.n_zero_words = attn_prefill_ctr(B, S, c.window, d.nq, d.d, &ctr_off);
+    p.zero_words = p.n_zero_words ? reinterpret_cast<int*>(at<uint8_t>(ws, L.part) + ctr_off) : nullptr;
     fill_inv_freq(p.inv_freq, c.rot_dim, c.rope_theta);
     ZAYA_STAGE("cca", 1, launch_cca(p, st));
   }
   {
     AttnParams p{};
+    p.ctr_cleared = 1;
     p.q = at<void>(ws, L.q); p.k_cache = state->k_cache; p.v_cache = state->v_cache; p.mask = mask;
     p.out = at<void>(ws, L.premix);
     p.B = B; p.S = S; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = c.window;
