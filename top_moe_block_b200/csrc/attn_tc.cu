@@ -6,21 +6,27 @@
 // key j is not padding (nnterp "zaya" page: grouped-query eager softmax
 // attention).  A query with no visible key outputs 0.
 //
-// CTA = 128 queries of two query heads that share a kv head, 10 warps:
-//   warp 0     TMA: both heads' Q tiles once, then K and V tiles of 64 keys
-//              into a 3-slot and a 2-slot ring (128-byte swizzle, 64-wide d
-//              atoms), shared by the two heads;
-//   warp 1     one thread issues tcgen05.mma: per head, S(j) = Q K^T into one
-//              of two S buffers in tensor memory; once the softmax has written
-//              P(j) over it, O += P V with P read straight from tensor memory
-//              (A operand in TMEM) and V from shared memory as an MN-major
+// CTA = 128 queries of one query head, 6 warps, two CTAs per SM (256 TMEM
+// columns and ~98 KB of shared memory each), so that one CTA's pipeline fill
+// and drain (Q load, first S, the O readout or partial write) overlap the
+// other's steady state (measured 72 us against 77 us for one CTA of two heads
+// per SM at S = 4096):
+//   warp 0     TMA: the head's Q tile once, then K and V tiles of 64 keys
+//              into a 2-slot and a 2-slot ring (128-byte swizzle, 64-wide d
+//              atoms);
+//   warp 1     one thread issues tcgen05.mma: S(j) = Q K^T into one of two S
+//              buffers in tensor memory; once the softmax has written P(j)
+//              over it, O += P V with P read straight from tensor memory (A
+//              operand in TMEM) and V from shared memory as an MN-major
 //              operand, then S(j+2) into the same buffer: S runs two tiles
-//              ahead of the softmax and the two heads alternate;
-//   warps 2-9  softmax, a warpgroup per head, one thread per query row (its
-//              TMEM lane): row max and sum are thread-local; P goes back into
-//              the S columns as bf16 pairs (tcgen05.st).  The running max is
-//              only moved (and O rescaled in TMEM) when it grows by more than
-//              2^8, which keeps P <= 256 and the result exact.
+//              ahead of the softmax;
+//   warps 2-5  softmax, one thread per query row (its TMEM lane): row max
+//              and sum are thread-local; P goes back into the S columns as
+//              bf16 pairs (tcgen05.st).  The running max is only moved (and O
+//              rescaled in TMEM) when it grows by more than 2^8, which keeps
+//              P <= 256 and the result exact.
+// The code is written for kHPC query heads per CTA (sharing the K / V tiles);
+// kHPC = 2 with one CTA per SM measured slower.
 // Shared memory carries only Q, K and V (P never leaves tensor memory): a
 // version with P staged in shared memory was measured to be limited by
 // shared-memory bandwidth, and one with a single S buffer per head by the
@@ -29,10 +35,10 @@
 // only on tiles that straddle the diagonal, the window edge, the sequence
 // end or a padding mask.
 // Balance: causal rows differ in length (row tile i of a short sequence sees
-// i+1 key tiles), so when the longest row tile holds more key tiles than an
-// SM's share of the whole launch, row tiles are cut into key chunks of at
-// most two thirds of that share.  The host lists the (row tile, chunk, head pair,
-// sequence) items longest first; a chunk writes its unnormalised O with its
+// i+1 key tiles), so when the longest row tile holds more key tiles than a
+// CTA slot's share of the whole launch (two slots per SM), row tiles are cut
+// into key chunks of at most two thirds of that share.  The host lists the
+// (row tile, chunk, head, sequence) items longest first; a chunk writes its unnormalised O with its
 // running max and sum (fp32), and the last chunk of a row tile to finish
 // (a per-row-tile counter) merges all chunks in chunk order:
 // O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c, M = max_c m_c.
@@ -49,19 +55,19 @@ namespace {
 
 constexpr int kQT = 128;  // queries per CTA
 constexpr int kKT = 64;   // keys per tile
-constexpr int kHPC = 2;   // query heads per CTA (sharing one kv head)
-constexpr int kRing = 3;  // K ring depth (S runs two tiles ahead)
+constexpr int kHPC = 1;   // query heads per CTA (sharing one kv head)
+constexpr int kRing = 2;  // K ring depth (S runs two tiles ahead)
 constexpr int kRingV = 2; // V ring depth
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kMaxItems = 512;   // split-plan items carried in the kernel parameters
-constexpr int kPlanSms = 148;    // the SM count the split plan balances over
+constexpr int kMaxItems = 1024;  // split-plan items carried in the kernel parameters (16 KB)
+constexpr int kPlanSms = 296;    // the CTA slots the split plan balances over (148 SMs x 2)
 constexpr int kMinChunk = 4;     // fewest key tiles in a chunk
 
 struct AttnItems {
-  int n_items;   // 0: grid (row tiles, head pairs, sequences), no row tile split
+  int n_items;   // 0: grid (row tiles, head groups of kHPC, sequences), no row tile split
   float* po;     // partial O, per slot [kHPC][d][kQT] fp32 (row index fastest)
   float* pml;    // per slot [kHPC][2][kQT] fp32: running max (log2 units), running sum
-  int* ctr;      // per split (row tile, head pair, sequence): chunks finished
+  int* ctr;      // per split (row tile, head group, sequence): chunks finished
   uint4 it[kMaxItems];   // {rt | c << 16 | nc << 24, b | hp << 16, first slot of the group, counter}
 };
 
@@ -152,14 +158,15 @@ struct AttnTc {
   static constexpr int Q_BYTES = SUB * Q_ATOM;     // one head's Q tile
   static constexpr int KV_BYTES = SUB * KV_ATOM;   // one K (or V) tile
   static constexpr int SMEM_USED = 1024 + kHPC * Q_BYTES + (kRing + kRingV) * KV_BYTES + 512;
-  // at least 120 KB so a second CTA never shares the SM (and its TMEM)
-  static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-  static constexpr uint32_t TMEM_COLS = 512;       // per head: S0 / P0 [0, 64), S1 / P1 [64, 128), O [128, 128 + D)
+  static constexpr int SMEM = SMEM_USED;           // two CTAs per SM
+  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+  // per head: S0 / P0 [0, 64), S1 / P1 [64, 128), O [128, 128 + D); two CTAs share the 512 columns
+  static constexpr uint32_t TMEM_COLS = kHPC * 256;
   static constexpr uint32_t HEAD_COLS = 256;
   static constexpr uint32_t O_COL = 2 * kKT;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, kKT);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32_bmn(128, D);
-  static_assert(kHPC * (2 * kKT + D) <= 512, "tensor memory");
+  static_assert(kHPC * (2 * kKT + D) <= 256, "tensor memory: two CTAs per SM");
 };
 
 // 2^x on the special-function unit (inputs <= 0 here; results below 2^-126
@@ -175,7 +182,7 @@ __device__ __forceinline__ bool key_visible(int q, int key, int window, int S, c
 }
 
 template <int D>
-__global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
+__global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams p,
                    const __grid_constant__ AttnItems items, int* status) {
@@ -197,7 +204,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + kHPC);
   int* s_last = reinterpret_cast<int*>(tmem_slot + 1);
 
-  // this CTA's item: a row tile of two heads, or one key chunk of it
+  // this CTA's item: a row tile of its kHPC heads, or one key chunk of it
   int qb, hp, b, chunk = 0, n_chunks = 1, slot0 = 0, ctr = 0;
   if (items.n_items) {
     const uint4 it = items.it[blockIdx.x];
@@ -254,7 +261,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
   griddep_begin();   // the prologue above overlaps the previous kernel; global memory only from here
 
   if (warp == 0) {
-    // ---------------- TMA producer: both heads' Q once, then K(j) and V(j) into their rings
+    // ---------------- TMA producer: the heads' Q once, then K(j) and V(j) into their rings
     if (elect_one()) {
       const int kv_row = (b * p.n_kv + g) * p.cap + n_begin + t_begin * kKT;
       mbar_arrive_expect_tx(q_full, kHPC * C::Q_BYTES);
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 1)
     // softmax writes P(j) over it; O += P(j) V(j) with P read from tensor
     // memory; then S(j+2) into the same buffer (the tensor pipe runs one
     // thread's MMAs in issue order, so S(j+2) is written after P(j) is read).
-    // S runs two tiles ahead of the softmax, and the two heads alternate.
+    // S runs two tiles ahead of the softmax (with kHPC > 1 the heads alternate).
     if (elect_one()) {
       bool ok = mbar_wait(q_full, 0, status);
       auto issue_qk = [&](int x, int j) {
