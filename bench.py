@@ -5,7 +5,10 @@
 
 A step is one pass of the whole block (every stage of the hot path) over one
 batch of the workload's synthetic input; the default workload is the
-full-width single-block prefill, B1 x S4096.  Under torchrun (N > 1) every
+full-width single-block prefill, B1 x S4096.  `--workload decode_stack_b64`
+times the decode workload instead: one step is one new token for each of 64
+sequences through the 40-block stack (8192 cached tokens, window 4096) and
+the tied lm_head, HBM-bound, reported against the HBM roofline.  Under torchrun (N > 1) every
 rank runs its own replica on its own GPU (independent sequences, no data
 exchange: weak scaling); NCCL carries only the barrier and the max-over-ranks
 of the device time.  Rank 0 prints one JSON line.
@@ -46,6 +49,8 @@ def parse_args():
     ap.add_argument("--workload", default="prefill_4k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stages", action="store_true", help="print the per-stage table to stderr")
+    ap.add_argument("--n-blocks", type=int, default=0,
+                    help="decode stack only: run this many blocks instead of the workload's (a small case for ncu)")
     return ap.parse_args()
 
 
@@ -86,6 +91,32 @@ def stage_work(cfg, routed_tokens, pairs):
         "dispatch": ("hbm", routed_tokens * H * 2 * 2 + (M - routed_tokens) * H * 8, "B"),
         "experts_gate_up": ("tensor", 2.0 * routed_tokens * H * 2 * I, "FLOP"),
         "experts_down_merge": ("tensor", 2.0 * routed_tokens * I * H, "FLOP"),
+    }
+
+
+def stage_work_decode(cfg, routed, distinct):
+    """Per-launch algorithmic HBM bytes of each stage of one decode step of a
+    block (and of the stack's embed / final norm / lm_head): weights once,
+    only the distinct experts hit, the window's K / V only, activations once."""
+    B, H, R, E1, I = cfg.batch, cfg.hidden, cfg.router_hidden, cfg.n_experts + 1, cfg.inter
+    qd, kvd, nqkv, d = cfg.q_dim, cfg.kv_dim, cfg.n_qkv, cfg.head_dim
+    keys = min(cfg.window, cfg.cache_prior + 1)
+    C = cfg.qk_channels
+    return {
+        "rmsnorm_attn": ("hbm", B * H * 4 + 2 * B * H * 2 + H * 2, "B"),
+        "qkv_gemm": ("hbm", nqkv * H * 2 + 2 * B * H * 2 + 2 * B * nqkv * 2, "B"),
+        "cca": ("hbm", 2 * B * nqkv * 2 + B * (qd + 2 * kvd) * 2 + B * C * 2 * 2 * 2 + B * H * 2, "B"),
+        "attention_decode": ("hbm", B * cfg.n_kv * keys * d * 2 * 2 + 2 * B * qd * 2, "B"),
+        "o_proj_merge": ("hbm", H * qd * 2 + B * qd * 2 + B * H * 4 * 2, "B"),
+        "rmsnorm_mlp": ("hbm", B * H * 4 + B * H * 2 + H * 2, "B"),
+        "router_down": ("hbm", R * H * 2 + B * H * 2 + B * R * 4, "B"),
+        "router_mlp": ("hbm", 2 * R * R * 4 + E1 * R * 4 + B * R * 4 * 2, "B"),
+        "dispatch": ("hbm", routed * H * 2 * 2 + (B - routed) * H * 8, "B"),
+        "experts_gate_up": ("hbm", distinct * 2 * I * H * 2 + routed * H * 2 + routed * I * 2, "B"),
+        "experts_down_merge": ("hbm", distinct * H * I * 2 + routed * I * 2 + B * H * 4 * 2, "B"),
+        "embed": ("hbm", B * H * 2 + B * H * 4, "B"),
+        "final_norm": ("hbm", B * H * 4 + B * H * 2, "B"),
+        "lm_head": ("hbm", cfg.vocab * H * 2 + B * H * 2 + B * cfg.vocab * 2, "B"),
     }
 
 
@@ -209,8 +240,12 @@ def run_ours(args, world, rank, local):
     from top_moe_block_b200 import build
     build.build()
     cfg = get_config(args.workload)
+    if cfg.mode == "decode" and cfg.n_blocks > 1:
+        if args.n_blocks > 0:
+            cfg = cfg.with_(n_blocks=args.n_blocks)
+        return run_decode(args, world, rank, local, cfg)
     if cfg.mode != "prefill" or cfg.n_blocks != 1:
-        raise SystemExit(f"workload {cfg.name}: only single-block prefill workloads are timed by bench.py")
+        raise SystemExit(f"workload {cfg.name}: bench.py times single-block prefill and the decode stack")
     dev = torch.device("cuda", local)
     W = gen_block_weights(cfg)
     Wd = {k: v.to(dev).contiguous() for k, v in W.items()}
@@ -334,6 +369,126 @@ def run_ours(args, world, rank, local):
         "cpu_baseline": cpu,
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items()},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, world, rank, local, cfg):
+    """The decode workload: one token per sequence through the whole stack."""
+    import torch
+    import top_moe_block_b200 as ZB
+    from synthetic import gen_block_weights, gen_decode_state, gen_stack_weights_extra, gen_token_ids
+    dev = torch.device("cuda", local)
+    B, H, V, L = cfg.batch, cfg.hidden, cfg.vocab, cfg.cache_prior
+    K = args.steps
+    cap = L + args.warmup + 3 * K + 8   # every step appends one token; the window keeps the work fixed
+    blocks = [gen_block_weights(cfg, block=i, device=dev) for i in range(cfg.n_blocks)]
+    extra = gen_stack_weights_extra(cfg, device=dev)
+    states = [gen_decode_state(cfg, i, cap, device=dev) for i in range(cfg.n_blocks)]
+    ids = gen_token_ids(cfg)[:, 0].contiguous().to(dev)
+    c = ZB.make_config(cfg)
+    ws = torch.zeros(ZB.zaya_stack_workspace_size(c, ZB.ZAYA_DECODE, B, 1), dtype=torch.uint8, device=dev)
+    logits = torch.empty(B, V, dtype=torch.bfloat16, device=dev)
+    w_s = [ZB.make_weights(w) for w in blocks]
+    st_s = [ZB.make_state(s) for s in states]
+    stream = torch.cuda.current_stream(dev)
+
+    # routed tokens and distinct experts of block 0 (taps of one block decode on a copy of its state)
+    st0 = {k: v.clone() for k, v in states[0].items()}
+    x0 = (extra["embed"][ids.long()].float() * cfg.emb_mult).contiguous()
+    r0 = torch.empty(B, cfg.router_hidden, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, dtype=torch.int32, device=dev)
+    wt = torch.empty(B, dtype=torch.float32, device=dev)
+    ws0 = torch.zeros(ZB.zaya_workspace_size(c, ZB.ZAYA_DECODE, B, 1), dtype=torch.uint8, device=dev)
+    ZB.zaya_block_decode(c, w_s[0], 0, B, x0, None, r0, ZB.make_state(st0),
+                         ZB.make_taps({"expert_indices": idx, "expert_weights": wt}), ws0, stream=stream)
+    torch.cuda.synchronize()
+    routed = int((wt > 0).sum().item())
+    distinct = int(torch.unique(idx[wt > 0]).numel())
+    del st0, ws0
+
+    def step():
+        ZB.zaya_stack_forward(c, w_s, extra["embed"], extra["final_norm_w"], ZB.ZAYA_DECODE, B, 1, ids, None,
+                              st_s, logits, 0, ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ZB.zaya_device_status(ws, stream) == 0
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = ZB.zaya_launch_count()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    launches = ZB.zaya_launch_count() - n0
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+    clocks = clk.summary()
+    ZB.zaya_profile_reset()
+    ZB.zaya_profile_enable(True)
+    for _ in range(K):
+        step()
+    torch.cuda.synchronize()
+    stages = ZB.zaya_profile_read()
+    ZB.zaya_profile_enable(False)
+    ids_h = ids.cpu().pin_memory()
+    logits_h = torch.empty(B, V, dtype=torch.bfloat16).pin_memory()
+    e2e = []
+    for _ in range(K):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ids.copy_(ids_h, non_blocking=True)
+        step()
+        logits_h.copy_(logits, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e.append(a.elapsed_time(b))
+    e2e_ms = max_over_ranks(sum(e2e), world) / K
+
+    ms_per_step = total_ms / K
+    tokens = sum(shard_tokens(B, world))
+    value = tokens / (ms_per_step / 1e3)
+    work = stage_work_decode(cfg, routed, distinct)
+    per_block = [k for k in work if k not in ("embed", "final_norm", "lm_head")]
+    step_bytes = cfg.n_blocks * sum(work[k][1] for k in per_block) + sum(work[k][1] for k in ("embed", "final_norm", "lm_head"))
+    peaks, peak_src = load_peaks()
+    roof = roofline(stages, work, peaks, peak_src, cfg)
+    step_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+    if rank == 0 and args.stages:
+        tot = sum(v[0] for v in stages.values())
+        for name, (ms, n) in sorted(stages.items(), key=lambda kv: -kv[1][0]):
+            amt = work.get(name, ("?", 0, ""))[1]
+            per = ms / max(n, 1)
+            print(f"{name:22s} {per * 1e3:9.1f} us  {100 * ms / tot:5.1f}%  {amt / (per / 1e3) / 1e9 if amt else 0:9.1f} GB/s",
+                  file=sys.stderr)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) caches and states, random-init weights of the ZAYA1-8B stack shapes)",
+        "config": {"workload": f"{cfg.name}: one decode step (1 new token for each of B{B} sequences) through "
+                               f"{cfg.n_blocks} ZAYA1 blocks + final norm + tied lm_head (vocab {V}), {L} cached "
+                               f"tokens per sequence, window {cfg.window}",
+                   "batch": B, "seq_len": 1, "tokens_per_step": B, "routed_tokens_block0": routed,
+                   "distinct_experts_block0": distinct,
+                   "hbm_bytes_per_step": step_bytes,
+                   "step_hbm": {"achieved_gbs": round(step_gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+                                "frac": round(step_gbs / peaks["hbm_gbs"], 4)},
+                   "l2": "not flushed: a step moves about 28 GB, far more than L2",
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)"},
+        "roofline": roof,
+        "cpu_baseline": None,
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": ids_h.numel() * 4, "d2h_bytes_per_step": logits_h.numel() * 2},
         "gpu_launches": int(launches),
         "clocks": clocks,
         "stages_us": {k: round(v[0] / max(v[1], 1) * 1e3, 2) for k, v in stages.items()},
