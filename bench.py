@@ -501,7 +501,8 @@ def kernel_source_sha(name):
     files = {"attention": "attn_tc.cu", "experts_gate_up": "gemm_tc.cu", "experts_down_merge": "gemm_tc.cu",
              "qkv_gemm": "gemm_tc.cu", "o_proj_merge": "gemm_tc.cu", "router_down": "gemm_tc.cu",
              "router_mlp": "router.cu", "dispatch": "router.cu", "cca": "cca.cu",
-             "rmsnorm_attn": "norm.cu", "rmsnorm_mlp": "norm.cu"}
+             "rmsnorm_attn": "norm.cu", "rmsnorm_mlp": "norm.cu", "attention_decode": "attn_decode.cu",
+             "lm_head": "gemm_tc.cu", "final_norm": "norm.cu", "embed": "norm.cu"}
     f = files.get(name)
     if not f:
         return None
