@@ -26,7 +26,11 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller; the
  *    library allocates nothing and keeps no state between calls.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
- *    the legacy default stream); nothing synchronises the host.
+ *    the legacy default stream); nothing synchronises the host.  The
+ *    library's kernels are launched with programmatic stream serialisation:
+ *    each may be scheduled while the previous kernel of the stream finishes,
+ *    but touches global memory only after that kernel has completed, so the
+ *    usual stream order holds for the caller's own work on the stream.
  *  - Row-major layouts; bf16 = IEEE bfloat16, fp32 = IEEE float.
  *  - Every weight matrix and vector of zaya_block_weights except k_temp,
  *    the router MLP biases and norm weight, and balancing, and every bf16
