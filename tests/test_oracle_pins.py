@@ -432,3 +432,127 @@ def test_prefill_rows_equals_full_prefill():
         np.testing.assert_array_equal(part["expert_cls"], full["expert_cls"][0, r0:r1])
         np.testing.assert_allclose(part["attention_keys"].transpose(1, 0, 2),
                                    full["attention_keys"][0][:, r0:r1], rtol=1e-9, atol=1e-9)
+
+
+# ---------------------------------------------------------------- carried router state
+
+def _carry_case(block_idx):
+    """The hand-worked carried-state example through the oracle's mlp half."""
+    ex = _load("worked_examples.json")["router_state_carry"]
+    R, H, E = ex["router_hidden"], ex["hidden"], ex["n_experts"]
+    cfg = get_config("tiny").with_(hidden=H, router_hidden=R, n_experts=E, inter=1, rms_eps=ex["rms_eps"])
+    W = {"ln2_w": np.array(ex["ln2_w"]), "router_down_w": np.array(ex["router_down_w"]),
+         "router_down_b": np.array(ex["router_down_b"]), "router_state_scale": np.array(ex["router_state_scale"]),
+         "router_norm_w": np.ones(R), "fc1_w": np.eye(R), "fc1_b": np.zeros(R), "fc2_w": np.eye(R),
+         "fc2_b": np.zeros(R), "out_w": np.eye(R)[:E + 1], "balancing": np.zeros(E + 1),
+         "w_gate_up": np.zeros((E, 2, H)), "w_down": np.zeros((E, H, 1)),
+         "merge_m": np.array([[0.0] * H, [1.0] * H, [0.0] * H, [1.0] * H])}
+    h = np.array([ex["stream_h"]])
+    rin = np.array([ex["router_state_in"]])
+    return ex, Z._mlp_half(cfg, W, h, rin, block_idx, np.ones(1, dtype=bool))
+
+
+def test_router_state_carry_worked_example():
+    """Block > 0: the state out is down_proj + bias + prev * router_states_scale
+    (after the add, the scale on the previous state), and the router MLP reads
+    that same state: its logits are gelu(gelu(rmsnorm(state))) for identity
+    fc1 / fc2 / out_proj, computed here with math.erf (zaya page, 'One expert
+    per token, chosen beside a skip class')."""
+    ex, o = _carry_case(block_idx=1)
+    np.testing.assert_array_equal(o["router_state"][0], ex["state_out_block1"])
+    g = lambda x: 0.5 * x * (1 + math.erf(x / math.sqrt(2)))
+    r = np.array(ex["state_out_block1"])
+    z = r / math.sqrt(np.mean(r * r))
+    np.testing.assert_allclose(o["router_logits"][0], [np.float32(g(g(v))) for v in z], rtol=1e-6)
+
+
+def test_router_state_not_carried_on_block0():
+    """Block 0 adds no carried state, even when one is passed in."""
+    ex, o = _carry_case(block_idx=0)
+    np.testing.assert_array_equal(o["router_state"][0], ex["state_out_block0"])
+
+
+def _silent_expert_stack(cfg, n_blocks, scale_zero=False):
+    """Blocks whose experts output zero (w_down = 0), so the stream does not
+    depend on the routing and only the carried router state links the
+    blocks' routers."""
+    blocks = []
+    for i in range(n_blocks):
+        W = dict(gen_block_weights(cfg, block=i))
+        W["w_down"] = torch.zeros_like(W["w_down"])
+        if scale_zero:
+            W["router_state_scale"] = torch.zeros_like(W["router_state_scale"])
+        blocks.append(W)
+    return blocks
+
+
+def _bump_block0_router(blocks):
+    out = [dict(W) for W in blocks]
+    out[0]["router_down_b"] = out[0]["router_down_b"] + 0.5
+    return out
+
+
+def test_router_state_reaches_every_later_block():
+    """An edit to block 0's routing input (its down_proj bias) changes the
+    router logits of blocks 1 and 2 through the carried state; with
+    router_states_scale = 0 on every block the later blocks' logits are
+    bit-identical (zaya page, 'One expert per token ...': the state carries
+    from block to block)."""
+    cfg = get_config("tiny").with_(seq=12, batch=1)
+    ids = np.arange(1, 13)[None, :] * 7 % cfg.vocab
+    extra = {"embed": torch.randn(cfg.vocab, cfg.hidden, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16),
+             "final_norm_w": torch.ones(cfg.hidden, dtype=torch.bfloat16)}
+
+    def logits_per_block(blocks):
+        te, x = Z.embed(cfg, extra["embed"], ids)
+        r, out = None, []
+        for i, W in enumerate(blocks):
+            o = Z.block_prefill(cfg, W, x, None, r, block_idx=i)
+            x, r = o["layer_output"], o["router_state"]
+            out.append((o["router_logits"], o["layer_output"]))
+        return out
+
+    for scale_zero in (False, True):
+        base = _silent_expert_stack(cfg, 3, scale_zero)
+        a = logits_per_block(base)
+        b = logits_per_block(_bump_block0_router(base))
+        assert not np.array_equal(a[0][0], b[0][0])            # block 0's own router sees the edit
+        for i in (1, 2):
+            np.testing.assert_array_equal(a[i][1], b[i][1])     # the stream is the same
+            if scale_zero:
+                np.testing.assert_array_equal(a[i][0], b[i][0])
+            else:
+                assert (a[i][0] != b[i][0]).any(axis=-1).all(), i   # every token's logits moved
+
+
+def test_router_state_chain_in_decode():
+    """The decode stack chains the router state the same way: block 2's
+    router logits follow an edit to block 0's down_proj bias only through a
+    nonzero router_states_scale."""
+    cfg = get_config("tiny").with_(seq=10, batch=2)
+    extra = {"embed": torch.randn(cfg.vocab, cfg.hidden, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16),
+             "final_norm_w": torch.ones(cfg.hidden, dtype=torch.bfloat16)}
+    ids = (np.arange(20).reshape(2, 10) * 5 + 1) % cfg.vocab
+    for scale_zero in (False, True):
+        base = _silent_expert_stack(cfg, 3, scale_zero)
+        pre = Z.stack_prefill(cfg, base, extra, ids)
+        states = [dict(s, cache_len=s["cache_len"]) for s in pre["states"]]
+        for s in states:
+            s["k_cache"] = np.concatenate([s["k_cache"], np.zeros_like(s["k_cache"][:, :, :1])], axis=2)
+            s["v_cache"] = np.concatenate([s["v_cache"], np.zeros_like(s["v_cache"][:, :, :1])], axis=2)
+        new_ids = np.array([3, 9])
+
+        def last_block_logits(blocks):
+            te, x = Z.embed(cfg, extra["embed"], new_ids)
+            r = None
+            for i, W in enumerate(blocks):
+                o = Z.block_decode(cfg, W, x, states[i], r, block_idx=i)
+                x, r = o["layer_output"], o["router_state"]
+            return o["router_logits"]
+
+        a = last_block_logits(base)
+        b = last_block_logits(_bump_block0_router(base))
+        if scale_zero:
+            np.testing.assert_array_equal(a, b)
+        else:
+            assert (a != b).any(axis=-1).all()
