@@ -41,6 +41,18 @@
  *    detected on the host before anything is launched.  Faults found on the
  *    device (a bounded wait that ran out, an index out of range) are written
  *    to a status word in the workspace and read with zaya_device_status().
+ *  - The workspace starts with a 256-byte header: the status word (int32 at
+ *    byte 0) and a wait limit (uint64 nanoseconds at byte 8; 0 means the
+ *    default of 2 s, and a test may set a shorter one to make the bounded
+ *    waits run out).  The header must be zero before the first call on a
+ *    workspace (cudaMemsetAsync); the calls never clear it themselves, so a
+ *    fault stays recorded across calls until zaya_device_status() reads and
+ *    clears it.
+ *  - Fail fast: once the status word holds a fault, the library's kernels
+ *    that wait on asynchronous copies skip their work, and a wait gives up as
+ *    soon as another has recorded a fault, so a failed call (or stack) ends
+ *    within one wait limit.  The outputs of a call that recorded a fault are
+ *    unspecified.
  */
 #ifndef ZAYA_H_
 #define ZAYA_H_
@@ -184,7 +196,10 @@ int zaya_block_prefill(const zaya_config* cfg, const zaya_block_weights* w, int3
  *  hidden fp32 [B, H] in/out.  router_state_in / _out fp32 [B, R].
  *  The token of sequence b sits at position cache_len[b]; it attends over
  *  positions max(0, t - window + 1) .. t; requires cache_len[b] < cache_cap
- *  (checked on the device: ZAYA_ERR_DEVICE_RANGE, nothing written).
+ *  for every b, checked on the device: if any sequence fails it, the status
+ *  word records ZAYA_ERR_DEVICE_RANGE and no sequence's caches, conv_state,
+ *  prev_hs or cache_len are written (hidden and the router state out are
+ *  then unspecified).
  *  conv_state, prev_hs, the caches and cache_len are updated. */
 int zaya_block_decode(const zaya_config* cfg, const zaya_block_weights* w, int32_t block_idx,
                       int32_t B, float* hidden, const float* router_state_in, float* router_state_out,
@@ -210,15 +225,24 @@ int zaya_block_decode(const zaya_config* cfg, const zaya_block_weights* w, int32
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
+ *  - Every argument is checked before anything is enqueued; an invalid
+ *    call returns its ZAYA_ERR_* code with no GPU work issued.
  *  - All calls share the one array and it keeps the previous call's
- *    contents; the call clears the device status word it needs at zero.
- *    Calls that overlap on the GPU (other streams, other threads) race on
- *    the array and corrupt each other: serialise them.
- *  - Device-side faults are recorded in the array's status word, which no
- *    entry point returns. */
+ *    contents; each call first clears the array's 256-byte header (status
+ *    word and wait limit) on `stream`.  Calls that overlap on the GPU (other
+ *    streams, other threads) race on the array and corrupt each other:
+ *    serialise them.
+ *  - Device-side faults of the last call are recorded in the array's status
+ *    word; zaya_noalloc_status() returns and clears it. */
 int zaya_block_decode_noalloc(const zaya_config* cfg, const zaya_block_weights* w, int32_t block_idx, int32_t B,
                               float* hidden, const float* router_state_in, float* router_state_out,
                               const zaya_block_state* state, const zaya_taps* taps, void* stream);
+
+/* Device status of zaya_block_decode_noalloc on the current device:
+ * synchronises `stream`, returns the status word of the library's fixed
+ * scratch (ZAYA_OK if none) and clears it.  Like the entry point it serves,
+ * it has no counterpart on the pages. */
+int zaya_noalloc_status(void* stream);
 
 /* The whole stack: embedding -> n_blocks blocks (router state chained on the
  * device) -> final norm -> tied lm_head (zaya page, "Printout" and "The

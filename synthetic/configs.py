@@ -55,6 +55,9 @@ class BlockConfig:
     skip_bias: float = 0.0       # balancing bias of the skip class when not calibrated
     temp_mode: str = "one"       # "one" -> temp = 1; "stress" -> U(0.8, 12.9) per kv head
     input_dtype: str = "fp32"    # "fp32": tiny workload (GPU takes bf16-rounded copies)
+    weight_dtype: str = "bf16"   # "bf16": drawn values rounded to bf16 (a bf16 checkpoint);
+                                 # "fp32": unrounded fp32 weights (the tiny workload); the GPU
+                                 # takes bf16-rounded copies of the matrices it reads in bf16
 
     # ---- derived sizes ----
     @property
@@ -97,14 +100,14 @@ _FULL = dict(hidden=2048, n_q=8, n_kv=2, head_dim=128, rot_dim=64, n_experts=16,
              router_w_std=1.0 / 16.0, router_b_std=0.5)
 
 CONFIGS = {
-    # Tiny single block, fp32 inputs and weights, seed 0.
+    # Tiny single block, fp32 inputs and weights (unrounded), seed 0.
     "tiny": BlockConfig(
         name="tiny", hidden=256, n_q=4, n_kv=1, head_dim=64, rot_dim=32, n_experts=4,
         inter=256, router_hidden=32, window=32, rope_theta=1e4, batch=1, seq=64,
         seed=0, vocab=512, emb_mult=math.sqrt(256.0),
         # N(0, 0.02) router-MLP weights make the 5 logits equal to ~1e-3 and send
         # every token to one class; 1/sqrt(R) keeps the choice token-dependent.
-        router_w_std=1.0 / math.sqrt(32.0), calibrated=1, skip_frac=0.25),
+        router_w_std=1.0 / math.sqrt(32.0), calibrated=1, skip_frac=0.25, weight_dtype="fp32"),
     # Full-width single block prefill, B1 x S4096; balancing biases fitted to
     # roughly uniform expert loads with no skip (the random-init router alone
     # sends half the tokens to one expert).

@@ -38,6 +38,13 @@ def bf16_values(t: torch.Tensor) -> torch.Tensor:
     return t.to(torch.bfloat16).to(torch.float32)
 
 
+_bf16_values = bf16_values
+
+
+def _identity(t: torch.Tensor) -> torch.Tensor:
+    return t
+
+
 def _normal(cfg, block, tag, shape, std, device, mean=0.0):
     g = _gen(cfg, block, tag, device)
     return torch.randn(shape, generator=g, device=device, dtype=torch.float32) * std + mean
@@ -69,10 +76,18 @@ def balancing_biases(cfg: BlockConfig) -> torch.Tensor:
 
 
 def gen_block_weights(cfg: BlockConfig, block: int | None = None, device="cpu") -> dict:
-    """One block's parameters, keyed by the C ABI's field names."""
+    """One block's parameters, keyed by the C ABI's field names.  With
+    ``weight_dtype == "fp32"`` every tensor is float32 and unrounded (the
+    caller rounds the matrices the C ABI takes in bf16); otherwise matrices
+    are bf16 and the small parameters hold bf16 values in float32."""
     blk = cfg.block_idx if block is None else block
     H, R, E, I, C = cfg.hidden, cfg.router_hidden, cfg.n_experts, cfg.inter, cfg.qk_channels
-    bf = torch.bfloat16
+    if cfg.weight_dtype == "fp32":
+        bf = torch.float32
+        bf16_values = _identity
+    else:
+        bf = torch.bfloat16
+        bf16_values = _bf16_values
     n = lambda tag, shape, std, mean=0.0: _normal(cfg, blk, tag, shape, std, device, mean)
     u = lambda tag, shape, lo, hi: _uniform(cfg, blk, tag, shape, lo, hi, device)
     w = {}

@@ -26,8 +26,14 @@ TOL_COS = 0.9995
 NEAR_TIE = 1e-5
 
 
+# Weight fields the C ABI reads in bf16 (the rest are fp32).
+BF16_FIELDS = ("ln1_w", "ln2_w", "w_qkv", "w_o", "router_down_w", "w_gate_up", "w_down")
+
+
 def dev_weights(W: dict, dev="cuda") -> dict:
-    return {k: v.to(dev).contiguous() for k, v in W.items()}
+    """The block's weights on the device in the C ABI's dtypes: unrounded
+    fp32 matrices (the tiny workload) become bf16-rounded copies."""
+    return {k: v.to(dev, torch.bfloat16 if k in BF16_FIELDS else torch.float32).contiguous() for k, v in W.items()}
 
 
 def new_state(cfg, B, cap, dev="cuda") -> dict:
@@ -198,3 +204,34 @@ def assert_block_ok(res):
     assert res["router_mismatch"] == 0, res
     lo = res["layer_output"]
     assert lo["rel_max"] <= TOL_REL_MAX and lo["cos"] >= TOL_COS, lo
+
+
+def check_prefill_rows(cfg, W, x_seq, rin_seq, gpu, ranges, block_idx, b=0):
+    """Sampled-row comparison of one GPU prefill block of a long unpadded
+    sequence (sequence b of the batch): for each row range, the oracle's
+    windowed evaluation of those rows (teacher-forced with the GPU's expert
+    choices) against the GPU's layer_output, and the oracle's router on the
+    GPU's mlp_norm_output against the GPU's choices.  Returns a list of
+    per-range results (near-ties counted, not failed)."""
+    S = x_seq.shape[0]
+    g_cls = gpu_classes(cfg, gpu).reshape(-1, S)[b]
+    m_in = gpu["mlp_norm_output"].reshape(-1, S, cfg.hidden)[b]
+    out = []
+    for r0, r1 in ranges:
+        ref = Z.block_prefill_rows(cfg, W, x_seq, r0, r1, rin_seq, block_idx=block_idx, force_cls=g_cls[r0:r1])
+        rin_rows = None if rin_seq is None else rin_seq[r0:r1]
+        t_cls, gap, _, _ = router_teacher_forced(cfg, W, m_in[r0:r1], rin_rows, block_idx)
+        near = gap < NEAR_TIE
+        res = {"rows": (r0, r1), "near_ties": int(near.sum()),
+               "router_mismatch": int(((t_cls != g_cls[r0:r1]) & ~near).sum())}
+        lo = gpu["layer_output"].reshape(-1, S, cfg.hidden)[b, r0:r1].numpy()
+        res["layer_output"] = report("layer_output", lo, ref["layer_output"])
+        out.append(res)
+    return out
+
+
+def assert_rows_ok(results):
+    for res in results:
+        assert res["router_mismatch"] == 0, res
+        lo = res["layer_output"]
+        assert lo["rel_max"] <= TOL_REL_MAX and lo["cos"] >= TOL_COS, res

@@ -109,3 +109,100 @@ def test_decode_after_prefill(name):
     k_new = st["k_cache"][0, :, S].float().cpu().numpy()
     assert Hn.rel_max(k_new, ref["state"]["k_cache"][0, :, S]) <= 2e-2
     np.testing.assert_array_equal(st["prev_hs"].cpu().float().numpy(), dec["attention_norm_output"].float().numpy())
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill_4k"])
+def test_key_temperature_stress(name):
+    """Key temperatures drawn U(0.8, 12.9) per kv head, the range of the
+    ZAYA1-8B checkpoint (zaya page, 'Queries and keys are convolved ...'):
+    softmax logits reach ~146, where the attention's lazy rescale of O
+    does its work."""
+    from tests import harness as Hn
+    cfg = get_config(name).with_(temp_mode="stress")
+    if name == "prefill_4k":
+        cfg = cfg.with_(seq=1024)
+    res = _run_prefill(cfg)
+    Hn.assert_block_ok(res)
+    for key in ("attention_output", "k_cache"):
+        assert res[key]["bf16_ok"], (key, res[key])
+
+
+def test_tiny_partial_rope_not_multiple_of_16():
+    """rot_dim = 24 (not a multiple of 16) takes the CCA kernel's general
+    form instead of the streaming one."""
+    from tests import harness as Hn
+    cfg = get_config("tiny").with_(rot_dim=24, seq=77)
+    res = _run_prefill(cfg)
+    Hn.assert_block_ok(res)
+    for key in ("k_cache", "attention_queries"):
+        assert res[key]["bf16_ok"], (key, res[key])
+
+
+def test_full_prefill_8k_window_edge_sampled():
+    """Full width at S = 8192 with window 4096 < S: from row 4096 on, every
+    query tile's window starts inside a key tile (head_dim 128).  Sampled
+    row ranges against the oracle's windowed evaluation: across the first
+    window edge, in the middle, and the last rows."""
+    from tests import harness as Hn
+    cfg = get_config("prefill_4k").with_(seq=8192)
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    gpu = Hn.gpu_prefill(cfg, Hn.dev_weights(W), inp["x"], None, inp["router_state_in"])
+    ranges = [(4088, 4104), (6000, 6020), (8192 - 40, 8192)]
+    res = Hn.check_prefill_rows(cfg, W, inp["x"][0], inp["router_state_in"][0], gpu, ranges, cfg.block_idx)
+    print(res)
+    Hn.assert_rows_ok(res)
+
+
+def test_decode_position_outside_cache_is_reported():
+    """A decode step whose position equals cache_cap for one sequence
+    records ZAYA_ERR_DEVICE_RANGE and writes no sequence's cache,
+    conv_state, prev_hs or cache_len."""
+    import top_moe_block_b200 as ZB
+    from tests import harness as Hn
+    cfg = get_config("tiny")
+    B, S = 3, 20
+    W = gen_block_weights(cfg)
+    Wd = Hn.dev_weights(W)
+    inp = gen_prefill_inputs(cfg.with_(seq=S + 1, batch=B))
+    st = Hn.new_state(cfg, B, S + 2)
+    Hn.gpu_prefill(cfg, Wd, inp["x"][:, :S], None, inp["router_state_in"][:, :S], state=st, taps=False)
+    st["cache_len"][1] = S + 2                       # == cache_cap
+    before = {k: v.clone() for k, v in st.items()}
+    c = ZB.make_config(cfg)
+    ws = Hn.workspace(ZB.zaya_workspace_size(c, ZB.ZAYA_DECODE, B, 1))
+    h = inp["x"][:, S].cuda().contiguous()
+    r_out = torch.empty(B, cfg.router_hidden, device="cuda")
+    ZB.zaya_block_decode(c, ZB.make_weights(Wd), cfg.block_idx, B, h, inp["router_state_in"][:, S].cuda().contiguous(),
+                         r_out, ZB.make_state(st), None, ws)
+    assert ZB.zaya_device_status(ws) == ZB._abi.ZAYA_ERR_DEVICE_RANGE
+    assert ZB.zaya_device_status(ws) == 0             # read and cleared
+    for k in before:
+        assert torch.equal(st[k], before[k]), k
+
+
+def test_wait_timeout_is_reported_and_the_context_recovers():
+    """With a 1 ns wait limit in the workspace header the bounded waits run
+    out: the call records ZAYA_ERR_TIMEOUT (nothing hangs or faults).  With
+    the header cleared, the same call on the same context matches the
+    oracle."""
+    import top_moe_block_b200 as ZB
+    from tests import harness as Hn
+    cfg = get_config("tiny")
+    W = gen_block_weights(cfg)
+    Wd = Hn.dev_weights(W)
+    inp = gen_prefill_inputs(cfg)
+    B, S = cfg.batch, cfg.seq
+    c = ZB.make_config(cfg)
+    ws = Hn.workspace(ZB.zaya_workspace_size(c, ZB.ZAYA_PREFILL, B, S))
+    ZB.set_wait_limit_ns(ws, 1)
+    hidden = inp["x"].cuda().contiguous()
+    r_out = torch.empty(B, S, cfg.router_hidden, device="cuda")
+    st = Hn.new_state(cfg, B, S)
+    ZB.zaya_block_prefill(c, ZB.make_weights(Wd), cfg.block_idx, B, S, hidden, None,
+                          inp["router_state_in"].cuda().contiguous(), r_out, ZB.make_state(st), None, ws)
+    assert ZB.zaya_device_status(ws) == ZB._abi.ZAYA_ERR_TIMEOUT
+    ZB.set_wait_limit_ns(ws, 0)
+    torch.cuda.synchronize()
+    gpu = Hn.gpu_prefill(cfg, Wd, inp["x"], None, inp["router_state_in"])
+    Hn.assert_block_ok(Hn.check_prefill_block(cfg, W, inp, gpu, verbose=False))

@@ -161,3 +161,46 @@ def test_decode_stack_b64_40_blocks():
     emb = extra_d["embed"].cpu()
     _, ref_logits = Z.lm_head(cfg, emb, extra_d["final_norm_w"].cpu(), Z.as64(x[rows]))
     _check_logits(logits[rows], ref_logits)
+
+
+def test_prefill_stack_32k_sampled():
+    """The long-prefill workload: B1 x S32768 through 40 full-width blocks,
+    window 4096, vocab 262144, logits at every position.  Blocks 0 and 39
+    are checked against the oracle on sampled rows (the last 48 positions
+    and the window edge 4094..4098, teacher-forced on the GPU's own block
+    input), and the logits on sampled positions."""
+    import top_moe_block_b200 as ZB
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config("prefill_stack_32k")
+    B, S, V = cfg.batch, cfg.seq, cfg.vocab
+    dev = "cuda"
+    blocks_d = [gen_block_weights(cfg, block=i, device=dev) for i in range(cfg.n_blocks)]
+    extra_d = gen_stack_weights_extra(cfg, device=dev)
+    ids = gen_token_ids(cfg).to(dev)
+    states = [Hn.new_state(cfg, B, S) for _ in range(cfg.n_blocks)]
+    c = ZB.make_config(cfg)
+    ws = Hn.workspace(ZB.zaya_stack_workspace_size(c, ZB.ZAYA_PREFILL, B, S), poison=False)
+    logits = torch.empty(B, S, V, dtype=torch.bfloat16, device=dev)
+    ZB.zaya_stack_forward(c, [ZB.make_weights(w) for w in blocks_d], extra_d["embed"], extra_d["final_norm_w"],
+                          ZB.ZAYA_PREFILL, B, S, ids, None, [ZB.make_state(s) for s in states], logits, 0, ws)
+    assert ZB.zaya_device_status(ws) == 0
+    del states, ws
+    ranges = [(S - 48, S), (4094, 4099)]
+    x = _embed_stream(cfg, extra_d["embed"], ids)
+    r = None
+    for i in range(cfg.n_blocks):
+        check = i in (0, cfg.n_blocks - 1)
+        out = Hn.gpu_prefill(cfg, blocks_d[i], x, None, r, block_idx=i, taps=check)
+        if check:
+            W = {k: v.cpu() for k, v in blocks_d[i].items()}
+            res = Hn.check_prefill_rows(cfg, W, x[0].cpu(), None if r is None else r[0].cpu(), out, ranges, i)
+            print(i, res)
+            Hn.assert_rows_ok(res)
+        x = out["layer_output"].to(dev)
+        r = out["router_state"].to(dev)
+        del out
+    rows = [0, 4095, 4096, S - 1]
+    emb = extra_d["embed"].cpu()
+    _, ref_logits = Z.lm_head(cfg, emb, extra_d["final_norm_w"].cpu(), Z.as64(x[0, rows]))
+    _check_logits(logits[0, rows], ref_logits)

@@ -51,6 +51,7 @@ def test_noalloc_decode_matches_workspace_decode(name, B):
         ZB.zaya_block_decode_noalloc(c, w, cfg.block_idx, B, h_new, rs, r_new, ZB.make_state(st_new))
         torch.cuda.synchronize()
         assert ZB.zaya_device_status(ws) == 0
+        assert ZB.zaya_noalloc_status() == 0        # the fixed scratch's own status word
         a, b = h_new.cpu().numpy(), h_ref.cpu().numpy()
         assert Hn.rel_max(a, b) <= Hn.TOL_REL_MAX and Hn.cosine(a, b) >= Hn.TOL_COS
         np.testing.assert_allclose(r_new.cpu().numpy(), r_ref.cpu().numpy(), rtol=1e-6, atol=1e-6)

@@ -19,7 +19,7 @@ from ._abi import (ZAYA_DECODE, ZAYA_OK, ZAYA_PREFILL, zaya_block_state,  # noqa
 __all__ = ["make_config", "make_weights", "make_state", "make_taps", "zaya_workspace_size",
            "zaya_stack_workspace_size", "zaya_block_prefill", "zaya_block_decode", "zaya_block_decode_noalloc",
            "zaya_stack_forward",
-           "zaya_device_status", "zaya_status_string", "zaya_abi_version", "zaya_profile_enable",
+           "zaya_device_status", "zaya_noalloc_status", "set_wait_limit_ns", "zaya_status_string", "zaya_abi_version", "zaya_profile_enable",
            "zaya_profile_reset", "zaya_profile_read", "zaya_launch_count", "ZayaError", "ZAYA_PREFILL",
            "ZAYA_DECODE"]
 
@@ -150,6 +150,17 @@ def zaya_stack_forward(cfg, blocks, embed, final_norm_w, mode, B, S, ids, attn_m
 
 def zaya_device_status(workspace, stream=None) -> int:
     return _abi.lib().zaya_device_status(_ptr(workspace), _stream_ptr(stream))
+
+
+def zaya_noalloc_status(stream=None) -> int:
+    """Status word of zaya_block_decode_noalloc's fixed scratch (read and cleared)."""
+    return _abi.lib().zaya_noalloc_status(_stream_ptr(stream))
+
+
+def set_wait_limit_ns(workspace, ns: int) -> None:
+    """Write the wait limit into the workspace header (bytes 8..16; 0 = the
+    default 2 s), stream-ordered on the current stream."""
+    workspace[8:16].copy_(torch.tensor([int(ns)], dtype=torch.int64).view(torch.uint8))
 
 
 def zaya_profile_enable(on: bool = True) -> None:

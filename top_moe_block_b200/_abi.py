@@ -81,6 +81,8 @@ def lib() -> C.CDLL:
         L.zaya_stack_forward.restype = C.c_int
         L.zaya_device_status.argtypes = [vp, vp]
         L.zaya_device_status.restype = C.c_int
+        L.zaya_noalloc_status.argtypes = [vp]
+        L.zaya_noalloc_status.restype = C.c_int
         L.zaya_status_string.argtypes = [C.c_int]
         L.zaya_status_string.restype = C.c_char_p
         L.zaya_profile_enable.argtypes = [C.c_int]

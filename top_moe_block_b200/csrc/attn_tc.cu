@@ -201,7 +201,8 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
   uint64_t* s_full = v_empty + kRingV;          // [kHPC][2]: S(j) of the head is in S buffer j & 1
   uint64_t* p_full = s_full + 2 * kHPC;         // [kHPC][2]: P(j) is in TMEM over S(j)
   uint64_t* pv_done = p_full + 2 * kHPC;        // [kHPC]: O += P(j) V(j) complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + kHPC);
+  uint64_t* o_ready = pv_done + kHPC;           // the MMA thread's last commit: every MMA of the CTA is done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_ready + 1);
   int* s_last = reinterpret_cast<int*>(tmem_slot + 1);
 
   // this CTA's item: a row tile of its kHPC heads, or one key chunk of it
@@ -247,6 +248,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
       mbar_init(&p_full[i], 4);
     }
     for (int i = 0; i < kHPC; ++i) mbar_init(&pv_done[i], 1);
+    mbar_init(o_ready, 1);
     fence_barrier_init();
     fence_proxy_async();
     prefetch_tmap(&tmQ);
@@ -259,10 +261,15 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   griddep_begin();   // the prologue above overlaps the previous kernel; global memory only from here
+  // A fault already recorded (an earlier wait ran out) means the launch chain
+  // has failed: no work.  Each role reads the word itself; roles that read
+  // differently meet in waits that give up on the recorded fault.
+  const WaitCtx wc = wait_ctx(status);
+  const int n_work = wc.skip ? 0 : n_tiles;
 
   if (warp == 0) {
     // ---------------- TMA producer: the heads' Q once, then K(j) and V(j) into their rings
-    if (elect_one()) {
+    if (elect_one() && !wc.skip) {
       const int kv_row = (b * p.n_kv + g) * p.cap + n_begin + t_begin * kKT;
       mbar_arrive_expect_tx(q_full, kHPC * C::Q_BYTES);
 #pragma unroll
@@ -272,21 +279,30 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
         for (int s = 0; s < C::SUB; ++s)
           tma_load_2d(sQ + x * C::Q_BYTES + s * C::Q_ATOM, &tmQ, q_full, s * 64, q_row);
       }
+      int nk = 0, nv = 0;   // K / V tiles whose copies were started
       for (int j = 0; j < n_tiles; ++j) {
         const int slot = j % kRing;
         const uint32_t par = ((j / kRing) & 1) ^ 1u;
-        if (!mbar_wait(&k_empty[slot], par, status)) break;
+        if (!mbar_wait(&k_empty[slot], par, wc)) break;
         mbar_arrive_expect_tx(&k_full[slot], C::KV_BYTES);
 #pragma unroll
         for (int s = 0; s < C::SUB; ++s)
           tma_load_2d(sK + slot * C::KV_BYTES + s * C::KV_ATOM, &tmK, &k_full[slot], s * 64, kv_row + j * kKT);
+        ++nk;
         const int vslot = j % kRingV;
-        if (!mbar_wait(&v_empty[vslot], ((j / kRingV) & 1) ^ 1u, status)) break;
+        if (!mbar_wait(&v_empty[vslot], ((j / kRingV) & 1) ^ 1u, wc)) break;
         mbar_arrive_expect_tx(&v_full[vslot], C::KV_BYTES);
 #pragma unroll
         for (int s = 0; s < C::SUB; ++s)
           tma_load_2d(sV + vslot * C::KV_BYTES + s * C::KV_ATOM, &tmV, &v_full[vslot], s * 64, kv_row + j * kKT);
+        ++nv;
       }
+      // every copy started must land before the CTA may exit: the last phase
+      // armed on each slot (tile j uses phase j / ring of slot j % ring)
+      mbar_drain(q_full, 0, status);
+      for (int j = (nk > kRing ? nk - kRing : 0); j < nk; ++j) mbar_drain(&k_full[j % kRing], (j / kRing) & 1, status);
+      for (int j = (nv > kRingV ? nv - kRingV : 0); j < nv; ++j)
+        mbar_drain(&v_full[j % kRingV], (j / kRingV) & 1, status);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer.  Per head: S(j) into S buffer j & 1; the
@@ -295,7 +311,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
     // thread's MMAs in issue order, so S(j+2) is written after P(j) is read).
     // S runs two tiles ahead of the softmax (with kHPC > 1 the heads alternate).
     if (elect_one()) {
-      bool ok = mbar_wait(q_full, 0, status);
+      bool ok = n_work > 0 && mbar_wait(q_full, 0, wc);
       auto issue_qk = [&](int x, int j) {
         const uint32_t ka = smem_u32(sK + (j % kRing) * C::KV_BYTES);
         const uint32_t qa = smem_u32(sQ + x * C::Q_BYTES);
@@ -309,7 +325,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
         tc_commit(&s_full[x * 2 + (j & 1)]);
       };
       for (int j = 0; ok && j < 2 && j < n_tiles; ++j) {   // S(0), S(1)
-        ok = mbar_wait(&k_full[j], 0, status);
+        ok = mbar_wait(&k_full[j], 0, wc);
         if (!ok) break;
         tc_fence_after();
         for (int x = 0; x < kHPC; ++x) issue_qk(x, j);
@@ -318,11 +334,11 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int vslot = j % kRingV, nslot = (j + 2) % kRing;
         const bool more = j + 2 < n_tiles;
-        if (more && !mbar_wait(&k_full[nslot], ((j + 2) / kRing) & 1, status)) break;
-        if (!mbar_wait(&v_full[vslot], (j / kRingV) & 1, status)) break;
+        if (more && !mbar_wait(&k_full[nslot], ((j + 2) / kRing) & 1, wc)) break;
+        if (!mbar_wait(&v_full[vslot], (j / kRingV) & 1, wc)) break;
         const uint32_t va = smem_u32(sV + vslot * C::KV_BYTES);
         for (int x = 0; ok && x < kHPC; ++x) {
-          if (!mbar_wait(&p_full[x * 2 + (j & 1)], (j >> 1) & 1, status)) {
+          if (!mbar_wait(&p_full[x * 2 + (j & 1)], (j >> 1) & 1, wc)) {
             ok = false;
             break;
           }
@@ -339,6 +355,10 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
         tc_commit(&v_empty[vslot]);
         if (more) tc_commit(&k_empty[nslot]);
       }
+      // the last commit, issued on every path: it arrives once every MMA above
+      // has completed -- O is final and the tensor memory may be freed
+      tc_commit(o_ready);
+      mbar_drain(o_ready, 0, status);
     }
   } else {
     // ---------------- softmax: warpgroup x handles head h0 + x, one thread per query row
@@ -351,10 +371,10 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
     const float sl2 = p.scale * 1.4426950408889634f;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
+    for (int j = 0; j < n_work; ++j) {
       // every wait that guards a .sync.aligned TMEM access is made warp-uniform
       const int buf = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x * 2 + buf], (j >> 1) & 1, status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x * 2 + buf], (j >> 1) & 1, wc))) {
         ok = false;
         break;
       }
@@ -391,7 +411,9 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
         const float f = (m_used == -INFINITY || !finite_new) ? 1.f : exp2f(m_used - m_new);
         if (j > 0 && __any_sync(0xffffffffu, m_used != -INFINITY)) {
           // O holds tiles < j: wait for PV(j-1), then scale O in TMEM
-          if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[x], (j - 1) & 1, status))) {
+          // S(j) was committed after PV(j-2), so pv_done is at most one phase behind
+          // PV(j-1) here and its parity names that phase unambiguously
+          if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[x], (j - 1) & 1, wc))) {
             ok = false;
             break;
           }
@@ -430,8 +452,10 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[x * 2 + buf]);
     }
-    const bool have = ok && n_tiles > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (n_tiles - 1) & 1, status));
+    // O is final once the MMA thread's last commit has arrived (a single-use
+    // barrier: pv_done could still be two phases short of PV(n-1) here, when
+    // PV(n-2) has not completed, which its parity cannot tell apart)
+    const bool have = ok && n_work > 0 && __all_sync(0xffffffffu, mbar_wait(o_ready, 0, wc));
     const int ld = p.n_q * D;
     auto* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * S + q) * ld + (h0 + x) * D;
     // this row's 32 output columns [c, c + 32), scaled, as bf16

@@ -130,8 +130,21 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
   const size_t ld = (size_t)p.n_qkv;
 
   const int pos = p.decode ? p.cache_len[b] : s;
-  if (pos < 0 || pos >= p.cache_cap) {
-    if (warp == 0 && lane == 0) set_status(p.status, ZAYA_ERR_DEVICE_RANGE);
+  // Decode appends at cache_len[b]: a position outside the cache is a fault.
+  // Every CTA checks all sequences, so a call with one bad position writes no
+  // sequence's cache, conv_state or prev_hs (the status word then makes the
+  // rest of the block skip its work, and cache_len stays as it was).
+  bool bad = false;
+  if (p.decode) {
+    for (int i = threadIdx.x; i < p.B; i += blockDim.x) {
+      const int c = p.cache_len[i];
+      bad |= (c < 0 || c >= p.cache_cap);
+    }
+  } else {
+    bad = pos < 0 || pos >= p.cache_cap;
+  }
+  if (__syncthreads_or(bad)) {
+    if (threadIdx.x == 0 && (pos < 0 || pos >= p.cache_cap)) set_status(p.status, ZAYA_ERR_DEVICE_RANGE);
     return;
   }
   Pre<D> pre;

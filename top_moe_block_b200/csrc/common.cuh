@@ -62,6 +62,37 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Upper bound for any wait on an mbarrier or flag: 2 s of wall time.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// The status word's 256-byte header: word 0 is the status; the 64-bit word
+// at byte 8 may hold a shorter wait limit in ns (0: kWaitLimitNs), which a
+// test sets to make the bounded waits run out.
+__device__ __forceinline__ int status_peek(const int* status) {
+  return status ? *reinterpret_cast<const volatile int*>(status) : 0;
+}
+
+// What a role's bounded waits need, read once after griddep_begin():
+// the status word, the wait limit, and whether a fault is already recorded
+// (`skip`: the launch chain has failed, so the kernel does no work).
+// `bail`: a wait gives up as soon as another wait has recorded a fault
+// (kernels whose roles may stop independently; CTA-pair kernels keep both
+// CTAs' producers in step instead and wait for their own limit).
+struct WaitCtx {
+  int* status;
+  uint64_t limit_ns;
+  uint32_t hint_ns;
+  bool bail;
+  bool skip;
+};
+__device__ __forceinline__ WaitCtx wait_ctx(int* status, bool bail = true) {
+  WaitCtx w;
+  w.status = status;
+  w.bail = bail;
+  w.skip = status_peek(status) != 0;
+  uint64_t lim = status ? *reinterpret_cast<const volatile uint64_t*>(status + 2) : 0ull;
+  w.limit_ns = lim ? lim : kWaitLimitNs;
+  w.hint_ns = w.limit_ns < 20000ull ? (uint32_t)w.limit_ns : 20000u;
+  return w;
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -79,29 +110,49 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// The waiting thread may be suspended in hardware (up to kSuspendNs) until the
+// The waiting thread may be suspended in hardware (up to the hint) until the
 // phase completes, instead of spinning on the issue slots its SM sub-partition
 // shares with the warps that do the work.
-constexpr uint32_t kSuspendNs = 20000;
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
 // Bounded wait: returns false (and records ZAYA_ERR_TIMEOUT) if the phase
-// does not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
+// does not complete within the limit; with w.bail it also returns false as
+// soon as the status word holds a fault recorded elsewhere, so one failed
+// wait ends the whole launch (and the launches after it) in one limit's time.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  if (mbar_try_wait(bar, parity, w.hint_ns)) return true;
+  const uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if ((++n & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+  while (!mbar_try_wait(bar, parity, w.hint_ns)) {
+    if ((++n & 15u) == 0) {
+      if (w.bail && status_peek(w.status)) return false;
+      if (globaltimer_ns() - t0 > w.limit_ns) {
+        set_status(w.status, ZAYA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+// Teardown wait for a kernel's own asynchronous work (TMA copies it issued,
+// tcgen05 MMAs and commits): before a CTA frees its tensor memory and exits,
+// everything it started must have landed.  Bounded by kWaitLimitNs whatever
+// the status word or the test limit says.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity, 20000u)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (!mbar_try_wait(bar, parity, 20000u)) {
+    if ((++n & 15u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
       set_status(status, ZAYA_ERR_TIMEOUT);
       return false;
     }

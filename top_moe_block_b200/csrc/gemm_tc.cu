@@ -308,7 +308,9 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* mdrain = tempty + 2;   // the MMA thread's last commit: all its MMAs are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdrain + 1);
+  int* s_skip = reinterpret_cast<int*>(tmem_slot + 1);   // CTA pair: rank 0's reading of the status word
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -325,6 +327,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], CG * EW);
     }
+    mbar_init(mdrain, 1);
     fence_barrier_init();
     fence_proxy_async();
     prefetch_tmap(&tmA);
@@ -336,19 +339,32 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
   }
   tc_fence_before();
   __syncwarp();
-  if constexpr (CG == 2) cluster_sync_all();   // both CTAs' barriers and TMEM are ready
-  else __syncthreads();
+  // The prologue above overlaps the previous kernel; global memory only from here.
+  // A fault already recorded in the status word (an earlier wait ran out)
+  // means the launch chain has failed: the kernel then does no work.  Both
+  // CTAs of a pair take rank 0's reading, so that they walk the same tiles.
+  griddep_begin();
+  WaitCtx wc = wait_ctx(p.status, /*bail=*/CG == 1);
+  if constexpr (CG == 2) {
+    if (rank == 0 && threadIdx.x == 0) *s_skip = wc.skip ? 1 : 0;
+    cluster_sync_all();   // both CTAs' barriers and TMEM are ready; rank 0's reading is published
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(mapa_shared(s_skip, 0)) : "memory");
+    wc.skip = v != 0;
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  griddep_begin();   // the prologue above overlaps the previous kernel; global memory only from here
 
-  const int ntiles = total_tiles<EPI, BN_OUT, TM>(p);
+  const int ntiles = wc.skip ? 0 : total_tiles<EPI, BN_OUT, TM>(p);
 
   if (warp == 0) {
     // ---------------- TMA producer (each CTA loads its own A rows and B half)
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
+      int n_armed = 0;
       for (int t = unit; t < ntiles; t += n_units) {
         const TileInfo ti = tile_info<EPI, BN_OUT, TM>(p, t);
         // this CTA's B rows: CG = 1 all BN rows (SWIGLU: gate then up); CG = 2 its half
@@ -367,7 +383,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         for (int kb = ti.kb0; kb < ti.kb0 + kPrefetchAhead && kb < kb_end; ++kb) prefetch_b(kb);
         for (int kb = ti.kb0; kb < kb_end; ++kb) {
           if (kb + kPrefetchAhead < kb_end) prefetch_b(kb + kPrefetchAhead);
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) goto producer_done;
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
           uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
           uint8_t* b_dst = sB + stage * C::B_STAGE_BYTES;
           if constexpr (CG == 2) {
@@ -385,13 +401,21 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
               tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
             }
           }
+          ++n_armed;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-    producer_done:;
+    producer_done:
+      // Before the CTA may exit, every copy this producer started has landed:
+      // wait for the last phase it armed on each slot (rank 0 arms both CTAs'
+      // bytes of a pair, so its wait covers the peer's copies too).
+      if (CG == 1 || rank == 0) {
+        for (int s2 = 0; s2 < STAGES && s2 < n_armed; ++s2)
+          mbar_drain(&full[s2], (s2 < stage) ? phase : (phase ^ 1u), p.status);
+      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (rank 0 of a pair issues for both CTAs)
@@ -402,13 +426,13 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
       for (int t = unit; t < ntiles; t += n_units, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, wc)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         const int nkb = tile_info<EPI, BN_OUT, TM>(p, t).nkb;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.status)) {
+          if (!mbar_wait(&full[stage], phase, wc)) {
             ok = false;
             break;
           }
@@ -435,6 +459,11 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         if constexpr (CG == 2) tc_commit_pair(&tfull[acc], 3);
         else tc_commit(&tfull[acc]);
       }
+      // last commit: once it arrives every MMA of this thread has completed,
+      // so the tensor memory may be freed
+      if constexpr (CG == 2) tc_commit_pair(mdrain, 1);
+      else tc_commit(mdrain);
+      mbar_drain(mdrain, 0, p.status);
     }
   } else {
     // ---------------- epilogue warps 2 .. 2+EW-1 (this CTA's 128 accumulator rows)
@@ -466,7 +495,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         named_barrier_sync(1, EW * 32);
       }
       // warp-uniform: the TMEM loads below are .sync.aligned
-      if (!aborted && !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, p.status))) aborted = true;
+      if (!aborted && !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, wc))) aborted = true;
       if (aborted) continue;
       tc_fence_after();
       const int row = ti.m0 + row_off + q * 32 + lane;

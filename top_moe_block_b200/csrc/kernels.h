@@ -177,6 +177,7 @@ struct DispatchParams {
   const float* merge_m;   // [4, H]
   void* tap_mlp_out;      // optional bf16 [M, H]
   int* cache_len_inc;     // optional [M] (decode)
+  const int* status;      // device status word: a recorded fault makes the kernel do nothing
   int M, H, E;
 };
 int launch_dispatch(const DispatchParams& p, cudaStream_t st);

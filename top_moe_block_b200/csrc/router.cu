@@ -251,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
       prefetch_tmap(&tmW);
     }
   }
+  const WaitCtx wc = wait_ctx(p.status);
   stage_w(0);   // the first fc1 chunk streams in under the state assembly
 
   // router state r = down_proj partial sums (in slab order) + bias (+ previous
@@ -354,9 +355,15 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
 #pragma unroll
   for (int j = 0; j < Sh::NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
   bool ok = true;   // TMA mode: false once a chunk wait has run out (status set)
+  int n_staged = 1;  // TMA mode, thread 0: chunks whose copies were started
   for (int q = 0; q < 2 * nch; ++q) {
     if (q + 1 < 2 * nch) {
-      stage_w(q + 1);
+      // after a failed wait no further chunk is started (its stage may still
+      // be receiving the chunk that never arrived in time)
+      if (!Sh::TMA || ok) {
+        stage_w(q + 1);
+        ++n_staged;
+      }
     } else {
       const __nv_bfloat16* ows = p.wsplit + (size_t)4 * R * R;   // [hi|lo][NP][R]
       for (int i = threadIdx.x; i < 2 * NP * (R / 8); i += kThreads) {
@@ -369,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     }
     asm volatile("cp.async.wait_group 1;" ::: "memory");
     if constexpr (Sh::TMA) {   // every thread sees chunk q land (bounded wait)
-      if (ok && !mbar_wait(&wfull[q & 1], (uint32_t)(q >> 1) & 1u, p.status)) ok = false;
+      if (ok && !mbar_wait(&wfull[q & 1], (uint32_t)(q >> 1) & 1u, wc)) ok = false;
     }
     __syncthreads();
     const __nv_bfloat16* wh = wring + (q & 1) * 2 * Sh::CHUNK;
@@ -384,6 +391,11 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     __syncthreads();
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+  if constexpr (Sh::TMA) {   // every chunk copy started has landed before the CTA can exit
+    if (threadIdx.x == 0)
+      for (int q = (n_staged > 2 ? n_staged - 2 : 0); q < n_staged; ++q)
+        mbar_drain(&wfull[q & 1], (uint32_t)(q >> 1) & 1u, p.status);
+  }
   __syncthreads();
   // out_proj (no bias) on tensor cores with the same hi / lo split: tile w < 2 * NP / 8
   // (warps stride over them) is rows 16 * (w & 1) .. + 16 by classes 8 * (w >> 1) .. + 8
@@ -508,6 +520,7 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
 // padding) tokens write merge 2 with a zero routed output.
 __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
   griddep_begin();
+  if (status_peek(p.status)) return;   // a fault earlier in the block: no merge, cache_len not advanced
   const int t = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   const int E1 = p.E + 1;

@@ -282,6 +282,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.m_in = m_in; p.x_perm = xperm; p.stream = hidden; p.merge_m = w->merge_m;
     p.tap_mlp_out = taps ? taps->mlp_output : nullptr;
     p.cache_len_inc = cache_len_inc;
+    p.status = status;
     p.M = M; p.H = d.H; p.E = d.E;
     ZAYA_STAGE("dispatch", 1, launch_dispatch(p, st));
   }
@@ -373,16 +374,27 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
   return block_tail(c, d, w, block_idx, M, hidden, rin, rout, taps, ws, L, nullptr, mask, sms, st);
 }
 
+// Every host-side check of a decode call except the workspace's (shared with
+// the entry point without a caller workspace, which runs them before it
+// enqueues anything).
+int check_decode_args(const zaya_config* cfg, const zaya_block_weights* w, int block_idx, int B, const float* hidden,
+                      const float* rin, const float* rout, const zaya_block_state* state, const zaya_taps* taps) {
+  ZAYA_TRY(check_config(cfg));
+  ZAYA_TRY(check_weights(w));
+  if (B <= 0 || !hidden || !rout) return ZAYA_ERR_INVALID_ARG;
+  if (block_idx < 0 || (block_idx > 0 && !rin) || rin == rout) return ZAYA_ERR_INVALID_ARG;
+  ZAYA_TRY(check_state(state, 1));
+  if (!a16(hidden) || !a16(rout)) return ZAYA_ERR_MISALIGNED;
+  if (taps && taps->attention_queries && !a16(taps->attention_queries)) return ZAYA_ERR_MISALIGNED;
+  return ZAYA_OK;
+}
+
 int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int block_idx, int B, float* hidden,
                       const float* rin, float* rout, const zaya_block_state* state, const zaya_taps* taps, void* ws,
                       size_t ws_bytes, cudaStream_t st) {
-  ZAYA_TRY(check_config(cfg));
-  ZAYA_TRY(check_weights(w));
-  if (B <= 0 || !hidden || !rout || !ws) return ZAYA_ERR_INVALID_ARG;
-  if (block_idx < 0 || (block_idx > 0 && !rin) || rin == rout) return ZAYA_ERR_INVALID_ARG;
-  ZAYA_TRY(check_state(state, 1));
-  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) || !a16(hidden) || !a16(rout)) return ZAYA_ERR_MISALIGNED;
-  if (taps && taps->attention_queries && !a16(taps->attention_queries)) return ZAYA_ERR_MISALIGNED;
+  ZAYA_TRY(check_decode_args(cfg, w, block_idx, B, hidden, rin, rout, state, taps));
+  if (!ws) return ZAYA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) return ZAYA_ERR_MISALIGNED;
   const zaya_config& c = *cfg;
   const Derived d = derive(c);
   const Ws L = plan(c, ZAYA_DECODE, B, 1);
@@ -632,16 +644,23 @@ extern "C" int zaya_block_decode_noalloc(const zaya_config* cfg, const zaya_bloc
                                          int32_t B, float* hidden, const float* router_state_in,
                                          float* router_state_out, const zaya_block_state* state,
                                          const zaya_taps* taps, void* stream) {
-  if (check_config(cfg) != ZAYA_OK) return check_config(cfg);
-  if (B <= 0) return ZAYA_ERR_INVALID_ARG;
+  // every argument check first: an invalid call enqueues nothing
+  ZAYA_TRY(check_decode_args(cfg, w, block_idx, B, hidden, router_state_in, router_state_out, state, taps));
   const size_t need = zaya_workspace_size(cfg, ZAYA_DECODE, B, 1);
   if (need == 0) return ZAYA_ERR_INVALID_ARG;
   if (need > kNoAllocScratchBytes) return ZAYA_ERR_WORKSPACE;
   void* scratch = nullptr;
   ZAYA_TRY(noalloc_scratch(&scratch));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The scratch keeps the previous call's contents; only the status word must start at zero.
+  // The scratch keeps the previous call's contents; only its 256-byte header
+  // (the status word and the wait limit) must start at zero.
   if (cudaMemsetAsync(scratch, 0, 256, st) != cudaSuccess) return ZAYA_ERR_CUDA;
   return zaya_block_decode(cfg, w, block_idx, B, hidden, router_state_in, router_state_out, state, taps, scratch,
                            kNoAllocScratchBytes, stream);
+}
+
+extern "C" int zaya_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  ZAYA_TRY(noalloc_scratch(&scratch));
+  return zaya_device_status(scratch, stream);
 }
