@@ -36,6 +36,19 @@ def dev_weights(W: dict, dev="cuda") -> dict:
     return {k: v.to(dev, torch.bfloat16 if k in BF16_FIELDS else torch.float32).contiguous() for k, v in W.items()}
 
 
+def eff(W: dict) -> dict:
+    """The weights as the GPU reads them (host copies): the matrices the C
+    ABI takes in bf16 rounded to bf16.  Unchanged for a bf16 checkpoint; for
+    the tiny workload's unrounded fp32 weights this is what the kernels see."""
+    return {k: (v.detach().cpu().to(torch.bfloat16) if k in BF16_FIELDS else v.detach().cpu().float())
+            for k, v in W.items()}
+
+
+def _fp32_matrices(W: dict) -> bool:
+    return any(W[k].dtype == torch.float32 and not torch.equal(W[k], W[k].to(torch.bfloat16).float())
+               for k in BF16_FIELDS if k in W)
+
+
 def new_state(cfg, B, cap, dev="cuda") -> dict:
     return dict(
         k_cache=torch.zeros(B, cfg.n_kv, cap, cfg.head_dim, dtype=torch.bfloat16, device=dev),
@@ -150,7 +163,13 @@ def report(name, gpu, ref) -> dict:
 
 
 def check_prefill_block(cfg, W, inp, gpu, block_idx=None, verbose=True):
-    """Full comparison of one GPU prefill block against the oracle."""
+    """Full comparison of one GPU prefill block against the oracle, on the
+    weights as the GPU reads them.  When the workload's weights are
+    unrounded fp32 (the tiny workload), layer_output is also compared with
+    the oracle run on those fp32 weights (same expert choices), with the
+    block tolerances."""
+    W_given = W
+    W = eff(W)
     bidx = cfg.block_idx if block_idx is None else block_idx
     B, S = inp["x"].shape[:2]
     M = B * S
@@ -183,6 +202,10 @@ def check_prefill_block(cfg, W, inp, gpu, block_idx=None, verbose=True):
     res["conv_state"] = report("conv", st["conv_state"].float().numpy(), o["state"]["conv_state"])
     res["prev_hs"] = report("prev_hs", st["prev_hs"].float().numpy(), o["state"]["prev_hs"])
     res["cache_len_ok"] = bool((st["cache_len"].numpy() == S).all())
+    if _fp32_matrices(W_given):
+        o32 = Z.block_prefill(cfg, W_given, inp["x"], inp.get("attn_mask"), rin, bidx, force_cls=g_cls.reshape(B, S))
+        res["fp32_weights"] = report("layer_output", gpu["layer_output"].float().numpy().reshape(M, -1),
+                                     o32["layer_output"].reshape(M, -1))
     if verbose:
         print({k: (round(v["rel_max"], 5), round(v["cos"], 6)) if isinstance(v, dict) else v for k, v in res.items()})
     return res
@@ -204,6 +227,9 @@ def assert_block_ok(res):
     assert res["router_mismatch"] == 0, res
     lo = res["layer_output"]
     assert lo["rel_max"] <= TOL_REL_MAX and lo["cos"] >= TOL_COS, lo
+    if "fp32_weights" in res:
+        lo = res["fp32_weights"]
+        assert lo["rel_max"] <= TOL_REL_MAX and lo["cos"] >= TOL_COS, ("against the fp32-weight oracle", lo)
 
 
 def check_prefill_rows(cfg, W, x_seq, rin_seq, gpu, ranges, block_idx, b=0):
@@ -214,6 +240,7 @@ def check_prefill_rows(cfg, W, x_seq, rin_seq, gpu, ranges, block_idx, b=0):
     GPU's mlp_norm_output against the GPU's choices.  Returns a list of
     per-range results (near-ties counted, not failed)."""
     S = x_seq.shape[0]
+    W = eff(W)
     g_cls = gpu_classes(cfg, gpu).reshape(-1, S)[b]
     m_in = gpu["mlp_norm_output"].reshape(-1, S, cfg.hidden)[b]
     out = []

@@ -100,8 +100,8 @@ def test_decode_after_prefill(name):
     host_state = {k: v.cpu().clone() for k, v in st.items()}
     dec = Hn.gpu_decode(cfg, Wd, x[:, S], st, rin[:, S])
     g_cls = Hn.gpu_classes(cfg, dec)
-    ref = Z.block_decode(cfg, W, x[:, S], host_state, rin[:, S], force_cls=g_cls)
-    t_cls, gap, _, _ = Hn.router_teacher_forced(cfg, W, dec["mlp_norm_output"], rin[:, S], cfg.block_idx)
+    ref = Z.block_decode(cfg, Hn.eff(W), x[:, S], host_state, rin[:, S], force_cls=g_cls)
+    t_cls, gap, _, _ = Hn.router_teacher_forced(cfg, Hn.eff(W), dec["mlp_norm_output"], rin[:, S], cfg.block_idx)
     assert ((t_cls == g_cls) | (gap < Hn.NEAR_TIE)).all()
     lo = Hn.report("layer_output", dec["layer_output"].numpy(), ref["layer_output"])
     assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, lo

@@ -106,7 +106,7 @@ def test_tiny_stack_decode_after_prefill():
         st = {k: v.cuda() for k, v in dec_states[i].items()}
         out = Hn.gpu_decode(cfg, bd[i], x, st, r, block_idx=i)
         g_cls = Hn.gpu_classes(cfg, out)
-        ref = Z.block_decode(cfg, W, x.cpu(), dec_states[i], None if r is None else r.cpu(), block_idx=i,
+        ref = Z.block_decode(cfg, Hn.eff(W), x.cpu(), dec_states[i], None if r is None else r.cpu(), block_idx=i,
                              force_cls=g_cls)
         lo = Hn.report("layer_output", out["layer_output"].numpy(), ref["layer_output"])
         assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, (i, lo)
@@ -150,11 +150,11 @@ def test_decode_stack_b64_40_blocks():
         if i in (0, 1, cfg.n_blocks - 1):
             W = {k: v.cpu() for k, v in blocks_d[i].items()}
             g_cls = Hn.gpu_classes(cfg, out)[rows]
-            ref = Z.block_decode(cfg, W, x[rows].cpu(), host, None if r is None else r[rows].cpu(), block_idx=i,
+            ref = Z.block_decode(cfg, Hn.eff(W), x[rows].cpu(), host, None if r is None else r[rows].cpu(), block_idx=i,
                                  force_cls=g_cls)
             lo = Hn.report("layer_output", out["layer_output"][rows].numpy(), ref["layer_output"])
             assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, (i, lo)
-            t_cls, gap, _, _ = Hn.router_teacher_forced(cfg, W, out["mlp_norm_output"][rows],
+            t_cls, gap, _, _ = Hn.router_teacher_forced(cfg, Hn.eff(W), out["mlp_norm_output"][rows],
                                                         None if r is None else r[rows].cpu(), i)
             assert ((t_cls == g_cls) | (gap < Hn.NEAR_TIE)).all(), i
         x, r = out["layer_output"].to(dev), out["router_state"].to(dev)
