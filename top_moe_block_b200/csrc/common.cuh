@@ -124,22 +124,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
       : "memory");
   return ok != 0;
 }
+// Non-suspending probe of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// A probe of the wait: suspending for the usual limit; with a test limit
+// shorter than the suspend hint, a plain test, so that a phase still in
+// flight at the first probe makes the wait run out.
+__device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  return hint_ns >= 20000u ? mbar_try_wait(bar, parity, hint_ns) : mbar_test_wait(bar, parity);
+}
 // Bounded wait: returns false (and records ZAYA_ERR_TIMEOUT) if the phase
 // does not complete within the limit; with w.bail it also returns false as
 // soon as the status word holds a fault recorded elsewhere, so one failed
 // wait ends the whole launch (and the launches after it) in one limit's time.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  if (mbar_try_wait(bar, parity, w.hint_ns)) return true;
+  if (mbar_probe(bar, parity, w.hint_ns)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
-  while (!mbar_try_wait(bar, parity, w.hint_ns)) {
-    if ((++n & 15u) == 0) {
-      if (w.bail && status_peek(w.status)) return false;
-      if (globaltimer_ns() - t0 > w.limit_ns) {
-        set_status(w.status, ZAYA_ERR_TIMEOUT);
-        return false;
-      }
+  while (!mbar_probe(bar, parity, w.hint_ns)) {
+    if (globaltimer_ns() - t0 > w.limit_ns) {
+      set_status(w.status, ZAYA_ERR_TIMEOUT);
+      return false;
     }
+    if ((++n & 7u) == 0 && w.bail && status_peek(w.status)) return false;
   }
   return true;
 }
