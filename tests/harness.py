@@ -33,15 +33,25 @@ BF16_FIELDS = ("ln1_w", "ln2_w", "w_qkv", "w_o", "router_down_w", "w_gate_up", "
 def dev_weights(W: dict, dev="cuda") -> dict:
     """The block's weights on the device in the C ABI's dtypes: unrounded
     fp32 matrices (the tiny workload) become bf16-rounded copies."""
-    return {k: v.to(dev, torch.bfloat16 if k in BF16_FIELDS else torch.float32).contiguous() for k, v in W.items()}
+    return {k: v.to(dev, _abi_dtype(k, v)).contiguous() for k, v in W.items()}
+
+
+def _abi_dtype(name, t):
+    """The dtype the C ABI reads a weight in: bf16 for the block's matrices
+    and norm weights, fp32 for its small parameters; other tensors (the
+    stack's bf16 embedding and final norm) keep theirs."""
+    if name in BF16_FIELDS:
+        return torch.bfloat16
+    if name in ZB._abi.WEIGHT_FIELDS:
+        return torch.float32
+    return t.dtype
 
 
 def eff(W: dict) -> dict:
     """The weights as the GPU reads them (host copies): the matrices the C
     ABI takes in bf16 rounded to bf16.  Unchanged for a bf16 checkpoint; for
     the tiny workload's unrounded fp32 weights this is what the kernels see."""
-    return {k: (v.detach().cpu().to(torch.bfloat16) if k in BF16_FIELDS else v.detach().cpu().float())
-            for k, v in W.items()}
+    return {k: v.detach().cpu().to(_abi_dtype(k, v)) for k, v in W.items()}
 
 
 def _fp32_matrices(W: dict) -> bool:
