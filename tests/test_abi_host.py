@@ -136,3 +136,36 @@ def test_argument_errors_are_reported_before_launch():
     assert rc == ZB._abi.ZAYA_ERR_INVALID_ARG
     rc = L.zaya_device_status(None, None)
     assert rc == ZB._abi.ZAYA_ERR_INVALID_ARG
+
+
+def test_noalloc_checks_arguments_before_enqueueing_anything():
+    """The entry point without a caller workspace checks every argument
+    before it touches a device (it clears its scratch header only after):
+    on a machine without a GPU an invalid call returns its code, and a
+    well-formed call too large for the fixed scratch returns
+    ZAYA_ERR_WORKSPACE."""
+    cfg = get_config("tiny")
+    c = ZB.make_config(cfg)
+    L = _abi.lib()
+    w = _abi.zaya_block_weights()
+    st = _abi.zaya_block_state()
+    fake = C.c_void_p(256)
+    rc = L.zaya_block_decode_noalloc(C.byref(c), C.byref(w), 1, 2, fake, fake, C.c_void_p(512), C.byref(st), None,
+                                     None)
+    assert rc == ZB._abi.ZAYA_ERR_INVALID_ARG                  # NULL weights
+    for name in _abi.WEIGHT_FIELDS:
+        setattr(w, name, 4096)
+    rc = L.zaya_block_decode_noalloc(C.byref(c), C.byref(w), 1, 2, fake, fake, C.c_void_p(512), C.byref(st), None,
+                                     None)
+    assert rc == ZB._abi.ZAYA_ERR_INVALID_ARG                  # NULL state
+    st.k_cache = st.v_cache = st.conv_state = st.prev_hs = st.cache_len = 4096
+    st.cache_cap = 4
+    rc = L.zaya_block_decode_noalloc(C.byref(c), C.byref(w), 1, 2, fake, fake, fake, C.byref(st), None, None)
+    assert rc == ZB._abi.ZAYA_ERR_INVALID_ARG                  # router state in aliases out
+    rc = L.zaya_block_decode_noalloc(C.byref(c), C.byref(w), 1, 2, C.c_void_p(260), fake, C.c_void_p(512),
+                                     C.byref(st), None, None)
+    assert rc == ZB._abi.ZAYA_ERR_MISALIGNED                   # stream not 16-byte aligned
+    big = ZB.make_config(get_config("prefill_4k"))
+    rc = L.zaya_block_decode_noalloc(C.byref(big), C.byref(w), 1, 4096, fake, fake, C.c_void_p(512), C.byref(st),
+                                     None, None)
+    assert rc == ZB._abi.ZAYA_ERR_WORKSPACE                    # beyond the fixed scratch

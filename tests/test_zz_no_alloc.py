@@ -73,7 +73,9 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     w = _abi.zaya_block_weights()
     for n in _abi.WEIGHT_FIELDS:
         setattr(w, n, 4096)
-    st = _abi.zaya_block_state()
+    st = _abi.zaya_block_state()   # well-formed but never dereferenced: the call must stop at the size
+    st.k_cache, st.v_cache, st.cache_len, st.conv_state, st.prev_hs = 1024, 2048, 3072, 4096, 5120
+    st.cache_cap = 8
     rc = _abi.lib().zaya_block_decode_noalloc(C.byref(c), C.byref(w), 1, B, C.c_void_p(256), C.c_void_p(512),
                                               C.c_void_p(768), C.byref(st), None, None)
     assert rc == _abi.ZAYA_ERR_WORKSPACE
