@@ -339,23 +339,27 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
   }
   tc_fence_before();
   __syncwarp();
-  // The prologue above overlaps the previous kernel; global memory only from here.
-  // A fault already recorded in the status word (an earlier wait ran out)
-  // means the launch chain has failed: the kernel then does no work.  Both
-  // CTAs of a pair take rank 0's reading, so that they walk the same tiles.
+  if constexpr (CG == 2) cluster_sync_all();   // both CTAs' barriers and TMEM are ready
+  else __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // The prologue above (with the tensor-memory allocation) overlaps the
+  // previous kernel, and is complete in every warp before any thread lets the
+  // next kernel launch.  Global memory only from here.  A fault already
+  // recorded in the status word (an earlier wait ran out) means the launch
+  // chain has failed: the kernel then does no work.  Both CTAs of a pair take
+  // rank 0's reading, so that they walk the same tiles.
   griddep_begin();
   WaitCtx wc = wait_ctx(p.status, /*bail=*/CG == 1);
   if constexpr (CG == 2) {
-    if (rank == 0 && threadIdx.x == 0) *s_skip = wc.skip ? 1 : 0;
-    cluster_sync_all();   // both CTAs' barriers and TMEM are ready; rank 0's reading is published
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(mapa_shared(s_skip, 0)) : "memory");
-    wc.skip = v != 0;
-  } else {
-    __syncthreads();
+    if (rank == 0 && threadIdx.x == 0) {
+      const uint32_t v = wc.skip ? 1u : 0u;
+      *s_skip = v;
+      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa_shared(s_skip, 1)), "r"(v) : "memory");
+    }
+    cluster_sync_all();   // rank 0's reading is published to both CTAs
+    wc.skip = *reinterpret_cast<volatile int*>(s_skip) != 0;
   }
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
 
   const int ntiles = wc.skip ? 0 : total_tiles<EPI, BN_OUT, TM>(p);
 
