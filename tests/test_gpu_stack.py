@@ -182,9 +182,21 @@ def test_prefill_stack_32k_sampled():
     c = ZB.make_config(cfg)
     ws = Hn.workspace(ZB.zaya_stack_workspace_size(c, ZB.ZAYA_PREFILL, B, S), poison=False)
     logits = torch.empty(B, S, V, dtype=torch.bfloat16, device=dev)
-    ZB.zaya_stack_forward(c, [ZB.make_weights(w) for w in blocks_d], extra_d["embed"], extra_d["final_norm_w"],
-                          ZB.ZAYA_PREFILL, B, S, ids, None, [ZB.make_state(s) for s in states], logits, 0, ws)
+    w_s, st_s = [ZB.make_weights(w) for w in blocks_d], [ZB.make_state(s) for s in states]
+    ZB.zaya_stack_forward(c, w_s, extra_d["embed"], extra_d["final_norm_w"], ZB.ZAYA_PREFILL, B, S, ids, None, st_s,
+                          logits, 0, ws)
     assert ZB.zaya_device_status(ws) == 0
+    rows = [0, 4095, 4096, S - 1]
+    first = logits[0, rows].clone()
+    # three more passes back to back (no host synchronisation between them):
+    # the launch chain crosses stack and block boundaries and must complete,
+    # with bit-identical results (every token's arithmetic is independent of
+    # its place in the expert permutation)
+    for _ in range(3):
+        ZB.zaya_stack_forward(c, w_s, extra_d["embed"], extra_d["final_norm_w"], ZB.ZAYA_PREFILL, B, S, ids, None,
+                              st_s, logits, 0, ws)
+    assert ZB.zaya_device_status(ws) == 0
+    assert torch.equal(logits[0, rows], first)
     del states, ws
     ranges = [(S - 48, S), (4094, 4099)]
     x = _embed_stream(cfg, extra_d["embed"], ids)
@@ -200,7 +212,6 @@ def test_prefill_stack_32k_sampled():
         x = out["layer_output"].to(dev)
         r = out["router_state"].to(dev)
         del out
-    rows = [0, 4095, 4096, S - 1]
     emb = extra_d["embed"].cpu()
     _, ref_logits = Z.lm_head(cfg, emb, extra_d["final_norm_w"].cpu(), Z.as64(x[0, rows]))
     _check_logits(logits[0, rows], ref_logits)

@@ -47,7 +47,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // carve-out) then overlap this kernel's run and its tail.  The dependents of a
 // grid launch only once all of its CTAs have made the call, i.e. are resident,
 // so a waiting dependent never holds resources an unscheduled CTA of its
-// predecessor needs.
+// predecessor needs.  A CTA counts as having let its dependents launch as soon
+// as ANY of its threads executes launch_dependents, so a kernel that allocates
+// tensor memory must finish the allocation in every warp (and synchronise)
+// before any thread calls griddep_begin(): otherwise a dependent's CTA can
+// take the columns first and wait for this kernel, which waits for the columns.
 __device__ __forceinline__ void griddep_begin() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -425,9 +429,12 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // Launch with programmatic stream serialisation (the kernel must begin with
 // griddep_begin()); extra launch attributes (a cluster shape) may be added.
+// `programmatic` = 0 launches the kernel in plain stream order instead (it
+// starts only once the previous kernel has completed; its griddep_begin()
+// then returns at once and still lets the next kernel launch early).
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                            const cudaLaunchAttribute* extra, int n_extra, Args&&... args) {
+inline cudaError_t launch_k_as(int programmatic, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                               cudaStream_t st, const cudaLaunchAttribute* extra, int n_extra, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -435,11 +442,16 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
   cfg.stream = st;
   cudaLaunchAttribute attr[4];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].val.programmaticStreamSerializationAllowed = programmatic;
   for (int i = 0; i < n_extra && i < 3; ++i) attr[1 + i] = extra[i];
   cfg.attrs = attr;
   cfg.numAttrs = 1 + (n_extra < 3 ? n_extra : 3);
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            const cudaLaunchAttribute* extra, int n_extra, Args&&... args) {
+  return launch_k_as(1, kern, grid, block, smem, st, extra, n_extra, static_cast<Args&&>(args)...);
 }
 
 }  // namespace zaya

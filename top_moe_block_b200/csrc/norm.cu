@@ -9,6 +9,13 @@
 // thread keeps it in registers and four 8-warp CTAs fit an SM; the second
 // read is served from cache; the weight is staged in shared memory.
 // HBM-bound (4 bytes read + 2 bytes written per element).
+// The norms are launched in plain stream order, not as programmatic
+// dependents: with their small CTAs waiting beside a CTA-pair GEMM (the
+// previous block's expert down projection) and the next CTA-pair GEMM (the
+// q/k/v projection) waiting on them in turn, a 40-block prefill stack at
+// S = 32768 stopped making progress in about one stack in three; launched in
+// stream order, 30 stacks of 30 completed (as they also did with the pair
+// GEMMs launched in stream order instead).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -167,19 +174,19 @@ int launch_rmsnorm(const float* x, int row_mul, int row_add, const void* w, void
   const int v = H % 512 ? 0 : H / 512;   // one CTA per row when H is a multiple of 512
   if (v == 1 || v == 2 || v == 4 || v == 8) {
     cudaError_t e;
-    if (v == 1) e = launch_k(rmsnorm_row_kernel<1>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
-    else if (v == 2) e = launch_k(rmsnorm_row_kernel<2>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
-    else if (v == 4) e = launch_k(rmsnorm_row_kernel<4>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
-    else e = launch_k(rmsnorm_row_kernel<8>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
+    if (v == 1) e = launch_k_as(0, rmsnorm_row_kernel<1>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
+    else if (v == 2) e = launch_k_as(0, rmsnorm_row_kernel<2>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
+    else if (v == 4) e = launch_k_as(0, rmsnorm_row_kernel<4>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
+    else e = launch_k_as(0, rmsnorm_row_kernel<8>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
     return e == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
   }
   const dim3 grid((rows + 7) / 8);
   switch (H / 128) {
-    case 2: launch_k(rmsnorm_kernel<2>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
-    case 4: launch_k(rmsnorm_kernel<4>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
-    case 8: launch_k(rmsnorm_kernel<8>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
-    case 16: launch_k(rmsnorm_kernel<16>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
-    case 32: launch_k(rmsnorm_kernel<32>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 2: launch_k_as(0, rmsnorm_kernel<2>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 4: launch_k_as(0, rmsnorm_kernel<4>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 8: launch_k_as(0, rmsnorm_kernel<8>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 16: launch_k_as(0, rmsnorm_kernel<16>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 32: launch_k_as(0, rmsnorm_kernel<32>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
     default: return ZAYA_ERR_UNSUPPORTED;
   }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
