@@ -569,14 +569,22 @@ def run_decode(K, warmup, world, rank, local, cfg, show_stages):
     return line
 
 
+def block_window(cfg, block_idx):
+    """The window block `block_idx` attends over: the config's, or (a hybrid
+    stack's full-attention blocks) the whole sequence."""
+    if cfg.sliding_period <= 0 or block_idx % cfg.sliding_period == cfg.sliding_phase:
+        return cfg.window
+    return cfg.seq
+
+
 def stack_prefill_flops(cfg, routed_per_block):
     """Tensor-core FLOPs of one stack prefill: every block's contractions
     (routed tokens, window pairs) and the tied lm_head at every position."""
     M, H, V = cfg.batch * cfg.seq, cfg.hidden, cfg.vocab
-    pairs = attention_pairs(cfg, None)
     blocks = 0.0
-    for routed in routed_per_block:
-        w = stage_work(cfg, routed, pairs)
+    for i, routed in enumerate(routed_per_block):
+        bc = cfg.with_(window=block_window(cfg, i))
+        w = stage_work(bc, routed, attention_pairs(bc, None))
         blocks += sum(v[1] for v in w.values() if v[0] == "tensor")
     return blocks, 2.0 * M * H * V
 
@@ -665,8 +673,10 @@ def run_stack_prefill(K, warmup, world, rank, local, cfg, show_stages):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (uniform random token ids, random-init weights of the ZAYA1-8B stack shapes)",
         "config": {"workload": f"{cfg.name}: prefill of B{B} x S{S} uniform random ids through embedding x "
-                               f"{cfg.emb_mult:.2f}, {cfg.n_blocks} ZAYA1 blocks (window {cfg.window}), final "
-                               f"norm and tied lm_head (vocab {V}) at every position",
+                               f"{cfg.emb_mult:.2f}, {cfg.n_blocks} ZAYA1 blocks (window {cfg.window}"
+                               + (f" on blocks {cfg.sliding_phase} mod {cfg.sliding_period}, every earlier token "
+                                  f"on the others" if cfg.sliding_period > 0 else "")
+                               + f"), final norm and tied lm_head (vocab {V}) at every position",
                    "batch": B, "seq_len": S, "tokens_per_step": M,
                    "tc_flops_per_step": {"blocks": blk, "lm_head": head,
                                          "routed_tokens_per_block": routed},

@@ -64,7 +64,7 @@
 extern "C" {
 #endif
 
-#define ZAYA_ABI_VERSION 1
+#define ZAYA_ABI_VERSION 2
 
 enum zaya_status {
   ZAYA_OK = 0,
@@ -97,6 +97,11 @@ typedef struct zaya_config {
   int32_t vocab;             /* stack only: embedding rows */
   int32_t cca_mean_residual; /* 1: add the CCA mean residual after the conv */
   int32_t v_delayed;         /* 1: second half of each value head from token t-1 */
+  int32_t sliding_period;    /* 0: every block attends over `window` keys.  P > 0: only blocks with
+                                block_idx % P == sliding_phase do; the others attend to every
+                                earlier token (ZAYA1-74B-preview: a 4097-token window on every
+                                other block; zaya page, "Queries and keys are convolved ...") */
+  int32_t sliding_phase;     /* 0 <= sliding_phase < sliding_period */
   float rope_theta;          /* inv_freq[i] = rope_theta^(-2i/rot_dim) */
   float rms_eps;             /* RMSNorm epsilon (1e-5) */
   float qk_norm_eps;         /* q,k -> x * sqrt(d) / max(|x|, qk_norm_eps) */

@@ -194,6 +194,22 @@ def attention(q, k, v, q_pos, k_pos, k_valid, window, scale):
     return out
 
 
+FULL_ATTENTION = 1 << 62   # a window no sequence reaches
+
+
+def block_window(cfg, block_idx):
+    """Keys (its own included) a query of block ``block_idx`` attends over.
+    Every block slides over ``cfg.window`` keys unless ``cfg.sliding_period``
+    is set: then only the blocks with block_idx % period == phase slide and
+    the others attend to every earlier token -- ZAYA1-74B-preview's hybrid,
+    a 4097-token window on every other block (zaya page, "Queries and keys
+    are convolved ...", last sentence)."""
+    period = getattr(cfg, "sliding_period", 0)
+    if period <= 0 or block_idx % period == cfg.sliding_phase:
+        return cfg.window
+    return FULL_ATTENTION
+
+
 # ---------------------------------------------------------------------------
 # router and experts (zaya page, "One expert per token, chosen beside a skip
 # class"; "Printout" for the router's modules)
@@ -358,7 +374,7 @@ def block_prefill(cfg, W, x, attn_mask=None, router_state_in=None, block_idx=Non
         v = _values(cfg, vc, vd_prev)
         k = round_bf16(k)
         v = round_bf16(v)
-        o = attention(q, k, v, pos, pos, real, cfg.window, cfg.scale)
+        o = attention(q, k, v, pos, pos, real, block_window(cfg, bidx), cfg.scale)
         premix = o.reshape(S, nq * d)
         attn_o = premix @ as64(W["w_o"]).T
         attn_out, h = merge(attn_o, x[b], as64(W["merge_a"]))
@@ -393,7 +409,8 @@ def block_prefill_rows(cfg, W, x, r0, r1, router_state_in=None, block_idx=None, 
     x = as64(x)
     bidx = cfg.block_idx if block_idx is None else block_idx
     d, nq = cfg.head_dim, cfg.n_q
-    lo = max(0, r0 - cfg.window + 1)     # first key any of the rows sees
+    window = block_window(cfg, bidx)
+    lo = max(0, r0 - window + 1)         # first key any of the rows sees
     t0 = max(0, lo - 3)                  # plus the conv / delayed-value history
     seg = x[t0:r1]
     a_in = block_norm(seg, as64(W["ln1_w"]), cfg.rms_eps)
@@ -411,7 +428,7 @@ def block_prefill_rows(cfg, W, x, r0, r1, router_state_in=None, block_idx=None, 
     kl = lo - t0
     qi = np.arange(r0, r1) - t0
     o = attention(q[qi], k[kl:], v[kl:], np.arange(r0, r1), np.arange(lo, r1), np.ones(r1 - lo, dtype=bool),
-                  cfg.window, cfg.scale)
+                  window, cfg.scale)
     premix = o.reshape(r1 - r0, nq * d)
     attn_o = premix @ as64(W["w_o"]).T
     attn_out, h = merge(attn_o, x[r0:r1], as64(W["merge_a"]))
@@ -457,10 +474,11 @@ def block_decode(cfg, W, x, state, router_state_in=None, block_idx=None, force_c
         v = round_bf16(v)
         kc[b, :, t] = k[0]
         vcache[b, :, t] = v[0]
-        lo = max(0, t - cfg.window + 1)
+        window = block_window(cfg, bidx)
+        lo = max(0, t - window + 1)
         kpos = np.arange(lo, t + 1)
         o = attention(q, kc[b, :, lo:t + 1].transpose(1, 0, 2), vcache[b, :, lo:t + 1].transpose(1, 0, 2),
-                      np.array([t]), kpos, np.ones(len(kpos), dtype=bool), cfg.window, cfg.scale)
+                      np.array([t]), kpos, np.ones(len(kpos), dtype=bool), window, cfg.scale)
         premix[b] = o.reshape(nq * d)
         conv_state[b] = np.stack([hist[1], u[0]], axis=1)
         qs.append(q[0]); ks.append(k[0]); vs.append(v[0])

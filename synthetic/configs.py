@@ -33,6 +33,8 @@ class BlockConfig:
     attn_scale: float = 0.0      # 0 -> 1/sqrt(head_dim)
     cca_mean_residual: int = 1   # add the CCA mean residual after the conv
     v_delayed: int = 1           # half of each value head from token t-1
+    sliding_period: int = 0      # 0: every block slides over `window` keys; P > 0: only blocks with
+    sliding_phase: int = 0       # block % P == phase slide, the others attend to every earlier token
     vocab: int = 0
     emb_mult: float = 1.0
     emb_shift: float = 0.0
@@ -123,6 +125,12 @@ CONFIGS = {
         name="decode_stack_b64", batch=64, seq=1, n_blocks=40, block_idx=0, mode="decode",
         cache_prior=8192, seed=3, skip_bias=-1.0, input_dtype="bf16",
         vocab=262144, emb_mult=math.sqrt(2048.0), **_FULL),
+    # The same stack with the 74B preview's hybrid attention: a 4097-token
+    # window on every other block (the odd ones), every earlier token on the others.
+    "prefill_stack_hybrid_32k": BlockConfig(
+        name="prefill_stack_hybrid_32k", batch=1, seq=32768, n_blocks=40, block_idx=0, seed=5,
+        skip_bias=-1.0, input_dtype="bf16", vocab=262144, emb_mult=math.sqrt(2048.0),
+        sliding_period=2, sliding_phase=1, **dict(_FULL, window=4097)),
     # Long prefill through the 40-block stack with embedding and tied lm_head.
     "prefill_stack_32k": BlockConfig(
         name="prefill_stack_32k", batch=1, seq=32768, n_blocks=40, block_idx=0, seed=4,

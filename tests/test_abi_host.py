@@ -63,7 +63,7 @@ def test_struct_layout_matches_header(tmp_path):
 
 
 def test_status_strings_and_version():
-    assert ZB.zaya_abi_version() == 1
+    assert ZB.zaya_abi_version() == 2
     for code in range(8):
         assert isinstance(ZB.zaya_status_string(code), str)
     assert ZB.zaya_status_string(0) == "ok"

@@ -206,3 +206,21 @@ def test_wait_timeout_is_reported_and_the_context_recovers():
     torch.cuda.synchronize()
     gpu = Hn.gpu_prefill(cfg, Wd, inp["x"], None, inp["router_state_in"])
     Hn.assert_block_ok(Hn.check_prefill_block(cfg, W, inp, gpu, verbose=False))
+
+
+@pytest.mark.parametrize("block_idx", [1, 2])
+def test_full_prefill_hybrid_8k_sampled(block_idx):
+    """The 74B preview's hybrid at full width, S = 8192: block 1 slides over
+    4097 keys, block 2 attends to every earlier token (zaya page, 'Queries
+    and keys are convolved ...', last sentence); sampled rows against the
+    oracle's windowed evaluation."""
+    from tests import harness as Hn
+    cfg = get_config("prefill_4k").with_(seq=8192, window=4097, sliding_period=2, sliding_phase=1,
+                                         block_idx=block_idx)
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    gpu = Hn.gpu_prefill(cfg, Hn.dev_weights(W), inp["x"], None, inp["router_state_in"])
+    ranges = [(4090, 4106), (8192 - 24, 8192)]
+    res = Hn.check_prefill_rows(cfg, W, inp["x"][0], inp["router_state_in"][0], gpu, ranges, block_idx)
+    print(res)
+    Hn.assert_rows_ok(res)

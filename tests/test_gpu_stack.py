@@ -37,11 +37,16 @@ def _check_logits(gpu_logits, ref_logits):
         Hn.rel_max(g, ref_logits), Hn.cosine(g, ref_logits))
 
 
-def test_tiny_stack_prefill():
+@pytest.mark.parametrize("hybrid", [False, True])
+def test_tiny_stack_prefill(hybrid):
+    """The tiny stack; `hybrid`: a 12-key window on the odd blocks, every
+    earlier token on the even ones (the 74B preview's alternation)."""
     import top_moe_block_b200 as ZB
     from oracle import zaya_oracle as Z
     from tests import harness as Hn
     cfg = get_config("tiny").with_(n_blocks=3, block_idx=0, batch=2, seq=50)
+    if hybrid:
+        cfg = cfg.with_(window=12, sliding_period=2, sliding_phase=1)
     B, S, V = cfg.batch, cfg.seq, cfg.vocab
     blocks = [gen_block_weights(cfg, block=i) for i in range(cfg.n_blocks)]
     bd = [Hn.dev_weights(w) for w in blocks]
@@ -72,13 +77,17 @@ def test_tiny_stack_prefill():
     np.testing.assert_array_equal(states[-1]["cache_len"].cpu().numpy(), S)
 
 
-def test_tiny_stack_decode_after_prefill():
+@pytest.mark.parametrize("hybrid", [False, True])
+def test_tiny_stack_decode_after_prefill(hybrid):
     """prefill(S) through the stack, then one decode step through the stack;
-    the decode logits against the oracle's decode of the GPU's states."""
+    the decode logits against the oracle's decode of the GPU's states.
+    `hybrid`: block 0 attends to every earlier token, block 1 over 8 keys."""
     import top_moe_block_b200 as ZB
     from oracle import zaya_oracle as Z
     from tests import harness as Hn
     cfg = get_config("tiny").with_(n_blocks=2, block_idx=0, batch=3, seq=40)
+    if hybrid:
+        cfg = cfg.with_(window=8, sliding_period=2, sliding_phase=1)
     B, S, V = cfg.batch, cfg.seq, cfg.vocab
     blocks = [gen_block_weights(cfg, block=i) for i in range(cfg.n_blocks)]
     bd = [Hn.dev_weights(w) for w in blocks]

@@ -556,3 +556,45 @@ def test_router_state_chain_in_decode():
             np.testing.assert_array_equal(a, b)
         else:
             assert (a != b).any(axis=-1).all()
+
+
+# ---------------------------------------------------------------- hybrid sliding / full blocks
+
+def test_hybrid_blocks_window_reach():
+    """With sliding_period = 2, sliding_phase = 1 (ZAYA1-74B-preview: a
+    window on every other block; zaya page, 'Queries and keys are convolved
+    ...', last sentence), an odd block keeps the window's reach (outputs at
+    i >= t+W+2 bit-identical after perturbing token t), an even block
+    attends to every earlier token (the output far beyond the window moves),
+    and a stack without the setting slides on every block."""
+    cfg = get_config("tiny").with_(seq=48, window=8, sliding_period=2, sliding_phase=1)
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    t = 3
+    far = t + cfg.window + 20
+    for bidx, slides in ((1, True), (3, True), (0, False), (2, False)):
+        assert (Z.block_window(cfg, bidx) == cfg.window) == slides
+        o = Z.block_prefill(cfg, W, inp["x"], None, inp["router_state_in"], block_idx=bidx)
+        x2 = inp["x"].clone()
+        x2[0, t] += 1.0
+        o2 = Z.block_prefill(cfg, W, x2, None, inp["router_state_in"], block_idx=bidx)
+        same = np.array_equal(o2["attention_premix"][0, t + cfg.window + 2:], o["attention_premix"][0, t + cfg.window + 2:])
+        assert same == slides, bidx
+        assert np.array_equal(o2["attention_premix"][0, far], o["attention_premix"][0, far]) == slides, bidx
+    plain = cfg.with_(sliding_period=0)
+    assert all(Z.block_window(plain, b) == cfg.window for b in range(4))
+
+
+def test_hybrid_full_block_is_plain_causal():
+    """A full-attention block equals the same block with a window longer
+    than the sequence, and its windowed row evaluation (keys back to 0)
+    equals the full prefill at those rows."""
+    cfg = get_config("tiny").with_(seq=60, window=8, sliding_period=2, sliding_phase=1)
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    o = Z.block_prefill(cfg, W, inp["x"], None, inp["router_state_in"], block_idx=2)
+    ref = Z.block_prefill(cfg.with_(window=10**6, sliding_period=0), W, inp["x"], None, inp["router_state_in"],
+                          block_idx=2)
+    np.testing.assert_array_equal(o["layer_output"], ref["layer_output"])
+    part = Z.block_prefill_rows(cfg, W, inp["x"][0], 40, 60, inp["router_state_in"][0], block_idx=2)
+    np.testing.assert_allclose(part["layer_output"], o["layer_output"][0, 40:60], rtol=1e-9, atol=1e-9)

@@ -19,8 +19,9 @@ namespace zaya {
 
 namespace {
 
-constexpr int kChunk = 256;   // keys per CTA
+constexpr int kChunk = 256;   // keys per CTA up to kMaxChunks chunks (longer spans: longer chunks)
 constexpr int kWarps = 4;
+constexpr int kMaxChunks = 64; // a head's partials in the workspace
 
 template <int D, int REP>
 __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams p) {
@@ -34,10 +35,10 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
   const int t_raw = p.cache_len[b];
   const int t = (t_raw >= 0 && t_raw < p.cap) ? t_raw : -1;
   const int lo = max(0, t - p.window + 1);
-  const int c_begin = lo + chunk * kChunk;
-  const int c_end = min(t + 1, c_begin + kChunk);
-  const int w_begin = c_begin + warp * (kChunk / kWarps);
-  const int w_end = min(c_end, w_begin + kChunk / kWarps);
+  const int c_begin = lo + chunk * p.chunk_keys;
+  const int c_end = min(t + 1, c_begin + p.chunk_keys);
+  const int w_begin = c_begin + warp * (p.chunk_keys / kWarps);
+  const int w_end = min(c_end, w_begin + p.chunk_keys / kWarps);
 
   const float sl2 = p.scale * 1.4426950408889634f;
   float q[REP][DPL];
@@ -197,13 +198,29 @@ __global__ void attn_decode_combine(const DecodeAttnParams p, int rep) {
 
 }  // namespace
 
-size_t decode_attn_ws_bytes(int B, int n_q, int d, int window) {
-  const int n_chunks = (window + kChunk - 1) / kChunk;
-  return (size_t)B * n_q * n_chunks * (d + 2) * sizeof(float);
+int decode_attn_max_chunks(int window) {
+  const long n = ((long)window + kChunk - 1) / kChunk;
+  return n < 1 ? 1 : (n > kMaxChunks ? kMaxChunks : (int)n);
+}
+
+size_t decode_attn_ws_bytes(int B, int n_q, int d, int max_chunks) {
+  return (size_t)B * n_q * max_chunks * (d + 2) * sizeof(float);
+}
+
+void decode_attn_split(int span, int max_chunks, int* n_chunks, int* chunk_keys) {
+  int n = (span + kChunk - 1) / kChunk;
+  int ck = kChunk;
+  if (n > max_chunks) {   // longer chunks, still whole multiples of 256 keys
+    ck = ((span + max_chunks - 1) / max_chunks + kChunk - 1) / kChunk * kChunk;
+    n = (span + ck - 1) / ck;
+  }
+  *n_chunks = n < 1 ? 1 : n;
+  *chunk_keys = ck;
 }
 
 int launch_attn_decode(const DecodeAttnParams& p, cudaStream_t st) {
   if (p.B <= 0) return ZAYA_OK;
+  if (p.n_chunks < 1 || p.n_chunks > kMaxChunks || p.chunk_keys % kChunk) return ZAYA_ERR_UNSUPPORTED;
   const int rep = p.n_q / p.n_kv;
   const dim3 grid(p.n_chunks, p.n_kv, p.B);
 #define ZAYA_DEC(DV, RV)                                                   \

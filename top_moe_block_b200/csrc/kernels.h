@@ -126,9 +126,16 @@ struct DecodeAttnParams {
   void* out;              // bf16 premix [B, n_q*d]
   float* part;            // workspace partials
   int B, cap, n_q, n_kv, d, window, n_chunks;
+  int chunk_keys;         // keys per CTA (a multiple of 256)
   float scale;
 };
-size_t decode_attn_ws_bytes(int B, int n_q, int d, int window);
+// Key chunks a head's decode attention may use for a window (256 keys per
+// chunk, at most 64 chunks; a full-attention block passes a window no cache reaches).
+int decode_attn_max_chunks(int window);
+// Workspace of the decode attention's partials for up to max_chunks chunks per head.
+size_t decode_attn_ws_bytes(int B, int n_q, int d, int max_chunks);
+// Key chunks for a span of keys: 256 keys per chunk up to max_chunks, longer chunks beyond it.
+void decode_attn_split(int span, int max_chunks, int* n_chunks, int* chunk_keys);
 int launch_attn_decode(const DecodeAttnParams& p, cudaStream_t st);
 
 // ------------------------------------------------------------------ router / MoE dispatch

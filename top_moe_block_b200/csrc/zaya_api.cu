@@ -125,7 +125,31 @@ int check_config(const zaya_config* c) {
   if (c->inter % 128) return ZAYA_ERR_UNSUPPORTED;
   if (c->router_hidden % 32 || c->router_hidden > 256) return ZAYA_ERR_UNSUPPORTED;
   if (c->rms_eps < 0.f || c->qk_norm_eps <= 0.f) return ZAYA_ERR_INVALID_ARG;
+  if (c->sliding_period < 0 || (c->sliding_period > 0 && (c->sliding_phase < 0 || c->sliding_phase >= c->sliding_period)))
+    return ZAYA_ERR_INVALID_ARG;
   return ZAYA_OK;
+}
+
+// Keys (its own included) a query of block `block_idx` attends over: the
+// config's window, or every earlier token on the blocks a hybrid stack does
+// not slide (a window no sequence of the library reaches).
+constexpr int kFullWindow = 1 << 30;
+int block_window(const zaya_config& c, int block_idx) {
+  if (c.sliding_period <= 0 || block_idx % c.sliding_period == c.sliding_phase) return c.window;
+  return kFullWindow;
+}
+// Most key chunks a decode step's attention uses over the config's blocks.
+int decode_chunks_any(const zaya_config& c) {
+  return decode_attn_max_chunks(c.sliding_period > 0 ? kFullWindow : c.window);
+}
+// Largest prefill attention workspace over the windows the config's blocks use.
+size_t attn_prefill_ws_any(const zaya_config& c, int B, int S, int nq, int nkv, int d) {
+  size_t n = attn_prefill_ws_bytes(B, S, c.window, nq, nkv, d);
+  if (c.sliding_period > 0) {
+    const size_t f = attn_prefill_ws_bytes(B, S, kFullWindow, nq, nkv, d);
+    if (f > n) n = f;
+  }
+  return n;
 }
 
 inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -171,8 +195,8 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.mt_start = o; o += up((size_t)(d.E + 2) * 4);
   w.xperm = o; o += up(M * d.H * 2);
   w.act = o; o += up(M * d.I * 2);
-  w.part = o; o += up(mode == ZAYA_DECODE ? decode_attn_ws_bytes(B, d.nq, d.d, c.window)
-                                           : attn_prefill_ws_bytes(B, S, c.window, d.nq, d.nkv, d.d));
+  w.part = o; o += up(mode == ZAYA_DECODE ? decode_attn_ws_bytes(B, d.nq, d.d, decode_chunks_any(c))
+                                           : attn_prefill_ws_any(c, B, S, d.nq, d.nkv, d.d));
   w.rpart = o; o += up((size_t)router_down_splits((int)M, d.H) * M * d.R * 4);
   w.wsplit = o; o += up(((size_t)4 * d.R * d.R + (size_t)2 * ((d.E + 1 + 7) / 8 * 8) * d.R) * 2);   // fc1, fc2, out_proj hi / lo
   w.slot = o; o += up(M * 4);
@@ -330,6 +354,7 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
   if (ws_bytes < L.total) return ZAYA_ERR_WORKSPACE;
   const int M = B * S;
   const int sms = num_sms_current();
+  const int window = block_window(c, block_idx);
   int* status = at<int>(ws, L.status);
   void* a_in = at<void>(ws, L.a_in);
   void* qkv = at<void>(ws, L.qkv);
@@ -355,7 +380,7 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     p.cca_res = c.cca_mean_residual; p.v_delayed = c.v_delayed; p.theta = c.rope_theta; p.eps = c.qk_norm_eps;
     p.decode = 0; p.status = status;
     size_t ctr_off = 0;   // the attention's split merge counters, cleared by this kernel
-    p.n_zero_words = attn_prefill_ctr(B, S, c.window, d.nq, d.d, &ctr_off);
+    p.n_zero_words = attn_prefill_ctr(B, S, window, d.nq, d.d, &ctr_off);
     p.zero_words = p.n_zero_words ? reinterpret_cast<int*>(at<uint8_t>(ws, L.part) + ctr_off) : nullptr;
     fill_inv_freq(p.inv_freq, c.rot_dim, c.rope_theta);
     ZAYA_STAGE("cca", 1, launch_cca(p, st));
@@ -365,10 +390,10 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     p.ctr_cleared = 1;
     p.q = at<void>(ws, L.q); p.k_cache = state->k_cache; p.v_cache = state->v_cache; p.mask = mask;
     p.out = at<void>(ws, L.premix);
-    p.B = B; p.S = S; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = c.window;
+    p.B = B; p.S = S; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = window;
     p.scale = d.scale;
     p.part = at<void>(ws, L.part);
-    p.part_bytes = attn_prefill_ws_bytes(B, S, c.window, d.nq, d.nkv, d.d);
+    p.part_bytes = attn_prefill_ws_bytes(B, S, window, d.nq, d.nkv, d.d);
     ZAYA_STAGE("attention", 1, launch_attn_prefill_tc(p, status, st));
   }
   return block_tail(c, d, w, block_idx, M, hidden, rin, rout, taps, ws, L, nullptr, mask, sms, st);
@@ -432,9 +457,10 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
     DecodeAttnParams p{};
     p.q = at<void>(ws, L.q); p.k_cache = state->k_cache; p.v_cache = state->v_cache; p.cache_len = state->cache_len;
     p.out = at<void>(ws, L.premix); p.part = at<float>(ws, L.part);
-    p.B = B; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = c.window;
-    const int span = c.window < state->cache_cap ? c.window : state->cache_cap;
-    p.n_chunks = (span + 255) / 256;
+    const int window = block_window(c, block_idx);
+    p.B = B; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = window;
+    const int span = window < state->cache_cap ? window : state->cache_cap;
+    decode_attn_split(span, decode_chunks_any(c), &p.n_chunks, &p.chunk_keys);
     p.scale = d.scale;
     ZAYA_STAGE("attention_decode", 2, launch_attn_decode(p, st));
   }
