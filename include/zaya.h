@@ -81,7 +81,8 @@ enum zaya_mode { ZAYA_PREFILL = 0, ZAYA_DECODE = 1 };
 
 /* Shapes and every choice the pages leave open, passed by value.
  * Supported: hidden % 128 == 0 and <= 4096; head_dim in {64, 128};
- * rot_dim even and <= head_dim; n_q % n_kv == 0; conv_width == 3;
+ * rot_dim even and <= head_dim; n_q % n_kv == 0; conv_width == 3 with
+ * conv_groups == 0, or conv_width == 2 with conv_groups == n_q + n_kv;
  * n_experts <= 64; inter % 128 == 0; router_hidden % 32 == 0 and <= 256. */
 typedef struct zaya_config {
   int32_t hidden;            /* H (2048 on ZAYA1-8B) */
@@ -89,7 +90,8 @@ typedef struct zaya_config {
   int32_t n_kv;              /* key/value heads (2); query head h uses kv head h / (n_q/n_kv) */
   int32_t head_dim;          /* d (128) */
   int32_t rot_dim;           /* rotated dims per head, pairs (i, i + rot_dim/2) (64) */
-  int32_t conv_width;        /* 3: taps over tokens (t-2, t-1, t) */
+  int32_t conv_width;        /* 3: one depthwise conv, taps over tokens (t-2, t-1, t);
+                                2: the printout's two convs of width 2 (conv_groups > 0) */
   int32_t n_experts;         /* E (16); the router scores E + 1 classes, the last is skip */
   int32_t inter;             /* expert width I (2048) */
   int32_t router_hidden;     /* R (256) */
@@ -102,6 +104,10 @@ typedef struct zaya_config {
                                 earlier token (ZAYA1-74B-preview: a 4097-token window on every
                                 other block; zaya page, "Queries and keys are convolved ...") */
   int32_t sliding_phase;     /* 0 <= sliding_phase < sliding_period */
+  int32_t conv_groups;       /* 0: conv_w is the width-3 depthwise conv.  G > 0: conv_qk_depthwise
+                                (k=2, conv_w [C,2], conv_b) then conv_qk_grouped (k=2, G groups,
+                                conv2_w, conv2_b) as the zaya page's printout lists them; the
+                                kernels take one group per q / k head (G = n_q + n_kv, 10 on ZAYA1-8B) */
   float rope_theta;          /* inv_freq[i] = rope_theta^(-2i/rot_dim) */
   float rms_eps;             /* RMSNorm epsilon (1e-5) */
   float qk_norm_eps;         /* q,k -> x * sqrt(d) / max(|x|, qk_norm_eps) */
@@ -117,7 +123,8 @@ typedef struct zaya_block_weights {
   const void* ln2_w;              /* bf16 [H]   post_attention_layernorm weight */
   const void* w_qkv;              /* bf16 [n_q*d + n_kv*d + n_kv*d, H]: rows q_proj, k_proj,
                                      v_proj_current (n_kv*d/2 rows), v_proj_delayed (n_kv*d/2) */
-  const float* conv_w;            /* fp32 [C, 3] taps for (t-2, t-1, t) over the q||k channels */
+  const float* conv_w;            /* fp32 [C, 3] taps for (t-2, t-1, t) over the q||k channels;
+                                     with conv_groups > 0: [C, 2] depthwise taps for (t-1, t) */
   const float* conv_b;            /* fp32 [C] */
   const float* k_temp;            /* fp32 [n_kv] key temperature */
   const void* w_o;                /* bf16 [H, n_q*d] o_proj */
@@ -136,6 +143,10 @@ typedef struct zaya_block_weights {
   const float* balancing;         /* fp32 [E+1] balancing_biases (selection only) */
   const void* w_gate_up;          /* bf16 [E, 2I, H]: rows [0,I) gate, [I,2I) up */
   const void* w_down;             /* bf16 [E, H, I] */
+  const float* conv2_w;           /* conv_groups > 0 only (else may be NULL): fp32 [C, C/G, 2]
+                                     conv_qk_grouped taps for (t-1, t) of the depthwise output,
+                                     Conv1d's [out, in/groups, k] layout */
+  const float* conv2_b;           /* conv_groups > 0 only: fp32 [C] */
 } zaya_block_weights;
 
 /* One block's decode state (in/out, caller-owned). */

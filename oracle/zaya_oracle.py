@@ -124,6 +124,31 @@ def causal_conv(u, w, b, hist):
     return w[:, 0] * ext[0:T] + w[:, 1] * ext[1:T + 1] + w[:, 2] * ext[2:T + 2] + b
 
 
+def causal_conv_two_stage(u, dw, db, gw, gb, hist, groups):
+    """ZayaCCAProjection's two causal convolutions as the ZAYA1-8B printout
+    lists them (zaya page, "Printout": conv_qk_depthwise Conv1d(C, C, k=2,
+    groups=C), then conv_qk_grouped Conv1d(C, C, k=2, groups=G); "Queries
+    and keys are convolved ...": the current and two previous tokens):
+
+      z[s, c] = dw[c, 0] u[s-1, c] + dw[c, 1] u[s, c] + db[c]
+      y[t, o] = sum_i gw[o, i, 0] z[t-1, g(o) Cg + i] + gw[o, i, 1] z[t, g(o) Cg + i] + gb[o]
+
+    with Cg = C / G and g(o) = o // Cg (PyTorch's Conv1d weight layout
+    [out, in / groups, k]).  u before the sequence is ``hist`` (u[-2],
+    u[-1]: zeros for a fresh sequence, conv_state in decode), and z[-1] is
+    computed from it the same way, so prefill and decode agree.  u [T,C];
+    hist [2,C]; dw [C,2]; gw [C,Cg,2]."""
+    ext = np.concatenate([hist, u], axis=0)                  # u[-2] .. u[T-1]
+    T, C = u.shape
+    z = dw[:, 0] * ext[:-1] + dw[:, 1] * ext[1:] + db       # z[-1] .. z[T-1]
+    Cg = C // groups
+    y = np.empty((T, C))
+    for g in range(groups):
+        sl = slice(g * Cg, (g + 1) * Cg)
+        y[:, sl] = z[:-1, sl] @ gw[sl, :, 0].T + z[1:, sl] @ gw[sl, :, 1].T + gb[sl]
+    return y
+
+
 def cca_mean_residual(q_pre, k_pre, n_q, n_kv):
     """Each query head gets the mean of its own projection and its key head's
     projection; each key head gets the mean of those query residuals over the
@@ -295,7 +320,11 @@ def _qk(cfg, W, q_pre, k_pre, hist, pos):
     T = q_pre.shape[0]
     d = cfg.head_dim
     u = np.concatenate([q_pre, k_pre], axis=1)
-    y = causal_conv(u, as64(W["conv_w"]), as64(W["conv_b"]), hist)
+    if getattr(cfg, "conv_groups", 0):
+        y = causal_conv_two_stage(u, as64(W["conv_w"]), as64(W["conv_b"]), as64(W["conv2_w"]), as64(W["conv2_b"]),
+                                  hist, cfg.conv_groups)
+    else:
+        y = causal_conv(u, as64(W["conv_w"]), as64(W["conv_b"]), hist)
     q = y[:, :cfg.q_dim].reshape(T, cfg.n_q, d)
     k = y[:, cfg.q_dim:].reshape(T, cfg.n_kv, d)
     if cfg.cca_mean_residual:

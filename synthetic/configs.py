@@ -28,6 +28,8 @@ class BlockConfig:
     window: int                  # key j visible to query i iff 0 <= i-j < window
     rope_theta: float
     conv_width: int = 3          # taps (t-2, t-1, t) over the q||k channels
+    conv_groups: int = 0         # 0: that one depthwise conv; G: the printout's two convs of width 2
+                                 # (depthwise, then grouped with G groups; conv_width = 2)
     rms_eps: float = 1e-5
     qk_norm_eps: float = 1e-6    # x * sqrt(d) / max(|x|, eps)
     attn_scale: float = 0.0      # 0 -> 1/sqrt(head_dim)
@@ -131,6 +133,11 @@ CONFIGS = {
         name="prefill_stack_hybrid_32k", batch=1, seq=32768, n_blocks=40, block_idx=0, seed=5,
         skip_bias=-1.0, input_dtype="bf16", vocab=262144, emb_mult=math.sqrt(2048.0),
         sliding_period=2, sliding_phase=1, **dict(_FULL, window=4097)),
+    # The full-width block with the printout's two-stage conv_qk (depthwise
+    # k=2, then grouped k=2 with 10 groups), B1 x S4096.
+    "prefill_4k_conv2": BlockConfig(
+        name="prefill_4k_conv2", batch=1, seq=4096, seed=6, calibrated=1, skip_frac=0.0,
+        input_dtype="bf16", conv_width=2, conv_groups=10, **_FULL),
     # Long prefill through the 40-block stack with embedding and tied lm_head.
     "prefill_stack_32k": BlockConfig(
         name="prefill_stack_32k", batch=1, seq=32768, n_blocks=40, block_idx=0, seed=4,

@@ -96,6 +96,10 @@ def gen_block_weights(cfg: BlockConfig, block: int | None = None, device="cpu") 
     w["w_qkv"] = n("w_qkv", (cfg.n_qkv, H), cfg.w_std).to(bf)
     w["conv_w"] = bf16_values(n("conv_w", (C, cfg.conv_width), 0.5))
     w["conv_b"] = bf16_values(n("conv_b", (C,), 0.02))
+    if cfg.conv_groups:   # the grouped conv: [C, C/G, 2] (Conv1d layout), std 1/sqrt(2 C/G)
+        cg = C // cfg.conv_groups
+        w["conv2_w"] = bf16_values(n("conv2_w", (C, cg, 2), 1.0 / (2 * cg) ** 0.5))
+        w["conv2_b"] = bf16_values(n("conv2_b", (C,), 0.02))
     if cfg.temp_mode == "one":
         w["k_temp"] = torch.ones(cfg.n_kv, dtype=torch.float32, device=device)
     elif cfg.temp_mode == "zero":

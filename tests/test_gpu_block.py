@@ -224,3 +224,52 @@ def test_full_prefill_hybrid_8k_sampled(block_idx):
     res = Hn.check_prefill_rows(cfg, W, inp["x"][0], inp["router_state_in"][0], gpu, ranges, block_idx)
     print(res)
     Hn.assert_rows_ok(res)
+
+
+@pytest.mark.parametrize("seq,batch,pad", [(64, 1, 0), (129, 2, 0), (80, 3, 40)])
+def test_tiny_two_stage_conv(seq, batch, pad):
+    """The printout's two convs (depthwise k=2, then grouped k=2 with one
+    group per head) in place of the width-3 conv: tiles with ragged tails, a
+    batch, and left padding."""
+    from tests import harness as Hn
+    cfg = get_config("tiny").with_(seq=seq, batch=batch, pad_max=pad, conv_width=2, conv_groups=5)
+    res = _run_prefill(cfg)
+    Hn.assert_block_ok(res)
+    for key in ("k_cache", "attention_queries", "conv_state"):
+        assert res[key]["rel_max"] <= Hn.TOL_REL_MAX, (key, res[key])
+
+
+def test_full_prefill_4k_two_stage_conv():
+    """Full width with the two-stage conv_qk (10 groups of 128 channels)."""
+    from tests import harness as Hn
+    res = _run_prefill(get_config("prefill_4k_conv2"))
+    Hn.assert_block_ok(res)
+    for key in ("k_cache", "attention_queries"):
+        assert res[key]["bf16_ok"], (key, res[key])
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill_4k_conv2"])
+def test_two_stage_conv_decode_after_prefill(name):
+    """prefill(S) then one decode step with the two-stage conv: the decode's
+    grouped conv takes u(t-2), u(t-1) from conv_state."""
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config(name)
+    if name == "tiny":
+        cfg = cfg.with_(conv_width=2, conv_groups=5)
+    S = 40
+    cfg = cfg.with_(seq=S, batch=2)
+    W = gen_block_weights(cfg)
+    Wd = Hn.dev_weights(W)
+    inp = gen_prefill_inputs(cfg.with_(seq=S + 1))
+    x, rin = inp["x"], inp["router_state_in"]
+    st = Hn.new_state(cfg, 2, S + 8)
+    Hn.gpu_prefill(cfg, Wd, x[:, :S], None, rin[:, :S], state=st)
+    host_state = {k: v.cpu().clone() for k, v in st.items()}
+    dec = Hn.gpu_decode(cfg, Wd, x[:, S], st, rin[:, S])
+    g_cls = Hn.gpu_classes(cfg, dec)
+    ref = Z.block_decode(cfg, Hn.eff(W), x[:, S], host_state, rin[:, S], force_cls=g_cls)
+    lo = Hn.report("layer_output", dec["layer_output"].numpy(), ref["layer_output"])
+    assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, lo
+    k_new = st["k_cache"][:, :, S].float().cpu().numpy()
+    assert Hn.rel_max(k_new, ref["state"]["k_cache"][:, :, S]) <= 2e-2

@@ -598,3 +598,66 @@ def test_hybrid_full_block_is_plain_causal():
     np.testing.assert_array_equal(o["layer_output"], ref["layer_output"])
     part = Z.block_prefill_rows(cfg, W, inp["x"][0], 40, 60, inp["router_state_in"][0], block_idx=2)
     np.testing.assert_allclose(part["layer_output"], o["layer_output"][0, 40:60], rtol=1e-9, atol=1e-9)
+
+
+# ---------------------------------------------------------------- two-stage conv_qk
+
+def test_conv_two_stage_worked_example():
+    """The printout's two causal convolutions (depthwise k=2, then grouped
+    k=2), hand-worked for one group of two channels, fresh and with a
+    conv_state history, and for two groups of one channel."""
+    ex = _load("worked_examples.json")["conv_two_stage"]
+    dw, db = np.array(ex["dw_taps_t-1_t"]), np.array(ex["db"])
+    gw = np.stack([np.array(ex["gw_tap_t-1"]), np.array(ex["gw_tap_t"])], axis=-1)   # [out, in, tap]
+    u = np.array(ex["u"])
+    y = Z.causal_conv_two_stage(u, dw, db, gw, np.array(ex["gb"]), np.zeros((2, 2)), 1)
+    np.testing.assert_allclose(y, ex["y_fresh"], atol=1e-12)
+    y = Z.causal_conv_two_stage(u, dw, db, gw, np.array(ex["gb"]), np.array(ex["hist"]), 1)
+    np.testing.assert_allclose(y, ex["y_with_state"], atol=1e-12)
+    g2 = ex["two_groups"]
+    y = Z.causal_conv_two_stage(u, dw, db, np.array(g2["gw"]), np.array(g2["gb"]), np.zeros((2, 2)), 2)
+    np.testing.assert_allclose(y, g2["y_fresh"], atol=1e-12)
+
+
+def test_conv_two_stage_reduces_to_the_depthwise_conv():
+    """With the grouped stage the identity on the current token (zero on the
+    previous one, no bias), the two-stage conv is the depthwise conv of
+    width 2: the width-3 conv with taps (0, dw0, dw1), itself pinned above."""
+    rng = np.random.default_rng(7)
+    T, C, G = 9, 12, 3
+    u, hist = rng.standard_normal((T, C)), rng.standard_normal((2, C))
+    dw, db = rng.standard_normal((C, 2)), rng.standard_normal(C)
+    gw = np.zeros((C, C // G, 2))
+    for o in range(C):
+        gw[o, o % (C // G), 1] = 1.0
+    y = Z.causal_conv_two_stage(u, dw, db, gw, np.zeros(C), hist, G)
+    ref = Z.causal_conv(u, np.concatenate([np.zeros((C, 1)), dw], axis=1), db, hist)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_conv_two_stage_block_reach_and_decode():
+    """A block with the two-stage conv keeps the width-3 reach (outputs at
+    i >= t+W+2 bit-identical after perturbing token t, the one at t+W+1
+    moved), and prefill(S) then decode equals prefill(S+1) at S."""
+    cfg = get_config("tiny").with_(seq=48, conv_width=2, conv_groups=5)
+    W = gen_block_weights(cfg)
+    inp = gen_prefill_inputs(cfg)
+    o = Z.block_prefill(cfg, W, inp["x"], None, inp["router_state_in"])
+    t = 4
+    x2 = inp["x"].clone()
+    x2[0, t] += 0.5
+    o2 = Z.block_prefill(cfg, W, x2, None, inp["router_state_in"])
+    edge = t + cfg.window + 1
+    np.testing.assert_array_equal(o2["attention_premix"][0, edge + 1:], o["attention_premix"][0, edge + 1:])
+    assert not np.array_equal(o2["attention_premix"][0, edge], o["attention_premix"][0, edge])
+    S = 30
+    pre = Z.block_prefill(cfg.with_(seq=S), W, inp["x"][:, :S], None, inp["router_state_in"][:, :S])
+    st = {k: v for k, v in pre["state"].items()}
+    st["k_cache"] = np.concatenate([st["k_cache"], np.zeros_like(st["k_cache"][:, :, :1])], axis=2)
+    st["v_cache"] = np.concatenate([st["v_cache"], np.zeros_like(st["v_cache"][:, :, :1])], axis=2)
+    dec = Z.block_decode(cfg, W, inp["x"][:, S], st, inp["router_state_in"][:, S],
+                         force_cls=o["expert_cls"][:, S])
+    full = Z.block_prefill(cfg.with_(seq=S + 1), W, inp["x"][:, :S + 1], None, inp["router_state_in"][:, :S + 1],
+                           force_cls=o["expert_cls"][:, :S + 1])
+    np.testing.assert_allclose(dec["layer_output"], full["layer_output"][:, S], rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(dec["attention_keys"], full["attention_keys"][:, :, S], rtol=1e-9, atol=1e-9)

@@ -176,10 +176,15 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
       const float a0 = pre.at(c, 0), a1 = pre.at(c, 1), a2 = pre.at(c, 2);
       u0[i] = a0;
       u1[i] = a1;
-      float acc = __ldg(p.conv_b + c);
-      acc = fmaf(__ldg(p.conv_w + 3 * c + 0), a2, acc);
-      acc = fmaf(__ldg(p.conv_w + 3 * c + 1), a1, acc);
-      acc = fmaf(__ldg(p.conv_w + 3 * c + 2), a0, acc);
+      float acc;
+      if (p.conv_y) {   // the two-stage conv, computed by the grouped-conv kernel
+        acc = p.conv_y[(size_t)tok * C + c];
+      } else {
+        acc = __ldg(p.conv_b + c);
+        acc = fmaf(__ldg(p.conv_w + 3 * c + 0), a2, acc);
+        acc = fmaf(__ldg(p.conv_w + 3 * c + 1), a1, acc);
+        acc = fmaf(__ldg(p.conv_w + 3 * c + 2), a0, acc);
+      }
       if (p.cca_res) {
         const float kpre = pre.at(nq * D + g * D + j, 0);
         if (is_q) {
@@ -330,15 +335,19 @@ __global__ void __launch_bounds__(512) cca_prefill_kernel(const CcaParams p) {
       load_bf<DPL>(ut + cbase, a0);
       load_bf<DPL>(u1 + cbase, a1);
       load_bf<DPL>(u2 + cbase, a2);
-      load_f<3 * DPL>(p.conv_w + 3 * cbase, w);
-      load_f<DPL>(p.conv_b + cbase, bias);
+      if (p.conv_y) {   // the two-stage conv, computed by the grouped-conv kernel
+        load_f<DPL>(p.conv_y + (row0 + s) * C + cbase, y);
+      } else {
+        load_f<3 * DPL>(p.conv_w + 3 * cbase, w);
+        load_f<DPL>(p.conv_b + cbase, bias);
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) {
-        float acc = bias[i];
-        acc = fmaf(w[3 * i + 0], a2[i], acc);
-        acc = fmaf(w[3 * i + 1], a1[i], acc);
-        acc = fmaf(w[3 * i + 2], a0[i], acc);
-        y[i] = acc;
+        for (int i = 0; i < DPL; ++i) {
+          float acc = bias[i];
+          acc = fmaf(w[3 * i + 0], a2[i], acc);
+          acc = fmaf(w[3 * i + 1], a1[i], acc);
+          acc = fmaf(w[3 * i + 2], a0[i], acc);
+          y[i] = acc;
+        }
       }
       if (p.cca_res) {
         float kpre[DPL];
@@ -497,10 +506,12 @@ __global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constan
   // of 768 threads per SM), loaded under the staging
   const int head = tid / LPH, l = tid % LPH;
   const int cb = head * D + l * 8;
-  for (int i = threadIdx.x; i < C / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(cbias)[i] = __ldg(reinterpret_cast<const float4*>(p.conv_b) + i);
-  for (int i = threadIdx.x; i < 3 * C / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(cw)[i] = __ldg(reinterpret_cast<const float4*>(p.conv_w) + i);
+  if (!p.conv_y) {
+    for (int i = threadIdx.x; i < C / 4; i += blockDim.x)
+      reinterpret_cast<float4*>(cbias)[i] = __ldg(reinterpret_cast<const float4*>(p.conv_b) + i);
+    for (int i = threadIdx.x; i < 3 * C / 4; i += blockDim.x)
+      reinterpret_cast<float4*>(cw)[i] = __ldg(reinterpret_cast<const float4*>(p.conv_w) + i);
+  }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
@@ -529,25 +540,32 @@ __global__ void __launch_bounds__(768, 1) cca_stream_kernel(const __grid_constan
       const int s = s0 + tt;
       if (s >= p.S) break;   // uniform over the head's lanes
       const __nv_bfloat16* row = u + (size_t)(tt + 2) * ld;
-      float x2[8], x1[8], x0[8], y[8], wv[24];
-      load8(row - 2 * ld + cb, x2);
+      float x1[8], x0[8], y[8];
       load8(row - ld + cb, x1);
       load8(row + cb, x0);
+      if (p.conv_y) {   // the two-stage conv, computed by the grouped-conv kernel
+        const float4* cy = reinterpret_cast<const float4*>(p.conv_y + (row0 + s) * C + cb);
+        const float4 y0 = cy[0], y1 = cy[1];
+        y[0] = y0.x; y[1] = y0.y; y[2] = y0.z; y[3] = y0.w; y[4] = y1.x; y[5] = y1.y; y[6] = y1.z; y[7] = y1.w;
+      } else {
+        float x2[8], wv[24];
+        load8(row - 2 * ld + cb, x2);
 #pragma unroll
-      for (int i = 0; i < 6; ++i) {
-        const float4 v = wq[i];
-        wv[4 * i] = v.x; wv[4 * i + 1] = v.y; wv[4 * i + 2] = v.z; wv[4 * i + 3] = v.w;
-      }
-      const float4 bb0 = reinterpret_cast<const float4*>(cbias + cb)[0];
-      const float4 bb1 = reinterpret_cast<const float4*>(cbias + cb)[1];
-      const float bb[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
+        for (int i = 0; i < 6; ++i) {
+          const float4 v = wq[i];
+          wv[4 * i] = v.x; wv[4 * i + 1] = v.y; wv[4 * i + 2] = v.z; wv[4 * i + 3] = v.w;
+        }
+        const float4 bb0 = reinterpret_cast<const float4*>(cbias + cb)[0];
+        const float4 bb1 = reinterpret_cast<const float4*>(cbias + cb)[1];
+        const float bb[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float acc = bb[i];
-        acc = fmaf(wv[3 * i], x2[i], acc);
-        acc = fmaf(wv[3 * i + 1], x1[i], acc);
-        acc = fmaf(wv[3 * i + 2], x0[i], acc);
-        y[i] = acc;
+        for (int i = 0; i < 8; ++i) {
+          float acc = bb[i];
+          acc = fmaf(wv[3 * i], x2[i], acc);
+          acc = fmaf(wv[3 * i + 1], x1[i], acc);
+          acc = fmaf(wv[3 * i + 2], x0[i], acc);
+          y[i] = acc;
+        }
       }
       if (p.cca_res) {
         if (is_q) {

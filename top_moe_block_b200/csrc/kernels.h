@@ -94,9 +94,26 @@ struct CcaParams {
   int* status;
   int* zero_words;        // prefill: words CTA 0 clears for the next kernel (attention's merge counters), or null
   int n_zero_words;
+  const float* conv_y;    // fp32 [rows, C]: the two-stage conv's output (used instead of the width-3 conv), or null
   float inv_freq[64];     // RoPE inverse frequencies theta^(-2i/rot), i < rot/2 (fp32)
 };
 int launch_cca(const CcaParams& p, cudaStream_t st);
+
+// The two-stage conv_qk's grouped stage (with its depthwise stage fused in):
+// y fp32 [rows, C], one group per q / k head.
+struct ConvGroupedParams {
+  const void* qkv;        // bf16 [rows, ld]: the pre-conv q||k projection in columns [0, C)
+  int ld;
+  const float* dw;        // [C, 2] depthwise taps (t-1, t)
+  const float* db;        // [C]
+  const float* gw;        // [C, D, 2] grouped taps (Conv1d layout [out, in / groups, k])
+  const float* gb;        // [C]
+  const int* mask;        // prefill [B, S] or null
+  const void* conv_state; // decode: bf16 [rows, C, 2] (u at t-2, t-1)
+  float* y;               // [rows, C]
+  int rows, S, C, decode;
+};
+int launch_conv_grouped(const ConvGroupedParams& p, int groups, int d, int num_sms, cudaStream_t st);
 
 // ------------------------------------------------------------------ attention
 struct AttnParams {

@@ -114,7 +114,9 @@ int check_config(const zaya_config* c) {
       c->router_hidden <= 0 || c->window <= 0 || c->rot_dim < 0)
     return ZAYA_ERR_INVALID_ARG;
   if (c->n_q % c->n_kv) return ZAYA_ERR_INVALID_ARG;
-  if (c->conv_width != 3) return ZAYA_ERR_UNSUPPORTED;
+  if (c->conv_groups < 0) return ZAYA_ERR_INVALID_ARG;
+  if (!((c->conv_width == 3 && c->conv_groups == 0) || (c->conv_width == 2 && c->conv_groups == c->n_q + c->n_kv)))
+    return ZAYA_ERR_UNSUPPORTED;
   if (c->hidden % 128 || c->hidden > 4096) return ZAYA_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return ZAYA_ERR_UNSUPPORTED;
   if (c->rot_dim > c->head_dim || c->rot_dim % 2 || (c->rot_dim / 2) % (c->head_dim / 32)) return ZAYA_ERR_UNSUPPORTED;
@@ -154,8 +156,9 @@ size_t attn_prefill_ws_any(const zaya_config& c, int B, int S, int nq, int nkv, 
 
 inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-int check_weights(const zaya_block_weights* w) {
+int check_weights(const zaya_block_weights* w, const zaya_config* c) {
   if (!w) return ZAYA_ERR_INVALID_ARG;
+  if (c->conv_groups > 0 && (!w->conv2_w || !w->conv2_b)) return ZAYA_ERR_INVALID_ARG;
   const void* ptrs[] = {w->ln1_w, w->ln2_w, w->w_qkv, w->conv_w, w->conv_b, w->k_temp, w->w_o, w->merge_a,
                         w->merge_m, w->router_down_w, w->router_down_b, w->router_state_scale, w->router_norm_w,
                         w->fc1_w, w->fc1_b, w->fc2_w, w->fc2_b, w->out_w, w->balancing, w->w_gate_up, w->w_down};
@@ -171,7 +174,7 @@ int check_weights(const zaya_block_weights* w) {
 
 struct Ws {
   size_t status, a_in, qkv, q, premix, m_in, logits, cls, w, pos, perm, group_off, mt_start, xperm, act, part, rpart,
-      wsplit, slot, ccount, total;
+      wsplit, slot, ccount, convy, total;
 };
 
 Ws plan(const zaya_config& c, int mode, int B, int S) {
@@ -201,6 +204,7 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.wsplit = o; o += up(((size_t)4 * d.R * d.R + (size_t)2 * ((d.E + 1 + 7) / 8 * 8) * d.R) * 2);   // fc1, fc2, out_proj hi / lo
   w.slot = o; o += up(M * 4);
   w.ccount = o; o += up((size_t)(d.E + 2) * 4);
+  w.convy = o; o += c.conv_groups > 0 ? up(M * d.C * 4) : 0;   // the two-stage conv's output (fp32)
   w.total = o;
   return w;
 }
@@ -342,7 +346,7 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
                        float* hidden, const int32_t* mask, const float* rin, float* rout, const zaya_block_state* state,
                        const zaya_taps* taps, void* ws, size_t ws_bytes, cudaStream_t st) {
   ZAYA_TRY(check_config(cfg));
-  ZAYA_TRY(check_weights(w));
+  ZAYA_TRY(check_weights(w, cfg));
   if (B <= 0 || S <= 0 || !hidden || !rout || !ws) return ZAYA_ERR_INVALID_ARG;
   if (block_idx < 0 || (block_idx > 0 && !rin) || rin == rout) return ZAYA_ERR_INVALID_ARG;
   ZAYA_TRY(check_state(state, S));
@@ -370,8 +374,15 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     if (!bn) return ZAYA_ERR_UNSUPPORTED;
     ZAYA_STAGE("qkv_gemm", 1, launch_gemm(EPI_STORE_BF16, bn, a_in, M, w->w_qkv, d.n_qkv, p, sms, st));
   }
+  if (c.conv_groups > 0) {
+    ConvGroupedParams p{};
+    p.qkv = qkv; p.ld = d.n_qkv; p.dw = w->conv_w; p.db = w->conv_b; p.gw = w->conv2_w; p.gb = w->conv2_b;
+    p.mask = mask; p.y = at<float>(ws, L.convy); p.rows = M; p.S = S; p.C = d.C; p.decode = 0;
+    ZAYA_STAGE("conv_grouped", 1, launch_conv_grouped(p, c.conv_groups, d.d, sms, st));
+  }
   {
     CcaParams p{};
+    p.conv_y = c.conv_groups > 0 ? at<float>(ws, L.convy) : nullptr;
     p.qkv = qkv; p.n_qkv = d.n_qkv; p.conv_w = w->conv_w; p.conv_b = w->conv_b; p.k_temp = w->k_temp;
     p.mask = mask; p.q_out = at<void>(ws, L.q); p.tap_q = taps ? taps->attention_queries : nullptr;
     p.k_cache = state->k_cache; p.v_cache = state->v_cache; p.cache_cap = state->cache_cap;
@@ -405,7 +416,7 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
 int check_decode_args(const zaya_config* cfg, const zaya_block_weights* w, int block_idx, int B, const float* hidden,
                       const float* rin, const float* rout, const zaya_block_state* state, const zaya_taps* taps) {
   ZAYA_TRY(check_config(cfg));
-  ZAYA_TRY(check_weights(w));
+  ZAYA_TRY(check_weights(w, cfg));
   if (B <= 0 || !hidden || !rout) return ZAYA_ERR_INVALID_ARG;
   if (block_idx < 0 || (block_idx > 0 && !rin) || rin == rout) return ZAYA_ERR_INVALID_ARG;
   ZAYA_TRY(check_state(state, 1));
@@ -441,8 +452,15 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
     if (!bn) return ZAYA_ERR_UNSUPPORTED;
     ZAYA_STAGE("qkv_gemm", 1, launch_gemm(EPI_STORE_BF16, bn, a_in, 2 * B, w->w_qkv, d.n_qkv, p, sms, st));
   }
+  if (c.conv_groups > 0) {
+    ConvGroupedParams p{};
+    p.qkv = qkv; p.ld = d.n_qkv; p.dw = w->conv_w; p.db = w->conv_b; p.gw = w->conv2_w; p.gb = w->conv2_b;
+    p.conv_state = state->conv_state; p.y = at<float>(ws, L.convy); p.rows = B; p.S = 1; p.C = d.C; p.decode = 1;
+    ZAYA_STAGE("conv_grouped", 1, launch_conv_grouped(p, c.conv_groups, d.d, sms, st));
+  }
   {
     CcaParams p{};
+    p.conv_y = c.conv_groups > 0 ? at<float>(ws, L.convy) : nullptr;
     p.qkv = qkv; p.n_qkv = d.n_qkv; p.conv_w = w->conv_w; p.conv_b = w->conv_b; p.k_temp = w->k_temp;
     p.mask = nullptr; p.q_out = at<void>(ws, L.q); p.tap_q = taps ? taps->attention_queries : nullptr;
     p.k_cache = state->k_cache; p.v_cache = state->v_cache; p.cache_cap = state->cache_cap;
