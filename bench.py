@@ -93,6 +93,9 @@ def stage_work(cfg, routed_tokens, pairs):
         "dispatch": ("hbm", routed_tokens * H * 2 * 2 + (M - routed_tokens) * H * 8, "B"),
         "experts_gate_up": ("tensor", 2.0 * routed_tokens * H * 2 * I, "FLOP"),
         "experts_down_merge": ("tensor", 2.0 * routed_tokens * I * H, "FLOP"),
+        # the two-stage conv_qk's grouped stage (TF32 tensor cores): C outputs x 2 taps x C/G inputs
+        **({"conv_grouped": ("tensor", 2.0 * M * cfg.qk_channels * 2 * (cfg.qk_channels // cfg.conv_groups),
+                             "FLOP")} if cfg.conv_groups else {}),
     }
 
 
