@@ -159,6 +159,7 @@ inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) ==
 int check_weights(const zaya_block_weights* w, const zaya_config* c) {
   if (!w) return ZAYA_ERR_INVALID_ARG;
   if (c->conv_groups > 0 && (!w->conv2_w || !w->conv2_b)) return ZAYA_ERR_INVALID_ARG;
+  if (c->conv_groups > 0 && (!a16(w->conv2_w) || !a16(w->conv2_b))) return ZAYA_ERR_MISALIGNED;
   const void* ptrs[] = {w->ln1_w, w->ln2_w, w->w_qkv, w->conv_w, w->conv_b, w->k_temp, w->w_o, w->merge_a,
                         w->merge_m, w->router_down_w, w->router_down_b, w->router_state_scale, w->router_norm_w,
                         w->fc1_w, w->fc1_b, w->fc2_w, w->fc2_b, w->out_w, w->balancing, w->w_gate_up, w->w_down};
