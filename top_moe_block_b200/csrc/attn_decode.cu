@@ -4,12 +4,16 @@
 // byte is read once (nnterp "zaya" page: grouped-query eager attention).
 //
 // HBM-bound (the window's K and V: 2 x d x 2 bytes per key and kv head).
-// Split-KV: CTA (chunk, kv head, sequence) covers 256 keys, 4 warps of 64.
-// Each lane owns d/32 dims: it streams 8-byte slices of the keys (a warp
-// reads whole 256-byte rows, coalesced), forms rep partial dot products per
-// key, and a butterfly reduce-scatter over the warp leaves one complete
-// (key, head) score per lane.  Online softmax per head, P.V accumulated on
-// the lane's own dims.  A second kernel merges the chunks.
+// Split-KV: CTA (chunk, kv head, sequence) covers chunk_keys keys, 4 warps of
+// a quarter each.  A warp streams its keys in 16-key slices (K and V rows by
+// cp.async into a two-slot ring, 16-byte chunks XOR-swizzled by key so the
+// ldmatrix reads are free of bank conflicts) and runs both products on the
+// tensor cores with mma.sync m16n8k16 (bf16 in, fp32 accumulate): the rep
+// query heads are the rows of A (padded to 16), S = Q K^T in fp32, online
+// softmax per row on the accumulator fragments, P rounded to bf16 becomes the
+// A operand of P V straight from registers, V read with ldmatrix.trans.  The
+// four warps' (max, sum, O) are merged in shared memory into the chunk's
+// partial; a second kernel merges the chunks.
 #include <math.h>
 
 #include "common.cuh"
@@ -22,14 +26,22 @@ namespace {
 constexpr int kChunk = 256;   // keys per CTA up to kMaxChunks chunks (longer spans: longer chunks)
 constexpr int kWarps = 4;
 constexpr int kMaxChunks = 64; // a head's partials in the workspace
+constexpr int kSub = 16;       // keys per slice (one k16 step of P V)
+
+template <int D>
+constexpr size_t decode_smem_bytes() { return (size_t)kWarps * 2 * 2 * kSub * D * 2; }
 
 template <int D, int REP>
 __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams p) {
-  constexpr int DPL = D / 32;
-  constexpr int KPG = 32 / REP;  // keys per group: KPG * REP == 32 scores per warp step
+  constexpr int NK = D / 16;   // k16 steps of Q K^T
+  constexpr int ND = D / 8;    // 8-dim n-tiles of P V
+  constexpr int CPR = D / 8;   // 16-byte chunks per K / V row
+  static_assert(REP <= 8, "query heads per kv head fill the upper half of A at most");
   griddep_begin();
+  extern __shared__ __align__(128) uint8_t dsm[];
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
+  const int gid = lane >> 2, tig = lane & 3;
   // A position outside the cache (already reported by the conv kernel) gives
   // an empty key range, so nothing outside the cache is read.
   const int t_raw = p.cache_len[b];
@@ -37,115 +49,136 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
   const int lo = max(0, t - p.window + 1);
   const int c_begin = lo + chunk * p.chunk_keys;
   const int c_end = min(t + 1, c_begin + p.chunk_keys);
-  const int w_begin = c_begin + warp * (p.chunk_keys / kWarps);
-  const int w_end = min(c_end, w_begin + p.chunk_keys / kWarps);
-
+  const int per_warp = p.chunk_keys / kWarps;
+  const int w_begin = c_begin + warp * per_warp;
+  const int w_end = min(c_end, w_begin + per_warp);
   const float sl2 = p.scale * 1.4426950408889634f;
-  float q[REP][DPL];
-  const auto* qg = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.n_q + g * REP) * D + lane * DPL;
-#pragma unroll
-  for (int hh = 0; hh < REP; ++hh)
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) q[hh][i] = bf2f(qg[hh * D + i]) * sl2;
 
-  const auto* Kg = static_cast<const __nv_bfloat16*>(p.k_cache) + ((size_t)b * p.n_kv + g) * p.cap * D + lane * DPL;
-  const auto* Vg = static_cast<const __nv_bfloat16*>(p.v_cache) + ((size_t)b * p.n_kv + g) * p.cap * D + lane * DPL;
+  // Q fragments: row gid of A is query head g * REP + gid (zero from REP on)
+  uint32_t qa[NK][2];
+  {
+    const auto* qrow = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.n_q + g * REP + gid) * D;
+#pragma unroll
+    for (int kk = 0; kk < NK; ++kk) {
+      qa[kk][0] = gid < REP ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * tig) : 0u;
+      qa[kk][1] = gid < REP ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * tig) : 0u;
+    }
+  }
+  const auto* Kg = static_cast<const __nv_bfloat16*>(p.k_cache) + ((size_t)b * p.n_kv + g) * p.cap * D;
+  const auto* Vg = static_cast<const __nv_bfloat16*>(p.v_cache) + ((size_t)b * p.n_kv + g) * p.cap * D;
+  __nv_bfloat16* sw = reinterpret_cast<__nv_bfloat16*>(dsm) + (size_t)warp * 2 * 2 * kSub * D;   // [slot][K|V][16][D]
+  // K and V rows key0 .. key0+15 into ring slot `slot`; keys past the warp's
+  // range are zero-filled (no global read)
+  auto load_slice = [&](int slot, int key0) {
+    __nv_bfloat16* dk = sw + (size_t)slot * 2 * kSub * D;
+    __nv_bfloat16* dv = dk + kSub * D;
+#pragma unroll
+    for (int i = lane; i < kSub * CPR; i += 32) {
+      const int r = i / CPR, c = i % CPR;
+      const int key = key0 + r;
+      const bool ok = key < w_end;
+      const size_t src = (size_t)(ok ? key : 0) * D + c * 8;
+      const int dst = r * D + ((c ^ (r & 7)) * 8);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dk + dst)), "l"(Kg + src),
+                   "r"(ok ? 16 : 0)
+                   : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dv + dst)), "l"(Vg + src),
+                   "r"(ok ? 16 : 0)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
 
-  float o[REP][DPL];
+  float m_run = -INFINITY, l_run = 0.f;   // row gid
+  float o[ND][4];
 #pragma unroll
-  for (int hh = 0; hh < REP; ++hh)
+  for (int j = 0; j < ND; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  const int n_sub = w_end > w_begin ? (w_end - w_begin + kSub - 1) / kSub : 0;
+  if (n_sub > 0) load_slice(0, w_begin);
+  const int mi = lane >> 3, rr = lane & 7;
+  for (int si = 0; si < n_sub; ++si) {
+    const int slot = si & 1;
+    if (si + 1 < n_sub) {
+      load_slice(slot ^ 1, w_begin + (si + 1) * kSub);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncwarp();
+    const __nv_bfloat16* sK = sw + (size_t)slot * 2 * kSub * D;
+    const __nv_bfloat16* sV = sK + kSub * D;
+    // S = Q K^T over the slice's 16 keys (two 8-key n-tiles)
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      const int key_r = (mi >> 1) * 8 + rr;   // matrices: keys 0-7 / 8-15 x dims lo / hi of the k16 step
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) o[hh][i] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;  // for head (lane % REP)
-
-  for (int base = w_begin; base < w_end; base += KPG) {
-    float kf[KPG][DPL], vf[KPG][DPL];
-#pragma unroll
-    for (int kk = 0; kk < KPG; ++kk) {
-      const int key = base + kk;
-      if (key < w_end) {
-        if constexpr (DPL == 4) {
-          const uint2 ku = *reinterpret_cast<const uint2*>(Kg + (size_t)key * D);
-          const uint2 vu = *reinterpret_cast<const uint2*>(Vg + (size_t)key * D);
-          const float2 k01 = unpack_bf2(ku.x), k23 = unpack_bf2(ku.y);
-          const float2 v01 = unpack_bf2(vu.x), v23 = unpack_bf2(vu.y);
-          kf[kk][0] = k01.x; kf[kk][1] = k01.y; kf[kk][2] = k23.x; kf[kk][3] = k23.y;
-          vf[kk][0] = v01.x; vf[kk][1] = v01.y; vf[kk][2] = v23.x; vf[kk][3] = v23.y;
-        } else {
-          const uint32_t ku = *reinterpret_cast<const uint32_t*>(Kg + (size_t)key * D);
-          const uint32_t vu = *reinterpret_cast<const uint32_t*>(Vg + (size_t)key * D);
-          const float2 k01 = unpack_bf2(ku), v01 = unpack_bf2(vu);
-          kf[kk][0] = k01.x; kf[kk][1] = k01.y;
-          vf[kk][0] = v01.x; vf[kk][1] = v01.y;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) kf[kk][i] = vf[kk][i] = 0.f;
+      for (int kk = 0; kk < NK; ++kk) {
+        const int ch = 2 * kk + (mi & 1);
+        uint32_t b00, b01, b10, b11;
+        ldsm_x4(smem_u32(sK + key_r * D + ((ch ^ (key_r & 7)) * 8)), b00, b01, b10, b11);
+        const uint32_t a[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
+        mma16816(s[0], a, b00, b01);
+        mma16816(s[1], a, b10, b11);
       }
     }
-    // partial scores, value index = kk * REP + hh
-    float v[32];
+    // online softmax on row gid: keys 2tig, 2tig+1 (tile 0) and 8+2tig, 9+2tig (tile 1)
+    const int key0 = w_begin + si * kSub;
+    float v[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};
+    const int kid[4] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig};
 #pragma unroll
-    for (int kk = 0; kk < KPG; ++kk)
+    for (int i = 0; i < 4; ++i) v[i] = (key0 + kid[i] < w_end) ? v[i] * sl2 : -INFINITY;
+    float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float base = (m_new == -INFINITY) ? 0.f : m_new;
+    const float corr = exp2f(m_run - base);
+    float pv[4], ps = 0.f;
 #pragma unroll
-      for (int hh = 0; hh < REP; ++hh) {
-        float a = 0.f;
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) a = fmaf(q[hh][i], kf[kk][i], a);
-        v[kk * REP + hh] = a;
-      }
-    // butterfly reduce-scatter: lane l ends with the full sum of value l
-#pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) {
-      const bool upper = (lane & s) != 0;
-#pragma unroll
-      for (int i = 0; i < s; ++i) {
-        const float send = upper ? v[i] : v[i + s];
-        const float keep = upper ? v[i + s] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-      }
+    for (int i = 0; i < 4; ++i) {
+      pv[i] = exp2f(v[i] - base);
+      ps += pv[i];
     }
-    const int my_key = base + lane / REP;
-    float sc = (my_key < w_end) ? v[0] : -INFINITY;
-    float gm = sc;
-#pragma unroll
-    for (int s = REP; s < 32; s <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, s));
-    const float m_new = fmaxf(m_run, gm);
-    const float bse = (m_new == -INFINITY) ? 0.f : m_new;
-    const float pk = exp2f(sc - bse);
-    float ps = pk;
-#pragma unroll
-    for (int s = REP; s < 32; s <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, s);
-    const float corr = exp2f(m_run - bse);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
     l_run = l_run * corr + ps;
     m_run = m_new;
 #pragma unroll
-    for (int hh = 0; hh < REP; ++hh) {
-      const float ch = __shfl_sync(0xffffffffu, corr, hh);
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) o[hh][i] *= ch;
+    for (int j = 0; j < ND; ++j) {
+      o[j][0] *= corr;
+      o[j][1] *= corr;
     }
+    // O += P V: P (bf16) is the A operand, V read transposed
+    const uint32_t pa[4] = {pack_bf2(pv[0], pv[1]), 0u, pack_bf2(pv[2], pv[3]), 0u};
+    {
+      const int key_r = (mi & 1) * 8 + rr;   // matrices: keys 0-7 / 8-15 x dims of n-tiles j / j+1
 #pragma unroll
-    for (int kk = 0; kk < KPG; ++kk)
-#pragma unroll
-      for (int hh = 0; hh < REP; ++hh) {
-        const float pv = __shfl_sync(0xffffffffu, pk, kk * REP + hh);
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) o[hh][i] = fmaf(pv, vf[kk][i], o[hh][i]);
+      for (int j = 0; j < ND; j += 2) {
+        const int ch = j + (mi >> 1);
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_t(smem_u32(sV + key_r * D + ((ch ^ (key_r & 7)) * 8)), r0, r1, r2, r3);
+        mma16816(o[j], pa, r0, r1);
+        mma16816(o[j + 1], pa, r2, r3);
       }
+    }
+    __syncwarp();   // the slot is read before the next iteration refills it
   }
 
-  // merge the 4 warps of this CTA, then write the chunk's partial result
-  __shared__ float sm_m[kWarps][REP], sm_l[kWarps][REP];
-  __shared__ float sm_o[kWarps][REP][D];
-  if (lane < REP) {
-    sm_m[warp][lane] = m_run;
-    sm_l[warp][lane] = l_run;
+  // merge the 4 warps of this CTA (the K / V ring is free now), then write the
+  // chunk's partial result
+  __syncthreads();
+  float* sm_o = reinterpret_cast<float*>(dsm);                 // [kWarps][REP][D]
+  float* sm_m = sm_o + kWarps * REP * D;                        // [kWarps][REP]
+  float* sm_l = sm_m + kWarps * REP;
+  if (gid < REP) {
+    if (tig == 0) {
+      sm_m[warp * REP + gid] = m_run;
+      sm_l[warp * REP + gid] = l_run;
+    }
+#pragma unroll
+    for (int j = 0; j < ND; ++j)
+      *reinterpret_cast<float2*>(sm_o + (warp * REP + gid) * D + 8 * j + 2 * tig) = make_float2(o[j][0], o[j][1]);
   }
-#pragma unroll
-  for (int hh = 0; hh < REP; ++hh)
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) sm_o[warp][hh][lane * DPL + i] = o[hh][i];
   __syncthreads();
   const size_t part_idx = (((size_t)b * p.n_kv + g) * p.n_chunks + chunk) * REP;
   float* pm = p.part;                                           // [.., REP] max
@@ -155,14 +188,14 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
     const int hh = idx / D, dd = idx % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w][hh]);
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w * REP + hh]);
     const float bse = (M == -INFINITY) ? 0.f : M;
     float L = 0.f, O = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-      const float f = exp2f(sm_m[w][hh] - bse);
-      L += sm_l[w][hh] * f;
-      O += sm_o[w][hh][dd] * f;
+      const float f = exp2f(sm_m[w * REP + hh] - bse);
+      L += sm_l[w * REP + hh] * f;
+      O += sm_o[(w * REP + hh) * D + dd] * f;
     }
     po[(part_idx + hh) * D + dd] = O;
     if (dd == 0) {
@@ -223,11 +256,18 @@ int launch_attn_decode(const DecodeAttnParams& p, cudaStream_t st) {
   if (p.n_chunks < 1 || p.n_chunks > kMaxChunks || p.chunk_keys % kChunk) return ZAYA_ERR_UNSUPPORTED;
   const int rep = p.n_q / p.n_kv;
   const dim3 grid(p.n_chunks, p.n_kv, p.B);
-#define ZAYA_DEC(DV, RV)                                                   \
-  if (p.d == DV && rep == RV) {                                            \
-    launch_k(attn_decode_kernel<DV, RV>, grid, dim3(32 * kWarps), 0, st, nullptr, 0, p);          \
-    launch_k(attn_decode_combine<DV>, dim3(p.B * p.n_q), dim3(DV), 0, st, nullptr, 0, p, RV);   \
-    return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;    \
+#define ZAYA_DEC(DV, RV)                                                                               \
+  if (p.d == DV && rep == RV) {                                                                        \
+    static bool set = false;                                                                           \
+    if (!set) {                                                                                        \
+      if (cudaFuncSetAttribute(attn_decode_kernel<DV, RV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                               (int)decode_smem_bytes<DV>()) != cudaSuccess)                          \
+        return ZAYA_ERR_CUDA;                                                                          \
+      set = true;                                                                                      \
+    }                                                                                                  \
+    launch_k(attn_decode_kernel<DV, RV>, grid, dim3(32 * kWarps), decode_smem_bytes<DV>(), st, nullptr, 0, p); \
+    launch_k(attn_decode_combine<DV>, dim3(p.B * p.n_q), dim3(DV), 0, st, nullptr, 0, p, RV);         \
+    return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;                                \
   }
   ZAYA_DEC(128, 4)
   ZAYA_DEC(64, 4)
