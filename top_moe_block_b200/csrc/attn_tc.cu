@@ -386,18 +386,22 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
       for (int c = 0; c < kKT / 32; ++c)
         tmem_ld32(tl + buf * kKT + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
       tmem_ld_wait();
-      // raw scores (masked keys -inf); the scale sl2 > 0 is applied with the
-      // exponent's subtraction in one fma
       float* v = reinterpret_cast<float*>(r);
-      if (!full_vis) {
+      if (full_vis) {
 #pragma unroll
-        for (int i = 0; i < kKT; ++i)
-          if (!key_visible(q, key0 + i, p.window, S, mask)) v[i] = -INFINITY;
+        for (int i = 0; i < kKT; ++i) v[i] = __uint_as_float(r[i]) * sl2;
+      } else {
+#pragma unroll
+        for (int i = 0; i < kKT; ++i) {
+          const float xv = __uint_as_float(r[i]) * sl2;
+          v[i] = key_visible(q, key0 + i, p.window, S, mask) ? xv : -INFINITY;
+        }
       }
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
       for (int i = 0; i < kKT; ++i) mx[i & 3] = fmaxf(mx[i & 3], v[i]);
-      const float m_new = fmaxf(m_used, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
+      const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float m_new = fmaxf(m_used, tmax);
       // Move the running max when it grew by more than 2^8 -- for the whole warp
       // at once, since the O rescale below is a warp-wide TMEM access.  Each
       // lane scales its own row by exp2(m_used - m_new) <= 1, so the result is
@@ -428,16 +432,15 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
         l *= f;
         if (finite_new) m_used = m_new;
       }
-      const float nbase = (m_used == -INFINITY) ? 0.f : -m_used;
+      const float base = (m_used == -INFINITY) ? 0.f : m_used;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
-      // P = 2^(v * sl2 - m_used) as bf16 pairs, written over the first kKT/2 columns of S(j)
+      // P = 2^(v - base) as bf16 pairs, written over the first kKT/2 columns of S(j)
 #pragma unroll
       for (int c = 0; c < kKT / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2_approx(fmaf(v[c * 32 + i], sl2, nbase));
-          const float p1 = ex2_approx(fmaf(v[c * 32 + i + 1], sl2, nbase));
+          const float p0 = ex2_approx(v[c * 32 + i] - base), p1 = ex2_approx(v[c * 32 + i + 1] - base);
           ls[(i >> 1) & 3] += p0 + p1;
           pk[i >> 1] = pack_bf2(p0, p1);
         }

@@ -311,7 +311,6 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
   uint64_t* mdrain = tempty + 2;   // the MMA thread's last commit: all its MMAs are done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdrain + 1);
   int* s_skip = reinterpret_cast<int*>(tmem_slot + 1);   // CTA pair: rank 0's reading of the status word
-  int* s_last = s_skip + 1;                               // split-K: this CTA finishes the tile
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -478,11 +477,6 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     const int row_off = (int)rank * BM;  // this CTA's first row inside the tile
     int local = 0;
     bool aborted = false;   // a wait ran out: keep walking the tiles (barrier partners) without waiting
-    // split-K with the epilogue in the last split (dense STORE_BF16 / MERGE_ATTN, one CTA per tile)
-    const bool fixup = CG == 1 && EPI != EPI_STORE_F32 && EPI != EPI_SWIGLU && EPI != EPI_MERGE_MLP &&
-                       p.k_splits > 1;
-    const int ksn = p.k_splits > 1 ? p.k_splits : 1;
-    const int mtn = (p.M + TM - 1) / TM;
     for (int t = unit; t < ntiles; t += n_units, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
@@ -506,74 +500,11 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
       }
       // warp-uniform: the TMEM loads below are .sync.aligned
       if (!aborted && !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, wc))) aborted = true;
+      if (aborted) continue;
+      tc_fence_after();
       const int row = ti.m0 + row_off + q * 32 + lane;
       const bool valid = row < ti.m_end;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-      if constexpr (CG == 1 && (EPI == EPI_STORE_BF16 || EPI == EPI_MERGE_ATTN)) {
-        if (fixup) {
-          // this split's fp32 partial of the thread's row into its slab, then the
-          // accumulator goes back to the MMA thread
-          if (!aborted) {
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = part * 32; c < BN_OUT; c += 32 * (EW / 4)) {
-              uint32_t r[32];
-              tmem_ld32(tbase + c, r);
-              tmem_ld_wait();
-              if (valid) {
-                float4* dst = reinterpret_cast<float4*>(p.slab + ((size_t)ti.split * p.M + row) * p.N + ti.n0 + c);
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                  dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                       __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-              }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
-          }
-          // the last split of this (m, n) tile to arrive sums the slabs in split
-          // order (the same result whichever arrives last) and runs the epilogue;
-          // every epilogue warp reaches both barriers on every path
-          __threadfence();
-          named_barrier_sync(2, EW * 32);
-          const int tid = (t % mtn) + mtn * ((t / mtn) / ksn);
-          if (et == 0) *s_last = atomicAdd(p.tile_ctr + tid, 1) == ksn - 1;
-          named_barrier_sync(2, EW * 32);
-          if (*s_last) {
-            __threadfence();
-#pragma unroll 1
-            for (int c = part * 32; c < BN_OUT; c += 32 * (EW / 4)) {
-              float sum[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) sum[j] = 0.f;
-              if (valid) {
-                for (int sp = 0; sp < ksn; ++sp) {
-                  const float4* src =
-                      reinterpret_cast<const float4*>(p.slab + ((size_t)sp * p.M + row) * p.N + ti.n0 + c);
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) {
-                    const float4 v = __ldcg(src + j);
-                    sum[4 * j] += v.x; sum[4 * j + 1] += v.y; sum[4 * j + 2] += v.z; sum[4 * j + 3] += v.w;
-                  }
-                }
-              }
-              uint32_t r[32], r2[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sum[j]);
-              if constexpr (is_merge<EPI>())
-                merge_chunk<EPI>(p, ti.m0 + row_off + q * 32, ti.m_end, ti.n0 + c, r, sT + (warp - 2) * 1024,
-                                 prm + c, BN_OUT);
-              else if (valid)
-                epilogue32<EPI>(p, row, ti.n0 + c, 0, r, r2, prm + c, BN_OUT);
-            }
-            if (et == 0) p.tile_ctr[tid] = 0;   // left zero for the next launch
-          }
-          continue;
-        }
-      }
-      if (aborted) continue;
-      tc_fence_after();
 #pragma unroll 1
       for (int c = part * 32; c < BN_OUT; c += 32 * (EW / 4)) {
         uint32_t r[32], r2[32];
@@ -690,10 +621,7 @@ int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b
                 int num_sms, cudaStream_t st) {
   if (p.K % BK != 0 || p.K <= 0) return ZAYA_ERR_UNSUPPORTED;
   const int ks = p.k_splits > 1 ? p.k_splits : 1;
-  if ((p.K / BK) % ks != 0) return ZAYA_ERR_UNSUPPORTED;
-  if (ks > 1 && (p.grouped || p.pair ||
-                 (epi != EPI_STORE_F32 && !((epi == EPI_STORE_BF16 || epi == EPI_MERGE_ATTN) && p.slab && p.tile_ctr))))
-    return ZAYA_ERR_UNSUPPORTED;
+  if ((p.K / BK) % ks != 0 || (ks > 1 && (p.grouped || epi != EPI_STORE_F32))) return ZAYA_ERR_UNSUPPORTED;
   const int bn_out = (epi == EPI_SWIGLU) ? bn / 2 : bn;
   if (p.N % bn_out != 0) return ZAYA_ERR_UNSUPPORTED;
   if (a_rows <= 0) return ZAYA_OK;

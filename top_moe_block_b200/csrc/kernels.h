@@ -40,12 +40,6 @@ struct GemmParams {
   const float* row_w;        // MERGE_MLP: per-token expert weight
   void* tap_bf16;            // MERGE_*: optional bf16 [tokens, N] contribution tap
   float* tap_f32;            // MERGE_ATTN: optional fp32 [tokens, N] layer_mid tap
-  // Split-K for the other dense epilogues (decode-sized M): each of k_splits
-  // slabs writes its fp32 partial to slab [k_splits, M, N]; the last split of
-  // a tile to finish (tile_ctr, one counter per (m, n) tile, zero at launch
-  // and left zero) sums the slabs in split order and runs the epilogue.
-  float* slab;
-  int* tile_ctr;
 };
 
 // Encodes a 2-D bf16 tensor map (rows x cols, row-major) with a box of
@@ -72,8 +66,7 @@ inline int router_down_splits(int M, int K) {
 // row_add]); extra rows [M, M+n_copy) of out are a copy of copy_src (decode:
 // prev_hs, whose projection gives the delayed values).
 int launch_rmsnorm(const float* x, int row_mul, int row_add, const void* w, void* out, void* tap, int M, int H,
-                   float eps, const void* copy_src, int n_copy, cudaStream_t st, int* zero_words = nullptr,
-                   int n_zero = 0);
+                   float eps, const void* copy_src, int n_copy, cudaStream_t st);
 int launch_embed(const int* ids, const void* table, float* stream, int M, int H, int vocab, float mult,
                  float shift, int* status, cudaStream_t st);
 

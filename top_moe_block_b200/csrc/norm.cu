@@ -28,14 +28,11 @@ __global__ void __launch_bounds__(256, 4) rmsnorm_kernel(const float* __restrict
                                                          const __nv_bfloat16* __restrict__ w,
                                                          __nv_bfloat16* __restrict__ out,
                                                          __nv_bfloat16* __restrict__ tap, int M, float eps,
-                                                         const __nv_bfloat16* __restrict__ copy_src, int n_copy,
-                                                         int* __restrict__ zero_words, int n_zero) {
+                                                         const __nv_bfloat16* __restrict__ copy_src, int n_copy) {
   constexpr int H = CHUNKS * 128;
   constexpr int G = CHUNKS < 8 ? CHUNKS : 8;   // float4 loads in flight per group
   __shared__ __align__(16) __nv_bfloat16 ws[H];   // the norm weight, staged once per CTA
   griddep_begin();
-  if (zero_words && blockIdx.x == 0)   // counters a later kernel of the block needs at zero
-    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
   const int row = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   for (int i = threadIdx.x; i < H / 8; i += blockDim.x)
@@ -97,13 +94,10 @@ __global__ void __launch_bounds__(128) rmsnorm_row_kernel(const float* __restric
                                                           const __nv_bfloat16* __restrict__ w,
                                                           __nv_bfloat16* __restrict__ out,
                                                           __nv_bfloat16* __restrict__ tap, int M, float eps,
-                                                          const __nv_bfloat16* __restrict__ copy_src, int n_copy,
-                                                          int* __restrict__ zero_words, int n_zero) {
+                                                          const __nv_bfloat16* __restrict__ copy_src, int n_copy) {
   constexpr int H = 512 * V;
   __shared__ float red[4];
   griddep_begin();
-  if (zero_words && blockIdx.x == 0)   // counters a later kernel of the block needs at zero
-    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0;
   const int row = blockIdx.x, t = threadIdx.x;
   if (row >= M) {  // verbatim copy rows (decode: prev_hs feeds the delayed values)
     const uint2* src = reinterpret_cast<const uint2*>(copy_src + (size_t)(row - M) * H);
@@ -170,7 +164,7 @@ __global__ void __launch_bounds__(256) embed_kernel(const int* __restrict__ ids,
 }  // namespace
 
 int launch_rmsnorm(const float* x, int row_mul, int row_add, const void* w, void* out, void* tap, int M, int H,
-                   float eps, const void* copy_src, int n_copy, cudaStream_t st, int* zero_words, int n_zero) {
+                   float eps, const void* copy_src, int n_copy, cudaStream_t st) {
   const int rows = M + n_copy;
   if (rows <= 0) return ZAYA_OK;
   const auto* wb = static_cast<const __nv_bfloat16*>(w);
@@ -180,19 +174,19 @@ int launch_rmsnorm(const float* x, int row_mul, int row_add, const void* w, void
   const int v = H % 512 ? 0 : H / 512;   // one CTA per row when H is a multiple of 512
   if (v == 1 || v == 2 || v == 4 || v == 8) {
     cudaError_t e;
-    if (v == 1) e = launch_k_as(0, rmsnorm_row_kernel<1>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero);
-    else if (v == 2) e = launch_k_as(0, rmsnorm_row_kernel<2>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero);
-    else if (v == 4) e = launch_k_as(0, rmsnorm_row_kernel<4>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero);
-    else e = launch_k_as(0, rmsnorm_row_kernel<8>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero);
+    if (v == 1) e = launch_k_as(0, rmsnorm_row_kernel<1>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
+    else if (v == 2) e = launch_k_as(0, rmsnorm_row_kernel<2>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
+    else if (v == 4) e = launch_k_as(0, rmsnorm_row_kernel<4>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
+    else e = launch_k_as(0, rmsnorm_row_kernel<8>, dim3(rows), dim3(128), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy);
     return e == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
   }
   const dim3 grid((rows + 7) / 8);
   switch (H / 128) {
-    case 2: launch_k_as(0, rmsnorm_kernel<2>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero); break;
-    case 4: launch_k_as(0, rmsnorm_kernel<4>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero); break;
-    case 8: launch_k_as(0, rmsnorm_kernel<8>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero); break;
-    case 16: launch_k_as(0, rmsnorm_kernel<16>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero); break;
-    case 32: launch_k_as(0, rmsnorm_kernel<32>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy, zero_words, n_zero); break;
+    case 2: launch_k_as(0, rmsnorm_kernel<2>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 4: launch_k_as(0, rmsnorm_kernel<4>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 8: launch_k_as(0, rmsnorm_kernel<8>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 16: launch_k_as(0, rmsnorm_kernel<16>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
+    case 32: launch_k_as(0, rmsnorm_kernel<32>, grid, dim3(256), 0, st, nullptr, 0, x, row_mul, row_add, wb, ob, tb, M, eps, cs, n_copy); break;
     default: return ZAYA_ERR_UNSUPPORTED;
   }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;

@@ -175,19 +175,8 @@ int check_weights(const zaya_block_weights* w, const zaya_config* c) {
 
 struct Ws {
   size_t status, a_in, qkv, q, premix, m_in, logits, cls, w, pos, perm, group_off, mt_start, xperm, act, part, rpart,
-      wsplit, slot, ccount, convy, kctr, total;
+      wsplit, slot, ccount, convy, total;
 };
-
-// Decode-sized projections (one 128-row tile) split K so that their weight
-// stream spreads over more SMs: 64-wide tiles, K in kDecodeSplits slabs whose
-// fp32 partials (in the attention-partials region, free at those times) the
-// last split of each tile sums.
-constexpr int kDecodeSplits = 4;
-constexpr int kDecodeBn = 64;
-int decode_splits(int rows, int N, int K) {
-  if (rows > 128 || N % kDecodeBn || (K / 64) % kDecodeSplits) return 1;
-  return kDecodeSplits;
-}
 
 Ws plan(const zaya_config& c, int mode, int B, int S) {
   const Derived d = derive(c);
@@ -210,22 +199,13 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.mt_start = o; o += up((size_t)(d.E + 2) * 4);
   w.xperm = o; o += up(M * d.H * 2);
   w.act = o; o += up(M * d.I * 2);
-  if (mode == ZAYA_DECODE) {
-    size_t part = decode_attn_ws_bytes(B, d.nq, d.d, decode_chunks_any(c));
-    const size_t s_qkv = (size_t)decode_splits(2 * B, d.n_qkv, d.H) * 2 * B * d.n_qkv * 4;
-    const size_t s_o = (size_t)decode_splits(B, d.H, d.qd) * B * d.H * 4;
-    if (s_qkv > part) part = s_qkv;
-    if (s_o > part) part = s_o;
-    w.part = o; o += up(part);
-  } else {
-    w.part = o; o += up(attn_prefill_ws_any(c, B, S, d.nq, d.nkv, d.d));
-  }
+  w.part = o; o += up(mode == ZAYA_DECODE ? decode_attn_ws_bytes(B, d.nq, d.d, decode_chunks_any(c))
+                                           : attn_prefill_ws_any(c, B, S, d.nq, d.nkv, d.d));
   w.rpart = o; o += up((size_t)router_down_splits((int)M, d.H) * M * d.R * 4);
   w.wsplit = o; o += up(((size_t)4 * d.R * d.R + (size_t)2 * ((d.E + 1 + 7) / 8 * 8) * d.R) * 2);   // fc1, fc2, out_proj hi / lo
   w.slot = o; o += up(M * 4);
   w.ccount = o; o += up((size_t)(d.E + 2) * 4);
   w.convy = o; o += c.conv_groups > 0 ? up(M * d.C * 4) : 0;   // the two-stage conv's output (fp32)
-  w.kctr = o; o += mode == ZAYA_DECODE ? up((size_t)(d.n_qkv + d.H) / kDecodeBn * 4) : 0;   // split-K tile counters
   w.total = o;
   return w;
 }
@@ -285,13 +265,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.tap_bf16 = taps ? taps->attention_output : nullptr;
     p.tap_f32 = taps ? taps->layer_mid : nullptr;
     const int c3[] = {256, 128, 64};
-    int bn = pick_bn(M, d.H, c3, 3, sms);   // single-CTA tiles measured faster here than pairs
-    if (cache_len_inc && decode_splits(M, d.H, d.qd) > 1) {   // decode: split K
-      bn = kDecodeBn;
-      p.k_splits = decode_splits(M, d.H, d.qd);
-      p.slab = at<float>(ws, L.part);
-      p.tile_ctr = at<int>(ws, L.kctr) + d.n_qkv / kDecodeBn;
-    }
+    const int bn = pick_bn(M, d.H, c3, 3, sms);   // single-CTA tiles measured faster here than pairs
     ZAYA_STAGE("o_proj_merge", 1, launch_gemm(EPI_MERGE_ATTN, bn, at<void>(ws, L.premix), M, w->w_o, d.H, p, sms, st));
   }
   void* m_in = at<void>(ws, L.m_in);
@@ -467,23 +441,15 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
   int* status = at<int>(ws, L.status);
   void* a_in = at<void>(ws, L.a_in);
   void* qkv = at<void>(ws, L.qkv);
-  // rows [0,B): attention_norm_output; rows [B,2B): prev_hs (its projection gives the delayed values);
-  // the norm also clears the split-K tile counters of the block's projections
+  // rows [0,B): attention_norm_output; rows [B,2B): prev_hs (its projection gives the delayed values)
   ZAYA_STAGE("rmsnorm_attn", 1, launch_rmsnorm(hidden, 1, 0, w->ln1_w, a_in,
                                                taps ? taps->attention_norm_output : nullptr, M, d.H, c.rms_eps,
-                                               state->prev_hs, B, st, at<int>(ws, L.kctr),
-                                               (d.n_qkv + d.H) / kDecodeBn));
+                                               state->prev_hs, B, st));
   {
     GemmParams p{};
     p.M = 2 * B; p.N = d.n_qkv; p.K = d.H; p.status = status; p.out = qkv; p.ldo = d.n_qkv;
     const int c3[] = {256, 128, 64};
-    int bn = pick_bn(2 * B, d.n_qkv, c3, 3, sms);
-    if (decode_splits(2 * B, d.n_qkv, d.H) > 1) {   // split K
-      bn = kDecodeBn;
-      p.k_splits = decode_splits(2 * B, d.n_qkv, d.H);
-      p.slab = at<float>(ws, L.part);
-      p.tile_ctr = at<int>(ws, L.kctr);
-    }
+    const int bn = pick_bn(2 * B, d.n_qkv, c3, 3, sms);
     if (!bn) return ZAYA_ERR_UNSUPPORTED;
     ZAYA_STAGE("qkv_gemm", 1, launch_gemm(EPI_STORE_BF16, bn, a_in, 2 * B, w->w_qkv, d.n_qkv, p, sms, st));
   }
