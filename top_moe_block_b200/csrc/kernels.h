@@ -176,12 +176,16 @@ struct RouterParams {
   float* w;               // [M]
   float* w_tap;           // optional [M]
   int* class_count;       // [E+1] tokens per class (cleared by the launch, then one atomic add per CTA and class)
+  int* lo_any;            // [n_lo_words]: per weight-split block, whether a weight has a nonzero lo part
+  int n_lo_words;         // router_split_blocks(R, E)
   int* slot;              // [M]: the token's place among its class's rows (order across CTAs unspecified)
   int* status;            // device status word (a bounded wait that ran out records ZAYA_ERR_TIMEOUT)
   int M, R, E;
   float eps;
 };
 int launch_router(const RouterParams& p, cudaStream_t st);
+// Blocks of the router's weight-split kernel (one lo_any word each).
+int router_split_blocks(int R, int E);
 
 
 // Copies m_in rows of routed tokens into their permuted rows; writes the

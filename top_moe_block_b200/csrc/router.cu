@@ -85,7 +85,7 @@ __device__ __forceinline__ void stage_chunk(__nv_bfloat16* dst, const __nv_bfloa
 // tensor cores (mma.sync m16n8k16) with both operands split into bf16 hi + lo:
 // a.W ~= a_hi.W_hi + a_hi.W_lo + a_lo.W_hi, fp32 accumulation.  ah / al are the
 // activation's hi / lo tiles ([32][kAS]); wh / wl the staged weight chunk.
-template <int R>
+template <int R, bool LO>   // LO: the weights have lo parts (else wl is not read)
 __device__ __forceinline__ void mlp_chunk(const __nv_bfloat16* ah_t, const __nv_bfloat16* al_t, float (*acc)[4],
                                           const __nv_bfloat16* wh, const __nv_bfloat16* wl, int c) {
   using Sh = RouterShape<R>;
@@ -107,13 +107,16 @@ __device__ __forceinline__ void mlp_chunk(const __nv_bfloat16* ah_t, const __nv_
       if (j + 1 < Sh::NTW) {
         const int row = nbase + j * 8 + (m >> 1) * 8 + (lane & 7);
         const int col = ks * 16 + (m & 1) * 8;
-        uint32_t bh0, bh1, bh2, bh3, bl0, bl1, bl2, bl3;
+        uint32_t bh0, bh1, bh2, bh3;
         ldsm_x4(smem_u32(wh) + wofs<R>(row, col), bh0, bh1, bh2, bh3);
-        ldsm_x4(smem_u32(wl) + wofs<R>(row, col), bl0, bl1, bl2, bl3);
         mma16816(acc[j], ah, bh0, bh1);
         mma16816(acc[j + 1], ah, bh2, bh3);
-        mma16816(acc[j], ah, bl0, bl1);
-        mma16816(acc[j + 1], ah, bl2, bl3);
+        if constexpr (LO) {
+          uint32_t bl0, bl1, bl2, bl3;
+          ldsm_x4(smem_u32(wl) + wofs<R>(row, col), bl0, bl1, bl2, bl3);
+          mma16816(acc[j], ah, bl0, bl1);
+          mma16816(acc[j + 1], ah, bl2, bl3);
+        }
         mma16816(acc[j], al, bh0, bh1);
         mma16816(acc[j + 1], al, bh2, bh3);
       } else {   // a single n-tile left: b fragments read directly (two bf16 per 32-bit word)
@@ -123,10 +126,12 @@ __device__ __forceinline__ void mlp_chunk(const __nv_bfloat16* ah_t, const __nv_
         const char* wlb = reinterpret_cast<const char*>(wl);
         const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(whb + wofs<R>(row, col));
         const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(whb + wofs<R>(row, col + 8));
-        const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(wlb + wofs<R>(row, col));
-        const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(wlb + wofs<R>(row, col + 8));
         mma16816(acc[j], ah, bh0, bh1);
-        mma16816(acc[j], ah, bl0, bl1);
+        if constexpr (LO) {
+          const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(wlb + wofs<R>(row, col));
+          const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(wlb + wofs<R>(row, col + 8));
+          mma16816(acc[j], ah, bl0, bl1);
+        }
         mma16816(acc[j], al, bh0, bh1);
       }
     }
@@ -177,12 +182,15 @@ __host__ __device__ constexpr int router_np(int e1) { return (e1 + 7) / 8 * 8; }
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ fc1, const float* __restrict__ fc2,
                                                            const float* __restrict__ out_w, int e1,
                                                            __nv_bfloat16* __restrict__ wsplit, int R,
-                                                           int* __restrict__ class_count) {
+                                                           int* __restrict__ class_count, int* __restrict__ lo_any) {
   griddep_begin();
   if (blockIdx.x == 0 && threadIdx.x < e1) class_count[threadIdx.x] = 0;
   const int n4 = R * R / 4, r4 = R / 4, np = router_np(e1);
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= 2 * n4 + np * r4) return;
+  // lo_any[block]: whether any weight of this block's share has a nonzero lo
+  // part (every block writes its word every launch)
+  bool lo_nz = false;
+  if (i < 2 * n4 + np * r4) {
   float4 x;
   __nv_bfloat16* hi;
   __nv_bfloat16* lo;
@@ -203,6 +211,10 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
   const float hx = round_bf(x.x), hy = round_bf(x.y), hz = round_bf(x.z), hw = round_bf(x.w);
   reinterpret_cast<uint2*>(hi)[e4] = make_uint2(pack_bf2(hx, hy), pack_bf2(hz, hw));
   reinterpret_cast<uint2*>(lo)[e4] = make_uint2(pack_bf2(x.x - hx, x.y - hy), pack_bf2(x.z - hz, x.w - hw));
+  lo_nz = (x.x != hx) || (x.y != hy) || (x.z != hz) || (x.w != hw);
+  }
+  lo_nz = __syncthreads_or(lo_nz);
+  if (threadIdx.x == 0) lo_any[blockIdx.x] = lo_nz ? 1 : 0;
 }
 
 template <int R>
@@ -226,6 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   const size_t n = (size_t)R * R;
   __shared__ int s_cnt[96], s_cls[kTM], s_rank[kTM];   // per-class counts of this CTA's tokens
   for (int c = threadIdx.x; c < 96; c += kThreads) s_cnt[c] = 0;
+  // Weights that are bf16 values (a bf16 checkpoint) have zero lo parts: then
+  // only the hi parts are loaded and the a.W_lo products are skipped (the
+  // result is the same; the activations keep their hi / lo split).
+  bool lo_w = false;
+  if (warp == 0) {
+    int any = 0;
+    for (int i = lane; i < p.n_lo_words; i += 32) any |= p.lo_any[i];
+    lo_w = __any_sync(0xffffffffu, any != 0);
+  }
+  lo_w = __syncthreads_or(lo_w);
   // weight chunk q of the fc1 -> fc2 sequence into ring stage q & 1: two TMA
   // boxes (hi, lo) of [R rows][64 columns] on the stage's barrier, issued by
   // thread 0; or (R = 32) one cp.async group of all threads
@@ -233,10 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     if constexpr (Sh::TMA) {
       if (threadIdx.x == 0) {
         uint64_t* bar = &wfull[q & 1];
-        mbar_arrive_expect_tx(bar, 2 * Sh::CHUNK * (uint32_t)sizeof(__nv_bfloat16));
+        mbar_arrive_expect_tx(bar, (lo_w ? 2 : 1) * Sh::CHUNK * (uint32_t)sizeof(__nv_bfloat16));
         const int row = (q / nch) * 2 * R;   // layer q / nch: hi rows, then lo rows
         tma_load_2d(wring + (q & 1) * 2 * Sh::CHUNK, &tmW, bar, (q % nch) * Sh::KCH, row);
-        tma_load_2d(wring + (q & 1) * 2 * Sh::CHUNK + Sh::CHUNK, &tmW, bar, (q % nch) * Sh::KCH, row + R);
+        if (lo_w) tma_load_2d(wring + (q & 1) * 2 * Sh::CHUNK + Sh::CHUNK, &tmW, bar, (q % nch) * Sh::KCH, row + R);
       }
     } else {
       const __nv_bfloat16* whi = p.wsplit + (size_t)(q / nch) * 2 * n;
@@ -366,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
       }
     } else {
       const __nv_bfloat16* ows = p.wsplit + (size_t)4 * R * R;   // [hi|lo][NP][R]
-      for (int i = threadIdx.x; i < 2 * NP * (R / 8); i += kThreads) {
+      for (int i = threadIdx.x; i < (lo_w ? 2 : 1) * NP * (R / 8); i += kThreads) {
         const int row = i / (R / 8), c = i % (R / 8);   // row over hi rows then lo rows
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(ow + row * OWS + c * 8)),
                      "l"(ows + (size_t)row * R + c * 8)
@@ -380,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     }
     __syncthreads();
     const __nv_bfloat16* wh = wring + (q & 1) * 2 * Sh::CHUNK;
-    mlp_chunk<R>(zh, zl, acc, wh, wh + Sh::CHUNK, q % nch);
+    if (lo_w) mlp_chunk<R, true>(zh, zl, acc, wh, wh + Sh::CHUNK, q % nch);
+    else mlp_chunk<R, false>(zh, zl, acc, wh, wh + Sh::CHUNK, q % nch);
     if (q == nch - 1) {   // fc1 done: its GELU output becomes fc2's operand (in place)
       __syncthreads();
       mlp_epilogue<R>(acc, b1, zh, zl, nullptr);
@@ -417,10 +440,12 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
       const int col = ks * 16 + 2 * tq;
       const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(owh + col);
       const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(owh + col + 8);
-      const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(owl + col);
-      const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(owl + col + 8);
       mma16816(c4, ah, bh0, bh1);
-      mma16816(c4, ah, bl0, bl1);
+      if (lo_w) {
+        const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(owl + col);
+        const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(owl + col + 8);
+        mma16816(c4, ah, bl0, bl1);
+      }
       mma16816(c4, al, bh0, bh1);
     }
     const int r0 = mt * 16 + g, n0 = nt * 8 + 2 * tq;
@@ -498,8 +523,9 @@ int launch_router_r(const RouterParams& p, cudaStream_t st) {
   using Sh = RouterShape<R>;
   const int np = router_np(p.E + 1);
   const int n_split = 2 * R * R / 4 + np * R / 4;
+  if (p.n_lo_words != (n_split + 255) / 256) return ZAYA_ERR_UNSUPPORTED;
   launch_k(router_split_kernel, dim3((n_split + 255) / 256), dim3(256), 0, st, nullptr, 0, p.fc1_w, p.fc2_w, p.out_w,
-           p.E + 1, p.wsplit, R, p.class_count);
+           p.E + 1, p.wsplit, R, p.class_count, p.lo_any);
   const size_t ow_elems = (size_t)2 * np * (R + 8);
   const size_t smem = Sh::SMEM + (ow_elems <= (size_t)2 * Sh::CHUNK ? 0 : ow_elems * sizeof(__nv_bfloat16));
   if (smem > 227 * 1024) return ZAYA_ERR_UNSUPPORTED;
@@ -625,6 +651,11 @@ __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
 }
 
 }  // namespace
+
+int router_split_blocks(int R, int E) {
+  const int n_split = 2 * R * R / 4 + router_np(E + 1) * R / 4;
+  return (n_split + 255) / 256;
+}
 
 int launch_router(const RouterParams& p, cudaStream_t st) {
   if (p.M <= 0) return ZAYA_OK;

@@ -175,7 +175,7 @@ int check_weights(const zaya_block_weights* w, const zaya_config* c) {
 
 struct Ws {
   size_t status, a_in, qkv, q, premix, m_in, logits, cls, w, pos, perm, group_off, mt_start, xperm, act, part, rpart,
-      wsplit, slot, ccount, convy, total;
+      wsplit, slot, ccount, convy, loany, total;
 };
 
 Ws plan(const zaya_config& c, int mode, int B, int S) {
@@ -206,6 +206,7 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.slot = o; o += up(M * 4);
   w.ccount = o; o += up((size_t)(d.E + 2) * 4);
   w.convy = o; o += c.conv_groups > 0 ? up(M * d.C * 4) : 0;   // the two-stage conv's output (fp32)
+  w.loany = o; o += up((size_t)router_split_blocks(d.R, d.E) * 4);
   w.total = o;
   return w;
 }
@@ -295,6 +296,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.w_tap = taps ? taps->expert_weights : nullptr;
     p.M = M; p.R = d.R; p.E = d.E; p.eps = c.rms_eps;
     p.class_count = at<int>(ws, L.ccount); p.slot = at<int>(ws, L.slot); p.status = status;
+    p.lo_any = at<int>(ws, L.loany); p.n_lo_words = router_split_blocks(d.R, d.E);
     ZAYA_STAGE("router_mlp", 2, launch_router(p, st));
   }
   int* group_off = at<int>(ws, L.group_off);
