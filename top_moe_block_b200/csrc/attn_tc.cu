@@ -6,20 +6,25 @@
 // key j is not padding (nnterp "zaya" page: grouped-query eager softmax
 // attention).  A query with no visible key outputs 0.
 //
-// CTA = 128 queries of one query head, 6 warps, two CTAs per SM (256 TMEM
+// CTA = 128 queries of one query head, 7 warps, two CTAs per SM (256 TMEM
 // columns and ~98 KB of shared memory each), so that one CTA's pipeline fill
 // and drain (Q load, first S, the O readout or partial write) overlap the
 // other's steady state (measured 72 us against 77 us for one CTA of two heads
 // per SM at S = 4096):
-//   warp 0     TMA: the head's Q tile once, then K and V tiles of 64 keys
-//              into a 2-slot and a 2-slot ring (128-byte swizzle, 64-wide d
-//              atoms);
+//   warp 0     TMA: the head's Q tile once, then K tiles of 64 keys into a
+//              2-slot ring (128-byte swizzle, 64-wide d atoms);
+//   warp 6     TMA: V tiles into their own 2-slot ring.  K and V have a
+//              thread each, so a K tile is requested as soon as its slot is
+//              free (S(j) done) rather than behind the previous V tile, whose
+//              slot frees only after P V (measured: the softmax waited ~1100
+//              cycles per tile for S with one thread loading both);
 //   warp 1     one thread issues tcgen05.mma: S(j) = Q K^T into one of two S
 //              buffers in tensor memory; once the softmax has written P(j)
 //              over it, O += P V with P read straight from tensor memory (A
 //              operand in TMEM) and V from shared memory as an MN-major
-//              operand, then S(j+2) into the same buffer: S runs two tiles
-//              ahead of the softmax;
+//              operand, then, once K(j+2) has landed, S(j+2) into the same
+//              buffer: S runs two tiles ahead of the softmax, and P V never
+//              waits for a K tile;
 //   warps 2-5  softmax, one thread per query row (its TMEM lane): row max
 //              and sum are thread-local; P goes back into the S columns as
 //              bf16 pairs (tcgen05.st).  The running max is only moved (and O
@@ -62,6 +67,8 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr int kMaxItems = 1024;  // split-plan items carried in the kernel parameters (16 KB)
 constexpr int kPlanSms = 296;    // the CTA slots the split plan balances over (148 SMs x 2)
 constexpr int kMinChunk = 4;     // fewest key tiles in a chunk
+constexpr int kVWarp = 2 + 4 * kHPC;            // the V loader
+constexpr int kThreads = 32 * (kVWarp + 1);     // producer, MMA, softmax warpgroups, V loader
 
 struct AttnItems {
   int n_items;   // 0: grid (row tiles, head groups of kHPC, sequences), no row tile split
@@ -182,7 +189,7 @@ __device__ __forceinline__ bool key_visible(int q, int key, int window, int S, c
 }
 
 template <int D>
-__global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams p,
                    const __grid_constant__ AttnItems items, int* status) {
@@ -268,7 +275,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
   const int n_work = wc.skip ? 0 : n_tiles;
 
   if (warp == 0) {
-    // ---------------- TMA producer: the heads' Q once, then K(j) and V(j) into their rings
+    // ---------------- TMA producer: the heads' Q once, then K(j) into its ring
     if (elect_one() && !wc.skip) {
       const int kv_row = (b * p.n_kv + g) * p.cap + n_begin + t_begin * kKT;
       mbar_arrive_expect_tx(q_full, kHPC * C::Q_BYTES);
@@ -279,7 +286,7 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
         for (int s = 0; s < C::SUB; ++s)
           tma_load_2d(sQ + x * C::Q_BYTES + s * C::Q_ATOM, &tmQ, q_full, s * 64, q_row);
       }
-      int nk = 0, nv = 0;   // K / V tiles whose copies were started
+      int nk = 0;   // K tiles whose copies were started
       for (int j = 0; j < n_tiles; ++j) {
         const int slot = j % kRing;
         const uint32_t par = ((j / kRing) & 1) ^ 1u;
@@ -289,6 +296,18 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
         for (int s = 0; s < C::SUB; ++s)
           tma_load_2d(sK + slot * C::KV_BYTES + s * C::KV_ATOM, &tmK, &k_full[slot], s * 64, kv_row + j * kKT);
         ++nk;
+      }
+      // every copy started must land before the CTA may exit: the last phase
+      // armed on each slot (tile j uses phase j / ring of slot j % ring)
+      mbar_drain(q_full, 0, status);
+      for (int j = (nk > kRing ? nk - kRing : 0); j < nk; ++j) mbar_drain(&k_full[j % kRing], (j / kRing) & 1, status);
+    }
+  } else if (warp == kVWarp) {
+    // ---------------- TMA producer: V(j) into its ring
+    if (elect_one() && !wc.skip) {
+      const int kv_row = (b * p.n_kv + g) * p.cap + n_begin + t_begin * kKT;
+      int nv = 0;   // V tiles whose copies were started
+      for (int j = 0; j < n_tiles; ++j) {
         const int vslot = j % kRingV;
         if (!mbar_wait(&v_empty[vslot], ((j / kRingV) & 1) ^ 1u, wc)) break;
         mbar_arrive_expect_tx(&v_full[vslot], C::KV_BYTES);
@@ -297,10 +316,6 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
           tma_load_2d(sV + vslot * C::KV_BYTES + s * C::KV_ATOM, &tmV, &v_full[vslot], s * 64, kv_row + j * kKT);
         ++nv;
       }
-      // every copy started must land before the CTA may exit: the last phase
-      // armed on each slot (tile j uses phase j / ring of slot j % ring)
-      mbar_drain(q_full, 0, status);
-      for (int j = (nk > kRing ? nk - kRing : 0); j < nk; ++j) mbar_drain(&k_full[j % kRing], (j / kRing) & 1, status);
       for (int j = (nv > kRingV ? nv - kRingV : 0); j < nv; ++j)
         mbar_drain(&v_full[j % kRingV], (j / kRingV) & 1, status);
     }
@@ -334,7 +349,6 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int vslot = j % kRingV, nslot = (j + 2) % kRing;
         const bool more = j + 2 < n_tiles;
-        if (more && !mbar_wait(&k_full[nslot], ((j + 2) / kRing) & 1, wc)) break;
         if (!mbar_wait(&v_full[vslot], (j / kRingV) & 1, wc)) break;
         const uint32_t va = smem_u32(sV + vslot * C::KV_BYTES);
         for (int x = 0; ok && x < kHPC; ++x) {
@@ -349,11 +363,15 @@ __global__ void __launch_bounds__(64 + 32 * 4 * kHPC, 2)
             tc_mma_bf16_ts(tmem_base + x * C::HEAD_COLS + C::O_COL, pa + kk * 8,
                            smem_desc_sw128(va + kk * 2048, C::KV_ATOM, 1024), C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&pv_done[x]);
-          if (more) issue_qk(x, j + 2);
         }
         if (!ok) break;
         tc_commit(&v_empty[vslot]);
-        if (more) tc_commit(&k_empty[nslot]);
+        if (more) {   // S(j+2) once K(j+2) has landed, after P V(j) in the pipe's order
+          if (!mbar_wait(&k_full[nslot], ((j + 2) / kRing) & 1, wc)) break;
+          tc_fence_after();
+          for (int x = 0; x < kHPC; ++x) issue_qk(x, j + 2);
+          tc_commit(&k_empty[nslot]);
+        }
       }
       // the last commit, issued on every path: it arrives once every MMA above
       // has completed -- O is final and the tensor memory may be freed
@@ -599,7 +617,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTc<128>::SMEM);
       set = true;
     }
-    launch_k(kern, grid, dim3(64 + 32 * 4 * kHPC), AttnTc<128>::SMEM, st, nullptr, 0, mq, mk, mv, p, items, status);
+    launch_k(kern, grid, dim3(kThreads), AttnTc<128>::SMEM, st, nullptr, 0, mq, mk, mv, p, items, status);
   } else {
     auto kern = attn_tc_kernel<64>;
     static bool set = false;
@@ -607,7 +625,7 @@ int launch_attn_prefill_tc(const AttnParams& p, int* status, cudaStream_t st) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTc<64>::SMEM);
       set = true;
     }
-    launch_k(kern, grid, dim3(64 + 32 * 4 * kHPC), AttnTc<64>::SMEM, st, nullptr, 0, mq, mk, mv, p, items, status);
+    launch_k(kern, grid, dim3(kThreads), AttnTc<64>::SMEM, st, nullptr, 0, mq, mk, mv, p, items, status);
   }
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }

@@ -17,6 +17,12 @@
 // Grouped mode (the experts): A rows are the tokens permuted by expert, B is
 // the stacked expert weights; the tile list is derived on the device from
 // the per-expert row offsets, so no host synchronisation is needed.
+// Grouped CTA pairs run swapped (D^T = W X^T): the expert's weight rows are
+// the MMA's M = 256 side and its tokens the N side, N = the tile's token count
+// rounded up to 16 (an expert's tokens split into ceil(n/256) near-equal
+// tiles), so a routed token costs 1/16 of padding at most instead of up to a
+// whole 256-row tile.  The epilogue then holds one feature per TMEM lane and
+// one token per column.
 //
 // Epilogues (what the block needs right after each contraction):
 //   STORE_BF16   q/k/v projections, lm_head logits
@@ -50,14 +56,17 @@ constexpr int kPrefetchAhead = 8;  // k-blocks of B pulled into L2 ahead of thei
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA (227 KB)
 
-template <int BN, int EPI, int CG = 1>
+template <int BN, int EPI, int CG = 1, bool SWAP = false>
 struct GemmCfg {
-  static constexpr int B_STAGE_BYTES = BN / CG * BK * 2;   // a CTA pair splits B's columns
+  static constexpr int B_STAGE_BYTES = BN / CG * BK * 2;   // a CTA pair splits B's columns (swapped: 128 token rows)
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
-  static constexpr int PARAM_BYTES = is_merge<EPI>() ? 2 * 4 * BN * 4 : 0;  // merge: [2 tiles][hb,hs,rb,rs][BN] fp32
-  // merge epilogues: a 32 x 32 fp32 transpose buffer per epilogue warp
-  static constexpr int T_BYTES = is_merge<EPI>() ? epi_warps<EPI>() * 32 * 32 * 4 : 0;
+  // merge: [2 tiles][hb,hs,rb,rs][BN] fp32 (swapped: per-lane registers instead)
+  static constexpr int PARAM_BYTES = (is_merge<EPI>() && !SWAP) ? 2 * 4 * BN * 4 : 0;
+  // merge epilogues: a 32 x 32 fp32 transpose buffer per epilogue warp; swapped
+  // SwiGLU: per chunk two feature groups x (16 gate + 16 up tokens) x 32 lanes, double-buffered
+  static constexpr int T_BYTES = (SWAP && EPI == EPI_SWIGLU) ? 2 * 2 * 32 * 32 * 4
+                                 : (is_merge<EPI>() ? epi_warps<EPI>() * 32 * 32 * 4 : 0);
   static constexpr int FIXED = PARAM_BYTES + T_BYTES + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr int DEF_STAGES = (STAGE_BYTES >= 49152) ? 4 : (STAGE_BYTES >= 32768 ? 6 : 8);  // ~192 KB ring
   static constexpr int FIT_STAGES = (kSmemLimit - FIXED) / STAGE_BYTES;
@@ -75,6 +84,8 @@ struct TileInfo {
   int n0;      // first output column
   int b_row;   // first B row (gate rows for SWIGLU)
   int b_row2;  // SWIGLU: first up row
+  int n_valid; // swapped: the tile's tokens (rows m0 .. m0 + n_valid of A)
+  int n_mma;   // swapped: MMA N, n_valid rounded up to 16
 };
 
 template <int EPI, int BN_OUT, int TM>   // TM: output rows per tile (128, or 256 for a CTA pair)
@@ -85,7 +96,7 @@ __device__ __forceinline__ int total_tiles(const GemmParams& p) {
   return p.mt_start[p.n_groups] * nt;   // mt_start counts TM-row tiles
 }
 
-template <int EPI, int BN_OUT, int TM>
+template <int EPI, int BN_OUT, int TM, bool SWAP = false>
 __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
   TileInfo ti;
   const int nt = p.N / BN_OUT;
@@ -113,11 +124,24 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
     ti.n0 = (local / mte) * BN_OUT;
     ti.b_row = e * p.b_rows_per_group + ti.n0;
     ti.b_row2 = e * p.b_rows_per_group + (p.b_rows_per_group >> 1) + ti.n0;
+    if constexpr (SWAP) {
+      // the expert's n tokens in mte near-equal tiles of `per` (a multiple of 16,
+      // at most 256); every tile holds at least one token since n > 256 (mte - 1)
+      const int n = ti.m_end - p.group_off[e];
+      const int per = ((n + mte - 1) / mte + 15) & ~15;
+      const int i = local % mte;
+      ti.m0 = p.group_off[e] + i * per;
+      ti.n_valid = min(per, n - i * per);
+      ti.n_mma = (ti.n_valid + 15) & ~15;
+    }
   }
   return ti;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the fast (branch-free) division: a few ulp in
+// fp32 ahead of the bf16 rounding of act, and no per-element branch that would
+// serialise the epilogue's chains (g -> -inf gives -0).
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // Epilogue of one row (this thread) x 32 consecutive columns.
 template <int EPI>
@@ -279,6 +303,68 @@ __device__ __forceinline__ void merge_chunk(const GemmParams& p, int row0, int m
   __syncwarp();
 }
 
+// Swapped merge epilogue of a warp's 32 features (lanes, from fw) x 32
+// permuted rows (columns, from row0; nj of them real): the accumulator goes
+// through a 32 x 32 fp32 shared-memory transpose to token-major 16-byte chunks
+// (XOR-swizzled by token), then each step covers 4 tokens x 128 contiguous
+// bytes of the fp32 stream, all eight steps' loads in flight first.  tokl /
+// wl: lane i holds row row0 + i's token and routing weight.
+__device__ __forceinline__ void merge_chunk_swap(const GemmParams& p, int nj, int fw, int tokl, float wl,
+                                                 const uint32_t (&r)[32], float* T) {
+  const int lane = lane_id();
+#pragma unroll
+  for (int j = 0; j < 32; ++j) T[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = __uint_as_float(r[j]);
+  __syncwarp();
+  const int jj = lane & 7, rsub = lane >> 3;
+  const int N = p.N;
+  const int col = fw + 4 * jj;
+  int tok[8];
+  float wt[8];
+  float4 xs[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    tok[i] = __shfl_sync(0xffffffffu, tokl, 4 * i + rsub);
+    wt[i] = __shfl_sync(0xffffffffu, wl, 4 * i + rsub);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    xs[i] = 4 * i + rsub < nj ? *reinterpret_cast<const float4*>(p.stream + (size_t)tok[i] * N + col)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4 hb4 = __ldg(reinterpret_cast<const float4*>(p.merge + col));
+  const float4 hs4 = __ldg(reinterpret_cast<const float4*>(p.merge + N + col));
+  const float4 rb4 = __ldg(reinterpret_cast<const float4*>(p.merge + 2 * N + col));
+  const float4 rs4 = __ldg(reinterpret_cast<const float4*>(p.merge + 3 * N + col));
+  const float* hbp = &hb4.x;
+  const float* hsp = &hs4.x;
+  const float* rbp = &rb4.x;
+  const float* rsp = &rs4.x;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = 4 * i + rsub;
+    if (rr >= nj) continue;
+    const float4 a4 = *reinterpret_cast<const float4*>(T + rr * 32 + ((jj ^ (rr & 7)) << 2));
+    const float* ap = &a4.x;
+    float4 x4 = xs[i];
+    float* xp = &x4.x;
+    float cb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float contrib = round_bf((ap[j] * wt[i] + hbp[j]) * hsp[j]);
+      cb[j] = contrib;
+      xp[j] = fmaf(xp[j] + rbp[j], rsp[j], contrib);
+    }
+    const size_t off = (size_t)tok[i] * N + col;
+    *reinterpret_cast<float4*>(p.stream + off) = x4;
+    if (p.tap_bf16) {
+      uint2 u;
+      u.x = pack_bf2(cb[0], cb[1]);
+      u.y = pack_bf2(cb[2], cb[3]);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.tap_bf16) + off) = u;
+    }
+  }
+  __syncwarp();
+}
+
 // CG = 1: one CTA per SM, 128 x BN tiles.  CG = 2: clusters of two CTAs
 // (cta_group::2), 256 x BN tiles: CTA rank r loads A rows [m0 + 128r, +128)
 // and its half of B's BN rows (SWIGLU: rank 0 the gate rows, rank 1 the up
@@ -287,11 +373,18 @@ __device__ __forceinline__ void merge_chunk(const GemmParams& p, int row0, int m
 // MMAs and its commits arrive on the `empty` / `tfull` barriers of both CTAs;
 // each CTA's epilogue reads its own 128 accumulator rows and releases the
 // accumulator on rank 0's `tempty`.
-template <int BN, int EPI, int CG>
+// SWAP (grouped CTA pairs): CTA rank r loads 128 weight rows into the A slot
+// (SWIGLU: gate rows [n0 + 64r, +64) then the up rows of the same features;
+// MERGE_MLP: output rows [n0 + 128r, +128)) and a box of tok_box token rows
+// from m0 + r * n_mma / 2 into the B slot, of which the MMA reads the first
+// n_mma / 2 <= tok_box; tmA then maps the tokens and tmB the weights.
+template <int BN, int EPI, int CG, bool SWAP>
 __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
-  using C = GemmCfg<BN, EPI, CG>;
+  static_assert(!SWAP || (CG == 2 && BN == 256 && (EPI == EPI_SWIGLU || EPI == EPI_MERGE_MLP)),
+                "swapped tiles: grouped expert GEMMs on CTA pairs");
+  using C = GemmCfg<BN, EPI, CG, SWAP>;
   constexpr int STAGES = C::STAGES;
   constexpr int BN_OUT = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
   constexpr int TM = BM * CG;   // output rows per tile
@@ -370,14 +463,18 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
       uint32_t phase = 0;
       int n_armed = 0;
       for (int t = unit; t < ntiles; t += n_units) {
-        const TileInfo ti = tile_info<EPI, BN_OUT, TM>(p, t);
+        const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP>(p, t);
         // this CTA's B rows: CG = 1 all BN rows (SWIGLU: gate then up); CG = 2 its half
         const int b_first = (CG == 1) ? ti.b_row
+                            : SWAP ? ti.b_row + (int)rank * (EPI == EPI_SWIGLU ? 64 : 128)
                             : (EPI == EPI_SWIGLU) ? (rank == 0 ? ti.b_row : ti.b_row2)
                                                   : ti.b_row + (int)rank * (BN / 2);
         const int kb_end = ti.kb0 + ti.nkb;
         auto prefetch_b = [&](int kb) {
-          if constexpr (EPI == EPI_SWIGLU && CG == 1) {
+          if constexpr (SWAP && EPI == EPI_SWIGLU) {
+            tma_prefetch_l2_2d(&tmB, kb * BK, b_first);
+            tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row2 + (int)rank * 64);
+          } else if constexpr (EPI == EPI_SWIGLU && CG == 1) {
             tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row);
             tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row2);
           } else {
@@ -390,7 +487,14 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
           if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) goto producer_done;
           uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
           uint8_t* b_dst = sB + stage * C::B_STAGE_BYTES;
-          if constexpr (CG == 2) {
+          if constexpr (SWAP) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (A_STAGE_BYTES + p.tok_box * BK * 2));   // both CTAs
+            const uint32_t bar = mapa_shared(&full[stage], 0);
+            tma_load_2d_pair(a_dst, &tmB, bar, kb * BK, b_first);   // weights: the MMA's A
+            if constexpr (EPI == EPI_SWIGLU)
+              tma_load_2d_pair(a_dst + 64 * BK * 2, &tmB, bar, kb * BK, ti.b_row2 + (int)rank * 64);
+            tma_load_2d_pair(b_dst, &tmA, bar, kb * BK, ti.m0 + (int)rank * (ti.n_mma >> 1));   // tokens: B
+          } else if constexpr (CG == 2) {
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);   // both CTAs' bytes
             const uint32_t bar = mapa_shared(&full[stage], 0);
             tma_load_2d_pair(a_dst, &tmA, bar, kb * BK, ti.m0 + (int)rank * BM);
@@ -433,7 +537,9 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, wc)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        const int nkb = tile_info<EPI, BN_OUT, TM>(p, t).nkb;
+        const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP>(p, t);
+        const int nkb = ti.nkb;
+        const uint32_t idesc = SWAP ? idesc_bf16_f32(TM, ti.n_mma) : IDESC;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, wc)) {
@@ -446,7 +552,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             if constexpr (CG == 2)
-              tc_mma_bf16_pair(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), IDESC,
+              tc_mma_bf16_pair(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), idesc,
                                (kb | k) != 0 ? 1u : 0u);
             else
               tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), IDESC,
@@ -469,6 +575,95 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
       else tc_commit(mdrain);
       mbar_drain(mdrain, 0, p.status);
     }
+  } else if constexpr (SWAP) {
+    // ---------------- epilogue warps, swapped tiles: TMEM lane = weight row, column = token
+    const int q = warp & 3;              // TMEM lanes [32q, 32q+32) are reachable from this warp
+    const int part = (warp - 2) >> 2;    // MERGE_MLP: column interleave of the two warps per lane quarter
+    const int N = p.N;
+    int local = 0;
+    uint32_t kc = 0;        // SWIGLU: chunks done, the parity of the up-value buffer
+    bool aborted = false;   // a wait ran out: keep walking the tiles (barrier partners) without waiting
+    for (int t = unit; t < ntiles; t += n_units, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP>(p, t);
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if constexpr (EPI == EPI_SWIGLU) {
+        // Lanes 0-63 hold the gate rows of features n0 + 64 rank + [0, 64), lanes
+        // 64-127 their up rows.  Per 32-token chunk, warp q works on feature
+        // group q & 1 and token half q >> 1: the gate warp hands its second
+        // half of gate values to the up warp of its group and takes the up
+        // warp's first half of up values (shared memory), then each warp writes
+        // act = bf16(silu(gate) * up) for its 16 tokens x 32 features.
+        const bool ok = !aborted && mbar_wait(&tfull[acc], acc_phase, wc);
+        if (named_barrier_any(1, EW * 32, !ok)) aborted = true;   // the four warps decide together
+        if (aborted) continue;
+        tc_fence_after();
+        const int fg = q & 1, th = q >> 1;
+        const int feat = ti.n0 + 64 * (int)rank + 32 * fg + lane;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll 1
+        for (int c = 0; c < ti.n_valid; c += 32, ++kc) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
+          tmem_ld_wait();
+          // [group][0: gate tokens 16-31 | 1: up tokens 0-15][16][32 lanes]
+          float* T = sT + (kc & 1) * 2048 + fg * 1024;
+          float* give = T + th * 512;    // gate warp gives gate (tokens 16-31), up warp gives up (tokens 0-15)
+          float* take = T + (th ^ 1) * 512;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) give[j * 32 + lane] = __uint_as_float(th == 0 ? r[j + 16] : r[j]);
+          named_barrier_sync(1, EW * 32);
+          float a[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float mine = __uint_as_float(th == 0 ? r[j] : r[j + 16]), other = take[j * 32 + lane];
+            a[j] = th == 0 ? silu_f(mine) * other : silu_f(other) * mine;
+          }
+          const int j0 = c + 16 * th;
+          const int nj = min(16, ti.n_valid - j0);
+          __nv_bfloat16* dst = out + (size_t)(ti.m0 + j0) * p.ldo + feat;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < nj) dst[(size_t)j * p.ldo] = __float2bfloat16_rn(a[j]);
+        }
+      } else {
+        // MERGE_MLP: lane = output feature, column = permuted row; a token's 32
+        // features of this warp are one 128-byte segment of its stream row.
+        // While the main loop runs: this warp's chunks are columns 32 part + 64 k
+        // (k < 4, N <= 256); lane j of chunk k fetches its token and routing
+        // weight and pulls the token's stream segment into L2.
+        const int fw = ti.n0 + 128 * (int)rank + 32 * q;   // this warp's first feature
+        int tokk[4];
+        float wk[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int cc = 32 * part + 64 * k + lane;
+          tokk[k] = cc < ti.n_valid ? p.perm[ti.m0 + cc] : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const bool in = 32 * part + 64 * k + lane < ti.n_valid;
+          wk[k] = in ? p.row_w[tokk[k]] : 0.f;
+          if (in) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.stream + (size_t)tokk[k] * N + fw));
+        }
+        if (!aborted && !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, wc))) aborted = true;
+        if (aborted) continue;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c = 32 * part + 64 * k;
+          if (c >= ti.n_valid) break;   // warp-uniform
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
+          tmem_ld_wait();
+          merge_chunk_swap(p, min(32, ti.n_valid - c), fw, tokk[k], wk[k], r, sT + (warp - 2) * 1024);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(&tempty[acc], 0));
+    }
   } else {
     // ---------------- epilogue warps 2 .. 2+EW-1 (this CTA's 128 accumulator rows)
     const int q = warp & 3;              // TMEM lanes [32q, 32q+32) are reachable from this warp
@@ -480,7 +675,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     for (int t = unit; t < ntiles; t += n_units, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      const TileInfo ti = tile_info<EPI, BN_OUT, TM>(p, t);
+      const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP>(p, t);
       float* prm = sPrm + acc * 4 * BN_OUT;
       if constexpr (is_merge<EPI>()) {
         // this tile's merge parameters (hb, hs, rb, rs for its columns) into shared memory
@@ -553,11 +748,11 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <int BN, int EPI, int CG>
+template <int BN, int EPI, int CG, bool SWAP = false>
 int launch_impl(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, int ntiles_hint, int num_sms,
                 cudaStream_t st) {
-  using C = GemmCfg<BN, EPI, CG>;
-  auto kern = gemm_tc_kernel<BN, EPI, CG>;
+  using C = GemmCfg<BN, EPI, CG, SWAP>;
+  auto kern = gemm_tc_kernel<BN, EPI, CG, SWAP>;
   static bool attr_set = false;
   static int max_pairs = 0;   // co-resident CTA pairs (CG = 2)
   if (!attr_set) {
@@ -627,15 +822,27 @@ int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b
   if (a_rows <= 0) return ZAYA_OK;
   const int cg = p.pair ? 2 : 1;
   if (cg == 2 && bn != 256 && bn != 128) return ZAYA_ERR_UNSUPPORTED;
+  // grouped expert GEMMs on CTA pairs run swapped (weights on the M side)
+  const bool swap = cg == 2 && p.grouped && (epi == EPI_SWIGLU || epi == EPI_MERGE_MLP);
+  if (swap && bn != 256) return ZAYA_ERR_UNSUPPORTED;
+  // swapped: a token box as tall as any tile's half of N can be (<= 128, and
+  // n_mma / 2 <= round16(a_rows) / 2 since an expert holds at most a_rows tokens)
+  GemmParams q = p;
+  q.tok_box = swap ? (a_rows >= 128 ? 128 : ((a_rows + 15) & ~15)) : BM;
   CUtensorMap ma, mb;
-  int rc = make_tmap_bf16(&ma, A, (uint64_t)a_rows, (uint64_t)p.K, BM);
+  int rc = make_tmap_bf16(&ma, A, (uint64_t)a_rows, (uint64_t)p.K, (uint32_t)q.tok_box);
   if (rc) return rc;
   // B box: a CTA pair splits the tile's B rows in two; SWIGLU loads gate and up rows as two boxes
-  rc = make_tmap_bf16(&mb, B, (uint64_t)b_rows, (uint64_t)p.K, (epi == EPI_SWIGLU || cg == 2) ? bn / 2 : bn);
+  // (swapped SWIGLU: 64 gate and 64 up rows per CTA)
+  const uint32_t b_box = (swap && epi == EPI_SWIGLU) ? 64 : (epi == EPI_SWIGLU || cg == 2) ? bn / 2 : bn;
+  rc = make_tmap_bf16(&mb, B, (uint64_t)b_rows, (uint64_t)p.K, b_box);
   if (rc) return rc;
   const int nt = p.N / bn_out;
   const int tm = BM * cg;
   int hint = p.grouped ? num_sms : ((p.M + tm - 1) / tm) * nt * ks;
+  if (swap)
+    return epi == EPI_SWIGLU ? launch_impl<256, EPI_SWIGLU, 2, true>(ma, mb, q, hint, num_sms, st)
+                             : launch_impl<256, EPI_MERGE_MLP, 2, true>(ma, mb, q, hint, num_sms, st);
 #define ZAYA_GEMM_CASE(BNV, EPIV)                                                  \
   if (bn == BNV && epi == EPIV)                                                    \
     return cg == 2 ? launch_impl<BNV, EPIV, 2>(ma, mb, p, hint, num_sms, st)       \

@@ -40,6 +40,7 @@ struct GemmParams {
   const float* row_w;        // MERGE_MLP: per-token expert weight
   void* tap_bf16;            // MERGE_*: optional bf16 [tokens, N] contribution tap
   float* tap_f32;            // MERGE_ATTN: optional fp32 [tokens, N] layer_mid tap
+  int tok_box;               // set by launch_gemm: swapped tiles' token box rows (16..128)
 };
 
 // Encodes a 2-D bf16 tensor map (rows x cols, row-major) with a box of
@@ -51,11 +52,16 @@ int make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t co
 int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b_rows, const GemmParams& p,
                 int num_sms, cudaStream_t st);
 
-// K slabs for the router down-projection of M rows (a power of two, at most
-// 8 and K/64): enough 128-row x slab tiles to fill the GPU while the fp32
-// partial slabs stay small.  Deterministic in M.
-inline int router_down_splits(int M, int K) {
+// Router down-projection plan for M rows and R outputs over K inputs.
+// 0: one pass over K whose epilogue adds the bias and the carried state and
+// writes the router state itself, chosen when 64-column tiles alone give 96 or
+// more CTAs.  Otherwise the number of K slabs (a power of two, at most 8 and
+// K/64) of fp32 partial sums that the router kernel adds in slab order: enough
+// 128-row x slab tiles to fill the GPU while the slabs stay small.
+// Deterministic in (M, R, K).
+inline int router_down_splits(int M, int R, int K) {
   const int mt = (M + 127) / 128;
+  if (R % 64 == 0 && mt * (R / 64) >= 96) return 0;
   int ks = 1;
   while (ks * 2 <= 8 && ks * 2 <= K / 64 && mt * ks * 2 <= 148) ks *= 2;
   return ks;
@@ -158,7 +164,7 @@ int launch_attn_decode(const DecodeAttnParams& p, cudaStream_t st);
 // ------------------------------------------------------------------ router / MoE dispatch
 struct RouterParams {
   const float* part;      // [n_splits, M, R] partial sums of m_in . W_down^T (split over K)
-  int n_splits;
+  int n_splits;           // 0: r_out already holds the state (bias and carried state added)
   const float* bias;      // [R] down_proj bias
   const float* prev;      // [M, R] previous block's router state, or null (block 0)
   const float* prev_scale;// [R] router_states_scale

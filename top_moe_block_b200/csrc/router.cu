@@ -278,13 +278,15 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
 
   // router state r = down_proj partial sums (in slab order) + bias (+ previous
   // state * scale).  Each thread owns kPos float4 positions; the loads of two
-  // slabs for all of them are issued before any add.
+  // slabs for all of them are issued before any add.  n_splits 0: the
+  // down-projection's epilogue has written r itself (to r_out), read as is.
   {
     constexpr int R4 = R / 4;
     constexpr int kPos = (kTM * R4 + kThreads - 1) / kThreads;
     const size_t slab = (size_t)p.M * R4;
-    const int ns = p.n_splits;
-    const float4* part = reinterpret_cast<const float4*>(p.part);
+    const bool fused = p.n_splits == 0;
+    const int ns = fused ? 1 : p.n_splits;
+    const float4* part = reinterpret_cast<const float4*>(fused ? p.r_out : p.part);
     float4 v[kPos];
     size_t off[kPos];
     bool live[kPos], here[kPos];
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
       }
     }
     float4 pv[kPos];
-    if (p.prev) {
+    if (p.prev && !fused) {
 #pragma unroll
       for (int u = 0; u < kPos; ++u) pv[u] = reinterpret_cast<const float4*>(p.prev)[off[u]];
     }
@@ -320,15 +322,17 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
       const int i = threadIdx.x + u * kThreads;
       const int tt = i / R4, k4 = i % R4;
       if (!here[u]) continue;
-      const float4 bb = __ldg(reinterpret_cast<const float4*>(p.bias) + k4);
-      v[u].x += bb.x; v[u].y += bb.y; v[u].z += bb.z; v[u].w += bb.w;
-      if (p.prev) {
-        const float4 sc = __ldg(reinterpret_cast<const float4*>(p.prev_scale) + k4);
-        v[u].x = fmaf(pv[u].x, sc.x, v[u].x); v[u].y = fmaf(pv[u].y, sc.y, v[u].y);
-        v[u].z = fmaf(pv[u].z, sc.z, v[u].z); v[u].w = fmaf(pv[u].w, sc.w, v[u].w);
+      if (!fused) {
+        const float4 bb = __ldg(reinterpret_cast<const float4*>(p.bias) + k4);
+        v[u].x += bb.x; v[u].y += bb.y; v[u].z += bb.z; v[u].w += bb.w;
+        if (p.prev) {
+          const float4 sc = __ldg(reinterpret_cast<const float4*>(p.prev_scale) + k4);
+          v[u].x = fmaf(pv[u].x, sc.x, v[u].x); v[u].y = fmaf(pv[u].y, sc.y, v[u].y);
+          v[u].z = fmaf(pv[u].z, sc.z, v[u].z); v[u].w = fmaf(pv[u].w, sc.w, v[u].w);
+        }
       }
       if (!live[u]) v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      else reinterpret_cast<float4*>(p.r_out)[off[u]] = v[u];
+      else if (!fused) reinterpret_cast<float4*>(p.r_out)[off[u]] = v[u];
       *reinterpret_cast<float4*>(z + tt * kZS + k4 * 4) = v[u];
     }
   }
@@ -659,7 +663,7 @@ int router_split_blocks(int R, int E) {
 
 int launch_router(const RouterParams& p, cudaStream_t st) {
   if (p.M <= 0) return ZAYA_OK;
-  if (p.E + 1 > 96 || p.n_splits < 1 || !p.wsplit || !p.class_count) return ZAYA_ERR_UNSUPPORTED;
+  if (p.E + 1 > 96 || p.n_splits < 0 || !p.wsplit || !p.class_count) return ZAYA_ERR_UNSUPPORTED;
   switch (p.R) {
     case 32: return launch_router_r<32>(p, st);
     case 64: return launch_router_r<64>(p, st);

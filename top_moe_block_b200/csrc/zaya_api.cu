@@ -201,7 +201,7 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.act = o; o += up(M * d.I * 2);
   w.part = o; o += up(mode == ZAYA_DECODE ? decode_attn_ws_bytes(B, d.nq, d.d, decode_chunks_any(c))
                                            : attn_prefill_ws_any(c, B, S, d.nq, d.nkv, d.d));
-  w.rpart = o; o += up((size_t)router_down_splits((int)M, d.H) * M * d.R * 4);
+  w.rpart = o; o += up((size_t)router_down_splits((int)M, d.R, d.H) * M * d.R * 4);
   w.wsplit = o; o += up(((size_t)4 * d.R * d.R + (size_t)2 * ((d.E + 1 + 7) / 8 * 8) * d.R) * 2);   // fc1, fc2, out_proj hi / lo
   w.slot = o; o += up(M * 4);
   w.ccount = o; o += up((size_t)(d.E + 2) * 4);
@@ -275,15 +275,21 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
   int* cls = at<int>(ws, L.cls);
   float* wgt = at<float>(ws, L.w);
   float* rpart = at<float>(ws, L.rpart);
-  const int ks = router_down_splits(M, d.H);
-  {  // router down_proj as fp32 partial sums over K slabs
+  const int ks = router_down_splits(M, d.R, d.H);
+  if (ks == 0) {  // router down_proj + bias + carried state in one pass, straight into the state out
+    GemmParams p{};
+    p.M = M; p.N = d.R; p.K = d.H; p.status = status;
+    p.out = rout; p.ldo = d.R; p.bias = w->router_down_b;
+    p.prev = (block_idx > 0) ? rin : nullptr; p.prev_scale = w->router_state_scale;
+    ZAYA_STAGE("router_down", 1, launch_gemm(EPI_ROUTER_DOWN, 64, m_in, M, w->router_down_w, d.R, p, sms, st));
+  } else {  // router down_proj as fp32 partial sums over K slabs
     GemmParams p{};
     p.M = M; p.N = d.R; p.K = d.H; p.k_splits = ks; p.status = status;
     p.out = rpart; p.ldo = d.R;
     const int bn = (d.R % 256 == 0) ? 256 : (d.R % 128 == 0) ? 128 : (d.R % 64 == 0) ? 64 : 32;
     ZAYA_STAGE("router_down", 1, launch_gemm(EPI_STORE_F32, bn, m_in, M, w->router_down_w, d.R, p, sms, st));
   }
-  {  // router state (slab sum + bias + carried state), router MLP, scoring, top-1
+  {  // router state (slab sum + bias + carried state, unless fused above), router MLP, scoring, top-1
     RouterParams p{};
     p.part = rpart; p.n_splits = ks; p.bias = w->router_down_b;
     p.prev = (block_idx > 0) ? rin : nullptr; p.prev_scale = w->router_state_scale; p.r_out = rout;
@@ -303,8 +309,9 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
   int* mt_start = at<int>(ws, L.mt_start);
   int* pos = at<int>(ws, L.pos);
   int* perm = at<int>(ws, L.perm);
-  // expert GEMMs of prefill-sized batches run on CTA pairs (256-row tiles)
-  const int pair = M >= kPairMinRows ? 1 : 0;
+  // the expert GEMMs run swapped on CTA pairs (256 weight rows x each expert's
+  // tokens, rounded to 16) whenever the widths allow: I a multiple of 128, H of 256
+  const int pair = (d.I % 128 == 0 && d.H % 256 == 0) ? 1 : 0;
   void* xperm = at<void>(ws, L.xperm);
   {  // the token -> expert-row permutation, the copy of routed rows, merge 2 of skipped rows
     DispatchParams p{};
