@@ -375,9 +375,10 @@ __device__ __forceinline__ void merge_chunk_swap(const GemmParams& p, int nj, in
 // accumulator on rank 0's `tempty`.
 // SWAP (grouped CTA pairs): CTA rank r loads 128 weight rows into the A slot
 // (SWIGLU: gate rows [n0 + 64r, +64) then the up rows of the same features;
-// MERGE_MLP: output rows [n0 + 128r, +128)) and a box of tok_box token rows
-// from m0 + r * n_mma / 2 into the B slot, of which the MMA reads the first
-// n_mma / 2 <= tok_box; tmA then maps the tokens and tmB the weights.
+// MERGE_MLP: output rows [n0 + 128r, +128)) and its n_mma / 2 token rows from
+// m0 + r * n_mma / 2 into the B slot, in boxes of tok_box (16) rows, so a
+// tile of few tokens loads few bytes; tmA then maps the tokens and tmB the
+// weights.
 template <int BN, int EPI, int CG, bool SWAP>
 __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -402,7 +403,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mdrain = tempty + 2;   // the MMA thread's last commit: all its MMAs are done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdrain + 1);
+  uint64_t* xbar = mdrain + 1;     // [2] swapped SwiGLU: a chunk's gate / up halves are in shared memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 2);
   int* s_skip = reinterpret_cast<int*>(tmem_slot + 1);   // CTA pair: rank 0's reading of the status word
 
   const int warp = warp_id();
@@ -421,6 +423,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
       mbar_init(&tempty[a], CG * EW);
     }
     mbar_init(mdrain, 1);
+    mbar_init(&xbar[0], EW);
+    mbar_init(&xbar[1], EW);
     fence_barrier_init();
     fence_proxy_async();
     prefetch_tmap(&tmA);
@@ -488,12 +492,17 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
           uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
           uint8_t* b_dst = sB + stage * C::B_STAGE_BYTES;
           if constexpr (SWAP) {
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (A_STAGE_BYTES + p.tok_box * BK * 2));   // both CTAs
+            // tokens: the n_mma / 2 rows of this CTA's half of N, in boxes of tok_box rows
+            const int n_box = ((ti.n_mma >> 1) + p.tok_box - 1) / p.tok_box;
+            if (rank == 0)   // both CTAs' bytes
+              mbar_arrive_expect_tx(&full[stage], 2 * (A_STAGE_BYTES + n_box * p.tok_box * BK * 2));
             const uint32_t bar = mapa_shared(&full[stage], 0);
             tma_load_2d_pair(a_dst, &tmB, bar, kb * BK, b_first);   // weights: the MMA's A
             if constexpr (EPI == EPI_SWIGLU)
               tma_load_2d_pair(a_dst + 64 * BK * 2, &tmB, bar, kb * BK, ti.b_row2 + (int)rank * 64);
-            tma_load_2d_pair(b_dst, &tmA, bar, kb * BK, ti.m0 + (int)rank * (ti.n_mma >> 1));   // tokens: B
+            const int t0 = ti.m0 + (int)rank * (ti.n_mma >> 1);
+            for (int bx = 0; bx < n_box; ++bx)
+              tma_load_2d_pair(b_dst + bx * p.tok_box * BK * 2, &tmA, bar, kb * BK, t0 + bx * p.tok_box);
           } else if constexpr (CG == 2) {
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);   // both CTAs' bytes
             const uint32_t bar = mapa_shared(&full[stage], 0);
@@ -595,8 +604,12 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         // half of gate values to the up warp of its group and takes the up
         // warp's first half of up values (shared memory), then each warp writes
         // act = bf16(silu(gate) * up) for its 16 tokens x 32 features.
-        const bool ok = !aborted && mbar_wait(&tfull[acc], acc_phase, wc);
-        if (named_barrier_any(1, EW * 32, !ok)) aborted = true;   // the four warps decide together
+        // The hand-over of chunk kc completes xbar[kc & 1] (one arrival per warp)
+        // for the (kc >> 1)-th time; a warp writes that buffer again two chunks
+        // later, after the hand-over in between has completed, i.e. after
+        // every warp has read it.  All waits are bounded: a warp that gives up
+        // leaves the others to give up at their next hand-over.
+        if (!aborted && !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, wc))) aborted = true;
         if (aborted) continue;
         tc_fence_after();
         const int fg = q & 1, th = q >> 1;
@@ -613,7 +626,12 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
           float* take = T + (th ^ 1) * 512;
 #pragma unroll
           for (int j = 0; j < 16; ++j) give[j * 32 + lane] = __uint_as_float(th == 0 ? r[j + 16] : r[j]);
-          named_barrier_sync(1, EW * 32);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xbar[kc & 1]);
+          if (!__all_sync(0xffffffffu, mbar_wait(&xbar[kc & 1], (kc >> 1) & 1, wc))) {
+            aborted = true;
+            break;
+          }
           float a[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -627,6 +645,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
           for (int j = 0; j < 16; ++j)
             if (j < nj) dst[(size_t)j * p.ldo] = __float2bfloat16_rn(a[j]);
         }
+        if (aborted) continue;
       } else {
         // MERGE_MLP: lane = output feature, column = permuted row; a token's 32
         // features of this warp are one 128-byte segment of its stream row.
@@ -825,10 +844,10 @@ int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b
   // grouped expert GEMMs on CTA pairs run swapped (weights on the M side)
   const bool swap = cg == 2 && p.grouped && (epi == EPI_SWIGLU || epi == EPI_MERGE_MLP);
   if (swap && bn != 256) return ZAYA_ERR_UNSUPPORTED;
-  // swapped: a token box as tall as any tile's half of N can be (<= 128, and
-  // n_mma / 2 <= round16(a_rows) / 2 since an expert holds at most a_rows tokens)
+  // swapped: token boxes of 16 rows (two 128-byte swizzle atoms), as many as
+  // a tile's half of N needs
   GemmParams q = p;
-  q.tok_box = swap ? (a_rows >= 128 ? 128 : ((a_rows + 15) & ~15)) : BM;
+  q.tok_box = swap ? 16 : BM;
   CUtensorMap ma, mb;
   int rc = make_tmap_bf16(&ma, A, (uint64_t)a_rows, (uint64_t)p.K, (uint32_t)q.tok_box);
   if (rc) return rc;

@@ -40,7 +40,7 @@ struct GemmParams {
   const float* row_w;        // MERGE_MLP: per-token expert weight
   void* tap_bf16;            // MERGE_*: optional bf16 [tokens, N] contribution tap
   float* tap_f32;            // MERGE_ATTN: optional fp32 [tokens, N] layer_mid tap
-  int tok_box;               // set by launch_gemm: swapped tiles' token box rows (16..128)
+  int tok_box;               // set by launch_gemm: swapped tiles' token box rows (16)
 };
 
 // Encodes a 2-D bf16 tensor map (rows x cols, row-major) with a box of
