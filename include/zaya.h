@@ -64,7 +64,7 @@
 extern "C" {
 #endif
 
-#define ZAYA_ABI_VERSION 2
+#define ZAYA_ABI_VERSION 3
 
 enum zaya_status {
   ZAYA_OK = 0,
@@ -108,6 +108,12 @@ typedef struct zaya_config {
                                 (k=2, conv_w [C,2], conv_b) then conv_qk_grouped (k=2, G groups,
                                 conv2_w, conv2_b) as the zaya page's printout lists them; the
                                 kernels take one group per q / k head (G = n_q + n_kv, 10 on ZAYA1-8B) */
+  int32_t kv_ring;           /* 0: position p of a sequence in cache slot p (cache_cap bounds the
+                                positions).  1: slot p % cache_cap, a window ring: decode needs
+                                cache_cap >= window and keeps only the last cache_cap positions,
+                                so a sequence decodes past cache_cap with a window-sized cache
+                                (the pages' decode reads the window only: zaya page, "Queries and
+                                keys are convolved ..."; every block must slide: sliding_period 0) */
   float rope_theta;          /* inv_freq[i] = rope_theta^(-2i/rot_dim) */
   float rms_eps;             /* RMSNorm epsilon (1e-5) */
   float qk_norm_eps;         /* q,k -> x * sqrt(d) / max(|x|, qk_norm_eps) */
@@ -196,9 +202,11 @@ size_t zaya_stack_workspace_size(const zaya_config* cfg, int32_t mode, int32_t B
  *                   (+ router_state_in * router_state_scale); the next
  *                   block's router_state_in.  Must not alias router_state_in.
  *  state            K/V of every position written to the caches at 0..S-1
- *                   (cache_cap >= S); cache_len[b] = S; conv_state and
- *                   prev_hs set from the last two tokens.  Continuing a
- *                   padded prefill in decode is not supported.
+ *                   (cache_cap >= S); with kv_ring, the last min(S, cache_cap)
+ *                   positions p at slots p % cache_cap (any S; the attention
+ *                   reads the prompt's keys from the workspace); cache_len[b]
+ *                   = S; conv_state and prev_hs set from the last two tokens.
+ *                   Continuing a padded prefill in decode is not supported.
  *  taps             NULL or optional outputs.
  *  workspace        >= zaya_workspace_size(cfg, ZAYA_PREFILL, B, S) bytes,
  *                   256-byte aligned.  Its first word is the device status. */
@@ -211,8 +219,10 @@ int zaya_block_prefill(const zaya_config* cfg, const zaya_block_weights* w, int3
 /* One new token for each of B sequences through a block with a cache.
  *  hidden fp32 [B, H] in/out.  router_state_in / _out fp32 [B, R].
  *  The token of sequence b sits at position cache_len[b]; it attends over
- *  positions max(0, t - window + 1) .. t; requires cache_len[b] < cache_cap
- *  for every b, checked on the device: if any sequence fails it, the status
+ *  positions max(0, t - window + 1) .. t; requires 0 <= cache_len[b] and,
+ *  without kv_ring, cache_len[b] < cache_cap for every b (with kv_ring the
+ *  token's K/V go to slot cache_len[b] % cache_cap, and cache_cap >= window
+ *  is checked on the host), checked on the device: if any sequence fails it, the status
  *  word records ZAYA_ERR_DEVICE_RANGE and no sequence's caches, conv_state,
  *  prev_hs or cache_len are written (hidden and the router state out are
  *  then unspecified).

@@ -37,6 +37,7 @@ class BlockConfig:
     v_delayed: int = 1           # half of each value head from token t-1
     sliding_period: int = 0      # 0: every block slides over `window` keys; P > 0: only blocks with
     sliding_phase: int = 0       # block % P == phase slide, the others attend to every earlier token
+    kv_ring: int = 0             # 1: K/V caches as window rings (slot = position % cache_cap)
     vocab: int = 0
     emb_mult: float = 1.0
     emb_shift: float = 0.0

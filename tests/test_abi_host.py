@@ -63,7 +63,7 @@ def test_struct_layout_matches_header(tmp_path):
 
 
 def test_status_strings_and_version():
-    assert ZB.zaya_abi_version() == 2
+    assert ZB.zaya_abi_version() == 3
     for code in range(8):
         assert isinstance(ZB.zaya_status_string(code), str)
     assert ZB.zaya_status_string(0) == "ok"
@@ -169,3 +169,32 @@ def test_noalloc_checks_arguments_before_enqueueing_anything():
     rc = L.zaya_block_decode_noalloc(C.byref(big), C.byref(w), 1, 4096, fake, fake, C.c_void_p(512), C.byref(st),
                                      None, None)
     assert rc == ZB._abi.ZAYA_ERR_WORKSPACE                    # beyond the fixed scratch
+
+
+def test_window_ring_arguments():
+    """kv_ring: a window ring needs every block to slide (no full-attention
+    blocks) and a cache of at least a window; both are checked before any
+    launch."""
+    cfg = get_config("tiny")
+    assert ZB.zaya_workspace_size(ZB.make_config(cfg.with_(kv_ring=1)), ZB.ZAYA_DECODE, 2, 1) > 0
+    assert ZB.zaya_workspace_size(ZB.make_config(cfg.with_(kv_ring=2)), ZB.ZAYA_DECODE, 2, 1) == 0
+    hybrid = cfg.with_(kv_ring=1, sliding_period=2, sliding_phase=1)
+    assert ZB.zaya_workspace_size(ZB.make_config(hybrid), ZB.ZAYA_DECODE, 2, 1) == 0
+    # the prefill workspace of a ring also holds the prompt's linear K / V
+    assert (ZB.zaya_workspace_size(ZB.make_config(cfg.with_(kv_ring=1)), ZB.ZAYA_PREFILL, 1, 64)
+            > ZB.zaya_workspace_size(ZB.make_config(cfg), ZB.ZAYA_PREFILL, 1, 64))
+    c = ZB.make_config(cfg.with_(kv_ring=1))
+    L = _abi.lib()
+    w = _abi.zaya_block_weights()
+    for name in _abi.WEIGHT_FIELDS:
+        setattr(w, name, 4096)
+    st = _abi.zaya_block_state()
+    st.k_cache = st.v_cache = st.conv_state = st.prev_hs = st.cache_len = 4096
+    st.cache_cap = cfg.window - 1
+    fake = C.c_void_p(256)
+    rc = L.zaya_block_decode(C.byref(c), C.byref(w), 1, 2, fake, fake, C.c_void_p(512), C.byref(st), None,
+                             fake, 1 << 20, None)
+    assert rc == ZB._abi.ZAYA_ERR_INVALID_ARG                  # ring shorter than the window
+    rc = L.zaya_block_prefill(C.byref(c), C.byref(w), 1, 1, 8, fake, None, fake, C.c_void_p(512), C.byref(st), None,
+                              fake, 1 << 20, None)
+    assert rc == ZB._abi.ZAYA_ERR_INVALID_ARG                  # the same in prefill

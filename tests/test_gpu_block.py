@@ -273,3 +273,62 @@ def test_two_stage_conv_decode_after_prefill(name):
     assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, lo
     k_new = st["k_cache"][:, :, S].float().cpu().numpy()
     assert Hn.rel_max(k_new, ref["state"]["k_cache"][:, :, S]) <= 2e-2
+
+
+def _ring_matches_linear(lin, ring, n, cap):
+    """The ring's kept rows (positions max(0, n - cap) .. n-1 at slots p % cap)
+    equal the linear cache's rows, bit for bit; the other state too."""
+    for p in range(max(0, n - cap), n):
+        for key in ("k_cache", "v_cache"):
+            assert torch.equal(lin[key][:, :, p], ring[key][:, :, p % cap]), (key, p)
+    for key in ("cache_len", "conv_state", "prev_hs"):
+        assert torch.equal(lin[key], ring[key]), key
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill_4k"])
+def test_window_ring_cache_matches_linear_cache(name):
+    """kv_ring: a window-sized cache that keeps position p at slot p % cap.
+    A prompt longer than the ring, then decode steps across the ring's wrap:
+    every output equals the linear-cache run bit for bit (the same kernels
+    add the same keys in the same order; only the rows' addresses differ),
+    and the kept K / V rows equal the linear cache's.  The decode outputs are
+    also held against the oracle's decode on a dense state rebuilt from the
+    ring (positions outside the window are not read)."""
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config(name)
+    S, steps = (50, 5) if name == "tiny" else (300, 3)
+    if name == "prefill_4k":
+        cfg = cfg.with_(window=128)
+    cfg = cfg.with_(seq=S)
+    cap = cfg.window
+    rcfg = cfg.with_(kv_ring=1)
+    W = gen_block_weights(cfg)
+    Wd = Hn.dev_weights(W)
+    inp = gen_prefill_inputs(cfg.with_(seq=S + steps))
+    x, rin = inp["x"], inp["router_state_in"]
+    r_at = (lambda i: None) if rin is None else (lambda i: rin[:, i])
+    lin = Hn.new_state(cfg, 1, S + steps)
+    ring = Hn.new_state(cfg, 1, cap)
+    a = Hn.gpu_prefill(cfg, Wd, x[:, :S], None, None if rin is None else rin[:, :S], state=lin, taps=False)
+    b = Hn.gpu_prefill(rcfg, Wd, x[:, :S], None, None if rin is None else rin[:, :S], state=ring, taps=False)
+    assert torch.equal(a["layer_output"], b["layer_output"])
+    assert torch.equal(a["router_state"], b["router_state"])
+    _ring_matches_linear(lin, ring, S, cap)
+    for k in range(steps):
+        n = S + k
+        host = {key: v.cpu().clone() for key, v in ring.items()}
+        dense = dict(host)
+        for key in ("k_cache", "v_cache"):
+            full = torch.zeros(host[key].shape[0], host[key].shape[1], n + 1, host[key].shape[3], dtype=host[key].dtype)
+            for p in range(max(0, n - cap), n):
+                full[:, :, p] = host[key][:, :, p % cap]
+            dense[key] = full
+        da = Hn.gpu_decode(cfg, Wd, x[:, n], lin, r_at(n))
+        db = Hn.gpu_decode(rcfg, Wd, x[:, n], ring, r_at(n))
+        assert torch.equal(da["layer_output"], db["layer_output"]), k
+        _ring_matches_linear(lin, ring, n + 1, cap)
+        g_cls = Hn.gpu_classes(cfg, db)
+        ref = Z.block_decode(cfg, Hn.eff(W), x[:, n], dense, r_at(n), force_cls=g_cls)
+        lo = Hn.report("layer_output", db["layer_output"].numpy(), ref["layer_output"])
+        assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, (k, lo)

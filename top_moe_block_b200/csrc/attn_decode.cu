@@ -45,13 +45,16 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
   // A position outside the cache (already reported by the conv kernel) gives
   // an empty key range, so nothing outside the cache is read.
   const int t_raw = p.cache_len[b];
-  const int t = (t_raw >= 0 && t_raw < p.cap) ? t_raw : -1;
+  const int t = (t_raw >= 0 && (p.ring || t_raw < p.cap)) ? t_raw : -1;
   const int lo = max(0, t - p.window + 1);
   const int c_begin = lo + chunk * p.chunk_keys;
   const int c_end = min(t + 1, c_begin + p.chunk_keys);
   const int per_warp = p.chunk_keys / kWarps;
   const int w_begin = c_begin + warp * per_warp;
   const int w_end = min(c_end, w_begin + per_warp);
+  // cache row of key w_begin: a window ring keeps position p at slot p % cap;
+  // the warp's keys span fewer than cap positions, so they wrap at most once
+  const int row0 = p.ring && w_begin < w_end ? w_begin % p.cap : w_begin;
   const float sl2 = p.scale * 1.4426950408889634f;
 
   // Q fragments: row gid of A is query head g * REP + gid (zero from REP on)
@@ -77,7 +80,9 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
       const int r = i / CPR, c = i % CPR;
       const int key = key0 + r;
       const bool ok = key < w_end;
-      const size_t src = (size_t)(ok ? key : 0) * D + c * 8;
+      int row = row0 + (key - w_begin);
+      if (row >= p.cap) row -= p.cap;
+      const size_t src = (size_t)(ok ? row : 0) * D + c * 8;
       const int dst = r * D + ((c ^ (r & 7)) * 8);
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dk + dst)), "l"(Kg + src),
                    "r"(ok ? 16 : 0)

@@ -130,23 +130,24 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
   const size_t ld = (size_t)p.n_qkv;
 
   const int pos = p.decode ? p.cache_len[b] : s;
-  // Decode appends at cache_len[b]: a position outside the cache is a fault.
+  // Decode appends at cache_len[b]: a position outside the cache is a fault
+  // (a window ring takes any position >= 0, at slot pos % cache_cap).
   // Every CTA checks all sequences, so a call with one bad position writes no
   // sequence's cache, conv_state or prev_hs (the status word then makes the
   // rest of the block skip its work, and cache_len stays as it was).
+  const bool ring = p.decode && p.ring;
+  auto outside = [&](int c) { return c < 0 || (!ring && c >= p.cache_cap); };
   bool bad = false;
   if (p.decode) {
-    for (int i = threadIdx.x; i < p.B; i += blockDim.x) {
-      const int c = p.cache_len[i];
-      bad |= (c < 0 || c >= p.cache_cap);
-    }
+    for (int i = threadIdx.x; i < p.B; i += blockDim.x) bad |= outside(p.cache_len[i]);
   } else {
-    bad = pos < 0 || pos >= p.cache_cap;
+    bad = outside(pos);
   }
   if (__syncthreads_or(bad)) {
-    if (threadIdx.x == 0 && (pos < 0 || pos >= p.cache_cap)) set_status(p.status, ZAYA_ERR_DEVICE_RANGE);
+    if (threadIdx.x == 0 && outside(pos)) set_status(p.status, ZAYA_ERR_DEVICE_RANGE);
     return;
   }
+  const int slot = ring ? pos % p.cache_cap : pos;   // the cache row of this position
   Pre<D> pre;
   pre.qkv = qkv;
   pre.ld = ld;
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
         for (int i = 0; i < DPL; ++i) t[i] = f2bf(y[i]);
       }
     } else {
-      dst = static_cast<__nv_bfloat16*>(p.k_cache) + (((size_t)b * nkv + head) * p.cache_cap + pos) * D + lane * DPL;
+      dst = static_cast<__nv_bfloat16*>(p.k_cache) + (((size_t)b * nkv + head) * p.cache_cap + slot) * D + lane * DPL;
     }
 #pragma unroll
     for (int i = 0; i < DPL; ++i) dst[i] = f2bf(y[i]);
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
     const int vc0 = nq * D + nkv * D;
     const int vd0 = vc0 + nkv * (D / 2);
     __nv_bfloat16* dst =
-        static_cast<__nv_bfloat16*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + pos) * D + lane * DPL;
+        static_cast<__nv_bfloat16*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + slot) * D + lane * DPL;
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
       const int j = lane * DPL + i;
@@ -688,6 +689,45 @@ int launch_cca(const CcaParams& p, cudaStream_t st) {
     launch_k(cca_kernel<64>, dim3(tokens), dim3(threads), 0, st, nullptr, 0, p);
   else
     return ZAYA_ERR_UNSUPPORTED;
+  return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
+}
+
+
+namespace {
+
+// One thread per 16-byte piece of a kept row: K and V rows of positions
+// max(0, S - cap) .. S-1 of every (sequence, kv head).
+__global__ void __launch_bounds__(256) ring_store_kernel(const uint4* __restrict__ k_lin, const uint4* __restrict__ v_lin,
+                                                         uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                                                         int BG, int S, int cap, int vpr, int* status) {
+  griddep_begin();
+  if (status_peek(status)) return;
+  const int keep = S < cap ? S : cap;
+  const long total = (long)BG * keep * vpr;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+    const int v = (int)(i % vpr);
+    const long r = i / vpr;
+    const int bg = (int)(r / keep);
+    const int pos = S - keep + (int)(r % keep);
+    const size_t src = ((size_t)bg * S + pos) * vpr + v;
+    const size_t dst = ((size_t)bg * cap + pos % cap) * vpr + v;
+    k_cache[dst] = k_lin[src];
+    v_cache[dst] = v_lin[src];
+  }
+}
+
+}  // namespace
+
+int launch_ring_store(const void* k_lin, const void* v_lin, void* k_cache, void* v_cache, int B, int n_kv, int S,
+                      int cap, int d, int* status, cudaStream_t st) {
+  if (B <= 0 || S <= 0) return ZAYA_OK;
+  if (cap <= 0 || d % 8) return ZAYA_ERR_UNSUPPORTED;
+  const int vpr = d / 8;
+  const long total = (long)B * n_kv * (S < cap ? S : cap) * vpr;
+  const int blocks = (int)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
+  launch_k(ring_store_kernel, dim3(blocks), dim3(256), 0, st, nullptr, 0, static_cast<const uint4*>(k_lin),
+           static_cast<const uint4*>(v_lin), static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), B * n_kv, S,
+           cap, vpr, status);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 

@@ -97,6 +97,7 @@ struct CcaParams {
   int cca_res, v_delayed;
   float theta, eps;
   int decode;             // 1: one token per sequence, history from conv_state
+  int ring;               // decode: 1 = the caches are window rings (position p at slot p % cache_cap)
   int* status;
   int* zero_words;        // prefill: words CTA 0 clears for the next kernel (attention's merge counters), or null
   int n_zero_words;
@@ -104,6 +105,11 @@ struct CcaParams {
   float inv_freq[64];     // RoPE inverse frequencies theta^(-2i/rot), i < rot/2 (fp32)
 };
 int launch_cca(const CcaParams& p, cudaStream_t st);
+// Window-ring prefill: positions max(0, S - cap) .. S-1 of the linear K / V
+// (bf16 [B, n_kv, S, d]) into ring slots p % cap of the caches
+// (bf16 [B, n_kv, cap, d]).
+int launch_ring_store(const void* k_lin, const void* v_lin, void* k_cache, void* v_cache, int B, int n_kv, int S,
+                      int cap, int d, int* status, cudaStream_t st);
 
 // The two-stage conv_qk's grouped stage (with its depthwise stage fused in):
 // y fp32 [rows, C], one group per q / k head.
@@ -150,6 +156,7 @@ struct DecodeAttnParams {
   float* part;            // workspace partials
   int B, cap, n_q, n_kv, d, window, n_chunks;
   int chunk_keys;         // keys per CTA (a multiple of 256)
+  int ring;               // 1: position p at slot p % cap
   float scale;
 };
 // Key chunks a head's decode attention may use for a window (256 keys per

@@ -129,6 +129,8 @@ int check_config(const zaya_config* c) {
   if (c->rms_eps < 0.f || c->qk_norm_eps <= 0.f) return ZAYA_ERR_INVALID_ARG;
   if (c->sliding_period < 0 || (c->sliding_period > 0 && (c->sliding_phase < 0 || c->sliding_phase >= c->sliding_period)))
     return ZAYA_ERR_INVALID_ARG;
+  // a window ring needs a window on every block
+  if (c->kv_ring != 0 && (c->kv_ring != 1 || c->sliding_period > 0)) return ZAYA_ERR_INVALID_ARG;
   return ZAYA_OK;
 }
 
@@ -175,7 +177,7 @@ int check_weights(const zaya_block_weights* w, const zaya_config* c) {
 
 struct Ws {
   size_t status, a_in, qkv, q, premix, m_in, logits, cls, w, pos, perm, group_off, mt_start, xperm, act, part, rpart,
-      wsplit, slot, ccount, convy, loany, total;
+      wsplit, slot, ccount, convy, loany, kvlin, total;
 };
 
 Ws plan(const zaya_config& c, int mode, int B, int S) {
@@ -207,6 +209,9 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.ccount = o; o += up((size_t)(d.E + 2) * 4);
   w.convy = o; o += c.conv_groups > 0 ? up(M * d.C * 4) : 0;   // the two-stage conv's output (fp32)
   w.loany = o; o += up((size_t)router_split_blocks(d.R, d.E) * 4);
+  // window-ring prefill: the prompt's K and V (bf16 [B, n_kv, S, d] each) for
+  // the attention; the ring keeps the last cache_cap positions
+  w.kvlin = o; o += (c.kv_ring && mode == ZAYA_PREFILL) ? 2 * up(M * d.nkv * d.d * 2) : 0;
   w.total = o;
   return w;
 }
@@ -359,7 +364,8 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
   ZAYA_TRY(check_weights(w, cfg));
   if (B <= 0 || S <= 0 || !hidden || !rout || !ws) return ZAYA_ERR_INVALID_ARG;
   if (block_idx < 0 || (block_idx > 0 && !rin) || rin == rout) return ZAYA_ERR_INVALID_ARG;
-  ZAYA_TRY(check_state(state, S));
+  // a window ring holds any prompt's last cache_cap positions, and at least a window
+  ZAYA_TRY(check_state(state, cfg->kv_ring ? block_window(*cfg, block_idx) : S));
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) || !a16(hidden) || !a16(rout)) return ZAYA_ERR_MISALIGNED;
   if (taps && taps->attention_queries && !a16(taps->attention_queries)) return ZAYA_ERR_MISALIGNED;
   const zaya_config& c = *cfg;
@@ -372,6 +378,16 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
   int* status = at<int>(ws, L.status);
   void* a_in = at<void>(ws, L.a_in);
   void* qkv = at<void>(ws, L.qkv);
+  // K / V of the prompt for the attention: the caches themselves, or, for a
+  // window ring, linear copies in the workspace stored into the ring after it
+  void* kc = state->k_cache;
+  void* vc = state->v_cache;
+  int kcap = state->cache_cap;
+  if (c.kv_ring) {
+    kc = at<void>(ws, L.kvlin);
+    vc = at<uint8_t>(ws, L.kvlin) + up((size_t)M * d.nkv * d.d * 2);
+    kcap = S;
+  }
   ZAYA_STAGE("rmsnorm_attn", 1, launch_rmsnorm(hidden, 1, 0, w->ln1_w, a_in,
                                                taps ? taps->attention_norm_output : nullptr, M, d.H, c.rms_eps,
                                                nullptr, 0, st));
@@ -395,7 +411,7 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     p.conv_y = c.conv_groups > 0 ? at<float>(ws, L.convy) : nullptr;
     p.qkv = qkv; p.n_qkv = d.n_qkv; p.conv_w = w->conv_w; p.conv_b = w->conv_b; p.k_temp = w->k_temp;
     p.mask = mask; p.q_out = at<void>(ws, L.q); p.tap_q = taps ? taps->attention_queries : nullptr;
-    p.k_cache = state->k_cache; p.v_cache = state->v_cache; p.cache_cap = state->cache_cap;
+    p.k_cache = kc; p.v_cache = vc; p.cache_cap = kcap;
     p.cache_len = state->cache_len; p.conv_state = state->conv_state; p.prev_hs = state->prev_hs; p.a_in = a_in;
     p.B = B; p.S = S; p.H = d.H; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.rot = c.rot_dim;
     p.cca_res = c.cca_mean_residual; p.v_delayed = c.v_delayed; p.theta = c.rope_theta; p.eps = c.qk_norm_eps;
@@ -409,14 +425,17 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
   {
     AttnParams p{};
     p.ctr_cleared = 1;
-    p.q = at<void>(ws, L.q); p.k_cache = state->k_cache; p.v_cache = state->v_cache; p.mask = mask;
+    p.q = at<void>(ws, L.q); p.k_cache = kc; p.v_cache = vc; p.mask = mask;
     p.out = at<void>(ws, L.premix);
-    p.B = B; p.S = S; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = window;
+    p.B = B; p.S = S; p.cap = kcap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = window;
     p.scale = d.scale;
     p.part = at<void>(ws, L.part);
     p.part_bytes = attn_prefill_ws_bytes(B, S, window, d.nq, d.nkv, d.d);
     ZAYA_STAGE("attention", 1, launch_attn_prefill_tc(p, status, st));
   }
+  if (c.kv_ring)
+    ZAYA_STAGE("ring_store", 1, launch_ring_store(kc, vc, state->k_cache, state->v_cache, B, d.nkv, S,
+                                                  state->cache_cap, d.d, status, st));
   return block_tail(c, d, w, block_idx, M, hidden, rin, rout, taps, ws, L, nullptr, mask, sms, st);
 }
 
@@ -429,7 +448,7 @@ int check_decode_args(const zaya_config* cfg, const zaya_block_weights* w, int b
   ZAYA_TRY(check_weights(w, cfg));
   if (B <= 0 || !hidden || !rout) return ZAYA_ERR_INVALID_ARG;
   if (block_idx < 0 || (block_idx > 0 && !rin) || rin == rout) return ZAYA_ERR_INVALID_ARG;
-  ZAYA_TRY(check_state(state, 1));
+  ZAYA_TRY(check_state(state, cfg->kv_ring ? block_window(*cfg, block_idx) : 1));
   if (!a16(hidden) || !a16(rout)) return ZAYA_ERR_MISALIGNED;
   if (taps && taps->attention_queries && !a16(taps->attention_queries)) return ZAYA_ERR_MISALIGNED;
   return ZAYA_OK;
@@ -477,7 +496,7 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
     p.cache_len = state->cache_len; p.conv_state = state->conv_state; p.prev_hs = state->prev_hs; p.a_in = a_in;
     p.B = B; p.S = 1; p.H = d.H; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.rot = c.rot_dim;
     p.cca_res = c.cca_mean_residual; p.v_delayed = c.v_delayed; p.theta = c.rope_theta; p.eps = c.qk_norm_eps;
-    p.decode = 1; p.status = status;
+    p.decode = 1; p.ring = c.kv_ring; p.status = status;
     fill_inv_freq(p.inv_freq, c.rot_dim, c.rope_theta);
     ZAYA_STAGE("cca", 1, launch_cca(p, st));
   }
@@ -487,6 +506,7 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
     p.out = at<void>(ws, L.premix); p.part = at<float>(ws, L.part);
     const int window = block_window(c, block_idx);
     p.B = B; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = window;
+    p.ring = c.kv_ring;
     const int span = window < state->cache_cap ? window : state->cache_cap;
     decode_attn_split(span, decode_chunks_any(c), &p.n_chunks, &p.chunk_keys);
     p.scale = d.scale;
