@@ -71,6 +71,36 @@ def round_bf16(x) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+E4M3_MAX = 448.0   # the largest finite OCP FP8 E4M3 value, 1.75 * 2^8
+
+
+def round_e4m3(x) -> np.ndarray:
+    """Round to the nearest OCP FP8 E4M3 value (4 exponent bits, bias 7, 3
+    mantissa bits; normals down to 2^-6, subnormals k * 2^-9), ties to an
+    even mantissa, magnitudes beyond the largest finite value saturating to
+    +-448 (the fp8 KV cache of the NVFP4 README's serving command,
+    "--kv-cache-dtype fp8", stores keys and values in this format).
+
+    The step between neighbours is 2^(e - 3) in the binade [2^e, 2^(e+1))
+    for e >= -6 and 2^-9 below it; rounding |x| / step to an integer (ties
+    to even) and scaling back lands on the nearest value, a carry into the
+    next binade included."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))      # a = f * 2^ex, f in [0.5, 1)
+    e = np.maximum(ex - 1, -6)
+    step = np.ldexp(1.0, (e - 3).astype(np.int64))
+    q = np.round(a / step) * step                    # numpy rounds half to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.where(np.isnan(x), np.nan, np.copysign(q, x))
+
+
+def cache_kv(cfg, t):
+    """Keys / values as the cache holds them: bf16, or with ``cfg.kv_fp8``
+    the bf16 value rounded on to E4M3."""
+    return round_e4m3(t) if getattr(cfg, "kv_fp8", 0) else t
+
+
 # ---------------------------------------------------------------------------
 # elementwise pieces
 # ---------------------------------------------------------------------------
@@ -414,8 +444,10 @@ def block_prefill(cfg, W, x, attn_mask=None, router_state_in=None, block_idx=Non
                           ("attention_keys", k.transpose(1, 0, 2)), ("attention_values", v.transpose(1, 0, 2)),
                           ("attention_premix", premix), ("attention_output", attn_out), ("layer_mid", h)):
             taps[name].append(val)
-        state["k_cache"].append(k.transpose(1, 0, 2))
-        state["v_cache"].append(v.transpose(1, 0, 2))
+        # the prompt attended over its bf16 keys and values above; the cache
+        # keeps them in its own format (E4M3 with kv_fp8)
+        state["k_cache"].append(cache_kv(cfg, k).transpose(1, 0, 2))
+        state["v_cache"].append(cache_kv(cfg, v).transpose(1, 0, 2))
         last2 = np.concatenate([hist, u], axis=0)[-2:]          # pre-conv q||k at S-2, S-1
         state["conv_state"].append(last2.T)                     # [C, 2]
         state["prev_hs"].append(a_in[-1])
@@ -501,8 +533,10 @@ def block_decode(cfg, W, x, state, router_state_in=None, block_idx=None, force_c
         v = _values(cfg, vc[b:b + 1], vd_prev[b:b + 1])
         k = round_bf16(k)
         v = round_bf16(v)
-        kc[b, :, t] = k[0]
-        vcache[b, :, t] = v[0]
+        # the token's keys / values go into the cache first, in its format,
+        # and the attention reads every position from the cache
+        kc[b, :, t] = cache_kv(cfg, k[0])
+        vcache[b, :, t] = cache_kv(cfg, v[0])
         window = block_window(cfg, bidx)
         lo = max(0, t - window + 1)
         kpos = np.arange(lo, t + 1)

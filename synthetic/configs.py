@@ -38,6 +38,7 @@ class BlockConfig:
     sliding_period: int = 0      # 0: every block slides over `window` keys; P > 0: only blocks with
     sliding_phase: int = 0       # block % P == phase slide, the others attend to every earlier token
     kv_ring: int = 0             # 1: K/V caches as window rings (slot = position % cache_cap)
+    kv_fp8: int = 0              # 1: K/V caches hold OCP FP8 E4M3 (the prompt attends over bf16)
     vocab: int = 0
     emb_mult: float = 1.0
     emb_shift: float = 0.0

@@ -661,3 +661,84 @@ def test_conv_two_stage_block_reach_and_decode():
                            force_cls=o["expert_cls"][:, :S + 1])
     np.testing.assert_allclose(dec["layer_output"], full["layer_output"][:, S], rtol=1e-9, atol=1e-9)
     np.testing.assert_allclose(dec["attention_keys"], full["attention_keys"][:, :, S], rtol=1e-9, atol=1e-9)
+
+
+# ---------------------------------------------------------------- fp8 KV cache
+
+def _e4m3_table():
+    """Every finite OCP FP8 E4M3 code and its value, decoded from the format's
+    definition: sign bit, 4 exponent bits (bias 7), 3 mantissa bits;
+    exponent 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN (no infinities)."""
+    codes, vals = [], []
+    for code in range(256):
+        s, e, m = code >> 7, (code >> 3) & 15, code & 7
+        if e == 15 and m == 7:
+            continue
+        v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+        codes.append(code)
+        vals.append(-v if s else v)
+    return np.array(codes), np.array(vals)
+
+
+def test_e4m3_rounding_against_the_format():
+    """round_e4m3 against the code table: every finite value is a fixed point;
+    a point just inside either neighbour's half goes to that neighbour; an
+    exact midpoint goes to the neighbour with the even mantissa; magnitudes
+    past 448 saturate; the largest value is 448 and the smallest subnormal
+    2^-9 (NVFP4 README, "--kv-cache-dtype fp8": keys and values stored in
+    8-bit floating point)."""
+    codes, vals = _e4m3_table()
+    assert vals.max() == 448.0 and vals[(vals > 0)].min() == 2.0 ** -9
+    np.testing.assert_array_equal(Z.round_e4m3(vals), vals)
+    pos = np.unique(vals[vals >= 0])
+    code_of = {v: c for c, v in zip(codes, vals) if v >= 0}
+    for lo, hi in zip(pos[:-1], pos[1:]):
+        mid = 0.5 * (lo + hi)
+        gap = hi - lo
+        assert Z.round_e4m3(mid - gap * 1e-3) == lo
+        assert Z.round_e4m3(mid + gap * 1e-3) == hi
+        even = lo if code_of[lo] % 2 == 0 else hi
+        assert Z.round_e4m3(mid) == even, (lo, hi)
+        assert Z.round_e4m3(-mid) == -even
+    for big in (448.5, 463.9, 464.0, 500.0, 1e9):
+        assert Z.round_e4m3(big) == 448.0 and Z.round_e4m3(-big) == -448.0
+
+
+def test_fp8_cache_prefill_and_decode(tiny):
+    """kv_fp8: the prompt attends over its bf16 keys / values, so every
+    prefill output is the bf16 cache's; the cache then holds E4M3 values
+    within half a step of the bf16 ones; a decode step computes its token's
+    keys as the bf16 run does and writes them in E4M3 before attending over
+    the cache, so its attention differs from the bf16 decode's by about
+    E4M3's precision (three mantissa bits), no more."""
+    cfg, W, inp, out = tiny
+    c8 = cfg.with_(kv_fp8=1)
+    x, r = inp["x"], inp["router_state_in"]
+    S = cfg.seq
+    p16 = Z.block_prefill(cfg, W, x[:, :S - 1], None, r[:, :S - 1])
+    p8 = Z.block_prefill(c8, W, x[:, :S - 1], None, r[:, :S - 1])
+    for key in ("layer_output", "router_state", "attention_output", "mlp_output"):
+        np.testing.assert_array_equal(p8[key], p16[key])
+    for key in ("k_cache", "v_cache"):
+        c16, c8v = p16["state"][key], p8["state"][key]
+        np.testing.assert_array_equal(Z.round_e4m3(c8v), c8v)
+        step = np.ldexp(1.0, np.maximum(np.frexp(np.abs(c16) + (c16 == 0))[1] - 1, -6) - 3)
+        assert (np.abs(c8v - c16) <= 0.5 * step + 1e-300).all()
+        assert (c8v != c16).any()
+    cap = S + 2
+
+    def state_of(st):
+        kc = np.zeros((1, cfg.n_kv, cap, cfg.head_dim))
+        vc = np.zeros_like(kc)
+        kc[:, :, :S - 1] = st["k_cache"]
+        vc[:, :, :S - 1] = st["v_cache"]
+        return dict(k_cache=kc, v_cache=vc, conv_state=st["conv_state"], prev_hs=st["prev_hs"],
+                    cache_len=st["cache_len"])
+
+    d8 = Z.block_decode(c8, W, x[:, S - 1], state_of(p8["state"]), r[:, S - 1])
+    d16 = Z.block_decode(cfg, W, x[:, S - 1], state_of(p16["state"]), r[:, S - 1])
+    # the token's own K / V entered the cache rounded to E4M3
+    np.testing.assert_array_equal(d8["state"]["k_cache"][:, :, S - 1], Z.round_e4m3(d16["state"]["k_cache"][:, :, S - 1]))
+    np.testing.assert_array_equal(d8["attention_keys"], d16["attention_keys"])
+    rel = np.abs(d8["attention_premix"] - d16["attention_premix"]).max() / np.abs(d16["attention_premix"]).max()
+    assert 1e-4 < rel < 0.1, rel
