@@ -106,12 +106,13 @@ def stage_work_decode(cfg, routed, distinct):
     B, H, R, E1, I = cfg.batch, cfg.hidden, cfg.router_hidden, cfg.n_experts + 1, cfg.inter
     qd, kvd, nqkv, d = cfg.q_dim, cfg.kv_dim, cfg.n_qkv, cfg.head_dim
     keys = min(cfg.window, cfg.cache_prior + 1)
+    kv_b = 1 if getattr(cfg, "kv_fp8", 0) else 2   # bytes per cached key / value element
     C = cfg.qk_channels
     return {
         "rmsnorm_attn": ("hbm", B * H * 4 + 2 * B * H * 2 + H * 2, "B"),
         "qkv_gemm": ("hbm", nqkv * H * 2 + 2 * B * H * 2 + 2 * B * nqkv * 2, "B"),
         "cca": ("hbm", 2 * B * nqkv * 2 + B * (qd + 2 * kvd) * 2 + B * C * 2 * 2 * 2 + B * H * 2, "B"),
-        "attention_decode": ("hbm", B * cfg.n_kv * keys * d * 2 * 2 + 2 * B * qd * 2, "B"),
+        "attention_decode": ("hbm", B * cfg.n_kv * keys * d * kv_b * 2 + 2 * B * qd * 2, "B"),
         "o_proj_merge": ("hbm", H * qd * 2 + B * qd * 2 + B * H * 4 * 2, "B"),
         "rmsnorm_mlp": ("hbm", B * H * 4 + B * H * 2 + H * 2, "B"),
         "router_down": ("hbm", R * H * 2 + B * H * 2 + B * R * 4, "B"),

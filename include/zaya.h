@@ -114,6 +114,11 @@ typedef struct zaya_config {
                                 so a sequence decodes past cache_cap with a window-sized cache
                                 (the pages' decode reads the window only: zaya page, "Queries and
                                 keys are convolved ..."; every block must slide: sliding_period 0) */
+  int32_t kv_fp8;            /* 0: the caches hold bf16 keys / values.  1: OCP FP8 E4M3 bytes (the
+                                bf16 value rounded to nearest, ties to even, saturating at 448), as
+                                a serving engine's fp8 KV cache (NVFP4 README, "Throughput and
+                                memory": --kv-cache-dtype fp8); a prompt attends over its bf16
+                                keys / values, a decode step over the cache */
   float rope_theta;          /* inv_freq[i] = rope_theta^(-2i/rot_dim) */
   float rms_eps;             /* RMSNorm epsilon (1e-5) */
   float qk_norm_eps;         /* q,k -> x * sqrt(d) / max(|x|, qk_norm_eps) */
@@ -157,9 +162,9 @@ typedef struct zaya_block_weights {
 
 /* One block's decode state (in/out, caller-owned). */
 typedef struct zaya_block_state {
-  void* k_cache;        /* bf16 [B, n_kv, cache_cap, d]: keys after norm, temp and RoPE
-                           (this and the three state buffers below: 16-byte aligned) */
-  void* v_cache;        /* bf16 [B, n_kv, cache_cap, d] */
+  void* k_cache;        /* bf16 (kv_fp8: E4M3 bytes) [B, n_kv, cache_cap, d]: keys after norm,
+                           temp and RoPE (this and the three state buffers below: 16-byte aligned) */
+  void* v_cache;        /* bf16 (kv_fp8: E4M3 bytes) [B, n_kv, cache_cap, d] */
   int32_t cache_cap;    /* positions per sequence the caches hold */
   int32_t* cache_len;   /* device int32 [B]: prefill writes S; decode appends at cache_len[b]
                            and increments it */
@@ -203,8 +208,9 @@ size_t zaya_stack_workspace_size(const zaya_config* cfg, int32_t mode, int32_t B
  *                   block's router_state_in.  Must not alias router_state_in.
  *  state            K/V of every position written to the caches at 0..S-1
  *                   (cache_cap >= S); with kv_ring, the last min(S, cache_cap)
- *                   positions p at slots p % cache_cap (any S; the attention
- *                   reads the prompt's keys from the workspace); cache_len[b]
+ *                   positions p at slots p % cache_cap (any S); with kv_ring
+ *                   or kv_fp8 the attention reads the prompt's bf16 keys from
+ *                   the workspace and a store kernel fills the cache; cache_len[b]
  *                   = S; conv_state and prev_hs set from the last two tokens.
  *                   Continuing a padded prefill in decode is not supported.
  *  taps             NULL or optional outputs.

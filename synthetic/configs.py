@@ -129,6 +129,12 @@ CONFIGS = {
         name="decode_stack_b64", batch=64, seq=1, n_blocks=40, block_idx=0, mode="decode",
         cache_prior=8192, seed=3, skip_bias=-1.0, input_dtype="bf16",
         vocab=262144, emb_mult=math.sqrt(2048.0), **_FULL),
+    # The decode step with an fp8 (E4M3) KV cache, as the NVFP4 README serves
+    # the model (--kv-cache-dtype fp8).
+    "decode_stack_b64_fp8kv": BlockConfig(
+        name="decode_stack_b64_fp8kv", batch=64, seq=1, n_blocks=40, block_idx=0, mode="decode",
+        cache_prior=8192, seed=3, skip_bias=-1.0, input_dtype="bf16", kv_fp8=1,
+        vocab=262144, emb_mult=math.sqrt(2048.0), **_FULL),
     # The same stack with the 74B preview's hybrid attention: a 4097-token
     # window on every other block (the odd ones), every earlier token on the others.
     "prefill_stack_hybrid_32k": BlockConfig(

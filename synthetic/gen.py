@@ -160,6 +160,9 @@ def gen_decode_state(cfg: BlockConfig, block: int, cap: int, device="cpu") -> di
     v = torch.zeros_like(k)
     k[:, :, :L] = _normal(cfg, block, "k_cache", (B, cfg.n_kv, L, d), 1.0, device).to(torch.bfloat16)
     v[:, :, :L] = _normal(cfg, block, "v_cache", (B, cfg.n_kv, L, d), 1.0, device).to(torch.bfloat16)
+    if cfg.kv_fp8:   # an fp8 cache holds E4M3 codes (uint8) of the same draws
+        k = k.to(torch.float8_e4m3fn).view(torch.uint8)
+        v = v.to(torch.float8_e4m3fn).view(torch.uint8)
     return {
         "k_cache": k, "v_cache": v,
         "conv_state": _normal(cfg, block, "conv_state", (B, cfg.qk_channels, 2), 1.0,

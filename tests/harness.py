@@ -60,9 +60,10 @@ def _fp32_matrices(W: dict) -> bool:
 
 
 def new_state(cfg, B, cap, dev="cuda") -> dict:
+    kv = torch.uint8 if getattr(cfg, "kv_fp8", 0) else torch.bfloat16   # E4M3 bytes with kv_fp8
     return dict(
-        k_cache=torch.zeros(B, cfg.n_kv, cap, cfg.head_dim, dtype=torch.bfloat16, device=dev),
-        v_cache=torch.zeros(B, cfg.n_kv, cap, cfg.head_dim, dtype=torch.bfloat16, device=dev),
+        k_cache=torch.zeros(B, cfg.n_kv, cap, cfg.head_dim, dtype=kv, device=dev),
+        v_cache=torch.zeros(B, cfg.n_kv, cap, cfg.head_dim, dtype=kv, device=dev),
         cache_len=torch.zeros(B, dtype=torch.int32, device=dev),
         conv_state=torch.zeros(B, cfg.qk_channels, 2, dtype=torch.bfloat16, device=dev),
         prev_hs=torch.zeros(B, cfg.hidden, dtype=torch.bfloat16, device=dev))
@@ -272,3 +273,22 @@ def assert_rows_ok(results):
         assert res["router_mismatch"] == 0, res
         lo = res["layer_output"]
         assert lo["rel_max"] <= TOL_REL_MAX and lo["cos"] >= TOL_COS, res
+
+
+def _e4m3_lut() -> torch.Tensor:
+    """The value of every OCP FP8 E4M3 code (sign, 4 exponent bits with bias
+    7, 3 mantissa bits; exponent 0 subnormal; S.1111.111 NaN)."""
+    vals = []
+    for code in range(256):
+        s, e, m = code >> 7, (code >> 3) & 15, code & 7
+        if e == 15 and m == 7:
+            v = float("nan")
+        else:
+            v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+        vals.append(-v if s else v)
+    return torch.tensor(vals, dtype=torch.float64)
+
+
+def e4m3_values(t: torch.Tensor) -> torch.Tensor:
+    """E4M3 bytes (uint8) as their float64 values."""
+    return _e4m3_lut()[t.cpu().long()]

@@ -178,6 +178,9 @@ def test_window_ring_arguments():
     cfg = get_config("tiny")
     assert ZB.zaya_workspace_size(ZB.make_config(cfg.with_(kv_ring=1)), ZB.ZAYA_DECODE, 2, 1) > 0
     assert ZB.zaya_workspace_size(ZB.make_config(cfg.with_(kv_ring=2)), ZB.ZAYA_DECODE, 2, 1) == 0
+    assert ZB.zaya_workspace_size(ZB.make_config(cfg.with_(kv_fp8=2)), ZB.ZAYA_DECODE, 2, 1) == 0
+    assert (ZB.zaya_workspace_size(ZB.make_config(cfg.with_(kv_fp8=1)), ZB.ZAYA_PREFILL, 1, 64)
+            > ZB.zaya_workspace_size(ZB.make_config(cfg), ZB.ZAYA_PREFILL, 1, 64))
     hybrid = cfg.with_(kv_ring=1, sliding_period=2, sliding_phase=1)
     assert ZB.zaya_workspace_size(ZB.make_config(hybrid), ZB.ZAYA_DECODE, 2, 1) == 0
     # the prefill workspace of a ring also holds the prompt's linear K / V

@@ -332,3 +332,75 @@ def test_window_ring_cache_matches_linear_cache(name):
         ref = Z.block_decode(cfg, Hn.eff(W), x[:, n], dense, r_at(n), force_cls=g_cls)
         lo = Hn.report("layer_output", db["layer_output"].numpy(), ref["layer_output"])
         assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, (k, lo)
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill_4k"])
+def test_fp8_cache_prefill_and_decode(name):
+    """kv_fp8 (E4M3 K/V cache, the NVFP4 README's --kv-cache-dtype fp8): the
+    prompt attends over its bf16 keys / values, so every prefill output equals
+    the bf16-cache run bit for bit; the cache bytes are the E4M3 codes of the
+    bf16 run's keys and values, exactly; decode steps then read the E4M3 cache
+    and match the oracle's fp8-cache decode on the GPU's own state."""
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config(name)
+    S, steps = (40, 3) if name == "tiny" else (256, 2)
+    cfg = cfg.with_(seq=S)
+    c8 = cfg.with_(kv_fp8=1)
+    W = gen_block_weights(cfg)
+    Wd = Hn.dev_weights(W)
+    inp = gen_prefill_inputs(cfg.with_(seq=S + steps))
+    x, rin = inp["x"], inp["router_state_in"]
+    r_at = (lambda i: None) if rin is None else (lambda i: rin[:, i])
+    st16 = Hn.new_state(cfg, 1, S + steps)
+    st8 = Hn.new_state(c8, 1, S + steps)
+    a = Hn.gpu_prefill(cfg, Wd, x[:, :S], None, None if rin is None else rin[:, :S], state=st16, taps=False)
+    b = Hn.gpu_prefill(c8, Wd, x[:, :S], None, None if rin is None else rin[:, :S], state=st8, taps=False)
+    assert torch.equal(a["layer_output"], b["layer_output"])
+    assert torch.equal(a["router_state"], b["router_state"])
+    for key in ("k_cache", "v_cache"):
+        got = Hn.e4m3_values(st8[key][:, :, :S]).numpy()
+        want = Z.round_e4m3(st16[key][:, :, :S].float().cpu().numpy())
+        np.testing.assert_array_equal(got, want)
+    for key in ("cache_len", "conv_state", "prev_hs"):
+        assert torch.equal(st8[key], st16[key]), key
+    for k in range(steps):
+        n = S + k
+        host = {key: v.cpu().clone() for key, v in st8.items()}
+        host["k_cache"] = Hn.e4m3_values(host["k_cache"])
+        host["v_cache"] = Hn.e4m3_values(host["v_cache"])
+        dec = Hn.gpu_decode(c8, Wd, x[:, n], st8, r_at(n))
+        g_cls = Hn.gpu_classes(cfg, dec)
+        ref = Z.block_decode(c8, Hn.eff(W), x[:, n], host, r_at(n), force_cls=g_cls)
+        lo = Hn.report("layer_output", dec["layer_output"].numpy(), ref["layer_output"])
+        assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, (k, lo)
+        ao = Hn.report("attention_output", dec["attention_output"].float().numpy(), ref["attention_output"])
+        assert ao["cos"] >= 0.999, (k, ao)
+        new = Hn.e4m3_values(st8["k_cache"][:, :, n]).numpy()
+        want = ref["state"]["k_cache"][:, :, n]
+        step = np.ldexp(1.0, np.maximum(np.frexp(np.abs(want) + (want == 0))[1] - 1, -6) - 3)
+        assert (np.abs(new - want) <= step).all()   # one E4M3 step: the keys' bf16 inputs differ in rounding
+
+
+def test_fp8_window_ring_matches_linear_fp8_cache():
+    """kv_fp8 with kv_ring: a prompt longer than the ring and decode steps
+    across the wrap equal the linear fp8-cache run bit for bit."""
+    from tests import harness as Hn
+    cfg = get_config("tiny").with_(seq=50, kv_fp8=1)
+    S, steps, cap = 50, 4, cfg.window
+    rcfg = cfg.with_(kv_ring=1)
+    W = gen_block_weights(cfg)
+    Wd = Hn.dev_weights(W)
+    inp = gen_prefill_inputs(cfg.with_(seq=S + steps))
+    x, rin = inp["x"], inp["router_state_in"]
+    lin = Hn.new_state(cfg, 1, S + steps)
+    ring = Hn.new_state(cfg, 1, cap)
+    a = Hn.gpu_prefill(cfg, Wd, x[:, :S], None, rin[:, :S], state=lin, taps=False)
+    b = Hn.gpu_prefill(rcfg, Wd, x[:, :S], None, rin[:, :S], state=ring, taps=False)
+    assert torch.equal(a["layer_output"], b["layer_output"])
+    _ring_matches_linear(lin, ring, S, cap)
+    for k in range(steps):
+        da = Hn.gpu_decode(cfg, Wd, x[:, S + k], lin, rin[:, S + k])
+        db = Hn.gpu_decode(rcfg, Wd, x[:, S + k], ring, rin[:, S + k])
+        assert torch.equal(da["layer_output"], db["layer_output"]), k
+        _ring_matches_linear(lin, ring, S + k + 1, cap)

@@ -25,7 +25,7 @@ class zaya_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "hidden", "n_q", "n_kv", "head_dim", "rot_dim", "conv_width", "n_experts", "inter",
         "router_hidden", "window", "vocab", "cca_mean_residual", "v_delayed", "sliding_period",
-        "sliding_phase", "conv_groups", "kv_ring")] + [
+        "sliding_phase", "conv_groups", "kv_ring", "kv_fp8")] + [
         (n, C.c_float) for n in ("rope_theta", "rms_eps", "qk_norm_eps", "attn_scale", "emb_mult", "emb_shift")]
 
 

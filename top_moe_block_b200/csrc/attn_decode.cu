@@ -14,6 +14,11 @@
 // A operand of P V straight from registers, V read with ldmatrix.trans.  The
 // four warps' (max, sum, O) are merged in shared memory into the chunk's
 // partial; a second kernel merges the chunks.
+// An fp8 cache (E4M3 bytes): the slice's raw bytes stream into a two-slot
+// staging ring (half the bytes), each warp converts its slice to f16 (exact)
+// in the swizzled layout above, and both products run on f16 mma.sync with q
+// and P as f16 (q's bf16 values are exact in f16 within its range, P gains
+// precision).
 #include <math.h>
 
 #include "common.cuh"
@@ -28,10 +33,30 @@ constexpr int kWarps = 4;
 constexpr int kMaxChunks = 64; // a head's partials in the workspace
 constexpr int kSub = 16;       // keys per slice (one k16 step of P V)
 
+// bf16: per warp two slots of [K|V][16][D] bf16.  fp8: one f16 slot plus two
+// staging slots of raw bytes -- the same 16 KB per warp.
 template <int D>
 constexpr size_t decode_smem_bytes() { return (size_t)kWarps * 2 * 2 * kSub * D * 2; }
 
-template <int D, int REP>
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+template <bool F16>
+__device__ __forceinline__ void mma_k16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    mma16816(c, a, b0, b1);
+  }
+}
+
+template <int D, int REP, bool F8>
 __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams p) {
   constexpr int NK = D / 16;   // k16 steps of Q K^T
   constexpr int ND = D / 8;    // 8-dim n-tiles of P V
@@ -65,14 +90,44 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
     for (int kk = 0; kk < NK; ++kk) {
       qa[kk][0] = gid < REP ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * tig) : 0u;
       qa[kk][1] = gid < REP ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * tig) : 0u;
+      if constexpr (F8) {   // the products run in f16
+        const float2 x0 = unpack_bf2(qa[kk][0]), x1 = unpack_bf2(qa[kk][1]);
+        qa[kk][0] = pack_f16x2(x0.x, x0.y);
+        qa[kk][1] = pack_f16x2(x1.x, x1.y);
+      }
     }
   }
-  const auto* Kg = static_cast<const __nv_bfloat16*>(p.k_cache) + ((size_t)b * p.n_kv + g) * p.cap * D;
-  const auto* Vg = static_cast<const __nv_bfloat16*>(p.v_cache) + ((size_t)b * p.n_kv + g) * p.cap * D;
+  constexpr int ES = F8 ? 1 : 2;   // bytes per cached element
+  const auto* Kg = static_cast<const uint8_t*>(p.k_cache) + ((size_t)b * p.n_kv + g) * p.cap * D * ES;
+  const auto* Vg = static_cast<const uint8_t*>(p.v_cache) + ((size_t)b * p.n_kv + g) * p.cap * D * ES;
   __nv_bfloat16* sw = reinterpret_cast<__nv_bfloat16*>(dsm) + (size_t)warp * 2 * 2 * kSub * D;   // [slot][K|V][16][D]
-  // K and V rows key0 .. key0+15 into ring slot `slot`; keys past the warp's
-  // range are zero-filled (no global read)
+  // fp8: the f16 slice in slot 0, raw staging slots [2][K|V][16][D] bytes in slot 1's space
+  uint8_t* raw = reinterpret_cast<uint8_t*>(sw + 2 * kSub * D);
+  // K and V rows key0 .. key0+15 into ring slot `slot` (fp8: staging slot);
+  // keys past the warp's range are zero-filled (no global read)
   auto load_slice = [&](int slot, int key0) {
+    if constexpr (F8) {
+      constexpr int CR = D / 16;   // 16-byte chunks per raw row
+      uint8_t* dk = raw + (size_t)slot * 2 * kSub * D;
+      uint8_t* dv = dk + kSub * D;
+#pragma unroll
+      for (int i = lane; i < kSub * CR; i += 32) {
+        const int r = i / CR, c = i % CR;
+        const int key = key0 + r;
+        const bool ok = key < w_end;
+        int row = row0 + (key - w_begin);
+        if (row >= p.cap) row -= p.cap;
+        const size_t src = (size_t)(ok ? row : 0) * D + c * 16;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dk + r * D + c * 16)),
+                     "l"(Kg + src), "r"(ok ? 16 : 0)
+                     : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dv + r * D + c * 16)),
+                     "l"(Vg + src), "r"(ok ? 16 : 0)
+                     : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      return;
+    }
     __nv_bfloat16* dk = sw + (size_t)slot * 2 * kSub * D;
     __nv_bfloat16* dv = dk + kSub * D;
 #pragma unroll
@@ -82,7 +137,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
       const bool ok = key < w_end;
       int row = row0 + (key - w_begin);
       if (row >= p.cap) row -= p.cap;
-      const size_t src = (size_t)(ok ? row : 0) * D + c * 8;
+      const size_t src = ((size_t)(ok ? row : 0) * D + c * 8) * 2;
       const int dst = r * D + ((c ^ (r & 7)) * 8);
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dk + dst)), "l"(Kg + src),
                    "r"(ok ? 16 : 0)
@@ -110,7 +165,28 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
       asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncwarp();
-    const __nv_bfloat16* sK = sw + (size_t)slot * 2 * kSub * D;
+    if constexpr (F8) {   // the staged E4M3 slice, K rows then V rows, as f16 into slot 0
+      constexpr int CR = D / 16;
+      const uint8_t* rk = raw + (size_t)slot * 2 * kSub * D;
+#pragma unroll 2
+      for (int i = lane; i < 2 * kSub * CR; i += 32) {
+        const int kv = i / (kSub * CR), rem = i % (kSub * CR);
+        const int r = rem / CR, c = rem % CR;
+        const uint4 x = *reinterpret_cast<const uint4*>(rk + kv * kSub * D + r * D + c * 16);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          h[2 * j] = e4m3x2_to_f16x2((uint16_t)(w[j] & 0xffffu));
+          h[2 * j + 1] = e4m3x2_to_f16x2((uint16_t)(w[j] >> 16));
+        }
+        __nv_bfloat16* dst = sw + kv * kSub * D + r * D;
+        *reinterpret_cast<uint4*>(dst + (((2 * c) ^ (r & 7)) * 8)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ (r & 7)) * 8)) = make_uint4(h[4], h[5], h[6], h[7]);
+      }
+      __syncwarp();
+    }
+    const __nv_bfloat16* sK = F8 ? sw : sw + (size_t)slot * 2 * kSub * D;
     const __nv_bfloat16* sV = sK + kSub * D;
     // S = Q K^T over the slice's 16 keys (two 8-key n-tiles)
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -122,8 +198,8 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
         uint32_t b00, b01, b10, b11;
         ldsm_x4(smem_u32(sK + key_r * D + ((ch ^ (key_r & 7)) * 8)), b00, b01, b10, b11);
         const uint32_t a[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
-        mma16816(s[0], a, b00, b01);
-        mma16816(s[1], a, b10, b11);
+        mma_k16<F8>(s[0], a, b00, b01);
+        mma_k16<F8>(s[1], a, b10, b11);
       }
     }
     // online softmax on row gid: keys 2tig, 2tig+1 (tile 0) and 8+2tig, 9+2tig (tile 1)
@@ -154,7 +230,8 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
       o[j][1] *= corr;
     }
     // O += P V: P (bf16) is the A operand, V read transposed
-    const uint32_t pa[4] = {pack_bf2(pv[0], pv[1]), 0u, pack_bf2(pv[2], pv[3]), 0u};
+    const uint32_t pa[4] = {F8 ? pack_f16x2(pv[0], pv[1]) : pack_bf2(pv[0], pv[1]), 0u,
+                            F8 ? pack_f16x2(pv[2], pv[3]) : pack_bf2(pv[2], pv[3]), 0u};
     {
       const int key_r = (mi & 1) * 8 + rr;   // matrices: keys 0-7 / 8-15 x dims of n-tiles j / j+1
 #pragma unroll
@@ -162,8 +239,8 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const DecodeAttnParams
         const int ch = j + (mi >> 1);
         uint32_t r0, r1, r2, r3;
         ldsm_x4_t(smem_u32(sV + key_r * D + ((ch ^ (key_r & 7)) * 8)), r0, r1, r2, r3);
-        mma16816(o[j], pa, r0, r1);
-        mma16816(o[j + 1], pa, r2, r3);
+        mma_k16<F8>(o[j], pa, r0, r1);
+        mma_k16<F8>(o[j + 1], pa, r2, r3);
       }
     }
     __syncwarp();   // the slot is read before the next iteration refills it
@@ -261,27 +338,29 @@ int launch_attn_decode(const DecodeAttnParams& p, cudaStream_t st) {
   if (p.n_chunks < 1 || p.n_chunks > kMaxChunks || p.chunk_keys % kChunk) return ZAYA_ERR_UNSUPPORTED;
   const int rep = p.n_q / p.n_kv;
   const dim3 grid(p.n_chunks, p.n_kv, p.B);
-#define ZAYA_DEC(DV, RV)                                                                               \
-  if (p.d == DV && rep == RV) {                                                                        \
+#define ZAYA_DEC(DV, RV, F8V)                                                                          \
+  if (p.d == DV && rep == RV && (p.fp8 != 0) == F8V) {                                                 \
     static bool set = false;                                                                           \
     if (!set) {                                                                                        \
-      if (cudaFuncSetAttribute(attn_decode_kernel<DV, RV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+      if (cudaFuncSetAttribute(attn_decode_kernel<DV, RV, F8V>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                (int)decode_smem_bytes<DV>()) != cudaSuccess)                          \
         return ZAYA_ERR_CUDA;                                                                          \
       set = true;                                                                                      \
     }                                                                                                  \
-    launch_k(attn_decode_kernel<DV, RV>, grid, dim3(32 * kWarps), decode_smem_bytes<DV>(), st, nullptr, 0, p); \
+    launch_k(attn_decode_kernel<DV, RV, F8V>, grid, dim3(32 * kWarps), decode_smem_bytes<DV>(), st, nullptr, 0, p); \
     launch_k(attn_decode_combine<DV>, dim3(p.B * p.n_q), dim3(DV), 0, st, nullptr, 0, p, RV);         \
     return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;                                \
   }
-  ZAYA_DEC(128, 4)
-  ZAYA_DEC(64, 4)
-  ZAYA_DEC(128, 2)
-  ZAYA_DEC(64, 2)
-  ZAYA_DEC(128, 1)
-  ZAYA_DEC(64, 1)
-  ZAYA_DEC(128, 8)
-  ZAYA_DEC(64, 8)
+#define ZAYA_DEC2(DV, RV) ZAYA_DEC(DV, RV, false) ZAYA_DEC(DV, RV, true)
+  ZAYA_DEC2(128, 4)
+  ZAYA_DEC2(64, 4)
+  ZAYA_DEC2(128, 2)
+  ZAYA_DEC2(64, 2)
+  ZAYA_DEC2(128, 1)
+  ZAYA_DEC2(64, 1)
+  ZAYA_DEC2(128, 8)
+  ZAYA_DEC2(64, 8)
+#undef ZAYA_DEC2
 #undef ZAYA_DEC
   return ZAYA_ERR_UNSUPPORTED;
 }

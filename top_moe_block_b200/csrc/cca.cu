@@ -218,11 +218,19 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
 #pragma unroll
         for (int i = 0; i < DPL; ++i) t[i] = f2bf(y[i]);
       }
+    } else if (p.decode && p.fp8) {   // the cache's E4M3 of the bf16 key
+      dst = nullptr;
+      uint8_t* d8 = static_cast<uint8_t*>(p.k_cache) + (((size_t)b * nkv + head) * p.cache_cap + slot) * D + lane * DPL;
+#pragma unroll
+      for (int i = 0; i < DPL; i += 2)
+        *reinterpret_cast<uint16_t*>(d8 + i) = pack_e4m3x2(round_bf(y[i]), round_bf(y[i + 1]));
     } else {
       dst = static_cast<__nv_bfloat16*>(p.k_cache) + (((size_t)b * nkv + head) * p.cache_cap + slot) * D + lane * DPL;
     }
+    if (dst) {
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) dst[i] = f2bf(y[i]);
+      for (int i = 0; i < DPL; ++i) dst[i] = f2bf(y[i]);
+    }
 
     if (last) {  // conv_state <- pre-conv channels of tokens t-1, t
 #pragma unroll
@@ -239,6 +247,7 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
     const int vd0 = vc0 + nkv * (D / 2);
     __nv_bfloat16* dst =
         static_cast<__nv_bfloat16*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + slot) * D + lane * DPL;
+    float vv[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
       const int j = lane * DPL + i;
@@ -255,7 +264,16 @@ __global__ void __launch_bounds__(1024) cca_kernel(const CcaParams p) {
           v = pre.real1 ? bf2f(qkv[(size_t)(tok - 1) * ld + col]) : 0.f;
         }
       }
-      dst[i] = f2bf(v);
+      vv[i] = v;
+    }
+    if (p.decode && p.fp8) {   // the cache's E4M3 of the bf16 value
+      uint8_t* d8 = static_cast<uint8_t*>(p.v_cache) + (((size_t)b * nkv + g) * p.cache_cap + slot) * D + lane * DPL;
+#pragma unroll
+      for (int i = 0; i < DPL; i += 2)
+        *reinterpret_cast<uint16_t*>(d8 + i) = pack_e4m3x2(round_bf(vv[i]), round_bf(vv[i + 1]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) dst[i] = f2bf(vv[i]);
     }
     if (last && g == 0) {  // prev_hs <- attention_norm_output of this token
       const uint2* src = reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.a_in) + (size_t)tok * p.H);
@@ -695,11 +713,13 @@ int launch_cca(const CcaParams& p, cudaStream_t st) {
 
 namespace {
 
-// One thread per 16-byte piece of a kept row: K and V rows of positions
-// max(0, S - cap) .. S-1 of every (sequence, kv head).
-__global__ void __launch_bounds__(256) ring_store_kernel(const uint4* __restrict__ k_lin, const uint4* __restrict__ v_lin,
-                                                         uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
-                                                         int BG, int S, int cap, int vpr, int* status) {
+// One thread per 8 values (16 bytes of bf16) of a kept row: K and V of
+// positions max(0, S - cap) .. S-1 of every (sequence, kv head), to slot p
+// (ring: p % cap), as bf16 or as E4M3 bytes of the bf16 values.
+__global__ void __launch_bounds__(256) cache_store_kernel(const uint4* __restrict__ k_lin,
+                                                          const uint4* __restrict__ v_lin, void* __restrict__ k_cache,
+                                                          void* __restrict__ v_cache, int BG, int S, int cap, int vpr,
+                                                          int ring, int fp8, int* status) {
   griddep_begin();
   if (status_peek(status)) return;
   const int keep = S < cap ? S : cap;
@@ -710,24 +730,39 @@ __global__ void __launch_bounds__(256) ring_store_kernel(const uint4* __restrict
     const int bg = (int)(r / keep);
     const int pos = S - keep + (int)(r % keep);
     const size_t src = ((size_t)bg * S + pos) * vpr + v;
-    const size_t dst = ((size_t)bg * cap + pos % cap) * vpr + v;
-    k_cache[dst] = k_lin[src];
-    v_cache[dst] = v_lin[src];
+    const size_t dst = ((size_t)bg * cap + (ring ? pos % cap : pos)) * vpr + v;
+    const uint4 kx = k_lin[src], vx = v_lin[src];
+    if (fp8) {
+      auto enc = [](const uint4& x) {
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 a = unpack_bf2(w[2 * h]), c = unpack_bf2(w[2 * h + 1]);
+          o[h] = (uint32_t)pack_e4m3x2(a.x, a.y) | ((uint32_t)pack_e4m3x2(c.x, c.y) << 16);
+        }
+        return make_uint2(o[0], o[1]);
+      };
+      static_cast<uint2*>(k_cache)[dst] = enc(kx);
+      static_cast<uint2*>(v_cache)[dst] = enc(vx);
+    } else {
+      static_cast<uint4*>(k_cache)[dst] = kx;
+      static_cast<uint4*>(v_cache)[dst] = vx;
+    }
   }
 }
 
 }  // namespace
 
-int launch_ring_store(const void* k_lin, const void* v_lin, void* k_cache, void* v_cache, int B, int n_kv, int S,
-                      int cap, int d, int* status, cudaStream_t st) {
+int launch_cache_store(const void* k_lin, const void* v_lin, void* k_cache, void* v_cache, int B, int n_kv, int S,
+                       int cap, int d, int ring, int fp8, int* status, cudaStream_t st) {
   if (B <= 0 || S <= 0) return ZAYA_OK;
   if (cap <= 0 || d % 8) return ZAYA_ERR_UNSUPPORTED;
   const int vpr = d / 8;
   const long total = (long)B * n_kv * (S < cap ? S : cap) * vpr;
   const int blocks = (int)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
-  launch_k(ring_store_kernel, dim3(blocks), dim3(256), 0, st, nullptr, 0, static_cast<const uint4*>(k_lin),
-           static_cast<const uint4*>(v_lin), static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), B * n_kv, S,
-           cap, vpr, status);
+  launch_k(cache_store_kernel, dim3(blocks), dim3(256), 0, st, nullptr, 0, static_cast<const uint4*>(k_lin),
+           static_cast<const uint4*>(v_lin), k_cache, v_cache, B * n_kv, S, cap, vpr, ring, fp8, status);
   return cudaGetLastError() == cudaSuccess ? ZAYA_OK : ZAYA_ERR_CUDA;
 }
 

@@ -98,6 +98,7 @@ struct CcaParams {
   float theta, eps;
   int decode;             // 1: one token per sequence, history from conv_state
   int ring;               // decode: 1 = the caches are window rings (position p at slot p % cache_cap)
+  int fp8;                // decode: 1 = the caches hold E4M3 bytes
   int* status;
   int* zero_words;        // prefill: words CTA 0 clears for the next kernel (attention's merge counters), or null
   int n_zero_words;
@@ -105,11 +106,11 @@ struct CcaParams {
   float inv_freq[64];     // RoPE inverse frequencies theta^(-2i/rot), i < rot/2 (fp32)
 };
 int launch_cca(const CcaParams& p, cudaStream_t st);
-// Window-ring prefill: positions max(0, S - cap) .. S-1 of the linear K / V
-// (bf16 [B, n_kv, S, d]) into ring slots p % cap of the caches
-// (bf16 [B, n_kv, cap, d]).
-int launch_ring_store(const void* k_lin, const void* v_lin, void* k_cache, void* v_cache, int B, int n_kv, int S,
-                      int cap, int d, int* status, cudaStream_t st);
+// Prefill into a window ring or an fp8 cache: positions max(0, S - cap) ..
+// S-1 of the linear bf16 K / V ([B, n_kv, S, d]) into the caches ([B, n_kv,
+// cap, d]) at slot p (ring: p % cap), as bf16 or (fp8) E4M3 bytes.
+int launch_cache_store(const void* k_lin, const void* v_lin, void* k_cache, void* v_cache, int B, int n_kv, int S,
+                       int cap, int d, int ring, int fp8, int* status, cudaStream_t st);
 
 // The two-stage conv_qk's grouped stage (with its depthwise stage fused in):
 // y fp32 [rows, C], one group per q / k head.
@@ -157,6 +158,7 @@ struct DecodeAttnParams {
   int B, cap, n_q, n_kv, d, window, n_chunks;
   int chunk_keys;         // keys per CTA (a multiple of 256)
   int ring;               // 1: position p at slot p % cap
+  int fp8;                // 1: the caches hold E4M3 bytes
   float scale;
 };
 // Key chunks a head's decode attention may use for a window (256 keys per

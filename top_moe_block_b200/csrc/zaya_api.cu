@@ -131,6 +131,7 @@ int check_config(const zaya_config* c) {
     return ZAYA_ERR_INVALID_ARG;
   // a window ring needs a window on every block
   if (c->kv_ring != 0 && (c->kv_ring != 1 || c->sliding_period > 0)) return ZAYA_ERR_INVALID_ARG;
+  if (c->kv_fp8 != 0 && c->kv_fp8 != 1) return ZAYA_ERR_INVALID_ARG;
   return ZAYA_OK;
 }
 
@@ -209,9 +210,9 @@ Ws plan(const zaya_config& c, int mode, int B, int S) {
   w.ccount = o; o += up((size_t)(d.E + 2) * 4);
   w.convy = o; o += c.conv_groups > 0 ? up(M * d.C * 4) : 0;   // the two-stage conv's output (fp32)
   w.loany = o; o += up((size_t)router_split_blocks(d.R, d.E) * 4);
-  // window-ring prefill: the prompt's K and V (bf16 [B, n_kv, S, d] each) for
-  // the attention; the ring keeps the last cache_cap positions
-  w.kvlin = o; o += (c.kv_ring && mode == ZAYA_PREFILL) ? 2 * up(M * d.nkv * d.d * 2) : 0;
+  // window-ring or fp8-cache prefill: the prompt's bf16 K and V ([B, n_kv, S, d]
+  // each) for the attention, stored into the cache afterwards
+  w.kvlin = o; o += ((c.kv_ring || c.kv_fp8) && mode == ZAYA_PREFILL) ? 2 * up(M * d.nkv * d.d * 2) : 0;
   w.total = o;
   return w;
 }
@@ -379,11 +380,13 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
   void* a_in = at<void>(ws, L.a_in);
   void* qkv = at<void>(ws, L.qkv);
   // K / V of the prompt for the attention: the caches themselves, or, for a
-  // window ring, linear copies in the workspace stored into the ring after it
+  // window ring or an fp8 cache, bf16 linear copies in the workspace, stored
+  // into the cache after the attention
+  const bool via_ws = c.kv_ring || c.kv_fp8;
   void* kc = state->k_cache;
   void* vc = state->v_cache;
   int kcap = state->cache_cap;
-  if (c.kv_ring) {
+  if (via_ws) {
     kc = at<void>(ws, L.kvlin);
     vc = at<uint8_t>(ws, L.kvlin) + up((size_t)M * d.nkv * d.d * 2);
     kcap = S;
@@ -433,9 +436,9 @@ int block_prefill_impl(const zaya_config* cfg, const zaya_block_weights* w, int 
     p.part_bytes = attn_prefill_ws_bytes(B, S, window, d.nq, d.nkv, d.d);
     ZAYA_STAGE("attention", 1, launch_attn_prefill_tc(p, status, st));
   }
-  if (c.kv_ring)
-    ZAYA_STAGE("ring_store", 1, launch_ring_store(kc, vc, state->k_cache, state->v_cache, B, d.nkv, S,
-                                                  state->cache_cap, d.d, status, st));
+  if (via_ws)
+    ZAYA_STAGE("cache_store", 1, launch_cache_store(kc, vc, state->k_cache, state->v_cache, B, d.nkv, S,
+                                                    state->cache_cap, d.d, c.kv_ring, c.kv_fp8, status, st));
   return block_tail(c, d, w, block_idx, M, hidden, rin, rout, taps, ws, L, nullptr, mask, sms, st);
 }
 
@@ -496,7 +499,7 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
     p.cache_len = state->cache_len; p.conv_state = state->conv_state; p.prev_hs = state->prev_hs; p.a_in = a_in;
     p.B = B; p.S = 1; p.H = d.H; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.rot = c.rot_dim;
     p.cca_res = c.cca_mean_residual; p.v_delayed = c.v_delayed; p.theta = c.rope_theta; p.eps = c.qk_norm_eps;
-    p.decode = 1; p.ring = c.kv_ring; p.status = status;
+    p.decode = 1; p.ring = c.kv_ring; p.fp8 = c.kv_fp8; p.status = status;
     fill_inv_freq(p.inv_freq, c.rot_dim, c.rope_theta);
     ZAYA_STAGE("cca", 1, launch_cca(p, st));
   }
@@ -507,6 +510,7 @@ int block_decode_impl(const zaya_config* cfg, const zaya_block_weights* w, int b
     const int window = block_window(c, block_idx);
     p.B = B; p.cap = state->cache_cap; p.n_q = d.nq; p.n_kv = d.nkv; p.d = d.d; p.window = window;
     p.ring = c.kv_ring;
+    p.fp8 = c.kv_fp8;
     const int span = window < state->cache_cap ? window : state->cache_cap;
     decode_attn_split(span, decode_chunks_any(c), &p.n_chunks, &p.chunk_keys);
     p.scale = d.scale;
