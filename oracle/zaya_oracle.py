@@ -95,6 +95,17 @@ def round_e4m3(x) -> np.ndarray:
     return np.where(np.isnan(x), np.nan, np.copysign(q, x))
 
 
+def e4m3_decode(codes) -> np.ndarray:
+    """Values of OCP FP8 E4M3 codes (uint8): sign bit, 4 exponent bits (bias
+    7), 3 mantissa bits; exponent 0 holds the subnormals m/8 * 2^-6; code
+    S.1111.111 is NaN."""
+    c = np.asarray(codes).astype(np.int64)
+    s, e, m = c >> 7, (c >> 3) & 15, c & 7
+    v = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    v = np.where((e == 15) & (m == 7), np.nan, v)
+    return np.where(s == 1, -v, v)
+
+
 def cache_kv(cfg, t):
     """Keys / values as the cache holds them: bf16, or with ``cfg.kv_fp8``
     the bf16 value rounded on to E4M3."""
@@ -308,17 +319,39 @@ def expert_ffn(x, w_gate_up_e, w_down_e, inter):
     return (silu(gu[:, :inter]) * gu[:, inter:]) @ w_down_e.T
 
 
+def expert_ffn_fp8(x, wgu_e, sgu_e, wdn_e, sdn_e, s_in, s_act, inter):
+    """The SwiGLU expert with FP8 (E4M3) weights and activations, the scheme
+    of an FP8 W8A8 checkpoint (the pages' own deployments
+    quantise the experts, NVFP4 README "Quantization details"): weights are
+    E4M3 values wgu_e [2I,H], wdn_e [H,I] with one fp32 scale per output row
+    (sgu_e [2I], sdn_e [H]); each input is quantised with a static per-expert
+    scale, x_q = E4M3(x / s_in) and act_q = E4M3(act / s_act); a product
+    is the E4M3 dot product times its input's and its row's scales."""
+    xq = round_e4m3(x / s_in)
+    gu = (xq @ wgu_e.T) * (s_in * sgu_e[None, :])
+    act = silu(gu[:, :inter]) * gu[:, inter:]
+    aq = round_e4m3(act / s_act)
+    return (aq @ wdn_e.T) * (s_act * sdn_e[None, :])
+
+
 def moe(cfg, W, m_in, cls, w):
     """routed_output: w_t * expert_{c_t}(m_in_t); zero where c_t is skip."""
     E, I = cfg.n_experts, cfg.inter
     y = np.zeros_like(m_in)
     wgu = W["w_gate_up"]
     wdn = W["w_down"]
+    fp8 = getattr(cfg, "expert_fp8", 0)
     for e in range(E):
         rows = np.nonzero(cls == e)[0]
         if rows.size == 0:
             continue
-        y[rows] = w[rows, None] * expert_ffn(m_in[rows], as64(wgu[e]), as64(wdn[e]), I)
+        if fp8:   # E4M3 codes with per-row scales and the expert's static input scales
+            sc = as64(W["expert_act_scale"])[e]
+            f = expert_ffn_fp8(m_in[rows], e4m3_decode(np.asarray(wgu[e])), as64(W["w_gate_up_scale"])[e],
+                               e4m3_decode(np.asarray(wdn[e])), as64(W["w_down_scale"])[e], sc[0], sc[1], I)
+        else:
+            f = expert_ffn(m_in[rows], as64(wgu[e]), as64(wdn[e]), I)
+        y[rows] = w[rows, None] * f
     return y
 
 

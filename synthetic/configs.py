@@ -39,6 +39,7 @@ class BlockConfig:
     sliding_phase: int = 0       # block % P == phase slide, the others attend to every earlier token
     kv_ring: int = 0             # 1: K/V caches as window rings (slot = position % cache_cap)
     kv_fp8: int = 0              # 1: K/V caches hold OCP FP8 E4M3 (the prompt attends over bf16)
+    expert_fp8: int = 0          # 1: expert weights as E4M3 codes + per-row scales, E4M3 activations
     vocab: int = 0
     emb_mult: float = 1.0
     emb_shift: float = 0.0

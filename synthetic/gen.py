@@ -125,6 +125,16 @@ def gen_block_weights(cfg: BlockConfig, block: int | None = None, device="cpu") 
     w["balancing"] = balancing_biases(cfg).to(device)
     w["w_gate_up"] = n("w_gate_up", (E, 2 * I, H), cfg.w_std).to(bf)   # rows [0,I) gate, [I,2I) up
     w["w_down"] = n("w_down", (E, H, I), cfg.w_std).to(bf)
+    if cfg.expert_fp8:
+        # an FP8 checkpoint of the same draws: E4M3 codes (uint8) with one fp32
+        # scale per output row (its absolute maximum over 448), and static
+        # per-expert input scales (powers of two: inputs of |x| <= 14 fit)
+        for name in ("w_gate_up", "w_down"):
+            full = w[name].float()
+            scale = full.abs().amax(dim=-1).clamp_min(1e-30) / 448.0
+            w[name] = (full / scale[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+            w[name + "_scale"] = scale.to(torch.float32)
+        w["expert_act_scale"] = torch.full((E, 2), 2.0 ** -5, dtype=torch.float32, device=device)
     return w
 
 

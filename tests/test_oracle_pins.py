@@ -742,3 +742,43 @@ def test_fp8_cache_prefill_and_decode(tiny):
     np.testing.assert_array_equal(d8["attention_keys"], d16["attention_keys"])
     rel = np.abs(d8["attention_premix"] - d16["attention_premix"]).max() / np.abs(d16["attention_premix"]).max()
     assert 1e-4 < rel < 0.1, rel
+
+
+# ---------------------------------------------------------------- FP8 experts
+
+def test_e4m3_decode_against_the_format():
+    """e4m3_decode of every code equals the table decoded from the format's
+    definition, and every finite value is a fixed point of round_e4m3."""
+    codes, vals = _e4m3_table()
+    np.testing.assert_array_equal(Z.e4m3_decode(codes), vals)
+    assert np.isnan(Z.e4m3_decode([0x7F, 0xFF])).all()
+    np.testing.assert_array_equal(Z.round_e4m3(Z.e4m3_decode(codes)), vals)
+
+
+def test_fp8_expert_brute_force():
+    """expert_ffn_fp8 on tiny shapes against a per-element loop: the input
+    quantised as E4M3(x / s_in), each gate / up dot product of E4M3 values
+    times s_in and its row's scale, SwiGLU, the activation quantised as
+    E4M3(act / s_act), the down dot products times s_act and their rows'
+    scales (an FP8 W8A8 expert; NVFP4 README, "Quantization details", for
+    the pages' quantised experts)."""
+    rng = np.random.default_rng(7)
+    T, H, I = 3, 5, 4
+    codes_gu = rng.integers(0, 256, size=(2 * I, H))
+    codes_dn = rng.integers(0, 256, size=(H, I))
+    codes_gu[(codes_gu & 0x7F) == 0x7F] = 0x12     # no NaN codes
+    codes_dn[(codes_dn & 0x7F) == 0x7F] = 0x21
+    wgu, wdn = Z.e4m3_decode(codes_gu), Z.e4m3_decode(codes_dn)
+    sgu = rng.uniform(0.001, 0.01, size=2 * I)
+    sdn = rng.uniform(0.001, 0.01, size=H)
+    s_in, s_act = 2.0 ** -5, 2.0 ** -3
+    x = rng.normal(0, 2.0, size=(T, H))
+    got = Z.expert_ffn_fp8(x, wgu, sgu, wdn, sdn, s_in, s_act, I)
+    for t in range(T):
+        xq = [float(Z.round_e4m3(x[t, h] / s_in)) for h in range(H)]
+        gu = [sum(xq[h] * wgu[j, h] for h in range(H)) * s_in * sgu[j] for j in range(2 * I)]
+        act = [gu[i] / (1.0 + math.exp(-gu[i])) * gu[I + i] for i in range(I)]
+        aq = [float(Z.round_e4m3(a / s_act)) for a in act]
+        for o in range(H):
+            want = sum(aq[i] * wdn[o, i] for i in range(I)) * s_act * sdn[o]
+            assert abs(got[t, o] - want) <= 1e-12 * max(1.0, abs(want)), (t, o)
