@@ -91,8 +91,9 @@ def stage_work(cfg, routed_tokens, pairs):
         "router_down": ("tensor", 2.0 * M * H * R, "FLOP"),
         "router_mlp": ("alu", 2.0 * M * (2 * R * R + R * E1), "FLOP"),
         "dispatch": ("hbm", routed_tokens * H * 2 * 2 + (M - routed_tokens) * H * 8, "B"),
-        "experts_gate_up": ("tensor", 2.0 * routed_tokens * H * 2 * I, "FLOP"),
-        "experts_down_merge": ("tensor", 2.0 * routed_tokens * I * H, "FLOP"),
+        # FP8 experts ("tensor_f8"): held against the E4M3 dense peak
+        "experts_gate_up": ("tensor_f8" if cfg.expert_fp8 else "tensor", 2.0 * routed_tokens * H * 2 * I, "FLOP"),
+        "experts_down_merge": ("tensor_f8" if cfg.expert_fp8 else "tensor", 2.0 * routed_tokens * I * H, "FLOP"),
         # the two-stage conv_qk's grouped stage (TF32 tensor cores): C outputs x 2 taps x C/G inputs
         **({"conv_grouped": ("tensor", 2.0 * M * cfg.qk_channels * 2 * (cfg.qk_channels // cfg.conv_groups),
                              "FLOP")} if cfg.conv_groups else {}),
@@ -107,6 +108,7 @@ def stage_work_decode(cfg, routed, distinct):
     qd, kvd, nqkv, d = cfg.q_dim, cfg.kv_dim, cfg.n_qkv, cfg.head_dim
     keys = min(cfg.window, cfg.cache_prior + 1)
     kv_b = 1 if getattr(cfg, "kv_fp8", 0) else 2   # bytes per cached key / value element
+    ew = 1 if getattr(cfg, "expert_fp8", 0) else 2   # bytes per expert weight
     C = cfg.qk_channels
     return {
         "rmsnorm_attn": ("hbm", B * H * 4 + 2 * B * H * 2 + H * 2, "B"),
@@ -118,8 +120,8 @@ def stage_work_decode(cfg, routed, distinct):
         "router_down": ("hbm", R * H * 2 + B * H * 2 + B * R * 4, "B"),
         "router_mlp": ("hbm", 2 * R * R * 4 + E1 * R * 4 + B * R * 4 * 2, "B"),
         "dispatch": ("hbm", routed * H * 2 * 2 + (B - routed) * H * 8, "B"),
-        "experts_gate_up": ("hbm", distinct * 2 * I * H * 2 + routed * H * 2 + routed * I * 2, "B"),
-        "experts_down_merge": ("hbm", distinct * H * I * 2 + routed * I * 2 + B * H * 4 * 2, "B"),
+        "experts_gate_up": ("hbm", distinct * 2 * I * H * ew + routed * H * 2 + routed * I * 2, "B"),
+        "experts_down_merge": ("hbm", distinct * H * I * ew + routed * I * 2 + B * H * 4 * 2, "B"),
         "embed": ("hbm", B * H * 2 + B * H * 4, "B"),
         "final_norm": ("hbm", B * H * 4 + B * H * 2, "B"),
         "lm_head": ("hbm", cfg.vocab * H * 2 + B * H * 2 + B * cfg.vocab * 2, "B"),
@@ -719,13 +721,16 @@ def roofline(stages, work, peaks, peak_src, cfg, step_ms):
     ms, n = stages[name]
     bound, amount, unit = work.get(name, ("hbm", 0, "B"))
     per_ms = ms / max(n, 1)
-    if bound == "tensor":
+    if bound in ("tensor", "tensor_f8"):
         achieved = amount / (per_ms / 1e3) / 1e12
         long_step = step_ms >= 1000.0
         peak = (peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]) if long_step else peaks["bf16_tflops"]
         u = "TFLOP/s"
         peak_note = (f"bf16 dense, {peak_src} {'sustained' if long_step else 'burst'} "
                      f"(kernel timed inside a {step_ms:.3f} ms step)")
+        if bound == "tensor_f8":   # E4M3 operands: the measured bf16 peak x the nominal fp8 / bf16 ratio (2)
+            peak *= 2.0
+            peak_note = "E4M3 dense = 2 x " + peak_note
     elif bound == "alu":
         achieved = amount / (per_ms / 1e3) / 1e12
         peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12

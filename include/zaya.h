@@ -114,6 +114,12 @@ typedef struct zaya_config {
                                 so a sequence decodes past cache_cap with a window-sized cache
                                 (the pages' decode reads the window only: zaya page, "Queries and
                                 keys are convolved ..."; every block must slide: sliding_period 0) */
+  int32_t expert_fp8;        /* 1: the experts as an FP8 W8A8 checkpoint (the pages'
+                                deployments quantise the experts: NVFP4 README, "Quantization
+                                details"): E4M3 weight codes with per-row fp32 scales, inputs
+                                quantised to E4M3 with static per-expert scales, products on the
+                                tensor cores in E4M3 (tcgen05 kind::f8f6f4), fp32 accumulation;
+                                needs inter % 128 == 0 and hidden % 256 == 0 */
   int32_t kv_fp8;            /* 0: the caches hold bf16 keys / values.  1: OCP FP8 E4M3 bytes (the
                                 bf16 value rounded to nearest, ties to even, saturating at 448), as
                                 a serving engine's fp8 KV cache (NVFP4 README, "Throughput and
@@ -152,12 +158,19 @@ typedef struct zaya_block_weights {
   const float* fc2_b;             /* fp32 [R] */
   const float* out_w;             /* fp32 [E+1, R] router_mlp.out_proj (no bias) */
   const float* balancing;         /* fp32 [E+1] balancing_biases (selection only) */
-  const void* w_gate_up;          /* bf16 [E, 2I, H]: rows [0,I) gate, [I,2I) up */
-  const void* w_down;             /* bf16 [E, H, I] */
+  const void* w_gate_up;          /* bf16 [E, 2I, H]: rows [0,I) gate, [I,2I) up
+                                     (expert_fp8: E4M3 codes, uint8) */
+  const void* w_down;             /* bf16 [E, H, I] (expert_fp8: E4M3 codes) */
   const float* conv2_w;           /* conv_groups > 0 only (else may be NULL): fp32 [C, C/G, 2]
                                      conv_qk_grouped taps for (t-1, t) of the depthwise output,
                                      Conv1d's [out, in/groups, k] layout */
   const float* conv2_b;           /* conv_groups > 0 only: fp32 [C] */
+  const float* w_gate_up_scale;   /* expert_fp8 only (else may be NULL): fp32 [E, 2I], one scale per
+                                     row of w_gate_up (weight = code value x scale); 16-byte aligned */
+  const float* w_down_scale;      /* expert_fp8 only: fp32 [E, H], one per row of w_down */
+  const float* expert_act_scale;  /* expert_fp8 only: fp32 [E, 2] static input scales, powers of two:
+                                     [e][0] for mlp_norm_output into gate/up (x_q = E4M3(x / s)),
+                                     [e][1] for the SwiGLU output into down */
 } zaya_block_weights;
 
 /* One block's decode state (in/out, caller-owned). */

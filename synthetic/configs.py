@@ -40,6 +40,7 @@ class BlockConfig:
     kv_ring: int = 0             # 1: K/V caches as window rings (slot = position % cache_cap)
     kv_fp8: int = 0              # 1: K/V caches hold OCP FP8 E4M3 (the prompt attends over bf16)
     expert_fp8: int = 0          # 1: expert weights as E4M3 codes + per-row scales, E4M3 activations
+    calib: str = ""              # calibrated: the workload whose fitted balancing biases apply (default: own)
     vocab: int = 0
     emb_mult: float = 1.0
     emb_shift: float = 0.0
@@ -129,6 +130,15 @@ CONFIGS = {
     "decode_stack_b64": BlockConfig(
         name="decode_stack_b64", batch=64, seq=1, n_blocks=40, block_idx=0, mode="decode",
         cache_prior=8192, seed=3, skip_bias=-1.0, input_dtype="bf16",
+        vocab=262144, emb_mult=math.sqrt(2048.0), **_FULL),
+    # The prefill block and the decode step with the experts as an FP8 W8A8
+    # checkpoint (E4M3 codes, per-row scales, static input scales).
+    "prefill_4k_fp8x": BlockConfig(
+        name="prefill_4k_fp8x", batch=1, seq=4096, seed=1, calibrated=1, skip_frac=0.0,
+        input_dtype="bf16", expert_fp8=1, calib="prefill_4k", **_FULL),
+    "decode_stack_b64_fp8x": BlockConfig(
+        name="decode_stack_b64_fp8x", batch=64, seq=1, n_blocks=40, block_idx=0, mode="decode",
+        cache_prior=8192, seed=3, skip_bias=-1.0, input_dtype="bf16", expert_fp8=1,
         vocab=262144, emb_mult=math.sqrt(2048.0), **_FULL),
     # The decode step with an fp8 (E4M3) KV cache, as the NVFP4 README serves
     # the model (--kv-cache-dtype fp8).

@@ -65,7 +65,7 @@ def balancing_biases(cfg: BlockConfig) -> torch.Tensor:
     """
     E = cfg.n_experts
     if cfg.calibrated:
-        path = os.path.join(_HERE, f"balancing_{cfg.name}.json")
+        path = os.path.join(_HERE, f"balancing_{cfg.calib or cfg.name}.json")
         with open(path) as f:
             vals = json.load(f)["balancing_biases"]
         assert len(vals) == E + 1

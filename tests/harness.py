@@ -40,6 +40,8 @@ def _abi_dtype(name, t):
     """The dtype the C ABI reads a weight in: bf16 for the block's matrices
     and norm weights, fp32 for its small parameters; other tensors (the
     stack's bf16 embedding and final norm) keep theirs."""
+    if t.dtype == torch.uint8:   # E4M3 codes (FP8 experts) stay bytes
+        return torch.uint8
     if name in BF16_FIELDS:
         return torch.bfloat16
     if name in ZB._abi.WEIGHT_FIELDS:
@@ -56,7 +58,7 @@ def eff(W: dict) -> dict:
 
 def _fp32_matrices(W: dict) -> bool:
     return any(W[k].dtype == torch.float32 and not torch.equal(W[k], W[k].to(torch.bfloat16).float())
-               for k in BF16_FIELDS if k in W)
+               for k in BF16_FIELDS if k in W and W[k].dtype != torch.uint8)
 
 
 def new_state(cfg, B, cap, dev="cuda") -> dict:

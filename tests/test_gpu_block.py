@@ -404,3 +404,40 @@ def test_fp8_window_ring_matches_linear_fp8_cache():
         db = Hn.gpu_decode(rcfg, Wd, x[:, S + k], ring, rin[:, S + k])
         assert torch.equal(da["layer_output"], db["layer_output"]), k
         _ring_matches_linear(lin, ring, S + k + 1, cap)
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill_4k"])
+def test_fp8_experts_prefill(name):
+    """expert_fp8: the experts as an FP8 W8A8 checkpoint (E4M3 weight codes
+    with per-row scales, E4M3 activations with static scales) on tcgen05
+    kind::f8f6f4 swapped pair tiles, against the oracle's FP8 expert at the
+    block tolerances (every step before the experts is the bf16 block's)."""
+    from tests import harness as Hn
+    cfg = get_config(name).with_(expert_fp8=1)
+    if name == "prefill_4k":
+        cfg = cfg.with_(seq=1024)
+    res = _run_prefill(cfg)
+    Hn.assert_block_ok(res)
+    assert res["mlp_output"]["cos"] >= 0.999, res["mlp_output"]
+
+
+def test_fp8_experts_decode_after_prefill():
+    """expert_fp8 in decode: a few tokens per expert on 16-token swapped
+    tiles, E4M3 operands, against the oracle's decode."""
+    from oracle import zaya_oracle as Z
+    from tests import harness as Hn
+    cfg = get_config("prefill_4k").with_(seq=128, expert_fp8=1)
+    S = 128
+    W = gen_block_weights(cfg)
+    Wd = Hn.dev_weights(W)
+    inp = gen_prefill_inputs(cfg.with_(seq=S + 1))
+    x, rin = inp["x"], inp["router_state_in"]
+    st = Hn.new_state(cfg, 1, S + 4)
+    Hn.gpu_prefill(cfg, Wd, x[:, :S], None, None if rin is None else rin[:, :S], state=st, taps=False)
+    host = {k: v.cpu().clone() for k, v in st.items()}
+    r1 = None if rin is None else rin[:, S]
+    dec = Hn.gpu_decode(cfg, Wd, x[:, S], st, r1)
+    g_cls = Hn.gpu_classes(cfg, dec)
+    ref = Z.block_decode(cfg, Hn.eff(W), x[:, S], host, r1, force_cls=g_cls)
+    lo = Hn.report("layer_output", dec["layer_output"].numpy(), ref["layer_output"])
+    assert lo["rel_max"] <= Hn.TOL_REL_MAX and lo["cos"] >= Hn.TOL_COS, lo

@@ -25,13 +25,14 @@ class zaya_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "hidden", "n_q", "n_kv", "head_dim", "rot_dim", "conv_width", "n_experts", "inter",
         "router_hidden", "window", "vocab", "cca_mean_residual", "v_delayed", "sliding_period",
-        "sliding_phase", "conv_groups", "kv_ring", "kv_fp8")] + [
+        "sliding_phase", "conv_groups", "kv_ring", "expert_fp8", "kv_fp8")] + [
         (n, C.c_float) for n in ("rope_theta", "rms_eps", "qk_norm_eps", "attn_scale", "emb_mult", "emb_shift")]
 
 
 WEIGHT_FIELDS = ("ln1_w", "ln2_w", "w_qkv", "conv_w", "conv_b", "k_temp", "w_o", "merge_a", "merge_m",
                  "router_down_w", "router_down_b", "router_state_scale", "router_norm_w", "fc1_w", "fc1_b",
-                 "fc2_w", "fc2_b", "out_w", "balancing", "w_gate_up", "w_down", "conv2_w", "conv2_b")
+                 "fc2_w", "fc2_b", "out_w", "balancing", "w_gate_up", "w_down", "conv2_w", "conv2_b",
+                 "w_gate_up_scale", "w_down_scale", "expert_act_scale")
 
 
 class zaya_block_weights(C.Structure):

@@ -86,6 +86,7 @@ struct TileInfo {
   int b_row2;  // SWIGLU: first up row
   int n_valid; // swapped: the tile's tokens (rows m0 .. m0 + n_valid of A)
   int n_mma;   // swapped: MMA N, n_valid rounded up to 16
+  int e;       // grouped: the expert
 };
 
 template <int EPI, int BN_OUT, int TM>   // TM: output rows per tile (128, or 256 for a CTA pair)
@@ -96,12 +97,14 @@ __device__ __forceinline__ int total_tiles(const GemmParams& p) {
   return p.mt_start[p.n_groups] * nt;   // mt_start counts TM-row tiles
 }
 
-template <int EPI, int BN_OUT, int TM, bool SWAP = false>
+// KE: K elements per k-block (a 128-byte smem row: 64 bf16, 128 E4M3)
+template <int EPI, int BN_OUT, int TM, bool SWAP = false, int KE = BK>
 __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
   TileInfo ti;
   const int nt = p.N / BN_OUT;
   const int ks = p.k_splits > 1 ? p.k_splits : 1;
-  ti.nkb = p.K / BK / ks;
+  ti.nkb = p.K / KE / ks;
+  ti.e = 0;
   ti.split = 0;
   ti.kb0 = 0;
   if (!p.grouped) {
@@ -124,6 +127,7 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int t) {
     ti.n0 = (local / mte) * BN_OUT;
     ti.b_row = e * p.b_rows_per_group + ti.n0;
     ti.b_row2 = e * p.b_rows_per_group + (p.b_rows_per_group >> 1) + ti.n0;
+    ti.e = e;
     if constexpr (SWAP) {
       // the expert's n tokens in mte near-equal tiles of `per` (a multiple of 16,
       // at most 256); every tile holds at least one token since n > 256 (mte - 1)
@@ -310,7 +314,7 @@ __device__ __forceinline__ void merge_chunk(const GemmParams& p, int row0, int m
 // bytes of the fp32 stream, all eight steps' loads in flight first.  tokl /
 // wl: lane i holds row row0 + i's token and routing weight.
 __device__ __forceinline__ void merge_chunk_swap(const GemmParams& p, int nj, int fw, int tokl, float wl,
-                                                 const uint32_t (&r)[32], float* T) {
+                                                 const uint32_t (&r)[32], float* T, const float4* dsc) {
   const int lane = lane_id();
 #pragma unroll
   for (int j = 0; j < 32; ++j) T[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = __uint_as_float(r[j]);
@@ -342,7 +346,10 @@ __device__ __forceinline__ void merge_chunk_swap(const GemmParams& p, int nj, in
   for (int i = 0; i < 8; ++i) {
     const int rr = 4 * i + rsub;
     if (rr >= nj) continue;
-    const float4 a4 = *reinterpret_cast<const float4*>(T + rr * 32 + ((jj ^ (rr & 7)) << 2));
+    float4 a4 = *reinterpret_cast<const float4*>(T + rr * 32 + ((jj ^ (rr & 7)) << 2));
+    if (dsc) {   // E4M3 products: s_act times the rows' scales
+      a4.x *= dsc->x; a4.y *= dsc->y; a4.z *= dsc->z; a4.w *= dsc->w;
+    }
     const float* ap = &a4.x;
     float4 x4 = xs[i];
     float* xp = &x4.x;
@@ -379,12 +386,18 @@ __device__ __forceinline__ void merge_chunk_swap(const GemmParams& p, int nj, in
 // m0 + r * n_mma / 2 into the B slot, in boxes of tok_box (16) rows, so a
 // tile of few tokens loads few bytes; tmA then maps the tokens and tmB the
 // weights.
-template <int BN, int EPI, int CG, bool SWAP>
+// F8 (swapped only): E4M3 operands on kind::f8f6f4, a k-block is 128 elements
+// (the same 128-byte rows), and the epilogues apply the static input scale
+// and the per-row weight scale of the expert (the SwiGLU output is stored as
+// E4M3 codes of act / s_act for the down projection).
+template <int BN, int EPI, int CG, bool SWAP, bool F8 = false>
 __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
   static_assert(!SWAP || (CG == 2 && BN == 256 && (EPI == EPI_SWIGLU || EPI == EPI_MERGE_MLP)),
                 "swapped tiles: grouped expert GEMMs on CTA pairs");
+  static_assert(!F8 || SWAP, "E4M3 operands: swapped expert tiles only");
+  constexpr int KE = F8 ? 2 * BK : BK;   // K elements per k-block
   using C = GemmCfg<BN, EPI, CG, SWAP>;
   constexpr int STAGES = C::STAGES;
   constexpr int BN_OUT = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
@@ -467,7 +480,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
       uint32_t phase = 0;
       int n_armed = 0;
       for (int t = unit; t < ntiles; t += n_units) {
-        const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP>(p, t);
+        const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP, KE>(p, t);
         // this CTA's B rows: CG = 1 all BN rows (SWIGLU: gate then up); CG = 2 its half
         const int b_first = (CG == 1) ? ti.b_row
                             : SWAP ? ti.b_row + (int)rank * (EPI == EPI_SWIGLU ? 64 : 128)
@@ -476,13 +489,13 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         const int kb_end = ti.kb0 + ti.nkb;
         auto prefetch_b = [&](int kb) {
           if constexpr (SWAP && EPI == EPI_SWIGLU) {
-            tma_prefetch_l2_2d(&tmB, kb * BK, b_first);
-            tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row2 + (int)rank * 64);
+            tma_prefetch_l2_2d(&tmB, kb * KE, b_first);
+            tma_prefetch_l2_2d(&tmB, kb * KE, ti.b_row2 + (int)rank * 64);
           } else if constexpr (EPI == EPI_SWIGLU && CG == 1) {
-            tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row);
-            tma_prefetch_l2_2d(&tmB, kb * BK, ti.b_row2);
+            tma_prefetch_l2_2d(&tmB, kb * KE, ti.b_row);
+            tma_prefetch_l2_2d(&tmB, kb * KE, ti.b_row2);
           } else {
-            tma_prefetch_l2_2d(&tmB, kb * BK, b_first);
+            tma_prefetch_l2_2d(&tmB, kb * KE, b_first);
           }
         };
         for (int kb = ti.kb0; kb < ti.kb0 + kPrefetchAhead && kb < kb_end; ++kb) prefetch_b(kb);
@@ -497,25 +510,25 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
             if (rank == 0)   // both CTAs' bytes
               mbar_arrive_expect_tx(&full[stage], 2 * (A_STAGE_BYTES + n_box * p.tok_box * BK * 2));
             const uint32_t bar = mapa_shared(&full[stage], 0);
-            tma_load_2d_pair(a_dst, &tmB, bar, kb * BK, b_first);   // weights: the MMA's A
+            tma_load_2d_pair(a_dst, &tmB, bar, kb * KE, b_first);   // weights: the MMA's A
             if constexpr (EPI == EPI_SWIGLU)
-              tma_load_2d_pair(a_dst + 64 * BK * 2, &tmB, bar, kb * BK, ti.b_row2 + (int)rank * 64);
+              tma_load_2d_pair(a_dst + 64 * BK * 2, &tmB, bar, kb * KE, ti.b_row2 + (int)rank * 64);
             const int t0 = ti.m0 + (int)rank * (ti.n_mma >> 1);
             for (int bx = 0; bx < n_box; ++bx)
-              tma_load_2d_pair(b_dst + bx * p.tok_box * BK * 2, &tmA, bar, kb * BK, t0 + bx * p.tok_box);
+              tma_load_2d_pair(b_dst + bx * p.tok_box * BK * 2, &tmA, bar, kb * KE, t0 + bx * p.tok_box);
           } else if constexpr (CG == 2) {
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);   // both CTAs' bytes
             const uint32_t bar = mapa_shared(&full[stage], 0);
-            tma_load_2d_pair(a_dst, &tmA, bar, kb * BK, ti.m0 + (int)rank * BM);
-            tma_load_2d_pair(b_dst, &tmB, bar, kb * BK, b_first);
+            tma_load_2d_pair(a_dst, &tmA, bar, kb * KE, ti.m0 + (int)rank * BM);
+            tma_load_2d_pair(b_dst, &tmB, bar, kb * KE, b_first);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-            tma_load_2d(a_dst, &tmA, &full[stage], kb * BK, ti.m0);
+            tma_load_2d(a_dst, &tmA, &full[stage], kb * KE, ti.m0);
             if constexpr (EPI == EPI_SWIGLU) {
-              tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
-              tma_load_2d(b_dst + (BN / 2) * BK * 2, &tmB, &full[stage], kb * BK, ti.b_row2);
+              tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, ti.b_row);
+              tma_load_2d(b_dst + (BN / 2) * BK * 2, &tmB, &full[stage], kb * KE, ti.b_row2);
             } else {
-              tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, ti.b_row);
+              tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, ti.b_row);
             }
           }
           ++n_armed;
@@ -546,9 +559,9 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, wc)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP>(p, t);
+        const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP, KE>(p, t);
         const int nkb = ti.nkb;
-        const uint32_t idesc = SWAP ? idesc_bf16_f32(TM, ti.n_mma) : IDESC;
+        const uint32_t idesc = F8 ? idesc_e4m3_f32(TM, ti.n_mma) : SWAP ? idesc_bf16_f32(TM, ti.n_mma) : IDESC;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, wc)) {
@@ -560,7 +573,10 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
           const uint32_t b_addr = smem_u32(sB + stage * C::B_STAGE_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            if constexpr (CG == 2)
+            if constexpr (F8)
+              tc_mma_e4m3_pair(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), idesc,
+                               (kb | k) != 0 ? 1u : 0u);
+            else if constexpr (CG == 2)
               tc_mma_bf16_pair(d_tmem, smem_desc_k128(a_addr + k * 32), smem_desc_k128(b_addr + k * 32), idesc,
                                (kb | k) != 0 ? 1u : 0u);
             else
@@ -595,7 +611,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     for (int t = unit; t < ntiles; t += n_units, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP>(p, t);
+      const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP, KE>(p, t);
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
       if constexpr (EPI == EPI_SWIGLU) {
         // Lanes 0-63 hold the gate rows of features n0 + 64 rank + [0, 64), lanes
@@ -615,6 +631,15 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         const int fg = q & 1, th = q >> 1;
         const int feat = ti.n0 + 64 * (int)rank + 32 * fg + lane;
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+        // F8: the gate / up accumulators times s_in and their rows' scales; act
+        // leaves as E4M3 codes of act / s_act
+        float sg = 1.f, su = 1.f, inv_act = 1.f;
+        if constexpr (F8) {
+          const float s_in = __ldg(p.act_scale + 2 * ti.e);
+          sg = s_in * __ldg(p.w_scale + (size_t)ti.e * p.b_rows_per_group + feat);
+          su = s_in * __ldg(p.w_scale + (size_t)ti.e * p.b_rows_per_group + (p.b_rows_per_group >> 1) + feat);
+          inv_act = __fdiv_rn(1.f, __ldg(p.act_scale + 2 * ti.e + 1));
+        }
 #pragma unroll 1
         for (int c = 0; c < ti.n_valid; c += 32, ++kc) {
           uint32_t r[32];
@@ -636,14 +661,22 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float mine = __uint_as_float(th == 0 ? r[j] : r[j + 16]), other = take[j * 32 + lane];
-            a[j] = th == 0 ? silu_f(mine) * other : silu_f(other) * mine;
+            const float gate = (th == 0 ? mine : other) * sg, up = (th == 0 ? other : mine) * su;
+            a[j] = silu_f(gate) * up;
           }
           const int j0 = c + 16 * th;
           const int nj = min(16, ti.n_valid - j0);
-          __nv_bfloat16* dst = out + (size_t)(ti.m0 + j0) * p.ldo + feat;
+          if constexpr (F8) {
+            uint8_t* dst8 = static_cast<uint8_t*>(p.out) + (size_t)(ti.m0 + j0) * p.ldo + feat;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j < nj) dst[(size_t)j * p.ldo] = __float2bfloat16_rn(a[j]);
+            for (int j = 0; j < 16; ++j)
+              if (j < nj) dst8[(size_t)j * p.ldo] = (uint8_t)(pack_e4m3x2(a[j] * inv_act, 0.f) & 0xffu);
+          } else {
+            __nv_bfloat16* dst = out + (size_t)(ti.m0 + j0) * p.ldo + feat;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (j < nj) dst[(size_t)j * p.ldo] = __float2bfloat16_rn(a[j]);
+          }
         }
         if (aborted) continue;
       } else {
@@ -669,6 +702,13 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
         if (!aborted && !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, wc))) aborted = true;
         if (aborted) continue;
         tc_fence_after();
+        float4 dsc;   // F8: s_act x the scales of this lane's four output rows (after the transpose)
+        if constexpr (F8) {
+          const float s_act = __ldg(p.act_scale + 2 * ti.e + 1);
+          const float4 ws = __ldg(reinterpret_cast<const float4*>(p.w_scale + (size_t)ti.e * p.b_rows_per_group + fw +
+                                                                  4 * (lane & 7)));
+          dsc = make_float4(s_act * ws.x, s_act * ws.y, s_act * ws.z, s_act * ws.w);
+        }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int c = 32 * part + 64 * k;
@@ -676,7 +716,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
           uint32_t r[32];
           tmem_ld32(tbase + c, r);
           tmem_ld_wait();
-          merge_chunk_swap(p, min(32, ti.n_valid - c), fw, tokk[k], wk[k], r, sT + (warp - 2) * 1024);
+          merge_chunk_swap(p, min(32, ti.n_valid - c), fw, tokk[k], wk[k], r, sT + (warp - 2) * 1024,
+                           F8 ? &dsc : nullptr);
         }
       }
       tc_fence_before();
@@ -694,7 +735,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<EPI>(), 1)
     for (int t = unit; t < ntiles; t += n_units, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP>(p, t);
+      const TileInfo ti = tile_info<EPI, BN_OUT, TM, SWAP, KE>(p, t);
       float* prm = sPrm + acc * 4 * BN_OUT;
       if constexpr (is_merge<EPI>()) {
         // this tile's merge parameters (hb, hs, rb, rs for its columns) into shared memory
@@ -767,11 +808,11 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <int BN, int EPI, int CG, bool SWAP = false>
+template <int BN, int EPI, int CG, bool SWAP = false, bool F8 = false>
 int launch_impl(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, int ntiles_hint, int num_sms,
                 cudaStream_t st) {
   using C = GemmCfg<BN, EPI, CG, SWAP>;
-  auto kern = gemm_tc_kernel<BN, EPI, CG, SWAP>;
+  auto kern = gemm_tc_kernel<BN, EPI, CG, SWAP, F8>;
   static bool attr_set = false;
   static int max_pairs = 0;   // co-resident CTA pairs (CG = 2)
   if (!attr_set) {
@@ -817,6 +858,21 @@ int launch_impl(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& 
 
 }  // namespace
 
+// E4M3 bytes: a box of box_rows x 128 (one 128-byte swizzled row per row).
+int make_tmap_u8(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return ZAYA_ERR_CUDA;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || cols % 16) return ZAYA_ERR_MISALIGNED;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ZAYA_OK : ZAYA_ERR_CUDA;
+}
+
 int make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return ZAYA_ERR_CUDA;
@@ -833,6 +889,22 @@ int make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t co
 
 int launch_gemm(int epi, int bn, const void* A, int a_rows, const void* B, int b_rows, const GemmParams& p,
                 int num_sms, cudaStream_t st) {
+  if (p.fp8) {   // E4M3 expert GEMMs: swapped CTA pairs only
+    if (!p.grouped || !p.pair || bn != 256 || (epi != EPI_SWIGLU && epi != EPI_MERGE_MLP) || p.K % (2 * BK) ||
+        p.K <= 0 || !p.w_scale || !p.act_scale)
+      return ZAYA_ERR_UNSUPPORTED;
+    if (p.N % (epi == EPI_SWIGLU ? bn / 2 : bn)) return ZAYA_ERR_UNSUPPORTED;
+    if (a_rows <= 0) return ZAYA_OK;
+    GemmParams q = p;
+    q.tok_box = 16;
+    CUtensorMap ma, mb;
+    int rc = make_tmap_u8(&ma, A, (uint64_t)a_rows, (uint64_t)p.K, (uint32_t)q.tok_box);
+    if (rc) return rc;
+    rc = make_tmap_u8(&mb, B, (uint64_t)b_rows, (uint64_t)p.K, epi == EPI_SWIGLU ? 64 : 128);
+    if (rc) return rc;
+    return epi == EPI_SWIGLU ? launch_impl<256, EPI_SWIGLU, 2, true, true>(ma, mb, q, num_sms, num_sms, st)
+                             : launch_impl<256, EPI_MERGE_MLP, 2, true, true>(ma, mb, q, num_sms, num_sms, st);
+  }
   if (p.K % BK != 0 || p.K <= 0) return ZAYA_ERR_UNSUPPORTED;
   const int ks = p.k_splits > 1 ? p.k_splits : 1;
   if ((p.K / BK) % ks != 0 || (ks > 1 && (p.grouped || epi != EPI_STORE_F32))) return ZAYA_ERR_UNSUPPORTED;

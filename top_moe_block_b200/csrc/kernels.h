@@ -41,6 +41,9 @@ struct GemmParams {
   void* tap_bf16;            // MERGE_*: optional bf16 [tokens, N] contribution tap
   float* tap_f32;            // MERGE_ATTN: optional fp32 [tokens, N] layer_mid tap
   int tok_box;               // set by launch_gemm: swapped tiles' token box rows (16)
+  int fp8;                   // grouped experts: A rows and B weights are E4M3 bytes (tcgen05 kind::f8f6f4)
+  const float* w_scale;      // fp8: [E, b_rows_per_group] fp32 per-row weight scales
+  const float* act_scale;    // fp8: [E, 2] static input scales (gate/up input, down input)
 };
 
 // Encodes a 2-D bf16 tensor map (rows x cols, row-major) with a box of
@@ -215,7 +218,8 @@ struct DispatchParams {
   int* mt_start;          // [E+2] out: prefix of per-expert tile counts (tile_rows rows) (CTA 0)
   int tile_rows;
   const void* m_in;       // bf16 [M, H]
-  void* x_perm;           // bf16 [M, H]
+  void* x_perm;           // bf16 [M, H]; with in_scale E4M3 bytes of m_in / in_scale[2e]
+  const float* in_scale;  // FP8 experts: [E, 2] static input scales, or null
   float* stream;          // [M, H] in: layer_mid; skip rows -> layer_output
   const float* merge_m;   // [4, H]
   void* tap_mlp_out;      // optional bf16 [M, H]

@@ -620,7 +620,23 @@ __global__ void __launch_bounds__(256) dispatch_kernel(const DispatchParams p) {
     p.pos[t] = row;
     p.perm[row] = t;
   }
-  if (c < p.E) {
+  if (c < p.E && p.in_scale) {   // FP8 experts: the row as E4M3 codes of x / s_in
+    const float s_in = __ldg(p.in_scale + 2 * c);
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * H);
+    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.x_perm) + (size_t)row * H);
+    for (int ch = lane; ch < per_row; ch += 32) {
+      const uint4 v = src[ch];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 a = unpack_bf2(w[2 * h]), b = unpack_bf2(w[2 * h + 1]);
+        o[h] = (uint32_t)pack_e4m3x2(__fdiv_rn(a.x, s_in), __fdiv_rn(a.y, s_in)) |
+               ((uint32_t)pack_e4m3x2(__fdiv_rn(b.x, s_in), __fdiv_rn(b.y, s_in)) << 16);
+      }
+      dst[ch] = make_uint2(o[0], o[1]);
+    }
+  } else if (c < p.E) {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.m_in) + (size_t)t * H);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.x_perm) + (size_t)row * H);
     constexpr int kV = 8;

@@ -132,6 +132,8 @@ int check_config(const zaya_config* c) {
   // a window ring needs a window on every block
   if (c->kv_ring != 0 && (c->kv_ring != 1 || c->sliding_period > 0)) return ZAYA_ERR_INVALID_ARG;
   if (c->kv_fp8 != 0 && c->kv_fp8 != 1) return ZAYA_ERR_INVALID_ARG;
+  if (c->expert_fp8 != 0 && c->expert_fp8 != 1) return ZAYA_ERR_INVALID_ARG;
+  if (c->expert_fp8 && (c->inter % 128 || c->hidden % 256)) return ZAYA_ERR_UNSUPPORTED;   // swapped pair tiles
   return ZAYA_OK;
 }
 
@@ -163,6 +165,9 @@ int check_weights(const zaya_block_weights* w, const zaya_config* c) {
   if (!w) return ZAYA_ERR_INVALID_ARG;
   if (c->conv_groups > 0 && (!w->conv2_w || !w->conv2_b)) return ZAYA_ERR_INVALID_ARG;
   if (c->conv_groups > 0 && (!a16(w->conv2_w) || !a16(w->conv2_b))) return ZAYA_ERR_MISALIGNED;
+  if (c->expert_fp8 && (!w->w_gate_up_scale || !w->w_down_scale || !w->expert_act_scale)) return ZAYA_ERR_INVALID_ARG;
+  if (c->expert_fp8 && (!a16(w->w_gate_up_scale) || !a16(w->w_down_scale) || !a16(w->expert_act_scale)))
+    return ZAYA_ERR_MISALIGNED;
   const void* ptrs[] = {w->ln1_w, w->ln2_w, w->w_qkv, w->conv_w, w->conv_b, w->k_temp, w->w_o, w->merge_a,
                         w->merge_m, w->router_down_w, w->router_down_b, w->router_state_scale, w->router_norm_w,
                         w->fc1_w, w->fc1_b, w->fc2_w, w->fc2_b, w->out_w, w->balancing, w->w_gate_up, w->w_down};
@@ -324,6 +329,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.cls = cls; p.class_count = at<int>(ws, L.ccount); p.slot = at<int>(ws, L.slot);
     p.pos = pos; p.perm = perm; p.group_off = group_off; p.mt_start = mt_start; p.tile_rows = pair ? 256 : 128;
     p.m_in = m_in; p.x_perm = xperm; p.stream = hidden; p.merge_m = w->merge_m;
+    p.in_scale = c.expert_fp8 ? w->expert_act_scale : nullptr;
     p.tap_mlp_out = taps ? taps->mlp_output : nullptr;
     p.cache_len_inc = cache_len_inc;
     p.status = status;
@@ -336,6 +342,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.M = M; p.N = d.I; p.K = d.H; p.grouped = 1; p.group_off = group_off; p.mt_start = mt_start;
     p.n_groups = d.E; p.b_rows_per_group = 2 * d.I; p.status = status; p.pair = pair;
     p.out = act; p.ldo = d.I;
+    p.fp8 = c.expert_fp8; p.w_scale = w->w_gate_up_scale; p.act_scale = w->expert_act_scale;
     ZAYA_STAGE("experts_gate_up", 1, launch_gemm(EPI_SWIGLU, 256, xperm, M, w->w_gate_up, d.E * 2 * d.I, p, sms, st));
   }
   {  // experts: down + weight + merge 2, scattered back to token rows
@@ -344,6 +351,7 @@ int block_tail(const zaya_config& c, const Derived& d, const zaya_block_weights*
     p.n_groups = d.E; p.b_rows_per_group = d.H; p.status = status; p.pair = pair;
     p.stream = hidden; p.merge = w->merge_m; p.perm = perm; p.row_w = wgt;
     p.tap_bf16 = taps ? taps->mlp_output : nullptr;
+    p.fp8 = c.expert_fp8; p.w_scale = w->w_down_scale; p.act_scale = w->expert_act_scale;
     const int c2[] = {256, 128};
     const int bn = pair ? (d.H % 256 == 0 ? 256 : 128) : pick_bn_tiles((M + 127) / 128 + d.E / 2, d.H, c2, 2, sms);
     ZAYA_STAGE("experts_down_merge", 1, launch_gemm(EPI_MERGE_MLP, bn, act, M, w->w_down, d.E * d.H, p, sms, st));
