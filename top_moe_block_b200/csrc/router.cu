@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   __nv_bfloat16* wring = reinterpret_cast<__nv_bfloat16*>(
       Sh::TMA ? (reinterpret_cast<uintptr_t>(zl + kTM * kAS) + 1023) & ~uintptr_t(1023)
               : reinterpret_cast<uintptr_t>(zl + kTM * kAS));
-  __shared__ uint64_t wfull[4];   // TMA mode: chunk landed in ring stage s
+  __shared__ uint64_t wfull[2];   // TMA mode: chunk landed in ring stage s
   const int E1 = p.E + 1;
   const int t0 = blockIdx.x * kTM;
   const int warp = warp_id(), lane = lane_id();
@@ -248,23 +248,17 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     lo_w = __any_sync(0xffffffffu, any != 0);
   }
   lo_w = __syncthreads_or(lo_w);
-  // The ring holds four chunks' worth of bf16 (two stages of hi + lo).  With
-  // hi parts only it is a four-stage ring, so three chunks stream in while one
-  // is multiplied (a small batch's few CTAs are bound by the chunks' latency).
-  const int nst = (Sh::TMA && !lo_w) ? 4 : 2;
-  const int sstride = (Sh::TMA && !lo_w) ? Sh::CHUNK : 2 * Sh::CHUNK;
-  // weight chunk q of the fc1 -> fc2 sequence into ring stage q % nst: TMA
-  // boxes (hi, and lo if any) of [R rows][64 columns] on the stage's barrier,
-  // issued by thread 0; or (R = 32) one cp.async group of all threads
+  // weight chunk q of the fc1 -> fc2 sequence into ring stage q & 1: two TMA
+  // boxes (hi, lo) of [R rows][64 columns] on the stage's barrier, issued by
+  // thread 0; or (R = 32) one cp.async group of all threads
   auto stage_w = [&](int q) {
     if constexpr (Sh::TMA) {
       if (threadIdx.x == 0) {
-        uint64_t* bar = &wfull[q % nst];
-        __nv_bfloat16* dst = wring + (q % nst) * sstride;
+        uint64_t* bar = &wfull[q & 1];
         mbar_arrive_expect_tx(bar, (lo_w ? 2 : 1) * Sh::CHUNK * (uint32_t)sizeof(__nv_bfloat16));
         const int row = (q / nch) * 2 * R;   // layer q / nch: hi rows, then lo rows
-        tma_load_2d(dst, &tmW, bar, (q % nch) * Sh::KCH, row);
-        if (lo_w) tma_load_2d(dst + Sh::CHUNK, &tmW, bar, (q % nch) * Sh::KCH, row + R);
+        tma_load_2d(wring + (q & 1) * 2 * Sh::CHUNK, &tmW, bar, (q % nch) * Sh::KCH, row);
+        if (lo_w) tma_load_2d(wring + (q & 1) * 2 * Sh::CHUNK + Sh::CHUNK, &tmW, bar, (q % nch) * Sh::KCH, row + R);
       }
     } else {
       const __nv_bfloat16* whi = p.wsplit + (size_t)(q / nch) * 2 * n;
@@ -273,18 +267,14 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   };
   if constexpr (Sh::TMA) {
     if (threadIdx.x == 0) {
-      for (int s = 0; s < 4; ++s) mbar_init(&wfull[s], 1);
+      mbar_init(&wfull[0], 1);
+      mbar_init(&wfull[1], 1);
       fence_barrier_init();
       prefetch_tmap(&tmW);
     }
   }
   const WaitCtx wc = wait_ctx(p.status);
-  // the first fc1 chunks (one per stage but the last) stream in under the state assembly
-  int n_staged = 0;  // TMA mode, thread 0: chunks whose copies were started
-  for (int q = 0; q < nst - 1 && q < 2 * nch; ++q) {
-    stage_w(q);
-    ++n_staged;
-  }
+  stage_w(0);   // the first fc1 chunk streams in under the state assembly
 
   // router state r = down_proj partial sums (in slab order) + bias (+ previous
   // state * scale).  Each thread owns kPos float4 positions; the loads of two
@@ -386,25 +376,21 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   const int NP = router_np(E1);
   constexpr int OWS = R + 8;
   const bool ow_in_ring = (size_t)2 * NP * OWS <= (size_t)2 * Sh::CHUNK;
-  // the four-stage ring's last chunk sits in its last stage, so the first two
-  // stages are free by then
-  __nv_bfloat16* ow = !ow_in_ring ? wring + 4 * Sh::CHUNK
-                      : nst == 4  ? wring
-                                  : wring + ((2 * nch) & 1) * 2 * Sh::CHUNK;
+  __nv_bfloat16* ow = ow_in_ring ? wring + ((2 * nch) & 1) * 2 * Sh::CHUNK : wring + 4 * Sh::CHUNK;
   float acc[Sh::NTW][4];
 #pragma unroll
   for (int j = 0; j < Sh::NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
   bool ok = true;   // TMA mode: false once a chunk wait has run out (status set)
+  int n_staged = 1;  // TMA mode, thread 0: chunks whose copies were started
   for (int q = 0; q < 2 * nch; ++q) {
-    if (q + nst - 1 < 2 * nch) {
-      // into the stage chunk q - 1 has left; after a failed wait no further
-      // chunk is started (its stage may still be receiving the chunk that
-      // never arrived in time)
+    if (q + 1 < 2 * nch) {
+      // after a failed wait no further chunk is started (its stage may still
+      // be receiving the chunk that never arrived in time)
       if (!Sh::TMA || ok) {
-        stage_w(q + nst - 1);
+        stage_w(q + 1);
         ++n_staged;
       }
-    } else if (q + 1 == 2 * nch) {
+    } else {
       const __nv_bfloat16* ows = p.wsplit + (size_t)4 * R * R;   // [hi|lo][NP][R]
       for (int i = threadIdx.x; i < (lo_w ? 2 : 1) * NP * (R / 8); i += kThreads) {
         const int row = i / (R / 8), c = i % (R / 8);   // row over hi rows then lo rows
@@ -416,10 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
     }
     asm volatile("cp.async.wait_group 1;" ::: "memory");
     if constexpr (Sh::TMA) {   // every thread sees chunk q land (bounded wait)
-      if (ok && !mbar_wait(&wfull[q % nst], (uint32_t)(q / nst) & 1u, wc)) ok = false;
+      if (ok && !mbar_wait(&wfull[q & 1], (uint32_t)(q >> 1) & 1u, wc)) ok = false;
     }
     __syncthreads();
-    const __nv_bfloat16* wh = Sh::TMA ? wring + (q % nst) * sstride : wring + (q & 1) * 2 * Sh::CHUNK;
+    const __nv_bfloat16* wh = wring + (q & 1) * 2 * Sh::CHUNK;
     if (lo_w) mlp_chunk<R, true>(zh, zl, acc, wh, wh + Sh::CHUNK, q % nch);
     else mlp_chunk<R, false>(zh, zl, acc, wh, wh + Sh::CHUNK, q % nch);
     if (q == nch - 1) {   // fc1 done: its GELU output becomes fc2's operand (in place)
@@ -434,8 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(const RouterParams 
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   if constexpr (Sh::TMA) {   // every chunk copy started has landed before the CTA can exit
     if (threadIdx.x == 0)
-      for (int q = (n_staged > nst ? n_staged - nst : 0); q < n_staged; ++q)
-        mbar_drain(&wfull[q % nst], (uint32_t)(q / nst) & 1u, p.status);
+      for (int q = (n_staged > 2 ? n_staged - 2 : 0); q < n_staged; ++q)
+        mbar_drain(&wfull[q & 1], (uint32_t)(q >> 1) & 1u, p.status);
   }
   __syncthreads();
   // out_proj (no bias) on tensor cores with the same hi / lo split: tile w < 2 * NP / 8
