@@ -389,28 +389,50 @@ def run_prefill(args, world, rank, local, cfg):
     stages = ZB.zaya_profile_read()
     ZB.zaya_profile_enable(False)
 
-    # ---- pass 3: end to end from pinned host buffers (H2D in, D2H out, per step)
+    # ---- pass 3: end to end from pinned host buffers, streamed: every step
+    # copies its inputs in (H2D stream) and its layer_output and router state
+    # out (D2H stream); two device slots let step i's copies overlap the
+    # blocks of steps i -+ 1 on the compute stream (one call of the public API
+    # per step, as a caller streaming batches would make them)
     x_h = x0.cpu().pin_memory()
     rin_h = None if rin is None else rin.cpu().pin_memory()
-    out_h = torch.empty_like(x_h).pin_memory()
-    rout_h = torch.empty(B, S, R, dtype=torch.float32).pin_memory()
-    e2e = []
+    out_h = [torch.empty_like(x_h).pin_memory() for _ in range(2)]
+    rout_h = [torch.empty(B, S, R, dtype=torch.float32).pin_memory() for _ in range(2)]
+    hid2 = [hidden, torch.empty_like(hidden)]
+    rin2 = [rin, None if rin is None else torch.empty_like(rin)]
+    rout2 = [rout, torch.empty_like(rout)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(K)]
+    ev_done = [torch.cuda.Event() for _ in range(K)]
+    ev_out = [torch.cuda.Event() for _ in range(K)]
+    t_a, t_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_a.record(s_in)
     for i in range(K):
+        j = i & 1
+        with torch.cuda.stream(s_in):
+            if i >= 2:   # slot j's previous outputs have been read back (so its block is done too)
+                s_in.wait_event(ev_out[i - 2])
+            hid2[j].copy_(x_h, non_blocking=True)
+            if rin is not None:
+                rin2[j].copy_(rin_h, non_blocking=True)
+            ev_in[i].record(s_in)
+        stream.wait_event(ev_in[i])
         flush.fill_(i & 0xFF)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        hidden.copy_(x_h, non_blocking=True)
-        if rin is not None:
-            rin.copy_(rin_h, non_blocking=True)
-        step()
-        out_h.copy_(hidden, non_blocking=True)
-        rout_h.copy_(rout, non_blocking=True)
-        b.record(stream)
-        torch.cuda.synchronize()
-        e2e.append(a.elapsed_time(b))
-    e2e_ms = max_over_ranks(sum(e2e), world) / K
+        ZB.zaya_block_prefill(c, w_s, cfg.block_idx, B, S, hid2[j], mask, rin2[j], rout2[j], st_s, None, ws,
+                              stream=stream)
+        ev_done[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[i])
+            out_h[j].copy_(hid2[j], non_blocking=True)
+            rout_h[j].copy_(rout2[j], non_blocking=True)
+            ev_out[i].record(s_out)
+    t_b.record(s_out)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t_a.elapsed_time(t_b), world) / K
+    assert ZB.zaya_device_status(ws, stream) == 0
     h2d = x_h.numel() * 4 + (0 if rin_h is None else rin_h.numel() * 4)
-    d2h = out_h.numel() * 4 + rout_h.numel() * 4
+    d2h = out_h[0].numel() * 4 + rout_h[0].numel() * 4
 
     ms_per_step = total_ms / K
     tokens = sum(shard_tokens(M, world))
