@@ -114,8 +114,8 @@ typedef struct zaya_config {
                                 so a sequence decodes past cache_cap with a window-sized cache
                                 (the pages' decode reads the window only: zaya page, "Queries and
                                 keys are convolved ..."; every block must slide: sliding_period 0) */
-  int32_t expert_fp8;        /* 1: the experts as an FP8 W8A8 checkpoint (the pages'
-                                deployments quantise the experts: NVFP4 README, "Quantization
+  int32_t expert_fp8;        /* 1: the experts as an FP8 W8A8 checkpoint (the pages' deployments
+                                quantise the experts: NVFP4 README, "Quantization
                                 details"): E4M3 weight codes with per-row fp32 scales, inputs
                                 quantised to E4M3 with static per-expert scales, products on the
                                 tensor cores in E4M3 (tcgen05 kind::f8f6f4), fp32 accumulation;

@@ -321,8 +321,8 @@ def expert_ffn(x, w_gate_up_e, w_down_e, inter):
 
 def expert_ffn_fp8(x, wgu_e, sgu_e, wdn_e, sdn_e, s_in, s_act, inter):
     """The SwiGLU expert with FP8 (E4M3) weights and activations, the scheme
-    of an FP8 W8A8 checkpoint (the pages' own deployments
-    quantise the experts, NVFP4 README "Quantization details"): weights are
+    of an FP8 W8A8 checkpoint (the pages' own deployments quantise the
+    experts, NVFP4 README "Quantization details"): weights are
     E4M3 values wgu_e [2I,H], wdn_e [H,I] with one fp32 scale per output row
     (sgu_e [2I], sdn_e [H]); each input is quantised with a static per-expert
     scale, x_q = E4M3(x / s_in) and act_q = E4M3(act / s_act); a product
