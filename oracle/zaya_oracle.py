@@ -27,7 +27,12 @@ are rounded where the pages fix a dtype and nowhere else:
   conv_state [B,1280,2] carries (JANGTQ2 README, "Architecture Summary");
 * the KV cache holds bf16 keys and values (llm-atlas card, "kvCacheText":
   40 KiB per token = 40 layers x (K+V) x 2 heads x 128 x 2 bytes), so keys
-  and values are rounded to bf16 where they enter the attention;
+  and values are rounded to bf16 where they enter the attention; with the
+  fp8 cache option (``kv_fp8``, the NVFP4 README's ``--kv-cache-dtype fp8``)
+  the cache holds them rounded on to E4M3 and a decode step reads those;
+* with the FP8 expert option (``expert_fp8``) the experts take E4M3 weight
+  codes with per-row scales and quantise their inputs to E4M3 with static
+  scales (``expert_ffn_fp8``);
 * the router's choice is taken on float32 softmax scores
   (``logits.float().softmax(-1)``, zaya page, "One expert per token"), so the
   logits are rounded to fp32 and the softmax, the bias add and the argmax run
