@@ -60,3 +60,25 @@ def test_decode_bytes_closed_forms():
     assert gate_up + down > 16 * expert
     assert w["lm_head"][1] == 262144 * 2048 * 2 + 64 * 2048 * 2 + 64 * 262144 * 2
     assert all(v[0] == "hbm" for v in w.values())
+
+
+def test_fp8_variants_work_and_peaks():
+    """The fp8 variants' algorithmic work: the E4M3 cache halves the window's
+    K/V bytes, FP8 experts halve their weight bytes in decode and are held
+    against twice the bf16 dense peak in prefill (the nominal E4M3 / bf16
+    ratio times the measured bf16 figure)."""
+    b = _bench()
+    d16 = b.stage_work_decode(get_config("decode_stack_b64"), routed=64, distinct=6)
+    dkv = b.stage_work_decode(get_config("decode_stack_b64_fp8kv"), routed=64, distinct=6)
+    dx = b.stage_work_decode(get_config("decode_stack_b64_fp8x"), routed=64, distinct=6)
+    kv = 64 * 2 * 4096 * 128 * 2 * 2
+    assert d16["attention_decode"][1] - dkv["attention_decode"][1] == kv // 2
+    assert d16["experts_gate_up"][1] - dx["experts_gate_up"][1] == 6 * 2 * 2048 * 2048
+    assert d16["experts_down_merge"][1] - dx["experts_down_merge"][1] == 6 * 2048 * 2048
+    w = b.stage_work(get_config("prefill_4k_fp8x"), 4093, 8390656)
+    assert w["experts_gate_up"][0] == "tensor_f8" and w["qkv_gemm"][0] == "tensor"
+    peaks = {"bf16_tflops": 1665.3, "bf16_tflops_sustained": 1404.1, "hbm_gbs": 6455.6}
+    cfg = get_config("prefill_4k_fp8x")
+    r = b.roofline({"experts_gate_up": (0.0604, 1)}, w, peaks, "measured", cfg, 0.314)
+    assert r["peak"] == round(2 * 1665.3, 1) and r["bound"] == "tensor"
+    assert abs(r["achieved"] - w["experts_gate_up"][1] / 60.4e-6 / 1e12) < 0.01
